@@ -1,0 +1,222 @@
+/*
+ * rrf_oracle.c -- the oracle for the fused "R-way bf16 sum + residual +
+ * RMSNorm + dynamic per-row FP8 (e4m3fn) quantisation" operation.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is a plain, slow, single-threaded CPU
+ * statement of what the operation computes.  Only the test suite, the smoke
+ * check and the CPU-baseline leg of the benchmark may build, load or call it.
+ * It shares no code, header, table or constant with the CUDA library, and the
+ * library never calls it: a missing CUDA extension is an error, not a reason
+ * to fall back to this file.
+ *
+ * Sources (web pages, cited by title and section):
+ *  - Modular docs, Mojo function `allreduce_rmsnorm_fp8` (module
+ *    nn/allreduce_residual_rmsnorm_fp8), "Args": per-GPU input buffers with
+ *    last dim = cols, FP8 output of the input's shape, 1-D gamma of length
+ *    cols, epsilon, weight_offset ("additive offset for gamma weights"),
+ *    scale_ub ("upper bound for FP8 scale clamping"), per-row scales with last
+ *    dim 1; in_dtype bfloat16, out_dtype float8_e4m3fn, scales float32.
+ *  - local-inference-lab/b12x PR #283 "PCIeTwoShotBF16", opening description
+ *    and "Behavior": the partials are accumulated in fp32 in a fixed rank
+ *    order and the result is rounded to bf16 once, so it is deterministic and
+ *    lies within one bf16 rounding of the exact sum.
+ *  - NVIDIA/TensorRT-LLM PR #19836, "Description": the RESIDUAL_RMS_NORM
+ *    epilogue adds a residual before the norm.
+ *  - Tenstorrent rmsnorm_2d.py, `_resolve_2d_config` (add_unit_offset adds
+ *    1.0 to the weight): weight_offset is added to gamma before it scales.
+ *  - Huawei Ascend aclnnAlltoAllQuantMatmul, quant-mode list, mode 7
+ *    "per-token dynamic quantization": one scale per row, from the row's data.
+ *
+ * The pages name the parameters but print no formula.  This file takes the
+ * plainest reading, the textbook RMSNorm followed by amax-scaled FP8
+ * quantisation.  Per row i, with x_r the R bf16 inputs:
+ *   1. acc_j = f32(x_0[i,j]); acc_j = acc_j + f32(x_r[i,j]) for r = 1..R-1,
+ *      each an IEEE fp32 add (no fused multiply-add); s_j = RN_bf16(acc_j).
+ *   2. with a residual: h_j = RN_bf16(f32(s_j) + f32(res_in[i,j])), written
+ *      to res_out; without one: h_j = s_j.
+ *   3. ss = sum_j h_j^2 in float64 (each term and, at these sizes, the sum
+ *      are exact); ms = f32(ss) / f32(cols); r = 1 / sqrtf(ms + eps), all fp32.
+ *   4. y_j = (f32(h_j) * r) * (f32(gamma_j) + weight_offset), fp32.
+ *   5. amax = max_j |y_j|; scale = max(min(amax, scale_ub), 1e-12) / 448.
+ *   6. q_j = e4m3fn(y_j / scale), round to nearest even, finite values and
+ *      infinities beyond 448 saturate to +-448, NaN gives 0x7F.
+ *      scales[i] = scale (the dequantisation multiplier: y ~ f32(q) * scale).
+ *
+ * Build with -ffp-contract=off (no FMA contraction) and without fast-math, so
+ * every fp32 operation above is one IEEE-rounded operation.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <string.h>
+
+#define E4M3_MAX 448.0
+#define SCALE_FLOOR 1e-12f
+
+/* ---------------------------------------------------------------- bf16 --- */
+
+/* bf16 is the top 16 bits of an IEEE binary32. */
+float oracle_bf16_to_float(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+static double bf16_magnitude_for_rounding(uint16_t b) {
+    /* Rounding behaves as if the exponent range were unbounded and then
+     * overflows to infinity, so the encoding 0x7F80 (infinity) stands for
+     * 2^128 while the nearest neighbour is chosen. */
+    if ((b & 0x7FFF) == 0x7F80) return ldexp(1.0, 128);
+    return fabs((double)oracle_bf16_to_float(b));
+}
+
+/* Round an fp32 value to the nearest bf16, ties to the even encoding (IEEE
+ * round-to-nearest-even).  The candidates are the bf16 value nearer zero
+ * (truncation of the low 16 bits) and the next one away from zero. */
+uint16_t oracle_bf16_round(float f) {
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if (isnan(f)) return (uint16_t)((u >> 16) | 0x0040); /* stays a quiet NaN */
+    uint16_t lo = (uint16_t)(u >> 16);
+    if ((lo & 0x7FFF) >= 0x7F80) return lo; /* infinity stays infinity */
+    uint16_t hi = (uint16_t)(lo + 1);
+    double a = fabs((double)f);
+    double dlo = a - bf16_magnitude_for_rounding(lo);
+    double dhi = bf16_magnitude_for_rounding(hi) - a;
+    if (dlo < dhi) return lo;
+    if (dhi < dlo) return hi;
+    return (lo & 1) ? hi : lo;
+}
+
+/* -------------------------------------------------------------- e4m3fn --- */
+
+/* Value of an e4m3fn code: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa
+ * bits; exponent field 0 holds subnormals m * 2^-9; S.1111.111 is NaN; there
+ * is no infinity, so S.1111.110 = 1.75 * 2^8 = 448 is the largest finite. */
+double oracle_e4m3_decode(uint8_t c) {
+    int s = c >> 7, e = (c >> 3) & 0xF, m = c & 0x7;
+    if (e == 0xF && m == 0x7) return NAN;
+    double mag = (e == 0) ? ldexp((double)m, -9) : ldexp((double)(8 + m), e - 10);
+    return s ? -mag : mag;
+}
+
+/* Nearest e4m3fn code to v, ties to the even code, saturating: any finite or
+ * infinite magnitude above 448 becomes +-448; NaN becomes 0x7F.  The search
+ * runs over all 127 non-negative finite codes, which is slow on purpose. */
+uint8_t oracle_e4m3_encode(float v) {
+    if (isnan(v)) return 0x7F;
+    uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    double a = fabs((double)v);
+    if (a > E4M3_MAX) return (uint8_t)(sign | 0x7E);
+    int best = 0;
+    double best_d = INFINITY;
+    for (int c = 0; c <= 0x7E; ++c) {
+        double d = fabs(a - oracle_e4m3_decode((uint8_t)c));
+        if (d < best_d || (d == best_d && (c & 1) == 0)) {
+            best = c;
+            best_d = d;
+        }
+    }
+    return (uint8_t)(sign | best);
+}
+
+/* ---------------------------------------------------------- vectorised --- */
+
+void oracle_bf16_round_array(const float* in, uint16_t* out, int64_t n) {
+    for (int64_t k = 0; k < n; ++k) out[k] = oracle_bf16_round(in[k]);
+}
+
+void oracle_e4m3_encode_array(const float* in, uint8_t* out, int64_t n) {
+    for (int64_t k = 0; k < n; ++k) out[k] = oracle_e4m3_encode(in[k]);
+}
+
+/* ------------------------------------------------------------ the sum --- */
+
+/* Step 1 for one element: fp32 accumulation in the fixed order 0..R-1,
+ * starting from the first input (not from +0, so all -0 inputs give -0),
+ * then a single rounding to bf16. */
+static uint16_t sum_element(const uint16_t* const* x, int R, int64_t k) {
+    float acc = oracle_bf16_to_float(x[0][k]);
+    for (int r = 1; r < R; ++r) acc = acc + oracle_bf16_to_float(x[r][k]);
+    return oracle_bf16_round(acc);
+}
+
+/* The bf16 sum alone: out[i, j] = RN_bf16(sum over r in order of x_r[i, j]).
+ * All arrays are row-major [rows, cols] of bf16 bit patterns. */
+void oracle_sum(const uint16_t* const* x, int R, int64_t rows, int64_t cols,
+                uint16_t* out) {
+    for (int64_t i = 0; i < rows; ++i)
+        for (int64_t j = 0; j < cols; ++j) out[i * cols + j] = sum_element(x, R, i * cols + j);
+}
+
+/* ---------------------------------------------------------- fused row --- */
+
+/* Steps 1-6 for the rows [row0, row0 + nrows).  res_in / res_out are both
+ * NULL (no residual) or both non-NULL; they may be the same array.  The
+ * optional outputs h_out (the bf16 norm input, [rows, cols]) and v_out (the
+ * fp32 pre-quantisation value y / scale, [rows, cols]) serve the tests. */
+void oracle_sum_rmsnorm_fp8_rows(const uint16_t* const* x, int R, int64_t row0,
+                                 int64_t nrows, int64_t cols, const uint16_t* res_in,
+                                 uint16_t* res_out, const uint16_t* gamma, float eps,
+                                 float weight_offset, float scale_ub, uint8_t* q,
+                                 float* scales, uint16_t* h_out, float* v_out) {
+    for (int64_t i = row0; i < row0 + nrows; ++i) {
+        const int64_t base = i * cols;
+
+        /* steps 1-2: the norm input h, one bf16 per element */
+        double ss = 0.0;
+        for (int64_t j = 0; j < cols; ++j) {
+            uint16_t s = sum_element(x, R, base + j);
+            uint16_t h = s;
+            if (res_in != NULL) {
+                float t = oracle_bf16_to_float(s) + oracle_bf16_to_float(res_in[base + j]);
+                h = oracle_bf16_round(t);
+                res_out[base + j] = h;
+            }
+            if (h_out != NULL) h_out[base + j] = h;
+            double hd = (double)oracle_bf16_to_float(h);
+            ss += hd * hd; /* step 3, float64 */
+        }
+        const uint16_t* hrow = (h_out != NULL) ? h_out + base
+                              : (res_out != NULL) ? res_out + base
+                                                  : NULL;
+
+        /* step 3: r = 1 / sqrt(mean(h^2) + eps) in fp32 */
+        float ms = (float)ss / (float)cols;
+        float r = 1.0f / sqrtf(ms + eps);
+
+        /* steps 4-5: y and its absolute maximum */
+        float amax = 0.0f;
+        for (int64_t j = 0; j < cols; ++j) {
+            float h = hrow ? oracle_bf16_to_float(hrow[j])
+                           : oracle_bf16_to_float(sum_element(x, R, base + j));
+            float g = oracle_bf16_to_float(gamma[j]) + weight_offset;
+            float y = (h * r) * g;
+            float ay = fabsf(y);
+            if (ay > amax) amax = ay;
+        }
+        float scale = fmaxf(fminf(amax, scale_ub), SCALE_FLOOR) / 448.0f;
+        scales[i] = scale;
+
+        /* step 6: quantise */
+        for (int64_t j = 0; j < cols; ++j) {
+            float h = hrow ? oracle_bf16_to_float(hrow[j])
+                           : oracle_bf16_to_float(sum_element(x, R, base + j));
+            float g = oracle_bf16_to_float(gamma[j]) + weight_offset;
+            float y = (h * r) * g;
+            float v = y / scale;
+            if (v_out != NULL) v_out[base + j] = v;
+            q[base + j] = oracle_e4m3_encode(v);
+        }
+    }
+}
+
+/* The whole operation over all rows. */
+void oracle_sum_rmsnorm_fp8(const uint16_t* const* x, int R, int64_t rows, int64_t cols,
+                            const uint16_t* res_in, uint16_t* res_out,
+                            const uint16_t* gamma, float eps, float weight_offset,
+                            float scale_ub, uint8_t* q, float* scales) {
+    oracle_sum_rmsnorm_fp8_rows(x, R, 0, rows, cols, res_in, res_out, gamma, eps,
+                                weight_offset, scale_ub, q, scales, NULL, NULL);
+}

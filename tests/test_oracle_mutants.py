@@ -1,0 +1,72 @@
+"""Plant one plausible mistake at a time in a copy of the oracle's C source
+(on the CPU, in a temporary directory) and require the pins to catch it.
+
+This shows that the pins constrain every step of the oracle: a dropped term,
+a wrong order, sign, index, constant or rounding rule fails at least one.
+"""
+import os
+
+import pytest
+
+import oracle
+import oracle_pins
+
+# (name, text in rrf_oracle.c, replacement)
+MUTANTS = [
+    ("sum starts from +0",
+     "float acc = oracle_bf16_to_float(x[0][k]);\n    for (int r = 1; r < R; ++r)",
+     "float acc = 0.0f;\n    for (int r = 0; r < R; ++r)"),
+    ("last input dropped", "for (int r = 1; r < R; ++r)", "for (int r = 1; r < R - 1; ++r)"),
+    ("float64 accumulator", "float acc = oracle_bf16_to_float(x[0][k]);",
+     "double acc = oracle_bf16_to_float(x[0][k]);"),
+    ("reversed rank order",
+     "for (int r = 1; r < R; ++r) acc = acc + oracle_bf16_to_float(x[r][k]);",
+     "for (int r = R - 1; r >= 1; --r) acc = acc + oracle_bf16_to_float(x[r][k]);"),
+    ("residual not added",
+     "float t = oracle_bf16_to_float(s) + oracle_bf16_to_float(res_in[base + j]);",
+     "float t = oracle_bf16_to_float(s);"),
+    ("eps outside the square root", "1.0f / sqrtf(ms + eps)", "1.0f / (sqrtf(ms) + eps)"),
+    ("mean over cols - 1", "(float)ss / (float)cols", "(float)ss / (float)(cols - 1)"),
+    ("weight offset dropped", "oracle_bf16_to_float(gamma[j]) + weight_offset;",
+     "oracle_bf16_to_float(gamma[j]);"),
+    ("weight offset subtracted", "oracle_bf16_to_float(gamma[j]) + weight_offset;",
+     "oracle_bf16_to_float(gamma[j]) - weight_offset;"),
+    ("no scale_ub clamp", "fminf(amax, scale_ub)", "amax"),
+    ("no scale floor", "fmaxf(fminf(amax, scale_ub), SCALE_FLOOR)", "fminf(amax, scale_ub)"),
+    ("e4m3fnuz maximum 240", "/ 448.0f", "/ 240.0f"),
+    ("scale applied as a multiplier", "float v = y / scale;", "float v = y * scale;"),
+    ("amax over h instead of y", "float ay = fabsf(y);", "float ay = fabsf(h);"),
+    ("row stride lost", "const int64_t base = i * cols;", "const int64_t base = i;"),
+    ("transposed sum index", "out[i * cols + j] = sum_element(x, R, i * cols + j);",
+     "out[i * cols + j] = sum_element(x, R, j * rows + i);"),
+    ("e4m3 ties away from zero", "(d == best_d && (c & 1) == 0)", "(d == best_d)"),
+    ("e4m3 loses the sign of zero", "uint8_t sign = signbit(v) ? 0x80 : 0x00;",
+     "uint8_t sign = (v < 0) ? 0x80 : 0x00;"),
+    ("e4m3 overflow to NaN", "if (a > E4M3_MAX) return (uint8_t)(sign | 0x7E);",
+     "if (a > E4M3_MAX) return 0x7F;"),
+    ("e4m3 exponent bias off by one", "ldexp((double)(8 + m), e - 10)",
+     "ldexp((double)(8 + m), e - 11)"),
+    ("bf16 ties away from zero", "return (lo & 1) ? hi : lo;", "return hi;"),
+    ("bf16 truncation", "if (dhi < dlo) return hi;", "if (0) return hi;"),
+]
+
+
+def _build_mutant(tmp_path, old, new):
+    with open(os.path.join(os.path.dirname(oracle.__file__), "rrf_oracle.c")) as fh:
+        src = fh.read()
+    assert src.count(old) >= 1, f"mutation site not found: {old!r}"
+    path = tmp_path / "mutant.c"
+    path.write_text(src.replace(old, new))
+    return oracle.Oracle(oracle.build(force=True, src=str(path), out=str(tmp_path / "m.so")))
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_mutant(tmp_path, name, old, new):
+    mutant = _build_mutant(tmp_path, old, new)
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(mutant)
+        except (AssertionError, ValueError, FloatingPointError):
+            caught.append(pin.__name__)
+    assert caught, f"no pin caught the mutant '{name}'"
