@@ -1,0 +1,538 @@
+"""Benchmark of the fused bf16 sum + residual + RMSNorm + per-row FP8 call.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl rrf|reference]
+
+One step is one pass of the operation over one batch of the workload: for
+the default "decode" workload (R = 8 bf16 inputs, 7168 columns, residual on)
+the four calls at 1, 8, 32 and 64 rows.  Inputs are resident in HBM when the
+timed region starts and rotate over buffer sets whose total exceeds three
+times the L2 cache, so every step reads cold HBM.  K steps are timed with
+CUDA events on the launching stream, bracketed by a barrier and a device
+synchronisation on both sides; the time is the maximum over ranks.
+
+value = algorithmic bytes of all ranks' steps / time, in GB/s, where one
+fused call moves R*rows*cols*2 + 4*rows*cols (residual read + write) +
+2*cols (gamma) + rows*cols (fp8 codes) + 4*rows (scales) bytes.
+
+Multi-GPU (torchrun, one process per GPU, NCCL only for the barrier and the
+max-over-ranks timing): rows are independent, so every rank runs its own
+batch with no data-path collective (weak scaling).
+
+--impl reference times the CPU oracle (single-threaded C) on a bounded sample
+of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "fused sum+RMSNorm+FP8 achieved HBM GB/s (% of B200 peak) and us/call"
+L2_FLUSH_FACTOR = 3  # rotating pool >= 3 x L2
+
+
+# ---------------------------------------------------------------- helpers ---
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def shard_rows(rows: int, world: int, rank: int):
+    """Contiguous row block [start, stop) of `rank` when `rows` independent
+    rows are split over `world` ranks (the first rows % world ranks get one
+    more)."""
+    base, extra = divmod(rows, world)
+    start = rank * base + min(rank, extra)
+    return start, start + base + (1 if rank < extra else 0)
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Maximum of a per-rank float over all ranks (identity without a
+    process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def workload_cases(name: str):
+    """(rows, residual) of every call one step makes."""
+    w = workloads.WORKLOADS[name]
+    return [(rows, w.residual) for rows in w.rows]
+
+
+def step_bytes(name: str) -> int:
+    w = workloads.WORKLOADS[name]
+    return sum(workloads.fused_bytes(w.R, rows, w.cols, res) for rows, res in
+               workload_cases(name))
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            p = json.load(fh)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """Polls NVML for the SM clock and the active clock-event reasons of one
+    GPU on a background thread while the timed region runs."""
+
+    REASONS = {  # NVML clocks-event-reason bits
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting"}
+
+    def __init__(self, index: int):
+        self.samples, self.reasons = [], 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nvml = None
+
+    def _run(self):
+        n = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM))
+                self.reasons |= int(n.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+            except Exception:
+                break
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self):
+        if self._nvml is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        reasons = [name for bit, name in self.REASONS.items()
+                   if self.reasons & bit and name != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples)}
+
+
+# -------------------------------------------------------------- CUDA arm ---
+
+class DevicePool:
+    """Rotating buffer sets for one workload: per set and call, the R inputs,
+    the residual, gamma and the outputs, all resident in HBM."""
+
+    def __init__(self, name: str, device, min_bytes: int):
+        import torch
+        self.name = name
+        w = workloads.WORKLOADS[name]
+        self.cases = []
+        for rows, residual in workload_cases(name):
+            c = workloads.make_case(name, rows, device=device)
+            self.cases.append(c)
+        per_set = step_bytes(name)
+        self.n_sets = max(2, math.ceil(min_bytes / per_set))
+        self.sets = []
+        for _ in range(self.n_sets):
+            calls = []
+            for c in self.cases:
+                calls.append(dict(
+                    inputs=[x.clone() for x in c.inputs],
+                    residual=None if c.residual is None else c.residual.clone(),
+                    res_out=None if c.residual is None else torch.empty_like(c.residual),
+                    gamma=c.gamma.clone(),
+                    q=torch.empty(c.inputs[0].shape, dtype=torch.float8_e4m3fn, device=device),
+                    scales=torch.empty((c.rows, 1), dtype=torch.float32, device=device)))
+            self.sets.append(calls)
+        self.eps, self.wo, self.ub = w.eps, w.weight_offset, w.scale_ub
+
+    def run_step(self, rrf, k: int) -> int:
+        """Enqueue step k (every call of the workload on set k mod n); returns
+        the number of kernels launched."""
+        for b in self.sets[k % self.n_sets]:
+            rrf.rrf_sum_rmsnorm_fp8(b["inputs"], b["gamma"], self.eps, self.wo, self.ub,
+                                    residual_in=b["residual"], residual_out=b["res_out"],
+                                    q_out=b["q"], scales_out=b["scales"])
+        return len(self.cases)
+
+    def run_call(self, rrf, k: int, i: int) -> int:
+        b = self.sets[k % self.n_sets][i]
+        rrf.rrf_sum_rmsnorm_fp8(b["inputs"], b["gamma"], self.eps, self.wo, self.ub,
+                                residual_in=b["residual"], residual_out=b["res_out"],
+                                q_out=b["q"], scales_out=b["scales"])
+        return 1
+
+
+def time_region(fn, k_steps: int, device, stream):
+    """Device time of k_steps calls of fn(i), CUDA events on `stream`, with a
+    barrier and a synchronisation on both sides; max over ranks, seconds."""
+    import torch
+    barrier(device)
+    torch.cuda.synchronize(device)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(k_steps):
+        fn(i)
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    return max_over_ranks(start.elapsed_time(end) / 1e3, device)
+
+
+def capture_steps(fn, n: int, device):
+    """Capture fn(0) .. fn(n-1) into one CUDA graph; returns (graph, number
+    of kernels fn launched)."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    launched = 0
+    torch.cuda.synchronize(device)
+    with torch.cuda.graph(g):
+        for i in range(n):
+            launched += fn(i) or 1
+    torch.cuda.synchronize(device)
+    return g, launched
+
+
+def e2e_measure(rrf, name: str, k_steps: int, warmup: int, device, stream):
+    """The same metric through the public call with HOST buffers: every step
+    copies its inputs from pinned host memory, runs the calls and reads the
+    results back; copies included in the timed region."""
+    import torch
+    w = workloads.WORKLOADS[name]
+    host, dev = [], []
+    h2d = d2h = 0
+    for rows, residual in workload_cases(name):
+        c = workloads.make_case(name, rows)
+        hb = dict(inputs=[x.pin_memory() for x in c.inputs],
+                  residual=None if c.residual is None else c.residual.pin_memory(),
+                  gamma=c.gamma.pin_memory(),
+                  q=torch.empty(c.inputs[0].shape, dtype=torch.uint8).pin_memory(),
+                  scales=torch.empty((rows, 1), dtype=torch.float32).pin_memory(),
+                  res_out=None if c.residual is None else
+                  torch.empty_like(c.residual).pin_memory())
+        db = dict(inputs=[torch.empty_like(x, device=device) for x in c.inputs],
+                  residual=None if c.residual is None else
+                  torch.empty_like(c.residual, device=device),
+                  gamma=torch.empty_like(c.gamma, device=device),
+                  q=torch.empty(c.inputs[0].shape, dtype=torch.float8_e4m3fn, device=device),
+                  scales=torch.empty((rows, 1), dtype=torch.float32, device=device),
+                  res_out=None if c.residual is None else
+                  torch.empty_like(c.residual, device=device))
+        h2d += sum(x.numel() * 2 for x in c.inputs) + c.gamma.numel() * 2 + \
+            (c.residual.numel() * 2 if c.residual is not None else 0)
+        d2h += rows * w.cols + rows * 4 + (rows * w.cols * 2 if residual else 0)
+        host.append(hb)
+        dev.append(db)
+
+    def step(_):
+        for hb, db in zip(host, dev):
+            for xd, xh in zip(db["inputs"], hb["inputs"]):
+                xd.copy_(xh, non_blocking=True)
+            if hb["residual"] is not None:
+                db["residual"].copy_(hb["residual"], non_blocking=True)
+            db["gamma"].copy_(hb["gamma"], non_blocking=True)
+            rrf.rrf_sum_rmsnorm_fp8(db["inputs"], db["gamma"], w.eps, w.weight_offset,
+                                    w.scale_ub, residual_in=db["residual"],
+                                    residual_out=db["res_out"], q_out=db["q"],
+                                    scales_out=db["scales"])
+            hb["q"].copy_(db["q"].view(torch.uint8), non_blocking=True)
+            hb["scales"].copy_(db["scales"], non_blocking=True)
+            if hb["res_out"] is not None:
+                hb["res_out"].copy_(db["res_out"], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            step(i)
+        t = time_region(step, k_steps, device, stream)
+    return t, h2d, d2h
+
+
+def cpu_baseline(name: str, budget_s: float = 12.0):
+    """The oracle, as it stands, on a bounded sample of the workload: whole
+    steps of the workload (all its calls) until about budget_s seconds."""
+    import oracle
+    w = workloads.WORKLOADS[name]
+    bits = workloads.bits
+    if name == "prefill":
+        # one full step is 1.4 GB; the sample is a block of 8 rows per call
+        calls = [(workloads.make_case(name, 8, sub=0), 8)]
+        sample = "8 of the 8192 rows per call, R=8 x 8192 cols + residual"
+        step_b = workloads.fused_bytes(w.R, 8, w.cols, w.residual)
+    else:
+        calls = [(workloads.make_case(name, rows), rows) for rows, _ in workload_cases(name)]
+        sample = "whole steps (every call of the workload)"
+        step_b = step_bytes(name)
+    prepared = [([bits(x) for x in c.inputs], None if c.residual is None else bits(c.residual),
+                 bits(c.gamma), c) for c, _ in calls]
+
+    def one_step():
+        for xs, res, g, c in prepared:
+            oracle.sum_rmsnorm_fp8(xs, c.rows, c.cols, g, c.eps, c.weight_offset, c.scale_ub,
+                                   residual=res)
+
+    one_step()  # builds the library and warms the caches
+    n, t0 = 0, time.perf_counter()
+    while True:
+        one_step()
+        n += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(step_b * n / dt / 1e9, 6), "unit": "GB/s", "cores": 1,
+            "kind": "oracle", "sample": f"{n} x ({sample}), {dt:.1f} s, single-threaded C",
+            "ms_per_step": round(dt / n * 1e3, 3)}
+
+
+def run_rrf(args):
+    import torch
+    import torch.distributed as dist
+    import reduce_rmsnorm_fp8_b200 as rrf
+
+    rank, local_rank, world = dist_env()
+    if world != args.gpus and rank == 0:
+        print(f"note: --gpus {args.gpus} but WORLD_SIZE {world}; using WORLD_SIZE",
+              file=sys.stderr)
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    props = torch.cuda.get_device_properties(device)
+    l2 = props.L2_cache_size
+    peak, peak_kind = measured_peaks()
+
+    name = args.workload
+    w = workloads.WORKLOADS[name]
+    pool = DevicePool(name, device, L2_FLUSH_FACTOR * l2)
+    stream = torch.cuda.current_stream(device)
+    launches = 0
+
+    # ---- warm-up (eager), then K steps captured in one CUDA graph and timed
+    # as one replay: the step is launch-bound at decode sizes, and a graph
+    # removes the host's per-launch cost from the device timeline.
+    for i in range(args.warmup):
+        pool.run_step(rrf, i)
+    torch.cuda.synchronize(device)
+    graph, launches = capture_steps(lambda i: pool.run_step(rrf, args.warmup + i),
+                                    args.steps, device)
+    graph.replay()  # one untimed replay: graph upload
+    torch.cuda.synchronize(device)
+    with ClockSampler(device.index) as clocks:
+        t = time_region(lambda _: graph.replay(), 1, device, stream)
+    del graph
+    per_step = step_bytes(name)
+    value = world * per_step * args.steps / t / 1e9
+    kernel_us = t / launches * 1e6
+
+    # ---- per-call breakdown (separate graphs, same rotation)
+    cases = []
+    reps = max(args.steps, 100)
+    for i, c in enumerate(pool.cases):
+        gi, _ = capture_steps(lambda k, i=i: pool.run_call(rrf, args.warmup + k, i), reps,
+                              device)
+        gi.replay()
+        torch.cuda.synchronize(device)
+        tc = time_region(lambda _: gi.replay(), 1, device, stream)
+        del gi
+        b = workloads.fused_bytes(w.R, c.rows, c.cols, c.residual is not None)
+        launch = rrf.rrf_plan_fused(w.R, c.rows, c.cols, props.multi_processor_count)
+        cases.append({"rows": c.rows, "us_per_call": round(tc / reps * 1e6, 3),
+                      "GB_s": round(b * reps / tc / 1e9, 1),
+                      "frac": round(b * reps / tc / 1e9 / peak, 4),
+                      "rows_per_s": round(c.rows * reps / tc, 1),
+                      "launch": {"cluster": launch[0], "threads": launch[1],
+                                 "vecs_per_thread": launch[2]}})
+
+    # ---- end to end through host buffers
+    e2e = None
+    if not args.no_e2e:
+        te, h2d, d2h = e2e_measure(rrf, name, max(10, args.steps // 10), args.warmup, device,
+                                   torch.cuda.Stream(device))
+        ke = max(10, args.steps // 10)
+        e2e = {"value": round(world * per_step * ke / te / 1e9, 3), "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": round(te / ke * 1e3, 4)}
+
+    # ---- secondary: the prefill-size call, where the kernel can reach HBM speed
+    secondary = None
+    if not args.no_secondary and name != "prefill":
+        del pool
+        torch.cuda.empty_cache()
+        pf = DevicePool("prefill", device, 2 * l2)
+        for i in range(3):
+            pf.run_step(rrf, i)
+        kp = 20
+        gp, _ = capture_steps(lambda k: pf.run_step(rrf, k), kp, device)
+        gp.replay()
+        torch.cuda.synchronize(device)
+        tp = time_region(lambda _: gp.replay(), 1, device, stream)
+        del gp
+        bp = step_bytes("prefill")
+        secondary = {"workload": "prefill R=8 8192x8192 + residual, 2 rotating sets of 1.41 GB",
+                     "us_per_call": round(tp / kp * 1e6, 2),
+                     "GB_s": round(bp * kp / tp / 1e9, 1),
+                     "frac": round(bp * kp / tp / 1e9 / peak, 4), "calls": kp}
+        del pf
+        torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(name)
+
+    if rank == 0:
+        achieved = per_step * args.steps / t / 1e9
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(t / args.steps * 1e3, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "io": "bf16 inputs/residual/gamma -> e4m3fn codes + f32 scales + bf16 residual",
+            "data": "synthetic (seeded splitmix64 + Box-Muller, drawn on the GPU)",
+            "impl": "rrf",
+            "config": {"workload": f"{name}: R={w.R}, cols={w.cols}, rows {list(w.rows)} "
+                                   f"per step, residual={'on' if w.residual else 'off'}",
+                       "R": w.R, "cols": w.cols, "rows": list(w.rows),
+                       "bytes_per_step": per_step,
+                       "l2": f"rotating {pool_sets_note(name, l2)} buffer sets > "
+                             f"{L2_FLUSH_FACTOR}x L2 ({l2 >> 20} MiB)",
+                       "launch": "auto (rrf_sum_rmsnorm_fp8)",
+                       "timing": "K steps captured in one CUDA graph, one replay timed "
+                                 "with CUDA events",
+                       "parallelism": f"dp{world}"},
+            "us_per_call": round(t / launches * 1e6, 3),
+            "cases": cases,
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "traffic": None, "peak_kind": f"{peak_kind} hbm_gbs",
+                         "kernel": "fused_kernel (rrf_fused.cu)",
+                         "avg_launch_us": round(kernel_us, 3),
+                         "bytes_per_launch": round(per_step / len(w.rows))},
+            "gpu_launches": launches,
+            "clocks": clocks.summary(),
+            "e2e": e2e,
+            "prefill": secondary,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier(device_ids=[device.index])
+        dist.destroy_process_group()
+
+
+def pool_sets_note(name: str, l2: int) -> str:
+    return str(max(2, math.ceil(L2_FLUSH_FACTOR * l2 / step_bytes(name))))
+
+
+def run_reference(args):
+    """The oracle as the reference arm: rank 0 times it on the host cores.
+    Each step is a bounded sample of one step of the workload: the first two
+    rows of every call (rows are independent, so GB/s over the sample is the
+    oracle's throughput on the workload)."""
+    rank, _, world = dist_env()
+    if rank != 0:
+        return
+    name = args.workload
+    w = workloads.WORKLOADS[name]
+    import oracle
+    bits = workloads.bits
+    cases = [workloads.make_case(name, rows) if name != "prefill" else
+             workloads.make_case(name, 8, sub=0) for rows, _ in workload_cases(name)]
+    prepared = [([bits(x[:2]) for x in c.inputs],
+                 None if c.residual is None else bits(c.residual[:2]), bits(c.gamma), c)
+                for c in cases]
+    per_step = sum(workloads.fused_bytes(w.R, min(2, c.rows), w.cols, w.residual)
+                   for c in cases)
+
+    def step():
+        for xs, res, g, c in prepared:
+            oracle.sum_rmsnorm_fp8(xs, min(2, c.rows), c.cols, g, c.eps, c.weight_offset,
+                                   c.scale_ub, residual=res)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = per_step * args.steps / dt / 1e9
+    sample = f"first 2 rows of each of the {len(cases)} calls per step"
+    line = {"metric": METRIC, "value": round(value, 6), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": f"{name}: R={w.R}, cols={w.cols}, rows {list(w.rows)} "
+                                   f"per step, residual={'on' if w.residual else 'off'}",
+                       "sample": sample},
+            "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": 1,
+                             "kind": "oracle", "sample": f"{args.steps} steps, {sample}"},
+            "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description="fused sum + RMSNorm + FP8 benchmark")
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["rrf", "reference"], default="rrf")
+    ap.add_argument("--workload", choices=sorted(workloads.WORKLOADS), default="decode")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_rrf(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,197 @@
+/*
+ * rrf.h -- C ABI of the fused "R-way bf16 sum + residual + RMSNorm + per-row
+ * FP8 (e4m3fn) quantisation" library for NVIDIA B200 (sm_100a).
+ *
+ * The operation is the epilogue of an all-reduce, run on one GPU whose HBM
+ * already holds the R rank-partial buffers:
+ *
+ *   Modular docs, Mojo function `allreduce_rmsnorm_fp8` (module
+ *   nn/allreduce_residual_rmsnorm_fp8): a fused allreduce + RMSNorm + FP8
+ *   dynamic quantisation in one kernel launch that skips the HBM round trip
+ *   between the reduced buffer and the norm.  Its "Args" section fixes the
+ *   argument set used here: R input buffers (last dim = cols), an FP8 output
+ *   of the input's shape, gamma of length cols, epsilon, weight_offset (an
+ *   additive offset for gamma), scale_ub (upper bound for the FP8 scale) and
+ *   a float32 scale per row.  Its peer-to-peer transport and signal buffers
+ *   have no counterpart on one GPU.
+ *
+ *   local-inference-lab/b12x PR #283 "PCIeTwoShotBF16": the partials are
+ *   accumulated in fp32 in a fixed rank order and rounded to bf16 once, which
+ *   makes the result deterministic and within one bf16 rounding of the exact
+ *   sum.
+ *
+ * What one row i computes (x_r are the inputs; every operation is fp32 and
+ * rounded once unless stated; RN_bf16 is round-to-nearest-even to bf16):
+ *   s_j   = RN_bf16(((x_0 + x_1) + x_2) + ... + x_{R-1})      (rank order)
+ *   h_j   = RN_bf16(s_j + residual_in_j), stored to residual_out   (or s_j)
+ *   r     = 1 / sqrt(sum_j h_j^2 / cols + eps)
+ *   y_j   = (h_j * r) * (gamma_j + weight_offset)
+ *   scale = max(min(max_j |y_j|, scale_ub), 1e-12) / 448
+ *   q_j   = e4m3fn(y_j / scale), nearest even, saturating at +-448
+ *   scales[i] = scale            (dequantise as y ~ e4m3fn_value(q) * scale)
+ * The bf16 outputs (s, residual_out) are exact; the sum of squares is a
+ * fixed-order fp32 tree, so scales agree with a float64 evaluation to about
+ * 1e-6 relative, and a code may differ by one step from the float64 one only
+ * where y / scale sits at an e4m3 rounding midpoint.
+ *
+ * Conventions for every entry point
+ *  - Layout: every 2-D array is contiguous row-major [rows, cols] (row stride
+ *    cols elements).  bf16 arrays hold IEEE bfloat16, fp8 arrays hold
+ *    e4m3fn codes (one byte each), scales are float32.
+ *  - Pointers: all data pointers are DEVICE pointers (or managed / host-
+ *    mapped memory the device can read).  The array `inputs` itself is a
+ *    HOST array of R device pointers; it is copied into the launch's
+ *    parameters, so it may be freed as soon as the call returns.
+ *  - Ownership: the caller owns every buffer.  The library allocates no
+ *    device memory and keeps no state between calls apart from a per-device
+ *    cache of the SM count.
+ *  - Asynchrony: work is enqueued on `stream` (NULL = the legacy default
+ *    stream) and the call returns without synchronising.  Outputs are valid
+ *    in stream order only.
+ *  - Validation: every argument is checked on the host before any CUDA call.
+ *    On an error the call returns a non-zero rrf_status and enqueues
+ *    nothing.  rows == 0 is a valid empty call: it returns RRF_OK without
+ *    looking at any pointer (empty torch tensors have null data pointers).
+ *  - Aliasing: inputs may alias one another.  No output may overlap an
+ *    input or another output, except residual_out == residual_in exactly
+ *    (the in-place residual update).
+ *  - Thread safety: calls from several host threads are safe; calls that
+ *    overlap on the GPU and share an output race like any two kernels.
+ */
+#ifndef RRF_H
+#define RRF_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The same type as cudaStream_t; NULL is the legacy default stream. */
+struct CUstream_st;
+typedef struct CUstream_st* rrf_stream_t;
+
+typedef enum rrf_status {
+    RRF_OK = 0,
+    RRF_ERR_NULL = 1,        /* a required pointer is NULL                           */
+    RRF_ERR_RANKS = 2,       /* num_inputs outside [1, RRF_MAX_INPUTS]               */
+    RRF_ERR_SHAPE = 3,       /* rows < 0, cols <= 0, cols % 8 != 0, or too large     */
+    RRF_ERR_ALIGN = 4,       /* a data pointer is not 16-byte aligned (scales: 4)    */
+    RRF_ERR_ALIAS = 5,       /* an output overlaps an input or another output        */
+    RRF_ERR_VALUE = 6,       /* eps < 0 or not finite, scale_ub <= 0 or NaN,
+                                weight_offset not finite                              */
+    RRF_ERR_UNSUPPORTED = 7, /* a forced variant / cluster size / block size that
+                                cannot run this shape                                */
+    RRF_ERR_CUDA = 8         /* a CUDA call failed: see rrf_last_cuda_error()        */
+} rrf_status;
+
+/* At most this many input buffers (the pages' systems use 2, 4 or 8 ranks;
+ * the Ascend page allows up to 16). */
+#define RRF_MAX_INPUTS 16
+
+/* Largest cols the fused entry points accept (262144): a row is held in
+ * registers across up to 16 cooperating blocks of 256 threads, each thread
+ * holding 8 vectors of 8 elements. */
+#define RRF_MAX_COLS (16 * 256 * 8 * 8)
+
+/* rrf_sum -- the bf16 sum alone.
+ *   out[i, j] = RN_bf16(x_0[i, j] + x_1[i, j] + ... + x_{R-1}[i, j]), fp32
+ *   accumulation in rank order 0..R-1 (b12x PR #283, opening description).
+ * inputs     host array of num_inputs device pointers, each bf16 [rows, cols],
+ *            16-byte aligned
+ * num_inputs R, 1..RRF_MAX_INPUTS
+ * rows, cols rows >= 0; cols > 0 and a multiple of 8 (16-byte rows)
+ * out        device pointer, bf16 [rows, cols], 16-byte aligned, must not
+ *            overlap any input
+ * Errors: RRF_ERR_NULL, RRF_ERR_RANKS, RRF_ERR_SHAPE, RRF_ERR_ALIGN,
+ *         RRF_ERR_ALIAS, RRF_ERR_CUDA. */
+rrf_status rrf_sum(const void* const* inputs, int num_inputs, int64_t rows,
+                   int64_t cols, void* out, rrf_stream_t stream);
+
+/* rrf_sum_rmsnorm_fp8 -- the fused operation (Modular docs,
+ * `allreduce_rmsnorm_fp8`, "Args"; the residual form is the module name's
+ * "residual" and TensorRT-LLM PR #19836's RESIDUAL_RMS_NORM epilogue).
+ * inputs        host array of num_inputs device pointers, bf16 [rows, cols]
+ * num_inputs    R, 1..RRF_MAX_INPUTS
+ * rows, cols    rows >= 0; cols > 0, a multiple of 8, at most RRF_MAX_COLS
+ * residual_in   bf16 [rows, cols] or NULL; residual_out bf16 [rows, cols] or
+ *               NULL; both NULL (no residual) or both set; they may be equal
+ * gamma         bf16 [cols]
+ * eps           >= 0, finite (the pages type it as the input dtype; it is
+ *               used here as the fp32 value given)
+ * weight_offset finite, added to gamma in fp32 (1.0 for unit-offset gamma)
+ * scale_ub      > 0 (may be +inf: no clamp)
+ * q_out         fp8 e4m3fn codes [rows, cols], 16-byte aligned
+ * scales_out    float32 [rows], 4-byte aligned
+ * Every bf16 / fp8 pointer must be 16-byte aligned.
+ * Errors: RRF_ERR_NULL, RRF_ERR_RANKS, RRF_ERR_SHAPE, RRF_ERR_ALIGN,
+ *         RRF_ERR_ALIAS, RRF_ERR_VALUE, RRF_ERR_CUDA. */
+rrf_status rrf_sum_rmsnorm_fp8(const void* const* inputs, int num_inputs,
+                               int64_t rows, int64_t cols, const void* residual_in,
+                               void* residual_out, const void* gamma, float eps,
+                               float weight_offset, float scale_ub, void* q_out,
+                               float* scales_out, rrf_stream_t stream);
+
+/* Launch variants of the fused kernel. */
+#define RRF_VARIANT_AUTO 0    /* the built-in choice (rrf_plan_fused)              */
+#define RRF_VARIANT_ROW 1     /* one block per row                                 */
+#define RRF_VARIANT_CLUSTER 2 /* each row split across a thread-block cluster of
+                                 cluster_size blocks whose row statistics meet in
+                                 distributed shared memory (TensorRT-LLM PR
+                                 #19836: cluster.sync() before remote writes, one
+                                 arrive / wait per thread per barrier phase)      */
+
+/* rrf_sum_rmsnorm_fp8_ex -- rrf_sum_rmsnorm_fp8 with the launch forced, for
+ * tests and benchmarks.  variant is one of RRF_VARIANT_*; cluster_size is
+ * 2, 4, 8 or 16 for RRF_VARIANT_CLUSTER (0 = automatic) and ignored
+ * otherwise; block_threads is a multiple of 32 in [32, 1024] or 0
+ * (automatic).  Results are bit-identical across variants for the bf16
+ * outputs and agree within the stated tolerance for scales and codes.
+ * Errors: those of rrf_sum_rmsnorm_fp8, and RRF_ERR_UNSUPPORTED when the
+ * forced launch cannot cover the row. */
+rrf_status rrf_sum_rmsnorm_fp8_ex(const void* const* inputs, int num_inputs,
+                                  int64_t rows, int64_t cols, const void* residual_in,
+                                  void* residual_out, const void* gamma, float eps,
+                                  float weight_offset, float scale_ub, void* q_out,
+                                  float* scales_out, int variant, int cluster_size,
+                                  int block_threads, rrf_stream_t stream);
+
+/* rrf_plan_fused -- the launch rrf_sum_rmsnorm_fp8 would use on a GPU with
+ * sm_count SMs, without touching the GPU.  Writes the cluster size (1 = one
+ * block per row), the threads per block and the 16-byte vectors each thread
+ * holds.  Returns RRF_ERR_SHAPE / RRF_ERR_RANKS for shapes the library
+ * rejects. */
+rrf_status rrf_plan_fused(int num_inputs, int64_t rows, int64_t cols, int sm_count,
+                          int* cluster_size, int* block_threads, int* vecs_per_thread);
+
+/* rrf_check_sum_args / rrf_check_fused_args -- the host-side validation of
+ * rrf_sum / rrf_sum_rmsnorm_fp8 alone: the status those calls would return
+ * before any CUDA call (RRF_OK if the arguments are valid).  No GPU needed. */
+rrf_status rrf_check_sum_args(const void* const* inputs, int num_inputs, int64_t rows,
+                              int64_t cols, const void* out);
+rrf_status rrf_check_fused_args(const void* const* inputs, int num_inputs, int64_t rows,
+                                int64_t cols, const void* residual_in,
+                                const void* residual_out, const void* gamma, float eps,
+                                float weight_offset, float scale_ub, const void* q_out,
+                                const void* scales_out);
+
+/* Text for a status code (static storage, never NULL). */
+const char* rrf_status_string(rrf_status status);
+
+/* The cudaError_t of the last RRF_ERR_CUDA returned on this host thread
+ * (0 if none). */
+int rrf_last_cuda_error(void);
+
+/* Test hook for the error path: the next launch on this host thread reports
+ * the given cudaError_t value without launching anything (0 clears it), so
+ * the RRF_ERR_CUDA path can be tested without making a GPU fail. */
+void rrf_debug_fail_next_launch(int cuda_error);
+
+/* Library version, "major.minor.patch". */
+const char* rrf_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RRF_H */

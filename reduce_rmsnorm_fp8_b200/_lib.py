@@ -1,0 +1,225 @@
+"""ctypes binding of librrf.so: argument marshalling only."""
+from __future__ import annotations
+
+import ctypes
+import enum
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "librrf.so")
+
+RRF_MAX_INPUTS = 16
+RRF_MAX_COLS = 16 * 256 * 8 * 8
+RRF_VARIANT_AUTO = 0
+RRF_VARIANT_ROW = 1
+RRF_VARIANT_CLUSTER = 2
+
+
+class Status(enum.IntEnum):
+    OK = 0
+    ERR_NULL = 1
+    ERR_RANKS = 2
+    ERR_SHAPE = 3
+    ERR_ALIGN = 4
+    ERR_ALIAS = 5
+    ERR_VALUE = 6
+    ERR_UNSUPPORTED = 7
+    ERR_CUDA = 8
+
+
+class RrfError(RuntimeError):
+    """A non-zero rrf_status from the library."""
+
+    def __init__(self, status: int, cuda_error: int = 0):
+        self.status = Status(status)
+        self.cuda_error = cuda_error
+        msg = f"{self.status.name}: {rrf_status_string(status)}"
+        if self.status == Status.ERR_CUDA:
+            msg += f" (cudaError {cuda_error})"
+        super().__init__(msg)
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m reduce_rmsnorm_fp8_b200.build` "
+        "(the CUDA kernels are the only implementation; there is no fallback)")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_int = ctypes.c_int
+_f32 = ctypes.c_float
+_ptrs = ctypes.POINTER(ctypes.c_void_p)
+
+lib.rrf_sum.restype = _int
+lib.rrf_sum.argtypes = [_ptrs, _int, _i64, _i64, _vp, _vp]
+_fused_args = [_ptrs, _int, _i64, _i64, _vp, _vp, _vp, _f32, _f32, _f32, _vp, _vp]
+lib.rrf_sum_rmsnorm_fp8.restype = _int
+lib.rrf_sum_rmsnorm_fp8.argtypes = _fused_args + [_vp]
+lib.rrf_sum_rmsnorm_fp8_ex.restype = _int
+lib.rrf_sum_rmsnorm_fp8_ex.argtypes = _fused_args + [_int, _int, _int, _vp]
+lib.rrf_plan_fused.restype = _int
+lib.rrf_plan_fused.argtypes = [_int, _i64, _i64, _int, ctypes.POINTER(_int),
+                               ctypes.POINTER(_int), ctypes.POINTER(_int)]
+lib.rrf_check_sum_args.restype = _int
+lib.rrf_check_sum_args.argtypes = [_ptrs, _int, _i64, _i64, _vp]
+lib.rrf_check_fused_args.restype = _int
+lib.rrf_check_fused_args.argtypes = _fused_args
+lib.rrf_status_string.restype = ctypes.c_char_p
+lib.rrf_status_string.argtypes = [_int]
+lib.rrf_last_cuda_error.restype = _int
+lib.rrf_last_cuda_error.argtypes = []
+lib.rrf_debug_fail_next_launch.restype = None
+lib.rrf_debug_fail_next_launch.argtypes = [_int]
+lib.rrf_version.restype = ctypes.c_char_p
+lib.rrf_version.argtypes = []
+
+
+def rrf_status_string(status: int) -> str:
+    return lib.rrf_status_string(int(status)).decode()
+
+
+def rrf_last_cuda_error() -> int:
+    return lib.rrf_last_cuda_error()
+
+
+def rrf_debug_fail_next_launch(cuda_error: int) -> None:
+    lib.rrf_debug_fail_next_launch(int(cuda_error))
+
+
+def rrf_version() -> str:
+    return lib.rrf_version().decode()
+
+
+def _raise_on(status: int) -> None:
+    if status != 0:
+        raise RrfError(status, lib.rrf_last_cuda_error() if status == Status.ERR_CUDA else 0)
+
+
+def _ptr_table(ptrs):
+    return (ctypes.c_void_p * max(1, len(ptrs)))(*[p or None for p in ptrs])
+
+
+# ------------------------------------------------------- raw pointer calls ---
+
+def rrf_check_sum_args(input_ptrs, rows, cols, out_ptr) -> int:
+    return lib.rrf_check_sum_args(_ptr_table(input_ptrs), len(input_ptrs), rows, cols,
+                                  out_ptr or None)
+
+
+def rrf_check_fused_args(input_ptrs, rows, cols, residual_in, residual_out, gamma, eps,
+                         weight_offset, scale_ub, q_out, scales_out) -> int:
+    return lib.rrf_check_fused_args(_ptr_table(input_ptrs), len(input_ptrs), rows, cols,
+                                    residual_in or None, residual_out or None, gamma or None,
+                                    eps, weight_offset, scale_ub, q_out or None,
+                                    scales_out or None)
+
+
+def rrf_plan_fused(num_inputs: int, rows: int, cols: int, sm_count: int):
+    """The launch the library would pick: (cluster_size, block_threads,
+    vecs_per_thread)."""
+    c, t, v = _int(), _int(), _int()
+    _raise_on(lib.rrf_plan_fused(num_inputs, rows, cols, sm_count, ctypes.byref(c),
+                                 ctypes.byref(t), ctypes.byref(v)))
+    return c.value, t.value, v.value
+
+
+def rrf_sum_ptr(input_ptrs, rows, cols, out_ptr, stream=0) -> None:
+    """rrf_sum on raw device pointers and a raw cudaStream_t handle."""
+    _raise_on(lib.rrf_sum(_ptr_table(input_ptrs), len(input_ptrs), rows, cols,
+                          out_ptr or None, stream or None))
+
+
+def rrf_sum_rmsnorm_fp8_ptr(input_ptrs, rows, cols, residual_in, residual_out, gamma, eps,
+                            weight_offset, scale_ub, q_out, scales_out, variant=0,
+                            cluster_size=0, block_threads=0, stream=0) -> None:
+    """rrf_sum_rmsnorm_fp8_ex on raw device pointers and a raw stream handle."""
+    _raise_on(lib.rrf_sum_rmsnorm_fp8_ex(
+        _ptr_table(input_ptrs), len(input_ptrs), rows, cols, residual_in or None,
+        residual_out or None, gamma or None, eps, weight_offset, scale_ub, q_out or None,
+        scales_out or None, variant, cluster_size, block_threads, stream or None))
+
+
+# ------------------------------------------------------------ torch calls ---
+
+def _torch():
+    import torch
+    return torch
+
+
+def _rows_cols(inputs):
+    torch = _torch()
+    if len(inputs) == 0:
+        raise ValueError("need at least one input")
+    x0 = inputs[0]
+    for x in inputs:
+        if x.dtype != torch.bfloat16:
+            raise TypeError("inputs must be bfloat16")
+        if x.shape != x0.shape or x.device != x0.device:
+            raise ValueError("inputs must share shape and device")
+        if x.device.type != "cuda":
+            raise ValueError("inputs must be CUDA tensors")
+        if not x.is_contiguous():
+            raise ValueError("inputs must be contiguous")
+    if x0.dim() == 0:
+        raise ValueError("inputs must have a last dimension")
+    cols = x0.shape[-1]
+    rows = x0.numel() // cols if cols else 0
+    return rows, cols
+
+
+def _stream(device):
+    return _torch().cuda.current_stream(device).cuda_stream
+
+
+def rrf_sum(inputs, out=None):
+    """Sum of the bf16 CUDA tensors ``inputs`` (fp32 in list order, rounded
+    to bf16 once), into ``out`` (allocated if None).  Returns ``out``."""
+    torch = _torch()
+    rows, cols = _rows_cols(inputs)
+    dev = inputs[0].device
+    if out is None:
+        out = torch.empty_like(inputs[0])
+    with torch.cuda.device(dev):
+        rrf_sum_ptr([x.data_ptr() for x in inputs], rows, cols, out.data_ptr(),
+                    _stream(dev))
+    return out
+
+
+def rrf_sum_rmsnorm_fp8_ex(inputs, gamma, eps, weight_offset, scale_ub, residual_in=None,
+                           residual_out=None, q_out=None, scales_out=None, variant=0,
+                           cluster_size=0, block_threads=0):
+    """The fused operation with a forced launch (variant, cluster size, block
+    size; 0 = automatic).  Returns (q, scales, residual_out)."""
+    torch = _torch()
+    rows, cols = _rows_cols(inputs)
+    x0 = inputs[0]
+    dev = x0.device
+    if gamma.dtype != torch.bfloat16 or gamma.numel() != cols or gamma.device != dev:
+        raise ValueError("gamma must be a bf16 tensor of length cols on the inputs' device")
+    if residual_in is not None and residual_out is None:
+        residual_out = torch.empty_like(residual_in)
+    if q_out is None:
+        q_out = torch.empty(x0.shape, dtype=torch.float8_e4m3fn, device=dev)
+    if scales_out is None:
+        scales_out = torch.empty(tuple(x0.shape[:-1]) + (1,), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        rrf_sum_rmsnorm_fp8_ptr(
+            [x.data_ptr() for x in inputs], rows, cols,
+            residual_in.data_ptr() if residual_in is not None else 0,
+            residual_out.data_ptr() if residual_out is not None else 0,
+            gamma.data_ptr(), eps, weight_offset, scale_ub, q_out.data_ptr(),
+            scales_out.data_ptr(), variant, cluster_size, block_threads, _stream(dev))
+    return q_out, scales_out, residual_out
+
+
+def rrf_sum_rmsnorm_fp8(inputs, gamma, eps, weight_offset, scale_ub, residual_in=None,
+                        residual_out=None, q_out=None, scales_out=None):
+    """The fused operation.  ``inputs``: R bf16 CUDA tensors [..., cols];
+    ``gamma``: bf16 [cols]; ``residual_in`` (optional) bf16 like the inputs,
+    written to ``residual_out`` (a new tensor if None; pass residual_in for an
+    in-place update).  Returns (q: float8_e4m3fn like the inputs, scales:
+    float32 [..., 1], residual_out or None)."""
+    return rrf_sum_rmsnorm_fp8_ex(inputs, gamma, eps, weight_offset, scale_ub, residual_in,
+                                  residual_out, q_out, scales_out)

@@ -1,0 +1,338 @@
+// rrf_api.cu -- the C ABI declared in include/rrf.h: host-side validation,
+// the launch planner and the entry points.  Every argument is checked before
+// any CUDA call; the library allocates nothing and keeps only a per-device
+// SM-count cache.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "rrf.h"
+#include "rrf_internal.h"
+
+namespace rrf {
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+thread_local int t_fail_next_launch = 0;
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];
+
+rrf_status cuda_fail(cudaError_t e) {
+    t_last_cuda_error = (int)e;
+    return RRF_ERR_CUDA;
+}
+
+// SM count of the current device, cached per device.
+rrf_status current_sm_count(int* sm_count) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev >= 0 && dev < kMaxDevices) {
+        int cached = g_sm_count[dev].load(std::memory_order_relaxed);
+        if (cached > 0) {
+            *sm_count = cached;
+            return RRF_OK;
+        }
+    }
+    int n = 0;
+    e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev >= 0 && dev < kMaxDevices) g_sm_count[dev].store(n, std::memory_order_relaxed);
+    *sm_count = n;
+    return RRF_OK;
+}
+
+// A pending injected failure (test hook) replaces the launch.
+bool take_injected_failure(cudaError_t* e) {
+    if (t_fail_next_launch == 0) return false;
+    *e = (cudaError_t)t_fail_next_launch;
+    t_fail_next_launch = 0;
+    return true;
+}
+
+bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
+
+struct Range {
+    uintptr_t lo, hi;  // [lo, hi)
+};
+
+Range range_of(const void* p, int64_t bytes) {
+    return Range{(uintptr_t)p, (uintptr_t)p + (uintptr_t)bytes};
+}
+
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
+
+rrf_status check_shape(int num_inputs, int64_t rows, int64_t cols, int64_t max_cols) {
+    if (num_inputs < 1 || num_inputs > RRF_MAX_INPUTS) return RRF_ERR_RANKS;
+    if (rows < 0 || cols <= 0 || cols % 8 != 0 || cols > max_cols) return RRF_ERR_SHAPE;
+    // every array's byte size (2 bytes per element) must fit in int64; the
+    // grid (at most 16 blocks per row) must fit in 2^31 - 1 blocks
+    if (rows > 0 && rows > (INT64_MAX / 2) / cols) return RRF_ERR_SHAPE;
+    if (rows > (int64_t)INT32_MAX / 16) return RRF_ERR_SHAPE;
+    return RRF_OK;
+}
+
+rrf_status check_inputs(const void* const* inputs, int num_inputs) {
+    if (inputs == nullptr) return RRF_ERR_NULL;
+    for (int r = 0; r < num_inputs; ++r) {
+        if (inputs[r] == nullptr) return RRF_ERR_NULL;
+        if (!aligned(inputs[r], 16)) return RRF_ERR_ALIGN;
+    }
+    return RRF_OK;
+}
+
+}  // namespace
+
+// --------------------------------------------------------------- planner ---
+
+static int round_up32(int64_t x) { return (int)((x + 31) / 32 * 32); }
+
+// Threads per block and vectors per thread for a row slice of `slice`
+// vectors: the fewest vectors per thread that keep the block at <= 256
+// threads (any size up to the compiled bound at 8 vectors per thread), or,
+// with forced_threads, the fewest that let that many threads cover the slice.
+static bool pick_block(int R, int64_t slice, int forced_threads, FusedLaunch* l) {
+    const int rb = input_bound(R);
+    for (int vpt = 1; vpt <= 8; vpt *= 2) {
+        const int max_t = fused_max_threads(rb, vpt);
+        int t;
+        if (forced_threads != 0) {
+            t = forced_threads;
+            if (t > max_t || (int64_t)t * vpt < slice) continue;
+        } else {
+            t = round_up32((slice + vpt - 1) / vpt);
+            if ((t > 256 && vpt < 8) || t > max_t) continue;
+        }
+        l->threads = t;
+        l->vecs_per_thread = vpt;
+        return true;
+    }
+    return false;
+}
+
+// Launch for a given cluster size (0 = the planner's choice) and block size
+// (0 = automatic).
+static rrf_status shape_launch(int R, int64_t rows, int64_t cols, int sm_count, int cluster,
+                               int forced_threads, FusedLaunch* out) {
+    rrf_status st = check_shape(R, rows, cols, RRF_MAX_COLS);
+    if (st != RRF_OK) return st;
+    if (sm_count < 1) sm_count = 1;
+    const int64_t vecs = cols / 8;
+    int c = cluster;
+    if (c == 0) {
+        // Split rows across the blocks of a cluster until the grid covers the
+        // SMs, keeping at least 32 vectors (one warp's worth) per block; then
+        // split further while one block cannot hold its slice.
+        c = 1;
+        while (c < 16 && rows * c < sm_count && vecs / (2 * c) >= 32) c *= 2;
+        while (c < 16 && !pick_block(R, (vecs + c - 1) / c, forced_threads, out)) c *= 2;
+    }
+    if (!pick_block(R, (vecs + c - 1) / c, forced_threads, out))
+        return cluster == 0 && forced_threads == 0 ? RRF_ERR_SHAPE : RRF_ERR_UNSUPPORTED;
+    out->cluster = c;
+    return RRF_OK;
+}
+
+rrf_status plan_fused(int R, int64_t rows, int64_t cols, int sm_count, FusedLaunch* out) {
+    return shape_launch(R, rows, cols, sm_count, 0, 0, out);
+}
+
+cudaError_t launch_fused(const FusedArgs& a, int64_t rows, const FusedLaunch& l, bool residual,
+                         cudaStream_t stream) {
+    switch (input_bound(a.R)) {
+        case 2: return launch_fused_rb2(a, rows, l, residual, stream);
+        case 4: return launch_fused_rb4(a, rows, l, residual, stream);
+        case 8: return launch_fused_rb8(a, rows, l, residual, stream);
+        default: return launch_fused_rb16(a, rows, l, residual, stream);
+    }
+}
+
+}  // namespace rrf
+
+using namespace rrf;
+
+// ------------------------------------------------------------ validation ---
+
+extern "C" rrf_status rrf_check_sum_args(const void* const* inputs, int num_inputs,
+                                         int64_t rows, int64_t cols, const void* out) {
+    rrf_status st = check_shape(num_inputs, rows, cols, INT64_MAX);
+    if (st != RRF_OK || rows == 0) return st;
+    if ((st = check_inputs(inputs, num_inputs)) != RRF_OK) return st;
+    if (out == nullptr) return RRF_ERR_NULL;
+    if (!aligned(out, 16)) return RRF_ERR_ALIGN;
+    const int64_t bytes = rows * cols * 2;
+    const Range o = range_of(out, bytes);
+    for (int r = 0; r < num_inputs; ++r)
+        if (overlap(o, range_of(inputs[r], bytes))) return RRF_ERR_ALIAS;
+    return RRF_OK;
+}
+
+extern "C" rrf_status rrf_check_fused_args(const void* const* inputs, int num_inputs,
+                                           int64_t rows, int64_t cols,
+                                           const void* residual_in,
+                                           const void* residual_out, const void* gamma,
+                                           float eps, float weight_offset, float scale_ub,
+                                           const void* q_out, const void* scales_out) {
+    rrf_status st = check_shape(num_inputs, rows, cols, RRF_MAX_COLS);
+    if (st != RRF_OK) return st;
+    if (!(std::isfinite(eps) && eps >= 0.0f)) return RRF_ERR_VALUE;
+    if (!std::isfinite(weight_offset)) return RRF_ERR_VALUE;
+    if (std::isnan(scale_ub) || !(scale_ub > 0.0f)) return RRF_ERR_VALUE;
+    if (rows == 0) return RRF_OK;
+    if ((st = check_inputs(inputs, num_inputs)) != RRF_OK) return st;
+    if ((residual_in == nullptr) != (residual_out == nullptr)) return RRF_ERR_NULL;
+    if (gamma == nullptr || q_out == nullptr || scales_out == nullptr) return RRF_ERR_NULL;
+    if (!aligned(gamma, 16) || !aligned(q_out, 16) || !aligned(scales_out, 4))
+        return RRF_ERR_ALIGN;
+    if (residual_in != nullptr && (!aligned(residual_in, 16) || !aligned(residual_out, 16)))
+        return RRF_ERR_ALIGN;
+
+    const int64_t bf16_bytes = rows * cols * 2;
+    Range reads[RRF_MAX_INPUTS + 2];
+    int n_reads = 0;
+    for (int r = 0; r < num_inputs; ++r) reads[n_reads++] = range_of(inputs[r], bf16_bytes);
+    reads[n_reads++] = range_of(gamma, cols * 2);
+    const bool in_place = residual_in != nullptr && residual_in == residual_out;
+    if (residual_in != nullptr && !in_place)
+        reads[n_reads++] = range_of(residual_in, bf16_bytes);
+
+    Range writes[3];
+    int n_writes = 0;
+    writes[n_writes++] = range_of(q_out, rows * cols);
+    writes[n_writes++] = range_of(scales_out, rows * 4);
+    if (residual_out != nullptr) writes[n_writes++] = range_of(residual_out, bf16_bytes);
+
+    for (int w = 0; w < n_writes; ++w) {
+        for (int r = 0; r < n_reads; ++r)
+            if (overlap(writes[w], reads[r])) return RRF_ERR_ALIAS;
+        for (int w2 = w + 1; w2 < n_writes; ++w2)
+            if (overlap(writes[w], writes[w2])) return RRF_ERR_ALIAS;
+    }
+    return RRF_OK;
+}
+
+// ----------------------------------------------------------- entry points ---
+
+extern "C" rrf_status rrf_sum(const void* const* inputs, int num_inputs, int64_t rows,
+                              int64_t cols, void* out, rrf_stream_t stream) {
+    rrf_status st = rrf_check_sum_args(inputs, num_inputs, rows, cols, out);
+    if (st != RRF_OK || rows == 0) return st;
+    int sm_count = 0;
+    if ((st = current_sm_count(&sm_count)) != RRF_OK) return st;
+    SumArgs a = {};
+    for (int r = 0; r < num_inputs; ++r) a.in[r] = static_cast<const uint4*>(inputs[r]);
+    a.out = static_cast<uint4*>(out);
+    a.R = num_inputs;
+    a.n_vecs = rows * cols / 8;
+    cudaError_t e;
+    if (!take_injected_failure(&e)) e = launch_sum(a, sm_count, (cudaStream_t)stream);
+    return e == cudaSuccess ? RRF_OK : cuda_fail(e);
+}
+
+extern "C" rrf_status rrf_sum_rmsnorm_fp8_ex(const void* const* inputs, int num_inputs,
+                                             int64_t rows, int64_t cols,
+                                             const void* residual_in, void* residual_out,
+                                             const void* gamma, float eps,
+                                             float weight_offset, float scale_ub,
+                                             void* q_out, float* scales_out, int variant,
+                                             int cluster_size, int block_threads,
+                                             rrf_stream_t stream) {
+    rrf_status st = rrf_check_fused_args(inputs, num_inputs, rows, cols, residual_in,
+                                         residual_out, gamma, eps, weight_offset, scale_ub,
+                                         q_out, scales_out);
+    if (st != RRF_OK) return st;
+    if (variant < RRF_VARIANT_AUTO || variant > RRF_VARIANT_CLUSTER) return RRF_ERR_UNSUPPORTED;
+    if (block_threads != 0 && (block_threads < 32 || block_threads > 1024 || block_threads % 32))
+        return RRF_ERR_UNSUPPORTED;
+    if (variant == RRF_VARIANT_CLUSTER && cluster_size != 0 && cluster_size != 2 &&
+        cluster_size != 4 && cluster_size != 8 && cluster_size != 16)
+        return RRF_ERR_UNSUPPORTED;
+    if (rows == 0) return RRF_OK;
+
+    int sm_count = 0;
+    if ((st = current_sm_count(&sm_count)) != RRF_OK) return st;
+    int cluster = 0;
+    if (variant == RRF_VARIANT_ROW) cluster = 1;
+    if (variant == RRF_VARIANT_CLUSTER) {
+        cluster = cluster_size;
+        if (cluster == 0) {
+            FusedLaunch planned = {};
+            if ((st = plan_fused(num_inputs, rows, cols, sm_count, &planned)) != RRF_OK) return st;
+            cluster = planned.cluster > 1 ? planned.cluster : 2;
+        }
+    }
+    FusedLaunch l = {};
+    if ((st = shape_launch(num_inputs, rows, cols, sm_count, cluster, block_threads, &l)) !=
+        RRF_OK)
+        return st;
+    const int64_t vecs = cols / 8;
+
+    FusedArgs a = {};
+    for (int r = 0; r < num_inputs; ++r) a.in[r] = static_cast<const uint4*>(inputs[r]);
+    a.res_in = static_cast<const uint4*>(residual_in);
+    a.res_out = static_cast<uint4*>(residual_out);
+    a.gamma = static_cast<const uint4*>(gamma);
+    a.q = static_cast<uint2*>(q_out);
+    a.scales = scales_out;
+    a.R = num_inputs;
+    a.vecs = (int)vecs;
+    a.cluster = l.cluster;
+    a.slice_vecs = (int)((vecs + l.cluster - 1) / l.cluster);
+    a.cols_f = (float)cols;
+    a.eps = eps;
+    a.weight_offset = weight_offset;
+    a.scale_ub = scale_ub;
+    cudaError_t e;
+    if (!take_injected_failure(&e))
+        e = launch_fused(a, rows, l, residual_in != nullptr, (cudaStream_t)stream);
+    return e == cudaSuccess ? RRF_OK : cuda_fail(e);
+}
+
+extern "C" rrf_status rrf_sum_rmsnorm_fp8(const void* const* inputs, int num_inputs,
+                                          int64_t rows, int64_t cols,
+                                          const void* residual_in, void* residual_out,
+                                          const void* gamma, float eps, float weight_offset,
+                                          float scale_ub, void* q_out, float* scales_out,
+                                          rrf_stream_t stream) {
+    return rrf_sum_rmsnorm_fp8_ex(inputs, num_inputs, rows, cols, residual_in, residual_out,
+                                  gamma, eps, weight_offset, scale_ub, q_out, scales_out,
+                                  RRF_VARIANT_AUTO, 0, 0, stream);
+}
+
+extern "C" rrf_status rrf_plan_fused(int num_inputs, int64_t rows, int64_t cols, int sm_count,
+                                     int* cluster_size, int* block_threads,
+                                     int* vecs_per_thread) {
+    if (!cluster_size || !block_threads || !vecs_per_thread) return RRF_ERR_NULL;
+    FusedLaunch l = {};
+    rrf_status st = plan_fused(num_inputs, rows, cols, sm_count, &l);
+    if (st != RRF_OK) return st;
+    *cluster_size = l.cluster;
+    *block_threads = l.threads;
+    *vecs_per_thread = l.vecs_per_thread;
+    return RRF_OK;
+}
+
+extern "C" const char* rrf_status_string(rrf_status status) {
+    switch (status) {
+        case RRF_OK: return "ok";
+        case RRF_ERR_NULL: return "a required pointer is null (or only one residual pointer given)";
+        case RRF_ERR_RANKS: return "num_inputs outside [1, 16]";
+        case RRF_ERR_SHAPE: return "invalid shape: rows < 0, cols <= 0, cols % 8 != 0, or too large";
+        case RRF_ERR_ALIGN: return "misaligned pointer: data needs 16 bytes, scales 4 bytes";
+        case RRF_ERR_ALIAS: return "an output overlaps an input or another output";
+        case RRF_ERR_VALUE: return "invalid scalar: eps < 0 or not finite, scale_ub <= 0 or NaN, weight_offset not finite";
+        case RRF_ERR_UNSUPPORTED: return "the forced launch cannot cover this shape";
+        case RRF_ERR_CUDA: return "a CUDA call failed (see rrf_last_cuda_error)";
+    }
+    return "unknown status";
+}
+
+extern "C" int rrf_last_cuda_error(void) { return t_last_cuda_error; }
+
+extern "C" void rrf_debug_fail_next_launch(int cuda_error) { t_fail_next_launch = cuda_error; }
+
+extern "C" const char* rrf_version(void) { return "0.1.0"; }

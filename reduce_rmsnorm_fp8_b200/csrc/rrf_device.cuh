@@ -1,0 +1,193 @@
+// rrf_device.cuh -- device-side building blocks of the sum and fused kernels:
+// 16-byte memory access, bf16 / e4m3fn conversion, warp / block / cluster
+// reductions.  sm_100a only.
+#pragma once
+
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+namespace rrf {
+
+// ------------------------------------------------------------------ memory --
+
+// Streamed 16-byte load of data read exactly once: read-only path, no L1
+// allocation, 256-byte L2 prefetch of the surrounding line.
+__device__ __forceinline__ uint4 ld_once(const uint4* p) {
+    uint4 v;
+    asm("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+        : "l"(p));
+    return v;
+}
+
+// 16-byte load of data every block of the grid reads (gamma): read-only path,
+// cached.
+__device__ __forceinline__ uint4 ld_shared_by_all(const uint4* p) {
+    uint4 v;
+    asm("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+        : "l"(p));
+    return v;
+}
+
+// Streaming stores (evict-first): results are not re-read by this kernel.
+__device__ __forceinline__ void st_once(uint4* p, uint4 v) {
+    asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};"
+                 :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ void st_once(uint2* p, uint2 v) {
+    asm volatile("st.global.cs.v2.u32 [%0], {%1, %2};" :: "l"(p), "r"(v.x), "r"(v.y)
+                 : "memory");
+}
+
+// -------------------------------------------------------------------- bf16 --
+
+// A 16-byte vector holds 8 bf16; 32-bit word k holds elements 2k (low half)
+// and 2k+1 (high half).  bf16 -> fp32 widening is exact: the bf16 bits are the
+// top half of the fp32 bits.
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 v, float f[8]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        f[2 * k] = __uint_as_float(w[k] << 16);
+        f[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+    }
+}
+
+// Two fp32 -> two bf16, round to nearest even (cvt.rn.bf16x2.f32 puts its
+// first source in the upper half).
+__device__ __forceinline__ uint32_t f32x2_to_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+__device__ __forceinline__ uint4 f32_to_bf16x8(const float f[8]) {
+    uint4 v;
+    v.x = f32x2_to_bf16x2(f[0], f[1]);
+    v.y = f32x2_to_bf16x2(f[2], f[3]);
+    v.z = f32x2_to_bf16x2(f[4], f[5]);
+    v.w = f32x2_to_bf16x2(f[6], f[7]);
+    return v;
+}
+
+// acc += widen(x), one IEEE fp32 add per element (no contraction).
+__device__ __forceinline__ void add_bf16x8(float acc[8], const uint4 x) {
+    float f[8];
+    bf16x8_to_f32(x, f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = __fadd_rn(acc[e], f[e]);
+}
+
+// Sum of squares of 8 bf16 as a balanced tree (each square is exact in fp32).
+__device__ __forceinline__ float sumsq_bf16x8(const uint4 v) {
+    float f[8];
+    bf16x8_to_f32(v, f);
+    const float a = __fmaf_rn(f[0], f[0], f[1] * f[1]);
+    const float b = __fmaf_rn(f[2], f[2], f[3] * f[3]);
+    const float c = __fmaf_rn(f[4], f[4], f[5] * f[5]);
+    const float d = __fmaf_rn(f[6], f[6], f[7] * f[7]);
+    return (a + b) + (c + d);
+}
+
+// ------------------------------------------------------------------ e4m3fn --
+
+// Two fp32 -> two e4m3fn codes, round to nearest even, saturating to +-448
+// (cvt.rn.satfinite.e4m3x2.f32 through the cuda_fp8.h intrinsic); the first
+// element lands in the low byte.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+    return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
+}
+
+__device__ __forceinline__ uint2 f32_to_e4m3x8(const float f[8]) {
+    uint2 q;
+    q.x = f32x2_to_e4m3x2(f[0], f[1]) | (f32x2_to_e4m3x2(f[2], f[3]) << 16);
+    q.y = f32x2_to_e4m3x2(f[4], f[5]) | (f32x2_to_e4m3x2(f[6], f[7]) << 16);
+    return q;
+}
+
+// -------------------------------------------------------------- reductions --
+// Butterfly (xor) reductions: at every level lane i combines its value with
+// lane i ^ off's, and a + b == b + a in IEEE arithmetic, so every lane ends
+// with the same bits and the result does not depend on which lane reads it.
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
+    return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, off));
+    return v;
+}
+
+// Block-wide sum / max, returned to every thread.  `scratch` holds one float
+// per warp and must not be reused until every thread has returned.
+__device__ __forceinline__ float block_sum(float v, float* scratch) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    v = warp_sum(v);
+    if (lane == 0) scratch[warp] = v;
+    __syncthreads();
+    return warp_sum(lane < nwarps ? scratch[lane] : 0.0f);
+}
+
+__device__ __forceinline__ float block_max(float v, float* scratch) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    v = warp_max(v);
+    if (lane == 0) scratch[warp] = v;
+    __syncthreads();
+    return warp_max(lane < nwarps ? scratch[lane] : 0.0f);
+}
+
+// ------------------------------------------------------ thread-block cluster --
+// Cluster barrier phases follow the rules the TensorRT-LLM PR #19836 write-up
+// spells out: every thread arrives and waits exactly once per phase, no
+// thread leaves before the last phase, and a block writes a peer's shared
+// memory only after a completed phase has shown that the peer has started.
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_arrive_release() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait_acquire() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Store v into the shared-memory word `local` of cluster block `peer`.
+__device__ __forceinline__ void st_peer_shared(float* local, uint32_t peer, float v) {
+    const uint32_t laddr = (uint32_t)__cvta_generic_to_shared(local);
+    uint32_t raddr;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(raddr) : "r"(laddr), "r"(peer));
+    asm volatile("st.shared::cluster.f32 [%0], %1;" :: "r"(raddr), "f"(v) : "memory");
+}
+
+// Cluster-wide combination of one value per block: block `rank` writes its
+// value into slot[rank] of every block (threads 0..C-1 write one peer each),
+// one barrier phase publishes the writes, and every block reduces the C slots
+// with the same butterfly, so all blocks hold the same bits.
+template <bool IS_MAX>
+__device__ __forceinline__ float cluster_combine(float block_value, float* slots,
+                                                 uint32_t rank, int C) {
+    if ((int)threadIdx.x < C) st_peer_shared(&slots[rank], threadIdx.x, block_value);
+    cluster_arrive_release();
+    cluster_wait_acquire();
+    const int lane = threadIdx.x & 31;
+    const float t = lane < C ? slots[lane] : 0.0f;
+    return IS_MAX ? warp_max(t) : warp_sum(t);
+}
+
+}  // namespace rrf

@@ -1,0 +1,191 @@
+// rrf_fused.cu -- the fused bf16 sum + residual + RMSNorm + per-row FP8 kernel.
+//
+// One row is covered by C blocks (C = 1: one block per row; C > 1: a
+// thread-block cluster, the row's statistics meeting in distributed shared
+// memory).  Each block owns a contiguous slice of the row's 16-byte vectors;
+// each thread owns up to VPT of them, strided by the block size so that a
+// warp's accesses are contiguous.  Every input byte is read from HBM once;
+// the row's bf16 norm input h stays in registers between the three passes
+// (gamma is re-read from cache):
+//   1. load the R inputs (+ residual), fp32 sum in rank order, round to bf16,
+//      add the residual and round again, store residual_out, sum of squares;
+//   2. r = 1 / sqrt(mean + eps); y = (h * r) * (gamma + weight_offset); amax;
+//   3. scale = max(min(amax, scale_ub), 1e-12) / 448; codes of y / scale.
+// The sum of squares and amax are reduced warp -> block -> cluster.  Sources:
+// Modular docs `allreduce_rmsnorm_fp8` (one launch, no HBM round trip between
+// the reduction and the norm), b12x PR #283 (fixed-order fp32, round once),
+// TensorRT-LLM PR #19836 (cluster partial-sum exchange and its barrier rules).
+#include <cuda_runtime.h>
+
+#include "rrf_device.cuh"
+#include "rrf_internal.h"
+
+#ifndef RRF_RB
+#error "compile with -DRRF_RB=<2|4|8|16>"
+#endif
+
+namespace rrf {
+namespace {
+
+constexpr float kE4m3Max = 448.0f;
+constexpr float kScaleFloor = 1e-12f;
+
+template <int RB, int VPT, bool RES, bool CLUSTER>
+__global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const FusedArgs a) {
+    __shared__ float warp_ss[32];
+    __shared__ float warp_amax[32];
+    __shared__ float cl_ss[16];
+    __shared__ float cl_amax[16];
+
+    // Phase 0 of the cluster barrier: announce that this block has started.
+    // Its wait comes just before the first write into a peer's shared memory.
+    if (CLUSTER) cluster_arrive_relaxed();
+
+    const int tid = threadIdx.x;
+    const int T = blockDim.x;
+    const uint32_t rank = CLUSTER ? cluster_rank() : 0u;
+    const int64_t row = CLUSTER ? (int64_t)(blockIdx.x / a.cluster) : (int64_t)blockIdx.x;
+    const int v_begin = (int)rank * a.slice_vecs;
+    const int v_end = min(v_begin + a.slice_vecs, a.vecs);
+    const int64_t row_base = row * (int64_t)a.vecs;
+
+    uint4 h[VPT];
+    float ss = 0.0f;
+
+    // ---- pass 1: sum, residual, sum of squares
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+        const int v = v_begin + tid + k * T;
+        if (v < v_end) {
+            uint4 x[RB];
+#pragma unroll
+            for (int r = 0; r < RB; ++r)
+                if (r < a.R) x[r] = ld_once(a.in[r] + row_base + v);
+            uint4 res;
+            if (RES) res = ld_once(a.res_in + row_base + v);
+
+            float acc[8];
+            bf16x8_to_f32(x[0], acc);
+#pragma unroll
+            for (int r = 1; r < RB; ++r)
+                if (r < a.R) add_bf16x8(acc, x[r]);
+            uint4 s = f32_to_bf16x8(acc);
+            if (RES) {
+                float t[8];
+                bf16x8_to_f32(s, t);
+                add_bf16x8(t, res);
+                s = f32_to_bf16x8(t);
+                st_once(a.res_out + row_base + v, s);
+            }
+            h[k] = s;
+            ss += sumsq_bf16x8(s);
+        }
+    }
+
+    float total_ss = block_sum(ss, warp_ss);
+    if (CLUSTER) {
+        cluster_wait_acquire();  // phase 0 done: every block of the cluster runs
+        total_ss = cluster_combine<false>(total_ss, cl_ss, rank, a.cluster);
+    }
+    const float ms = total_ss / a.cols_f;
+    const float rinv = 1.0f / sqrtf(ms + a.eps);
+
+    // ---- pass 2: y and its absolute maximum
+    float amax = 0.0f;
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+        const int v = v_begin + tid + k * T;
+        if (v < v_end) {
+            float hf[8], gf[8];
+            bf16x8_to_f32(h[k], hf);
+            bf16x8_to_f32(ld_shared_by_all(a.gamma + v), gf);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float y = __fmul_rn(__fmul_rn(hf[e], rinv), __fadd_rn(gf[e], a.weight_offset));
+                amax = fmaxf(amax, fabsf(y));
+            }
+        }
+    }
+    amax = block_max(amax, warp_amax);
+    if (CLUSTER) amax = cluster_combine<true>(amax, cl_amax, rank, a.cluster);
+
+    const float scale = fmaxf(fminf(amax, a.scale_ub), kScaleFloor) / kE4m3Max;
+    const float inv_scale = 1.0f / scale;
+
+    // ---- pass 3: quantise
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+        const int v = v_begin + tid + k * T;
+        if (v < v_end) {
+            float hf[8], gf[8], qv[8];
+            bf16x8_to_f32(h[k], hf);
+            bf16x8_to_f32(ld_shared_by_all(a.gamma + v), gf);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float y = __fmul_rn(__fmul_rn(hf[e], rinv), __fadd_rn(gf[e], a.weight_offset));
+                qv[e] = __fmul_rn(y, inv_scale);
+            }
+            st_once(a.q + row_base + v, f32_to_e4m3x8(qv));
+        }
+    }
+    if (tid == 0 && rank == 0) a.scales[row] = scale;
+}
+
+template <int RB, int VPT, bool RES, bool CLUSTER>
+cudaError_t launch_one(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
+                       cudaStream_t stream) {
+    auto kernel = fused_kernel<RB, VPT, RES, CLUSTER>;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(rows * l.cluster), 1, 1);
+    cfg.blockDim = dim3((unsigned)l.threads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    if (CLUSTER) {
+        if (l.cluster > 8) {
+            // Clusters of 16 are outside the portable limit of 8 and must be
+            // enabled per kernel.
+            cudaError_t e = cudaFuncSetAttribute(
+                kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            if (e != cudaSuccess) return e;
+        }
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)l.cluster;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    return cudaLaunchKernelEx(&cfg, kernel, a);
+}
+
+template <int RB, bool RES, bool CLUSTER>
+cudaError_t launch_vpt(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
+                       cudaStream_t stream) {
+    switch (l.vecs_per_thread) {
+        case 1: return launch_one<RB, 1, RES, CLUSTER>(a, rows, l, stream);
+        case 2: return launch_one<RB, 2, RES, CLUSTER>(a, rows, l, stream);
+        case 4: return launch_one<RB, 4, RES, CLUSTER>(a, rows, l, stream);
+        case 8: return launch_one<RB, 8, RES, CLUSTER>(a, rows, l, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+// This translation unit is compiled once per input bound (RRF_RB = 2, 4, 8,
+// 16) so the instantiations build in parallel; it defines launch_fused_rb<RB>.
+#define RRF_CAT2(a, b) a##b
+#define RRF_CAT(a, b) RRF_CAT2(a, b)
+cudaError_t RRF_CAT(launch_fused_rb, RRF_RB)(const FusedArgs& a, int64_t rows,
+                                             const FusedLaunch& l, bool residual,
+                                             cudaStream_t stream) {
+    const bool cluster = l.cluster > 1;
+    if (residual)
+        return cluster ? launch_vpt<RRF_RB, true, true>(a, rows, l, stream)
+                       : launch_vpt<RRF_RB, true, false>(a, rows, l, stream);
+    return cluster ? launch_vpt<RRF_RB, false, true>(a, rows, l, stream)
+                   : launch_vpt<RRF_RB, false, false>(a, rows, l, stream);
+}
+
+}  // namespace rrf

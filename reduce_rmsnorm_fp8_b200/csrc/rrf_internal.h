@@ -1,0 +1,78 @@
+// rrf_internal.h -- shared between the host API (rrf_api.cu) and the kernel
+// translation units (rrf_sum.cu, rrf_fused.cu).  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "rrf.h"
+
+namespace rrf {
+
+// Everything a launch needs, passed by value as the kernel parameter.  Input
+// pointers address 16-byte vectors of 8 bf16 elements.
+struct SumArgs {
+    const uint4* in[RRF_MAX_INPUTS];
+    uint4* out;
+    int R;
+    int64_t n_vecs;  // rows * cols / 8
+};
+
+struct FusedArgs {
+    const uint4* in[RRF_MAX_INPUTS];
+    const uint4* res_in;   // null without a residual
+    uint4* res_out;        // null without a residual
+    const uint4* gamma;    // [cols / 8]
+    uint2* q;              // 8 e4m3fn codes per 16-byte input vector
+    float* scales;         // [rows]
+    int R;
+    int vecs;              // cols / 8 (vectors per row)
+    int slice_vecs;        // vectors per block of a row's cluster: ceil(vecs / C)
+    int cluster;           // C, blocks per row (1 = no cluster)
+    float cols_f;          // cols as fp32, the mean's divisor
+    float eps;
+    float weight_offset;
+    float scale_ub;
+};
+
+struct FusedLaunch {
+    int cluster;          // blocks per row
+    int threads;          // threads per block
+    int vecs_per_thread;  // 1, 2, 4 or 8
+};
+
+// The fused kernel is compiled for input-count bounds RB in {2, 4, 8, 16}
+// (inputs past R are predicated off) and VPT in {1, 2, 4, 8} vectors per
+// thread.
+constexpr int input_bound(int R) { return R <= 2 ? 2 : (R <= 4 ? 4 : (R <= 8 ? 8 : 16)); }
+
+// Largest block the fused kernel is compiled for: a thread holds RB loads in
+// flight and VPT vectors of its row slice in registers, so the register
+// budget per thread (65536 / threads) must grow with both.  Chosen from the
+// ptxas register counts so that no instantiation spills more than a few bytes.
+constexpr int fused_max_threads(int rb, int vpt) {
+    return rb <= 4 ? (vpt <= 4 ? 1024 : 512)
+                   : (rb == 8 ? (vpt <= 2 ? 1024 : (vpt == 4 ? 512 : 256))
+                              : (vpt <= 4 ? 512 : 256));
+}
+
+// Kernel launchers (one per translation unit).  They return the CUDA error of
+// the launch (cudaSuccess when it was enqueued).
+cudaError_t launch_sum(const SumArgs& a, int sm_count, cudaStream_t stream);
+// One fused launcher per compiled input bound RB (inputs past R are
+// predicated off); launch_fused picks the smallest RB >= R.
+cudaError_t launch_fused_rb2(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
+                             bool residual, cudaStream_t stream);
+cudaError_t launch_fused_rb4(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
+                             bool residual, cudaStream_t stream);
+cudaError_t launch_fused_rb8(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
+                             bool residual, cudaStream_t stream);
+cudaError_t launch_fused_rb16(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
+                              bool residual, cudaStream_t stream);
+cudaError_t launch_fused(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
+                         bool residual, cudaStream_t stream);
+
+// The launch shape the library picks (pure host arithmetic).
+rrf_status plan_fused(int R, int64_t rows, int64_t cols, int sm_count, FusedLaunch* out);
+
+}  // namespace rrf

@@ -1,0 +1,54 @@
+// rrf_sum.cu -- the bf16 sum of R buffers: fp32 accumulation in rank order,
+// one rounding to bf16 (b12x PR #283 "PCIeTwoShotBF16": fixed-order fp32
+// accumulation rounded once, deterministic).
+//
+// A grid-stride loop over 16-byte vectors: per vector the R loads are issued
+// back to back before any add, each input byte is read once, the output is
+// written once with streaming stores.
+#include <cuda_runtime.h>
+
+#include "rrf_device.cuh"
+#include "rrf_internal.h"
+
+namespace rrf {
+namespace {
+
+template <int RB>
+__global__ void __launch_bounds__(256) sum_kernel(const SumArgs a) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < a.n_vecs; i += stride) {
+        uint4 x[RB];
+#pragma unroll
+        for (int r = 0; r < RB; ++r)
+            if (r < a.R) x[r] = ld_once(a.in[r] + i);
+        float acc[8];
+        bf16x8_to_f32(x[0], acc);
+#pragma unroll
+        for (int r = 1; r < RB; ++r)
+            if (r < a.R) add_bf16x8(acc, x[r]);
+        st_once(a.out + i, f32_to_bf16x8(acc));
+    }
+}
+
+template <int RB>
+cudaError_t launch_rb(const SumArgs& a, int sm_count, cudaStream_t stream) {
+    constexpr int kThreads = 256;
+    // Enough blocks for every vector, capped at a few resident waves; the
+    // grid-stride loop covers the rest.
+    const int64_t need = (a.n_vecs + kThreads - 1) / kThreads;
+    const int64_t cap = (int64_t)sm_count * 8;
+    const unsigned blocks = (unsigned)(need < cap ? need : cap);
+    sum_kernel<RB><<<blocks, kThreads, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_sum(const SumArgs& a, int sm_count, cudaStream_t stream) {
+    if (a.R <= 2) return launch_rb<2>(a, sm_count, stream);
+    if (a.R <= 4) return launch_rb<4>(a, sm_count, stream);
+    if (a.R <= 8) return launch_rb<8>(a, sm_count, stream);
+    return launch_rb<16>(a, sm_count, stream);
+}
+
+}  // namespace rrf

@@ -1,0 +1,207 @@
+"""The C ABI without a GPU: the library loads, exports every function the
+header declares, validates arguments on the host and plans launches.  No
+compute entry point is called here."""
+import os
+import re
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rrf.h")
+
+
+@pytest.fixture(scope="module")
+def rrf():
+    from reduce_rmsnorm_fp8_b200 import build
+    build.build()
+    import reduce_rmsnorm_fp8_b200 as m
+    return m
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(rrf_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for want in ("rrf_sum", "rrf_sum_rmsnorm_fp8", "rrf_sum_rmsnorm_fp8_ex",
+                 "rrf_status_string", "rrf_last_cuda_error"):
+        assert want in names
+
+
+def test_library_exports_every_declared_function(rrf):
+    out = subprocess.run(["nm", "-D", "--defined-only", rrf.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (rrf_[a-z0-9_]+)$", out, flags=re.M))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for name in declared_functions():
+        getattr(rrf.lib, name)  # resolvable through ctypes
+
+
+def test_header_compiles_as_plain_c(tmp_path):
+    src = tmp_path / "t.c"
+    src.write_text('#include "rrf.h"\nint main(void) { return RRF_OK; }\n')
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER),
+                    str(src), "-o", str(tmp_path / "t")], check=True)
+
+
+def test_constants_match_header(rrf):
+    text = open(HEADER).read()
+    assert rrf.RRF_MAX_INPUTS == int(re.search(r"#define RRF_MAX_INPUTS (\d+)", text).group(1))
+    expr = re.search(r"#define RRF_MAX_COLS \(([^)]*)\)", text).group(1)
+    assert rrf.RRF_MAX_COLS == eval(expr)
+    for name in ("RRF_VARIANT_AUTO", "RRF_VARIANT_ROW", "RRF_VARIANT_CLUSTER"):
+        assert getattr(rrf, name) == int(re.search(rf"#define {name} (\d+)", text).group(1))
+    for st in rrf.Status:
+        assert re.search(rf"RRF_{st.name} = {int(st)}\b", text), st
+
+
+def test_status_strings_and_version(rrf):
+    for st in rrf.Status:
+        assert rrf.rrf_status_string(st)
+    assert rrf.rrf_status_string(99) == "unknown status"
+    assert re.fullmatch(r"\d+\.\d+\.\d+", rrf.rrf_version())
+    assert rrf.rrf_last_cuda_error() == 0
+
+
+# ----------------------------------------------------------- validation ---
+
+A = 1 << 20  # fake, 16-byte aligned addresses: validation never dereferences them
+
+
+def fused_ok_args(R=4, rows=8, cols=64):
+    n = rows * cols
+    ins = [A * (r + 1) for r in range(R)]
+    base = A * 64
+    return dict(input_ptrs=ins, rows=rows, cols=cols, residual_in=base,
+                residual_out=base + 4 * A, gamma=base + 8 * A, eps=1e-5, weight_offset=0.0,
+                scale_ub=1200.0, q_out=base + 12 * A, scales_out=base + 16 * A)
+
+
+def check(rrf, **kw):
+    return rrf.Status(rrf.rrf_check_fused_args(**kw))
+
+
+def test_fused_validation_accepts_valid(rrf):
+    assert check(rrf, **fused_ok_args()) == rrf.Status.OK
+    kw = fused_ok_args()
+    kw["residual_out"] = kw["residual_in"]  # in-place residual
+    assert check(rrf, **kw) == rrf.Status.OK
+    kw = fused_ok_args()
+    kw["residual_in"] = kw["residual_out"] = 0  # no residual
+    assert check(rrf, **kw) == rrf.Status.OK
+    kw = fused_ok_args()
+    kw["scale_ub"] = float("inf")
+    assert check(rrf, **kw) == rrf.Status.OK
+
+
+@pytest.mark.parametrize("change,status", [
+    (dict(input_ptrs=[]), "ERR_RANKS"),
+    (dict(input_ptrs=[A * (r + 1) for r in range(17)]), "ERR_RANKS"),
+    (dict(rows=-1), "ERR_SHAPE"),
+    (dict(cols=0), "ERR_SHAPE"),
+    (dict(cols=60), "ERR_SHAPE"),
+    (dict(cols=16 * 256 * 8 * 8 + 8), "ERR_SHAPE"),
+    (dict(rows=2 ** 40), "ERR_SHAPE"),
+    (dict(eps=-1e-6), "ERR_VALUE"),
+    (dict(eps=float("nan")), "ERR_VALUE"),
+    (dict(eps=float("inf")), "ERR_VALUE"),
+    (dict(scale_ub=0.0), "ERR_VALUE"),
+    (dict(scale_ub=-1.0), "ERR_VALUE"),
+    (dict(scale_ub=float("nan")), "ERR_VALUE"),
+    (dict(weight_offset=float("inf")), "ERR_VALUE"),
+    (dict(gamma=0), "ERR_NULL"),
+    (dict(q_out=0), "ERR_NULL"),
+    (dict(scales_out=0), "ERR_NULL"),
+    (dict(residual_out=0), "ERR_NULL"),
+    (dict(residual_in=0), "ERR_NULL"),
+    (dict(input_ptrs=[A, 0]), "ERR_NULL"),
+    (dict(input_ptrs=[A, A * 2 + 8]), "ERR_ALIGN"),
+    (dict(gamma=A * 72 + 2), "ERR_ALIGN"),
+    (dict(q_out=A * 76 + 8), "ERR_ALIGN"),
+    (dict(scales_out=A * 80 + 2), "ERR_ALIGN"),
+    (dict(residual_in=A * 64 + 16 + 4), "ERR_ALIGN"),
+    (dict(q_out=A * 1 + 16), "ERR_ALIAS"),           # inside input 0
+    (dict(scales_out=A * 72), "ERR_ALIAS"),          # on gamma
+    (dict(residual_out=A * 64 + 16), "ERR_ALIAS"),   # overlaps residual_in, not equal
+    (dict(q_out=A * 68 + 256), "ERR_ALIAS"),         # inside residual_out
+    (dict(scales_out=A * 76 + 100), "ERR_ALIAS"),    # inside q_out
+])
+def test_fused_validation_rejects(rrf, change, status):
+    kw = fused_ok_args()
+    kw.update(change)
+    assert check(rrf, **kw) == rrf.Status[status]
+
+
+def test_empty_rows_is_valid_without_pointers(rrf):
+    st = rrf.rrf_check_fused_args([0, 0], 0, 64, 0, 0, 0, 1e-6, 0.0, 1.0, 0, 0)
+    assert st == rrf.Status.OK
+    assert rrf.rrf_check_sum_args([0], 0, 64, 0) == rrf.Status.OK
+    # the scalars and the shape are still checked
+    assert rrf.rrf_check_fused_args([0], 0, 64, 0, 0, 0, -1.0, 0.0, 1.0, 0, 0) == \
+        rrf.Status.ERR_VALUE
+    assert rrf.rrf_check_sum_args([0], 0, 63, 0) == rrf.Status.ERR_SHAPE
+
+
+def test_sum_validation(rrf):
+    ins = [A, 2 * A, 3 * A]
+    assert rrf.rrf_check_sum_args(ins, 16, 64, 8 * A) == rrf.Status.OK
+    assert rrf.rrf_check_sum_args(ins, 16, 64, 0) == rrf.Status.ERR_NULL
+    assert rrf.rrf_check_sum_args(ins, 16, 64, 8 * A + 4) == rrf.Status.ERR_ALIGN
+    assert rrf.rrf_check_sum_args(ins, 16, 64, 2 * A + 64) == rrf.Status.ERR_ALIAS
+    assert rrf.rrf_check_sum_args(ins, 16, 12, 8 * A) == rrf.Status.ERR_SHAPE
+    assert rrf.rrf_check_sum_args([A] * 17, 16, 64, 8 * A) == rrf.Status.ERR_RANKS
+    # sum-only has no column limit beyond memory
+    assert rrf.rrf_check_sum_args(ins, 1, 1 << 22, 1 << 40) == rrf.Status.OK
+
+
+# -------------------------------------------------------------- planner ---
+
+@pytest.mark.parametrize("R,rows,cols,sm,want", [
+    (8, 8192, 8192, 148, (1, 256, 4)),   # prefill: one block per row
+    (8, 1, 7168, 148, (16, 64, 1)),      # decode rows 1: cluster of 16
+    (8, 8, 7168, 148, (16, 64, 1)),
+    (8, 32, 7168, 148, (8, 128, 1)),
+    (8, 64, 7168, 148, (4, 224, 1)),
+    (4, 37, 7168, 148, (4, 224, 1)),
+    (4, 256, 4096, 148, (1, 256, 2)),
+    (2, 4, 256, 148, (1, 32, 1)),        # too short to split
+    (4, 1, 8, 148, (1, 32, 1)),
+    (4, 4, 262144, 148, (16, 256, 8)),   # the longest row
+])
+def test_plan(rrf, R, rows, cols, sm, want):
+    assert rrf.rrf_plan_fused(R, rows, cols, sm) == want
+
+
+def test_plan_covers_every_row(rrf):
+    for R in (1, 3, 8, 16):
+        for cols in (8, 256, 2880, 7168, 7176, 8192, 8200, 16384, 131072, 262144):
+            for rows in (1, 37, 4096):
+                c, t, v = rrf.rrf_plan_fused(R, rows, cols, 148)
+                assert c in (1, 2, 4, 8, 16) and 32 <= t <= 1024 and t % 32 == 0
+                assert v in (1, 2, 4, 8)
+                assert c * t * v * 8 >= cols, (R, rows, cols)
+
+
+def test_plan_rejects(rrf):
+    with pytest.raises(rrf.RrfError) as e:
+        rrf.rrf_plan_fused(4, 1, 16 * 256 * 8 * 8 + 8, 148)
+    assert e.value.status == rrf.Status.ERR_SHAPE
+    with pytest.raises(rrf.RrfError):
+        rrf.rrf_plan_fused(0, 1, 64, 148)
+
+
+def test_import_fails_loudly_without_library(tmp_path):
+    """Without librrf.so the package refuses to import: there is no fallback."""
+    import shutil
+    pkg = tmp_path / "reduce_rmsnorm_fp8_b200"
+    shutil.copytree(os.path.join(ROOT, "reduce_rmsnorm_fp8_b200"), pkg,
+                    ignore=shutil.ignore_patterns("*.so", "_build", "__pycache__"))
+    r = subprocess.run([sys.executable, "-c", "import reduce_rmsnorm_fp8_b200"],
+                       cwd=tmp_path, capture_output=True, text=True)
+    assert r.returncode != 0 and "librrf.so is missing" in r.stderr

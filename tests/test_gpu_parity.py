@@ -1,0 +1,271 @@
+"""GPU parity: the CUDA library against the oracle on the same seeded inputs.
+
+Every workload is run through the C ABI (via the thin binding) and compared
+element by element with the oracle: bit-exact bf16 sum and residual, scales
+within 1e-6 relative, fp8 codes equal up to the stated midpoint allowance.
+The full-size prefill case is checked on sampled rows, in the launch the
+benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import parity
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def rrf():
+    import reduce_rmsnorm_fp8_b200 as m
+    return m
+
+
+def dev_case(name, rows=None, **kw):
+    return parity.to_device(workloads.make_case(name, rows, **kw))
+
+
+# ----------------------------------------------------------- the workloads ---
+
+def test_tiny(rrf):
+    c = dev_case("tiny")
+    parity.assert_fused_parity(parity.gpu_fused(c), parity.oracle_fused(c), "tiny")
+    assert np.array_equal(workloads.bits(rrf.rrf_sum(c.inputs)), parity.oracle_sum(c))
+
+
+@pytest.mark.parametrize("rows", [1, 8, 32, 64])
+def test_decode(rrf, rows):
+    c = dev_case("decode", rows)
+    parity.assert_fused_parity(parity.gpu_fused(c), parity.oracle_fused(c), f"decode {rows}")
+
+
+@pytest.mark.parametrize("rows", [37, 64])
+def test_odd_shapes_with_clamped_rows(rrf, rows):
+    c = dev_case("odd", rows)
+    ref = parity.oracle_fused(c)
+    parity.assert_fused_parity(parity.gpu_fused(c), ref, f"odd {rows}")
+    ub_scale = np.float32(c.scale_ub) / np.float32(448.0)
+    assert (ref["scales"] == ub_scale).any(), "no row reached the scale_ub clamp"
+    assert (ref["scales"] < ub_scale).any()
+
+
+@pytest.mark.parametrize("rows", [16, 32, 48, 64, 96, 128, 256])
+def test_sweep_sum_and_fused(rrf, rows):
+    c = dev_case("sweep", rows)
+    assert np.array_equal(workloads.bits(rrf.rrf_sum(c.inputs)), parity.oracle_sum(c))
+    parity.assert_fused_parity(parity.gpu_fused(c), parity.oracle_fused(c), f"sweep {rows}")
+
+
+def test_prefill_full_size_sampled_rows(rrf):
+    """8 x 8192 x 8192 with residual, drawn on the GPU; the outputs of the
+    whole call are checked on 40 rows spread over the batch (first and last
+    included) against the oracle on exactly those rows."""
+    c = workloads.make_case("prefill", device="cuda")
+    gpu = parity.gpu_fused(c)
+    rows = sorted(set([0, 1, c.rows - 1] + list(np.random.default_rng(4).choice(
+        c.rows, 37, replace=False))))
+    ref = parity.oracle_fused(c, rows=rows)
+    parity.assert_fused_parity(parity.select_rows(gpu, rows), ref, "prefill")
+    # every row's scale is positive and finite, and every residual row written
+    assert np.isfinite(gpu["scales"]).all() and (gpu["scales"] > 0).all()
+    del c
+    torch.cuda.empty_cache()
+
+
+def test_sum_prefill_size(rrf):
+    """rrf_sum at 8 x 8192 x 8192: bit-exact on sampled rows."""
+    c = workloads.make_case("prefill", device="cuda", residual=False)
+    s = rrf.rrf_sum(c.inputs)
+    rows = [0, 4095, 8191]
+    idx = torch.tensor(rows, device="cuda")
+    import oracle
+    ref = oracle.sum_bf16([workloads.bits(x.index_select(0, idx)) for x in c.inputs], 3, c.cols)
+    assert np.array_equal(workloads.bits(s.index_select(0, idx)), ref)
+    del c, s
+    torch.cuda.empty_cache()
+
+
+# ------------------------------------------------------ forced launch shapes ---
+
+@pytest.mark.parametrize("name,rows", [("decode", 64), ("odd", 37), ("decode", 1),
+                                       ("sweep", 16)])
+@pytest.mark.parametrize("variant,cluster", [(1, 0), (2, 2), (2, 4), (2, 8), (2, 16)])
+def test_forced_variants(rrf, name, rows, variant, cluster):
+    """Every cluster size (1 = one block per row) gives the same bf16 outputs
+    and matches the oracle within tolerance."""
+    c = dev_case(name, rows)
+    gpu = parity.gpu_fused(c, variant=variant, cluster_size=cluster)
+    parity.assert_fused_parity(gpu, parity.oracle_fused(c), f"{name} {rows} C={cluster}")
+
+
+@pytest.mark.parametrize("threads", [32, 64, 128, 256, 512])
+def test_forced_block_sizes(rrf, threads):
+    c = dev_case("odd", 64)
+    ref = parity.oracle_fused(c)
+    for variant, cluster in ((1, 0), (2, 4)):
+        try:
+            gpu = parity.gpu_fused(c, variant=variant, cluster_size=cluster,
+                                   block_threads=threads)
+        except rrf.RrfError as e:
+            assert e.status == rrf.Status.ERR_UNSUPPORTED  # slice too long for the block
+            continue
+        parity.assert_fused_parity(gpu, ref, f"threads={threads} C={cluster}")
+
+
+def test_variants_bitwise_identical_bf16(rrf):
+    c = dev_case("decode", 32)
+    outs = [parity.gpu_fused(c, variant=v, cluster_size=k)
+            for v, k in ((1, 0), (2, 2), (2, 4), (2, 8), (2, 16))]
+    for o in outs[1:]:
+        assert np.array_equal(o["res_out"], outs[0]["res_out"])
+
+
+# --------------------------------------------------------------- edge cases ---
+
+@pytest.mark.parametrize("cols", [8, 16, 264, 2880, 7176, 8200, 16384, 131072, 262144])
+def test_column_counts(rrf, cols):
+    """Ragged rows (vector counts that are not a multiple of the block) and
+    the hidden sizes the TensorRT-LLM padding discussion lists, up to the
+    longest row the library accepts."""
+    rows = 3 if cols >= 131072 else 5
+    c = dev_case("decode", rows, cols=cols, R=3)
+    parity.assert_fused_parity(parity.gpu_fused(c), parity.oracle_fused(c), f"cols {cols}")
+    assert np.array_equal(workloads.bits(rrf.rrf_sum(c.inputs)), parity.oracle_sum(c))
+
+
+@pytest.mark.parametrize("R", [1, 2, 3, 5, 8, 9, 16])
+def test_input_counts(rrf, R):
+    c = dev_case("odd", 37, R=R)
+    parity.assert_fused_parity(parity.gpu_fused(c), parity.oracle_fused(c), f"R={R}")
+    assert np.array_equal(workloads.bits(rrf.rrf_sum(c.inputs)), parity.oracle_sum(c))
+
+
+def test_in_place_residual(rrf):
+    c = dev_case("decode", 8)
+    parity.assert_fused_parity(parity.gpu_fused(c, in_place=True), parity.oracle_fused(c),
+                               "in place")
+
+
+def test_empty_batch(rrf):
+    x = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    g = torch.ones(256, dtype=torch.bfloat16, device="cuda")
+    q, s, r = rrf.rrf_sum_rmsnorm_fp8([x, x], g, 1e-6, 0.0, 1200.0, residual_in=x)
+    assert q.shape == (0, 256) and s.shape == (0, 1) and r.shape == (0, 256)
+    assert rrf.rrf_sum([x]).shape == (0, 256)
+
+
+def test_zero_rows_and_signed_zeros(rrf):
+    """All-zero rows: scale = 1e-12 / 448 and codes +-0 following the sign of
+    gamma + weight_offset; -0 inputs sum to -0."""
+    c = dev_case("tiny")
+    c.inputs = [torch.zeros_like(x) for x in c.inputs]
+    c.gamma = torch.tensor(np.where(np.arange(c.cols) % 3 == 0, -1.0, 1.0),
+                           dtype=torch.bfloat16, device="cuda")
+    gpu = parity.gpu_fused(c)
+    ref = parity.oracle_fused(c)
+    assert np.array_equal(gpu["q"], ref["q"])
+    assert (ref["q"][:, 0] == 0x80).all() and (ref["q"][:, 1] == 0x00).all()
+    assert np.array_equal(gpu["scales"], ref["scales"])
+    negz = [torch.full_like(x, -0.0) for x in c.inputs]
+    assert (workloads.bits(rrf.rrf_sum(negz)) == 0x8000).all()
+
+
+def test_saturation_and_no_clamp(rrf):
+    """scale_ub = +inf (no clamp) and a tiny scale_ub (every row clamped, most
+    codes saturated)."""
+    for ub in (float("inf"), 1e-3):
+        c = dev_case("odd", 37)
+        c.scale_ub = ub
+        ref = parity.oracle_fused(c)
+        parity.assert_fused_parity(parity.gpu_fused(c), ref, f"ub={ub}")
+    assert ((ref["q"] & 0x7F) == 0x7E).mean() > 0.5
+
+
+# ------------------------------------------------ determinism and graphs ---
+
+def test_repeat_and_graph_replay_bitwise(rrf):
+    """Repeated calls and three replays of a captured CUDA graph give the
+    same bits as the first eager call."""
+    c = dev_case("decode", 64)
+    first = parity.gpu_fused(c)
+    for _ in range(2):
+        again = parity.gpu_fused(c)
+        for k in first:
+            assert np.array_equal(first[k], again[k]), k
+    res_out = torch.empty_like(c.residual)
+    q = torch.empty(c.inputs[0].shape, dtype=torch.float8_e4m3fn, device="cuda")
+    s = torch.empty((c.rows, 1), dtype=torch.float32, device="cuda")
+    call = lambda: rrf.rrf_sum_rmsnorm_fp8(c.inputs, c.gamma, c.eps, c.weight_offset,
+                                           c.scale_ub, residual_in=c.residual,
+                                           residual_out=res_out, q_out=q, scales_out=s)
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        call()  # warm-up outside capture (sets the non-portable cluster attribute)
+    torch.cuda.current_stream().wait_stream(stream)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call()
+    for _ in range(3):
+        q.zero_()
+        s.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert np.array_equal(q.view(torch.uint8).cpu().numpy(), first["q"])
+        assert np.array_equal(s.reshape(-1).cpu().numpy(), first["scales"])
+        assert np.array_equal(workloads.bits(res_out), first["res_out"])
+
+
+# -------------------------------------------------- errors and guard bands ---
+
+def test_validation_on_device_tensors(rrf):
+    c = dev_case("tiny")
+    x = c.inputs
+    with pytest.raises(ValueError):  # the binding checks shapes before marshalling
+        rrf.rrf_sum([x[0], x[1][:, 8:]])
+    flat = torch.empty(c.rows * c.cols + 8, dtype=torch.bfloat16, device="cuda")
+    out = torch.empty_like(x[0])
+    with pytest.raises(rrf.RrfError) as e:  # an input misaligned by one element
+        rrf.rrf_sum_ptr([x[0].data_ptr(), flat.data_ptr() + 2], c.rows, c.cols,
+                        out.data_ptr())
+    assert e.value.status == rrf.Status.ERR_ALIGN
+    with pytest.raises(rrf.RrfError) as e:  # output over an input
+        rrf.rrf_sum_ptr([x[0].data_ptr(), x[1].data_ptr()], c.rows, c.cols, x[1].data_ptr())
+    assert e.value.status == rrf.Status.ERR_ALIAS
+    with pytest.raises(rrf.RrfError) as e:
+        rrf.rrf_sum_rmsnorm_fp8(x, c.gamma, -1.0, 0.0, 1.0)
+    assert e.value.status == rrf.Status.ERR_VALUE
+
+
+def test_injected_launch_failure_reports_cuda_error(rrf):
+    c = dev_case("tiny")
+    rrf.rrf_debug_fail_next_launch(719)
+    with pytest.raises(rrf.RrfError) as e:
+        rrf.rrf_sum_rmsnorm_fp8(c.inputs, c.gamma, c.eps, c.weight_offset, c.scale_ub)
+    assert e.value.status == rrf.Status.ERR_CUDA and e.value.cuda_error == 719
+    assert rrf.rrf_last_cuda_error() == 719
+    # the hook is one-shot and nothing was launched: the next call works
+    parity.assert_fused_parity(parity.gpu_fused(c), parity.oracle_fused(c), "after")
+
+
+def test_guard_bands_untouched(rrf):
+    """Outputs sit between canary bytes; a call writes nothing outside them."""
+    c = dev_case("odd", 37)
+    n = c.rows * c.cols
+    pad = 4096
+    qbuf = torch.full((n + 2 * pad,), 0xA5, dtype=torch.uint8, device="cuda")
+    sbuf = torch.full((c.rows + 2 * pad // 4,), 7.0, dtype=torch.float32, device="cuda")
+    rbuf = torch.full((n + 2 * pad,), 3.0, dtype=torch.bfloat16, device="cuda")
+    q = qbuf[pad:pad + n].view(torch.float8_e4m3fn).view(c.rows, c.cols)
+    s = sbuf[pad // 4:pad // 4 + c.rows].view(c.rows, 1)
+    r = rbuf[pad:pad + n].view(c.rows, c.cols)
+    rrf.rrf_sum_rmsnorm_fp8(c.inputs, c.gamma, c.eps, c.weight_offset, c.scale_ub,
+                            residual_in=c.residual, residual_out=r, q_out=q, scales_out=s)
+    torch.cuda.synchronize()
+    assert (qbuf[:pad] == 0xA5).all() and (qbuf[pad + n:] == 0xA5).all()
+    assert (sbuf[:pad // 4] == 7.0).all() and (sbuf[pad // 4 + c.rows:] == 7.0).all()
+    assert (rbuf[:pad] == 3.0).all() and (rbuf[pad + n:] == 3.0).all()
+    got = {"q": q.view(torch.uint8).cpu().numpy(), "scales": s.reshape(-1).cpu().numpy(),
+           "res_out": workloads.bits(r)}
+    parity.assert_fused_parity(got, parity.oracle_fused(c), "guarded")
