@@ -20,6 +20,16 @@ __device__ __forceinline__ uint4 ld_once(const uint4* p) {
     return v;
 }
 
+// The same for data the kernel may also write (an in-place residual): a
+// coherent load, still without L1 allocation.
+__device__ __forceinline__ uint4 ld_once_coherent(const uint4* p) {
+    uint4 v;
+    asm volatile("ld.global.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
 // 16-byte load of data every block of the grid reads (gamma): read-only path,
 // cached.
 __device__ __forceinline__ uint4 ld_shared_by_all(const uint4* p) {

@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
             for (int r = 0; r < RB; ++r)
                 if (r < a.R) x[r] = ld_once(a.in[r] + row_base + v);
             uint4 res;
-            if (RES) res = ld_once(a.res_in + row_base + v);
+            if (RES) res = ld_once_coherent(a.res_in + row_base + v);
 
             float acc[8];
             bf16x8_to_f32(x[0], acc);
