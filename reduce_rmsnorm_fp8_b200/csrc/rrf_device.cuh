@@ -21,12 +21,13 @@ __device__ __forceinline__ uint4 ld_once(const uint4* p) {
 }
 
 // The same for data the kernel may also write (an in-place residual): a
-// coherent load, still without L1 allocation.
+// coherent load, still without L1 allocation.  Each element is loaded once,
+// by the thread that later overwrites it, so the load may be scheduled freely.
 __device__ __forceinline__ uint4 ld_once_coherent(const uint4* p) {
     uint4 v;
-    asm volatile("ld.global.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
+    asm("ld.global.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+        : "l"(p));
     return v;
 }
 
