@@ -160,48 +160,50 @@ class ClockSampler:
 # -------------------------------------------------------------- CUDA arm ---
 
 class DevicePool:
-    """Rotating buffer sets for one workload: per set and call, the R inputs,
-    the residual, gamma and the outputs, all resident in HBM."""
+    """Rotating buffer sets, all resident in HBM: for each call of the
+    workload (or the listed row counts), n_sets copies of the R inputs, the
+    residual, gamma and the outputs, carved as views from one allocation per
+    tensor kind.  n_sets is chosen so the sets together exceed min_bytes of
+    algorithmic traffic, so a set is cold in L2 when its turn comes again."""
 
-    def __init__(self, name: str, device, min_bytes: int):
+    def __init__(self, name: str, device, min_bytes: int, rows_list=None):
         import torch
         self.name = name
         w = workloads.WORKLOADS[name]
-        self.cases = []
-        for rows, residual in workload_cases(name):
-            c = workloads.make_case(name, rows, device=device)
-            self.cases.append(c)
-        per_set = step_bytes(name)
-        self.n_sets = max(2, math.ceil(min_bytes / per_set))
-        self.sets = []
-        for _ in range(self.n_sets):
-            calls = []
-            for c in self.cases:
-                calls.append(dict(
-                    inputs=[x.clone() for x in c.inputs],
-                    residual=None if c.residual is None else c.residual.clone(),
-                    res_out=None if c.residual is None else torch.empty_like(c.residual),
-                    gamma=c.gamma.clone(),
-                    q=torch.empty(c.inputs[0].shape, dtype=torch.float8_e4m3fn, device=device),
-                    scales=torch.empty((c.rows, 1), dtype=torch.float32, device=device)))
-            self.sets.append(calls)
+        rows_list = list(w.rows) if rows_list is None else list(rows_list)
+        self.cases = [workloads.make_case(name, rows, device=device) for rows in rows_list]
+        per_set = sum(workloads.fused_bytes(w.R, c.rows, c.cols, c.residual is not None)
+                      for c in self.cases)
+        self.n_sets = n = max(2, math.ceil(min_bytes / per_set))
+        self.per_set_bytes = per_set
+        self.big = []
+        for c in self.cases:
+            shape = (n, c.rows, c.cols)
+            b = {"inputs": [x.unsqueeze(0).expand(shape).contiguous() for x in c.inputs],
+                 "gamma": c.gamma.unsqueeze(0).expand(n, c.cols).contiguous(),
+                 "q": torch.empty(shape, dtype=torch.float8_e4m3fn, device=device),
+                 "scales": torch.empty((n, c.rows, 1), dtype=torch.float32, device=device),
+                 "residual": None, "res_out": None}
+            if c.residual is not None:
+                b["residual"] = c.residual.unsqueeze(0).expand(shape).contiguous()
+                b["res_out"] = torch.empty(shape, dtype=torch.bfloat16, device=device)
+            self.big.append(b)
         self.eps, self.wo, self.ub = w.eps, w.weight_offset, w.scale_ub
 
-    def run_step(self, rrf, k: int) -> int:
-        """Enqueue step k (every call of the workload on set k mod n); returns
-        the number of kernels launched."""
-        for b in self.sets[k % self.n_sets]:
-            rrf.rrf_sum_rmsnorm_fp8(b["inputs"], b["gamma"], self.eps, self.wo, self.ub,
-                                    residual_in=b["residual"], residual_out=b["res_out"],
-                                    q_out=b["q"], scales_out=b["scales"])
-        return len(self.cases)
-
-    def run_call(self, rrf, k: int, i: int) -> int:
-        b = self.sets[k % self.n_sets][i]
-        rrf.rrf_sum_rmsnorm_fp8(b["inputs"], b["gamma"], self.eps, self.wo, self.ub,
-                                residual_in=b["residual"], residual_out=b["res_out"],
-                                q_out=b["q"], scales_out=b["scales"])
+    def call(self, rrf, k: int, i: int) -> int:
+        """Enqueue call i of the workload on set k mod n_sets; returns 1."""
+        b, s = self.big[i], k % self.n_sets
+        rrf.rrf_sum_rmsnorm_fp8(
+            [x[s] for x in b["inputs"]], b["gamma"][s], self.eps, self.wo, self.ub,
+            residual_in=None if b["residual"] is None else b["residual"][s],
+            residual_out=None if b["res_out"] is None else b["res_out"][s],
+            q_out=b["q"][s], scales_out=b["scales"][s])
         return 1
+
+    def run_step(self, rrf, k: int) -> int:
+        """Enqueue step k: every call of the workload on set k mod n_sets;
+        returns the number of kernels launched."""
+        return sum(self.call(rrf, k, i) for i in range(len(self.cases)))
 
 
 def time_region(fn, k_steps: int, device, stream):
@@ -235,52 +237,68 @@ def capture_steps(fn, n: int, device):
     return g, launched
 
 
+class _Arena:
+    """Views of one byte buffer, each starting on a 256-byte boundary."""
+
+    def __init__(self):
+        self.size, self.items = 0, []
+
+    def add(self, shape, dtype):
+        import torch
+        off = (self.size + 255) // 256 * 256
+        n = math.prod(shape) * torch.empty((), dtype=dtype).element_size()
+        self.items.append((off, n, shape, dtype))
+        self.size = off + n
+        return len(self.items) - 1
+
+    def views(self, buf):
+        return [buf[off:off + n].view(dtype).view(shape) for off, n, shape, dtype in self.items]
+
+
 def e2e_measure(rrf, name: str, k_steps: int, warmup: int, device, stream):
     """The same metric through the public call with HOST buffers: every step
-    copies its inputs from pinned host memory, runs the calls and reads the
-    results back; copies included in the timed region."""
+    copies its inputs (all calls' inputs, residuals and gammas, packed in one
+    pinned host buffer) to the device in one copy, runs the calls, and reads
+    all results (codes, scales, residual outputs) back in one copy; both
+    copies are inside the timed region."""
     import torch
     w = workloads.WORKLOADS[name]
-    host, dev = [], []
-    h2d = d2h = 0
-    for rows, residual in workload_cases(name):
-        c = workloads.make_case(name, rows)
-        hb = dict(inputs=[x.pin_memory() for x in c.inputs],
-                  residual=None if c.residual is None else c.residual.pin_memory(),
-                  gamma=c.gamma.pin_memory(),
-                  q=torch.empty(c.inputs[0].shape, dtype=torch.uint8).pin_memory(),
-                  scales=torch.empty((rows, 1), dtype=torch.float32).pin_memory(),
-                  res_out=None if c.residual is None else
-                  torch.empty_like(c.residual).pin_memory())
-        db = dict(inputs=[torch.empty_like(x, device=device) for x in c.inputs],
-                  residual=None if c.residual is None else
-                  torch.empty_like(c.residual, device=device),
-                  gamma=torch.empty_like(c.gamma, device=device),
-                  q=torch.empty(c.inputs[0].shape, dtype=torch.float8_e4m3fn, device=device),
-                  scales=torch.empty((rows, 1), dtype=torch.float32, device=device),
-                  res_out=None if c.residual is None else
-                  torch.empty_like(c.residual, device=device))
-        h2d += sum(x.numel() * 2 for x in c.inputs) + c.gamma.numel() * 2 + \
-            (c.residual.numel() * 2 if c.residual is not None else 0)
-        d2h += rows * w.cols + rows * 4 + (rows * w.cols * 2 if residual else 0)
-        host.append(hb)
-        dev.append(db)
+    cases = [workloads.make_case(name, rows) for rows, _ in workload_cases(name)]
+    ins, outs = _Arena(), _Arena()
+    slots = []
+    for c in cases:
+        shape = (c.rows, c.cols)
+        slot = {"inputs": [ins.add(shape, torch.bfloat16) for _ in c.inputs],
+                "gamma": ins.add((c.cols,), torch.bfloat16),
+                "residual": ins.add(shape, torch.bfloat16) if c.residual is not None else None,
+                "q": outs.add(shape, torch.uint8),
+                "scales": outs.add((c.rows, 1), torch.float32),
+                "res_out": outs.add(shape, torch.bfloat16) if c.residual is not None else None}
+        slots.append(slot)
+    h_in = torch.empty(ins.size, dtype=torch.uint8).pin_memory()
+    h_out = torch.empty(outs.size, dtype=torch.uint8).pin_memory()
+    d_in = torch.empty(ins.size, dtype=torch.uint8, device=device)
+    d_out = torch.empty(outs.size, dtype=torch.uint8, device=device)
+    hv, dv, ov = ins.views(h_in), ins.views(d_in), outs.views(d_out)
+    for c, slot in zip(cases, slots):  # the host data of the step
+        for x, i in zip(c.inputs, slot["inputs"]):
+            hv[i].copy_(x)
+        hv[slot["gamma"]].copy_(c.gamma)
+        if slot["residual"] is not None:
+            hv[slot["residual"]].copy_(c.residual)
+    h2d = sum(n for _, n, _, _ in ins.items)
+    d2h = sum(n for _, n, _, _ in outs.items)
 
     def step(_):
-        for hb, db in zip(host, dev):
-            for xd, xh in zip(db["inputs"], hb["inputs"]):
-                xd.copy_(xh, non_blocking=True)
-            if hb["residual"] is not None:
-                db["residual"].copy_(hb["residual"], non_blocking=True)
-            db["gamma"].copy_(hb["gamma"], non_blocking=True)
-            rrf.rrf_sum_rmsnorm_fp8(db["inputs"], db["gamma"], w.eps, w.weight_offset,
-                                    w.scale_ub, residual_in=db["residual"],
-                                    residual_out=db["res_out"], q_out=db["q"],
-                                    scales_out=db["scales"])
-            hb["q"].copy_(db["q"].view(torch.uint8), non_blocking=True)
-            hb["scales"].copy_(db["scales"], non_blocking=True)
-            if hb["res_out"] is not None:
-                hb["res_out"].copy_(db["res_out"], non_blocking=True)
+        d_in.copy_(h_in, non_blocking=True)
+        for slot in slots:
+            rrf.rrf_sum_rmsnorm_fp8(
+                [dv[i] for i in slot["inputs"]], dv[slot["gamma"]], w.eps, w.weight_offset,
+                w.scale_ub,
+                residual_in=None if slot["residual"] is None else dv[slot["residual"]],
+                residual_out=None if slot["res_out"] is None else ov[slot["res_out"]],
+                q_out=ov[slot["q"]].view(torch.float8_e4m3fn), scales_out=ov[slot["scales"]])
+        h_out.copy_(d_out, non_blocking=True)
 
     with torch.cuda.stream(stream):
         for i in range(warmup):
@@ -364,20 +382,25 @@ def run_rrf(args):
     with ClockSampler(device.index) as clocks:
         t = time_region(lambda _: graph.replay(), 1, device, stream)
     del graph
+    n_sets = pool.n_sets
     per_step = step_bytes(name)
     value = world * per_step * args.steps / t / 1e9
     kernel_us = t / launches * 1e6
 
-    # ---- per-call breakdown (separate graphs, same rotation)
+    # ---- per-call breakdown: each row count alone, with its own rotating
+    # pool above 3 x L2 (a pool shared with the other calls would leave a
+    # small call's sets hot in L2 when it runs alone)
     cases = []
     reps = max(args.steps, 100)
-    for i, c in enumerate(pool.cases):
-        gi, _ = capture_steps(lambda k, i=i: pool.run_call(rrf, args.warmup + k, i), reps,
-                              device)
+    for c in pool.cases:
+        cp = DevicePool(name, device, L2_FLUSH_FACTOR * l2, rows_list=[c.rows])
+        for i in range(3):
+            cp.call(rrf, i, 0)
+        gi, _ = capture_steps(lambda k: cp.call(rrf, 3 + k, 0), reps, device)
         gi.replay()
         torch.cuda.synchronize(device)
         tc = time_region(lambda _: gi.replay(), 1, device, stream)
-        del gi
+        del gi, cp
         b = workloads.fused_bytes(w.R, c.rows, c.cols, c.residual is not None)
         launch = rrf.rrf_plan_fused(w.R, c.rows, c.cols, props.multi_processor_count)
         cases.append({"rows": c.rows, "us_per_call": round(tc / reps * 1e6, 3),
@@ -386,6 +409,7 @@ def run_rrf(args):
                       "rows_per_s": round(c.rows * reps / tc, 1),
                       "launch": {"cluster": launch[0], "threads": launch[1],
                                  "vecs_per_thread": launch[2]}})
+    torch.cuda.empty_cache()
 
     # ---- end to end through host buffers
     e2e = None
@@ -437,7 +461,8 @@ def run_rrf(args):
                                    f"per step, residual={'on' if w.residual else 'off'}",
                        "R": w.R, "cols": w.cols, "rows": list(w.rows),
                        "bytes_per_step": per_step,
-                       "l2": f"rotating {pool_sets_note(name, l2)} buffer sets > "
+                       "l2": f"inputs larger than L2: {n_sets} rotating buffer sets, "
+                             f"{n_sets * per_step >> 20} MiB of traffic > "
                              f"{L2_FLUSH_FACTOR}x L2 ({l2 >> 20} MiB)",
                        "launch": "auto (rrf_sum_rmsnorm_fp8)",
                        "timing": "K steps captured in one CUDA graph, one replay timed "
@@ -461,10 +486,6 @@ def run_rrf(args):
     if world > 1:
         dist.barrier(device_ids=[device.index])
         dist.destroy_process_group()
-
-
-def pool_sets_note(name: str, l2: int) -> str:
-    return str(max(2, math.ceil(L2_FLUSH_FACTOR * l2 / step_bytes(name))))
 
 
 def run_reference(args):

@@ -141,20 +141,30 @@ rrf_status rrf_sum_rmsnorm_fp8(const void* const* inputs, int num_inputs,
                                  #19836: cluster.sync() before remote writes, one
                                  arrive / wait per thread per barrier phase)      */
 
+/* Launch flags of rrf_sum_rmsnorm_fp8_ex. */
+#define RRF_FLAG_NO_PDL 1     /* launch without programmatic dependent launch     */
+
 /* rrf_sum_rmsnorm_fp8_ex -- rrf_sum_rmsnorm_fp8 with the launch forced, for
  * tests and benchmarks.  variant is one of RRF_VARIANT_*; cluster_size is
  * 2, 4, 8 or 16 for RRF_VARIANT_CLUSTER (0 = automatic) and ignored
  * otherwise; block_threads is a multiple of 32 in [32, 1024] or 0
- * (automatic).  Results are bit-identical across variants for the bf16
- * outputs and agree within the stated tolerance for scales and codes.
+ * (automatic); flags is 0 or RRF_FLAG_NO_PDL.  Results are bit-identical
+ * across variants for the bf16 outputs and agree within the stated tolerance
+ * for scales and codes.
+ *
+ * Programmatic dependent launch: by default every kernel of this library is
+ * launched so that it may start while the previous kernel in the stream is
+ * still finishing; each kernel waits for that kernel (its completion and the
+ * visibility of its writes) before it touches global memory, so stream order
+ * is kept for every producer.  RRF_FLAG_NO_PDL launches the plain way.
  * Errors: those of rrf_sum_rmsnorm_fp8, and RRF_ERR_UNSUPPORTED when the
- * forced launch cannot cover the row. */
+ * forced launch cannot cover the row or flags holds an unknown bit. */
 rrf_status rrf_sum_rmsnorm_fp8_ex(const void* const* inputs, int num_inputs,
                                   int64_t rows, int64_t cols, const void* residual_in,
                                   void* residual_out, const void* gamma, float eps,
                                   float weight_offset, float scale_ub, void* q_out,
                                   float* scales_out, int variant, int cluster_size,
-                                  int block_threads, rrf_stream_t stream);
+                                  int block_threads, int flags, rrf_stream_t stream);
 
 /* rrf_plan_fused -- the launch rrf_sum_rmsnorm_fp8 would use on a GPU with
  * sm_count SMs, without touching the GPU.  Writes the cluster size (1 = one

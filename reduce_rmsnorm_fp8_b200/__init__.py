@@ -21,6 +21,7 @@ from __future__ import annotations
 from ._lib import (  # noqa: F401
     LIB_PATH,
     RRF_MAX_COLS,
+    RRF_FLAG_NO_PDL,
     RRF_MAX_INPUTS,
     RRF_VARIANT_AUTO,
     RRF_VARIANT_CLUSTER,

@@ -13,6 +13,7 @@ RRF_MAX_COLS = 16 * 256 * 8 * 8
 RRF_VARIANT_AUTO = 0
 RRF_VARIANT_ROW = 1
 RRF_VARIANT_CLUSTER = 2
+RRF_FLAG_NO_PDL = 1
 
 
 class Status(enum.IntEnum):
@@ -58,7 +59,7 @@ _fused_args = [_ptrs, _int, _i64, _i64, _vp, _vp, _vp, _f32, _f32, _f32, _vp, _v
 lib.rrf_sum_rmsnorm_fp8.restype = _int
 lib.rrf_sum_rmsnorm_fp8.argtypes = _fused_args + [_vp]
 lib.rrf_sum_rmsnorm_fp8_ex.restype = _int
-lib.rrf_sum_rmsnorm_fp8_ex.argtypes = _fused_args + [_int, _int, _int, _vp]
+lib.rrf_sum_rmsnorm_fp8_ex.argtypes = _fused_args + [_int, _int, _int, _int, _vp]
 lib.rrf_plan_fused.restype = _int
 lib.rrf_plan_fused.argtypes = [_int, _i64, _i64, _int, ctypes.POINTER(_int),
                                ctypes.POINTER(_int), ctypes.POINTER(_int)]
@@ -133,12 +134,12 @@ def rrf_sum_ptr(input_ptrs, rows, cols, out_ptr, stream=0) -> None:
 
 def rrf_sum_rmsnorm_fp8_ptr(input_ptrs, rows, cols, residual_in, residual_out, gamma, eps,
                             weight_offset, scale_ub, q_out, scales_out, variant=0,
-                            cluster_size=0, block_threads=0, stream=0) -> None:
+                            cluster_size=0, block_threads=0, flags=0, stream=0) -> None:
     """rrf_sum_rmsnorm_fp8_ex on raw device pointers and a raw stream handle."""
     _raise_on(lib.rrf_sum_rmsnorm_fp8_ex(
         _ptr_table(input_ptrs), len(input_ptrs), rows, cols, residual_in or None,
         residual_out or None, gamma or None, eps, weight_offset, scale_ub, q_out or None,
-        scales_out or None, variant, cluster_size, block_threads, stream or None))
+        scales_out or None, variant, cluster_size, block_threads, flags, stream or None))
 
 
 # ------------------------------------------------------------ torch calls ---
@@ -189,9 +190,10 @@ def rrf_sum(inputs, out=None):
 
 def rrf_sum_rmsnorm_fp8_ex(inputs, gamma, eps, weight_offset, scale_ub, residual_in=None,
                            residual_out=None, q_out=None, scales_out=None, variant=0,
-                           cluster_size=0, block_threads=0):
+                           cluster_size=0, block_threads=0, flags=0):
     """The fused operation with a forced launch (variant, cluster size, block
-    size; 0 = automatic).  Returns (q, scales, residual_out)."""
+    size; 0 = automatic; flags RRF_FLAG_NO_PDL).  Returns (q, scales,
+    residual_out)."""
     torch = _torch()
     rows, cols = _rows_cols(inputs)
     x0 = inputs[0]
@@ -210,7 +212,7 @@ def rrf_sum_rmsnorm_fp8_ex(inputs, gamma, eps, weight_offset, scale_ub, residual
             residual_in.data_ptr() if residual_in is not None else 0,
             residual_out.data_ptr() if residual_out is not None else 0,
             gamma.data_ptr(), eps, weight_offset, scale_ub, q_out.data_ptr(),
-            scales_out.data_ptr(), variant, cluster_size, block_threads, _stream(dev))
+            scales_out.data_ptr(), variant, cluster_size, block_threads, flags, _stream(dev))
     return q_out, scales_out, residual_out
 
 

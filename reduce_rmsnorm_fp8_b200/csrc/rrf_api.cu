@@ -92,9 +92,11 @@ rrf_status check_inputs(const void* const* inputs, int num_inputs) {
 static int round_up32(int64_t x) { return (int)((x + 31) / 32 * 32); }
 
 // Threads per block and vectors per thread for a row slice of `slice`
-// vectors: the fewest vectors per thread that keep the block at <= 256
+// vectors: the fewest vectors per thread that keep the block at <= 512
 // threads (any size up to the compiled bound at 8 vectors per thread), or,
 // with forced_threads, the fewest that let that many threads cover the slice.
+// (On B200 the 8 x 8192-column prefill row runs fastest as 512 threads x 2
+// vectors: 2 blocks and 1024 threads per SM keep the most loads in flight.)
 static bool pick_block(int R, int64_t slice, int forced_threads, FusedLaunch* l) {
     const int rb = input_bound(R);
     for (int vpt = 1; vpt <= 8; vpt *= 2) {
@@ -105,7 +107,7 @@ static bool pick_block(int R, int64_t slice, int forced_threads, FusedLaunch* l)
             if (t > max_t || (int64_t)t * vpt < slice) continue;
         } else {
             t = round_up32((slice + vpt - 1) / vpt);
-            if ((t > 256 && vpt < 8) || t > max_t) continue;
+            if ((t > 512 && vpt < 8) || t > max_t) continue;
         }
         l->threads = t;
         l->vecs_per_thread = vpt;
@@ -125,10 +127,13 @@ static rrf_status shape_launch(int R, int64_t rows, int64_t cols, int sm_count, 
     int c = cluster;
     if (c == 0) {
         // Split rows across the blocks of a cluster until the grid covers the
-        // SMs, keeping at least 32 vectors (one warp's worth) per block; then
-        // split further while one block cannot hold its slice.
+        // SMs, keeping at least 96 vectors per block and clusters of at most
+        // 8 (measured on B200: at 1-64 rows of 7168 columns, clusters of 16
+        // and slices under ~100 vectors lose more to the cluster barrier than
+        // they gain in parallel loads); then split further, up to 16, while
+        // one block cannot hold its slice.
         c = 1;
-        while (c < 16 && rows * c < sm_count && vecs / (2 * c) >= 32) c *= 2;
+        while (c < 8 && rows * c < sm_count && vecs / (2 * c) >= 96) c *= 2;
         while (c < 16 && !pick_block(R, (vecs + c - 1) / c, forced_threads, out)) c *= 2;
     }
     if (!pick_block(R, (vecs + c - 1) / c, forced_threads, out))
@@ -229,7 +234,7 @@ extern "C" rrf_status rrf_sum(const void* const* inputs, int num_inputs, int64_t
     a.R = num_inputs;
     a.n_vecs = rows * cols / 8;
     cudaError_t e;
-    if (!take_injected_failure(&e)) e = launch_sum(a, sm_count, (cudaStream_t)stream);
+    if (!take_injected_failure(&e)) e = launch_sum(a, sm_count, true, (cudaStream_t)stream);
     return e == cudaSuccess ? RRF_OK : cuda_fail(e);
 }
 
@@ -239,13 +244,14 @@ extern "C" rrf_status rrf_sum_rmsnorm_fp8_ex(const void* const* inputs, int num_
                                              const void* gamma, float eps,
                                              float weight_offset, float scale_ub,
                                              void* q_out, float* scales_out, int variant,
-                                             int cluster_size, int block_threads,
+                                             int cluster_size, int block_threads, int flags,
                                              rrf_stream_t stream) {
     rrf_status st = rrf_check_fused_args(inputs, num_inputs, rows, cols, residual_in,
                                          residual_out, gamma, eps, weight_offset, scale_ub,
                                          q_out, scales_out);
     if (st != RRF_OK) return st;
     if (variant < RRF_VARIANT_AUTO || variant > RRF_VARIANT_CLUSTER) return RRF_ERR_UNSUPPORTED;
+    if ((flags & ~RRF_FLAG_NO_PDL) != 0) return RRF_ERR_UNSUPPORTED;
     if (block_threads != 0 && (block_threads < 32 || block_threads > 1024 || block_threads % 32))
         return RRF_ERR_UNSUPPORTED;
     if (variant == RRF_VARIANT_CLUSTER && cluster_size != 0 && cluster_size != 2 &&
@@ -270,6 +276,7 @@ extern "C" rrf_status rrf_sum_rmsnorm_fp8_ex(const void* const* inputs, int num_
         RRF_OK)
         return st;
     const int64_t vecs = cols / 8;
+    l.pdl = (flags & RRF_FLAG_NO_PDL) == 0;
 
     FusedArgs a = {};
     for (int r = 0; r < num_inputs; ++r) a.in[r] = static_cast<const uint4*>(inputs[r]);
@@ -300,7 +307,7 @@ extern "C" rrf_status rrf_sum_rmsnorm_fp8(const void* const* inputs, int num_inp
                                           rrf_stream_t stream) {
     return rrf_sum_rmsnorm_fp8_ex(inputs, num_inputs, rows, cols, residual_in, residual_out,
                                   gamma, eps, weight_offset, scale_ub, q_out, scales_out,
-                                  RRF_VARIANT_AUTO, 0, 0, stream);
+                                  RRF_VARIANT_AUTO, 0, 0, 0, stream);
 }
 
 extern "C" rrf_status rrf_plan_fused(int num_inputs, int64_t rows, int64_t cols, int sm_count,

@@ -1,6 +1,7 @@
 // rrf_device.cuh -- device-side building blocks of the sum and fused kernels:
-// 16-byte memory access, bf16 / e4m3fn conversion, warp / block / cluster
-// reductions.  sm_100a only.
+// 16-byte memory access, bf16 / e4m3fn conversion, programmatic dependent
+// launch, cluster barriers and the warp / block / cluster reduction of a
+// row's statistics.  sm_100a only.
 #pragma once
 
 #include <cuda_fp8.h>
@@ -119,39 +120,20 @@ __device__ __forceinline__ uint2 f32_to_e4m3x8(const float f[8]) {
     return q;
 }
 
-// -------------------------------------------------------------- reductions --
-// Butterfly (xor) reductions: at every level lane i combines its value with
-// lane i ^ off's, and a + b == b + a in IEEE arithmetic, so every lane ends
-// with the same bits and the result does not depend on which lane reads it.
+// ------------------------------------------------ programmatic dependent launch --
+// A kernel launched with programmatic stream serialization may start while the
+// previous kernel in the stream is still running.  It must wait for that
+// kernel (completion and memory visibility) before it reads or writes global
+// memory; without the launch attribute the wait returns at once.
 
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
-    return v;
+__device__ __forceinline__ void wait_for_previous_grid() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, off));
-    return v;
-}
-
-// Block-wide sum / max, returned to every thread.  `scratch` holds one float
-// per warp and must not be reused until every thread has returned.
-__device__ __forceinline__ float block_sum(float v, float* scratch) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-    v = warp_sum(v);
-    if (lane == 0) scratch[warp] = v;
-    __syncthreads();
-    return warp_sum(lane < nwarps ? scratch[lane] : 0.0f);
-}
-
-__device__ __forceinline__ float block_max(float v, float* scratch) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-    v = warp_max(v);
-    if (lane == 0) scratch[warp] = v;
-    __syncthreads();
-    return warp_max(lane < nwarps ? scratch[lane] : 0.0f);
+// Let the next kernel in the stream be scheduled; it still waits for this
+// whole grid before touching memory.
+__device__ __forceinline__ void allow_next_grid() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ------------------------------------------------------ thread-block cluster --
@@ -178,27 +160,102 @@ __device__ __forceinline__ void cluster_wait_acquire() {
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Store v into the shared-memory word `local` of cluster block `peer`.
-__device__ __forceinline__ void st_peer_shared(float* local, uint32_t peer, float v) {
-    const uint32_t laddr = (uint32_t)__cvta_generic_to_shared(local);
-    uint32_t raddr;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(raddr) : "r"(laddr), "r"(peer));
-    asm volatile("st.shared::cluster.f32 [%0], %1;" :: "r"(raddr), "f"(v) : "memory");
+// --------------------------------------------------------- row statistics --
+// Butterfly (xor) reductions: at every level lane i merges its value with
+// lane i ^ off's; the merge is commutative, so every lane ends with the same
+// bits and the result does not depend on which lane reads it.
+//
+// What a row's norm needs from all of its elements, reduced in one pass: the
+// sum of squares of h and the amax candidate, the element (h, g' = gamma +
+// weight_offset) with the largest key |h * g'|.  The merge keeps the larger
+// candidate under a total order (key, then the bits of h, then of g'), so it
+// is commutative and associative like the sum, and butterfly reductions
+// leave the same bits in every lane.
+
+struct __align__(16) RowStats {  // 16-byte aligned: one v4 store per peer
+    float ss;   // sum of h^2
+    float key;  // |h * g'| of the candidate (-1: no element yet)
+    float h;
+    float g;
+};
+
+__device__ __forceinline__ RowStats stats_empty() { return RowStats{0.0f, -1.0f, 0.0f, 0.0f}; }
+
+__device__ __forceinline__ bool stats_better(float key, float h, float g, const RowStats& s) {
+    if (key != s.key) return key > s.key;  // NaN keys never win
+    const uint32_t hb = __float_as_uint(h), sh = __float_as_uint(s.h);
+    if (hb != sh) return hb > sh;
+    return __float_as_uint(g) > __float_as_uint(s.g);
 }
 
-// Cluster-wide combination of one value per block: block `rank` writes its
-// value into slot[rank] of every block (threads 0..C-1 write one peer each),
-// one barrier phase publishes the writes, and every block reduces the C slots
-// with the same butterfly, so all blocks hold the same bits.
-template <bool IS_MAX>
-__device__ __forceinline__ float cluster_combine(float block_value, float* slots,
-                                                 uint32_t rank, int C) {
-    if ((int)threadIdx.x < C) st_peer_shared(&slots[rank], threadIdx.x, block_value);
+// Offer one element to a thread's statistics (the sum of squares is
+// accumulated separately, per 8-element vector).
+__device__ __forceinline__ void stats_offer(RowStats& s, float h, float g) {
+    const float key = fabsf(__fmul_rn(h, g));
+    if (stats_better(key, h, g, s)) {
+        s.key = key;
+        s.h = h;
+        s.g = g;
+    }
+}
+
+__device__ __forceinline__ RowStats stats_merge(RowStats a, const RowStats& b) {
+    a.ss = a.ss + b.ss;
+    if (stats_better(b.key, b.h, b.g, a)) {
+        a.key = b.key;
+        a.h = b.h;
+        a.g = b.g;
+    }
+    return a;
+}
+
+__device__ __forceinline__ RowStats shfl_xor_stats(const RowStats& s, int off) {
+    RowStats o;
+    o.ss = __shfl_xor_sync(0xFFFFFFFFu, s.ss, off);
+    o.key = __shfl_xor_sync(0xFFFFFFFFu, s.key, off);
+    o.h = __shfl_xor_sync(0xFFFFFFFFu, s.h, off);
+    o.g = __shfl_xor_sync(0xFFFFFFFFu, s.g, off);
+    return o;
+}
+
+__device__ __forceinline__ RowStats warp_stats_reduce(RowStats s) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s = stats_merge(s, shfl_xor_stats(s, off));
+    return s;
+}
+
+// Block-wide statistics, returned to every thread (one __syncthreads).
+__device__ __forceinline__ RowStats block_stats(RowStats s, RowStats* scratch) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    s = warp_stats_reduce(s);
+    if (lane == 0) scratch[warp] = s;
+    __syncthreads();
+    return warp_stats_reduce(lane < nwarps ? scratch[lane] : stats_empty());
+}
+
+// Store a block's statistics into slot `rank` of cluster block `peer`.
+__device__ __forceinline__ void st_peer_stats(RowStats* slots, uint32_t rank, uint32_t peer,
+                                              const RowStats& s) {
+    const uint32_t laddr = (uint32_t)__cvta_generic_to_shared(&slots[rank]);
+    uint32_t raddr;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(raddr) : "r"(laddr), "r"(peer));
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};"
+                 :: "r"(raddr), "f"(s.ss), "f"(s.key), "f"(s.h), "f"(s.g)
+                 : "memory");
+}
+
+// Cluster-wide statistics: block `rank` writes its statistics into slot
+// `rank` of every block of the cluster (threads 0..C-1 write one peer each),
+// one barrier phase publishes the writes, and every block reduces the C
+// slots with the same butterfly, so all blocks hold the same bits.  The
+// caller has completed barrier phase 0 (every block has started).
+__device__ __forceinline__ RowStats cluster_stats_combine(const RowStats& block, RowStats* slots,
+                                                          uint32_t rank, int C) {
+    if ((int)threadIdx.x < C) st_peer_stats(slots, rank, threadIdx.x, block);
     cluster_arrive_release();
     cluster_wait_acquire();
     const int lane = threadIdx.x & 31;
-    const float t = lane < C ? slots[lane] : 0.0f;
-    return IS_MAX ? warp_max(t) : warp_sum(t);
+    return warp_stats_reduce(lane < C ? slots[lane] : stats_empty());
 }
 
 }  // namespace rrf

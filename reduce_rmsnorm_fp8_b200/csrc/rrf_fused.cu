@@ -5,17 +5,21 @@
 // memory).  Each block owns a contiguous slice of the row's 16-byte vectors;
 // each thread owns up to VPT of them, strided by the block size so that a
 // warp's accesses are contiguous.  Every input byte is read from HBM once;
-// the row's bf16 norm input h stays in registers between the three passes
-// (gamma is re-read from cache):
-//   1. load the R inputs (+ residual), fp32 sum in rank order, round to bf16,
-//      add the residual and round again, store residual_out, sum of squares;
-//   2. r = 1 / sqrt(mean + eps); y = (h * r) * (gamma + weight_offset); amax;
-//   3. scale = max(min(amax, scale_ub), 1e-12) / 448; codes of y / scale.
-// The sum of squares and amax are reduced warp -> block -> cluster.  Sources:
+// the row's bf16 norm input h stays in registers between the two passes:
+//   1. load the R inputs, the residual and gamma; fp32 sum in rank order,
+//      round to bf16, add the residual and round again, store residual_out;
+//      accumulate the sum of squares and keep the element with the largest
+//      |h * (gamma + weight_offset)|, the amax candidate;
+//   2. after one reduction of both statistics (warp -> block -> cluster):
+//      r = 1 / sqrt(mean + eps), amax = |y| at the candidate,
+//      scale = max(min(amax, scale_ub), 1e-12) / 448, and the codes of
+//      y = (h * r) * (gamma + weight_offset) times 1 / scale.  Sources:
 // Modular docs `allreduce_rmsnorm_fp8` (one launch, no HBM round trip between
 // the reduction and the norm), b12x PR #283 (fixed-order fp32, round once),
 // TensorRT-LLM PR #19836 (cluster partial-sum exchange and its barrier rules).
 #include <cuda_runtime.h>
+
+#include <atomic>
 
 #include "rrf_device.cuh"
 #include "rrf_internal.h"
@@ -32,14 +36,17 @@ constexpr float kScaleFloor = 1e-12f;
 
 template <int RB, int VPT, bool RES, bool CLUSTER>
 __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const FusedArgs a) {
-    __shared__ float warp_ss[32];
-    __shared__ float warp_amax[32];
-    __shared__ float cl_ss[16];
-    __shared__ float cl_amax[16];
+    __shared__ RowStats warp_stats[32];
+    __shared__ RowStats cluster_stats[16];
 
     // Phase 0 of the cluster barrier: announce that this block has started.
     // Its wait comes just before the first write into a peer's shared memory.
     if (CLUSTER) cluster_arrive_relaxed();
+    // With programmatic dependent launch this block may run ahead of the
+    // previous kernel: wait for it before any global access, then let the
+    // next kernel launch early (it waits for this grid the same way).
+    wait_for_previous_grid();
+    allow_next_grid();
 
     const int tid = threadIdx.x;
     const int T = blockDim.x;
@@ -48,11 +55,15 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
     const int v_begin = (int)rank * a.slice_vecs;
     const int v_end = min(v_begin + a.slice_vecs, a.vecs);
     const int64_t row_base = row * (int64_t)a.vecs;
+    // One vector per thread keeps gamma in registers between the passes;
+    // longer slices re-read it (an L1 hit) to save registers.
+    constexpr bool KEEP_GAMMA = VPT == 1;
 
     uint4 h[VPT];
-    float ss = 0.0f;
+    uint4 g[KEEP_GAMMA ? VPT : 1];
+    RowStats st = stats_empty();
 
-    // ---- pass 1: sum, residual, sum of squares
+    // ---- pass 1: sum, residual, sum of squares, amax candidate
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
         const int v = v_begin + tid + k * T;
@@ -63,6 +74,8 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
                 if (r < a.R) x[r] = ld_once(a.in[r] + row_base + v);
             uint4 res;
             if (RES) res = ld_once_coherent(a.res_in + row_base + v);
+            const uint4 gv = ld_shared_by_all(a.gamma + v);
+            if (KEEP_GAMMA) g[k] = gv;
 
             float acc[8];
             bf16x8_to_f32(x[0], acc);
@@ -78,48 +91,39 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
                 st_once(a.res_out + row_base + v, s);
             }
             h[k] = s;
-            ss += sumsq_bf16x8(s);
+            st.ss += sumsq_bf16x8(s);
+            float hf[8], gf[8];
+            bf16x8_to_f32(s, hf);
+            bf16x8_to_f32(gv, gf);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                stats_offer(st, hf[e], __fadd_rn(gf[e], a.weight_offset));
         }
     }
 
-    float total_ss = block_sum(ss, warp_ss);
+    // ---- one reduction of (sum of squares, amax candidate): block, cluster
+    st = block_stats(st, warp_stats);
     if (CLUSTER) {
         cluster_wait_acquire();  // phase 0 done: every block of the cluster runs
-        total_ss = cluster_combine<false>(total_ss, cl_ss, rank, a.cluster);
+        st = cluster_stats_combine(st, cluster_stats, rank, a.cluster);
     }
-    const float ms = total_ss / a.cols_f;
+    const float ms = st.ss / a.cols_f;
     const float rinv = 1.0f / sqrtf(ms + a.eps);
-
-    // ---- pass 2: y and its absolute maximum
-    float amax = 0.0f;
-#pragma unroll
-    for (int k = 0; k < VPT; ++k) {
-        const int v = v_begin + tid + k * T;
-        if (v < v_end) {
-            float hf[8], gf[8];
-            bf16x8_to_f32(h[k], hf);
-            bf16x8_to_f32(ld_shared_by_all(a.gamma + v), gf);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float y = __fmul_rn(__fmul_rn(hf[e], rinv), __fadd_rn(gf[e], a.weight_offset));
-                amax = fmaxf(amax, fabsf(y));
-            }
-        }
-    }
-    amax = block_max(amax, warp_amax);
-    if (CLUSTER) amax = cluster_combine<true>(amax, cl_amax, rank, a.cluster);
-
+    // The largest |y_j| is reached at the element with the largest |h_j g'_j|
+    // (y = (h * r) * g' is monotone in |h g'| up to rounding); evaluating y
+    // there with the per-element formula gives max_j |y_j|.
+    const float amax = fabsf(__fmul_rn(__fmul_rn(st.h, rinv), st.g));
     const float scale = fmaxf(fminf(amax, a.scale_ub), kScaleFloor) / kE4m3Max;
     const float inv_scale = 1.0f / scale;
 
-    // ---- pass 3: quantise
+    // ---- pass 2: quantise
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
         const int v = v_begin + tid + k * T;
         if (v < v_end) {
             float hf[8], gf[8], qv[8];
             bf16x8_to_f32(h[k], hf);
-            bf16x8_to_f32(ld_shared_by_all(a.gamma + v), gf);
+            bf16x8_to_f32(KEEP_GAMMA ? g[k] : ld_shared_by_all(a.gamma + v), gf);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const float y = __fmul_rn(__fmul_rn(hf[e], rinv), __fadd_rn(gf[e], a.weight_offset));
@@ -140,21 +144,34 @@ cudaError_t launch_one(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
     cfg.blockDim = dim3((unsigned)l.threads, 1, 1);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
+    cfg.attrs = attr;
+    cfg.numAttrs = 0;
+    if (l.pdl) {
+        attr[cfg.numAttrs].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[cfg.numAttrs].val.programmaticStreamSerializationAllowed = 1;
+        ++cfg.numAttrs;
+    }
     if (CLUSTER) {
         if (l.cluster > 8) {
             // Clusters of 16 are outside the portable limit of 8 and must be
-            // enabled per kernel.
-            cudaError_t e = cudaFuncSetAttribute(
-                kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            // enabled once per kernel and device.
+            static std::atomic<uint64_t> enabled_on{0};
+            int dev = 0;
+            cudaError_t e = cudaGetDevice(&dev);
             if (e != cudaSuccess) return e;
+            const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
+            if (bit == 0 || (enabled_on.load(std::memory_order_relaxed) & bit) == 0) {
+                e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+                if (e != cudaSuccess) return e;
+                enabled_on.fetch_or(bit, std::memory_order_relaxed);
+            }
         }
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = (unsigned)l.cluster;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        attr[cfg.numAttrs].id = cudaLaunchAttributeClusterDimension;
+        attr[cfg.numAttrs].val.clusterDim.x = (unsigned)l.cluster;
+        attr[cfg.numAttrs].val.clusterDim.y = 1;
+        attr[cfg.numAttrs].val.clusterDim.z = 1;
+        ++cfg.numAttrs;
     }
     return cudaLaunchKernelEx(&cfg, kernel, a);
 }

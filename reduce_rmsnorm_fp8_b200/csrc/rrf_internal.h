@@ -39,6 +39,7 @@ struct FusedLaunch {
     int cluster;          // blocks per row
     int threads;          // threads per block
     int vecs_per_thread;  // 1, 2, 4 or 8
+    bool pdl;             // launch with programmatic stream serialization
 };
 
 // The fused kernel is compiled for input-count bounds RB in {2, 4, 8, 16}
@@ -58,7 +59,7 @@ constexpr int fused_max_threads(int rb, int vpt) {
 
 // Kernel launchers (one per translation unit).  They return the CUDA error of
 // the launch (cudaSuccess when it was enqueued).
-cudaError_t launch_sum(const SumArgs& a, int sm_count, cudaStream_t stream);
+cudaError_t launch_sum(const SumArgs& a, int sm_count, bool pdl, cudaStream_t stream);
 // One fused launcher per compiled input bound RB (inputs past R are
 // predicated off); launch_fused picks the smallest RB >= R.
 cudaError_t launch_fused_rb2(const FusedArgs& a, int64_t rows, const FusedLaunch& l,

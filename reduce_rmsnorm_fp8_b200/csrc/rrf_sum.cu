@@ -15,6 +15,8 @@ namespace {
 
 template <int RB>
 __global__ void __launch_bounds__(256) sum_kernel(const SumArgs a) {
+    wait_for_previous_grid();  // see rrf_device.cuh: programmatic dependent launch
+    allow_next_grid();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < a.n_vecs; i += stride) {
         uint4 x[RB];
@@ -31,24 +33,32 @@ __global__ void __launch_bounds__(256) sum_kernel(const SumArgs a) {
 }
 
 template <int RB>
-cudaError_t launch_rb(const SumArgs& a, int sm_count, cudaStream_t stream) {
+cudaError_t launch_rb(const SumArgs& a, int sm_count, bool pdl, cudaStream_t stream) {
     constexpr int kThreads = 256;
     // Enough blocks for every vector, capped at a few resident waves; the
     // grid-stride loop covers the rest.
     const int64_t need = (a.n_vecs + kThreads - 1) / kThreads;
     const int64_t cap = (int64_t)sm_count * 8;
     const unsigned blocks = (unsigned)(need < cap ? need : cap);
-    sum_kernel<RB><<<blocks, kThreads, 0, stream>>>(a);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(blocks, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, sum_kernel<RB>, a);
 }
 
 }  // namespace
 
-cudaError_t launch_sum(const SumArgs& a, int sm_count, cudaStream_t stream) {
-    if (a.R <= 2) return launch_rb<2>(a, sm_count, stream);
-    if (a.R <= 4) return launch_rb<4>(a, sm_count, stream);
-    if (a.R <= 8) return launch_rb<8>(a, sm_count, stream);
-    return launch_rb<16>(a, sm_count, stream);
+cudaError_t launch_sum(const SumArgs& a, int sm_count, bool pdl, cudaStream_t stream) {
+    if (a.R <= 2) return launch_rb<2>(a, sm_count, pdl, stream);
+    if (a.R <= 4) return launch_rb<4>(a, sm_count, pdl, stream);
+    if (a.R <= 8) return launch_rb<8>(a, sm_count, pdl, stream);
+    return launch_rb<16>(a, sm_count, pdl, stream);
 }
 
 }  // namespace rrf

@@ -62,14 +62,14 @@ def oracle_sum(case: workloads.Case) -> np.ndarray:
 
 
 def gpu_fused(case: workloads.Case, variant=0, cluster_size=0, block_threads=0,
-              in_place=False) -> dict:
+              in_place=False, flags=0) -> dict:
     import reduce_rmsnorm_fp8_b200 as rrf
     res_in = None if case.residual is None else case.residual.clone()
     res_out = res_in if in_place else None
     q, scales, res_out = rrf.rrf_sum_rmsnorm_fp8_ex(
         case.inputs, case.gamma, case.eps, case.weight_offset, case.scale_ub,
         residual_in=res_in, residual_out=res_out, variant=variant,
-        cluster_size=cluster_size, block_threads=block_threads)
+        cluster_size=cluster_size, block_threads=block_threads, flags=flags)
     torch.cuda.synchronize()
     out = {"q": q.view(torch.uint8).cpu().numpy(), "scales": scales.reshape(-1).cpu().numpy()}
     if res_out is not None:

@@ -163,16 +163,18 @@ def test_sum_validation(rrf):
 # -------------------------------------------------------------- planner ---
 
 @pytest.mark.parametrize("R,rows,cols,sm,want", [
-    (8, 8192, 8192, 148, (1, 256, 4)),   # prefill: one block per row
-    (8, 1, 7168, 148, (16, 64, 1)),      # decode rows 1: cluster of 16
-    (8, 8, 7168, 148, (16, 64, 1)),
+    (8, 8192, 8192, 148, (1, 512, 2)),   # prefill: one block per row
+    (8, 1, 7168, 148, (8, 128, 1)),      # decode: clusters of 8 ...
+    (8, 8, 7168, 148, (8, 128, 1)),
     (8, 32, 7168, 148, (8, 128, 1)),
-    (8, 64, 7168, 148, (4, 224, 1)),
+    (8, 64, 7168, 148, (4, 224, 1)),     # ... of 4 once 4 x rows covers the SMs
     (4, 37, 7168, 148, (4, 224, 1)),
-    (4, 256, 4096, 148, (1, 256, 2)),
+    (4, 16, 4096, 148, (4, 128, 1)),
+    (4, 256, 4096, 148, (1, 512, 1)),
     (2, 4, 256, 148, (1, 32, 1)),        # too short to split
     (4, 1, 8, 148, (1, 32, 1)),
-    (4, 4, 262144, 148, (16, 256, 8)),   # the longest row
+    (4, 4, 262144, 148, (8, 512, 8)),    # the longest row: 8 blocks of 512 x 8 vectors
+    (16, 1, 262144, 148, (16, 512, 4)),  # with 16 inputs: 16 blocks of 512 x 4
 ])
 def test_plan(rrf, R, rows, cols, sm, want):
     assert rrf.rrf_plan_fused(R, rows, cols, sm) == want

@@ -45,9 +45,10 @@ def test_odd_shapes_with_clamped_rows(rrf, rows):
     c = dev_case("odd", rows)
     ref = parity.oracle_fused(c)
     parity.assert_fused_parity(parity.gpu_fused(c), ref, f"odd {rows}")
+    # 1% of the elements are 50x outliers, so every row of 7168 columns holds
+    # some and reaches the clamp: the scale is then exactly fp32(ub / 448)
     ub_scale = np.float32(c.scale_ub) / np.float32(448.0)
-    assert (ref["scales"] == ub_scale).any(), "no row reached the scale_ub clamp"
-    assert (ref["scales"] < ub_scale).any()
+    assert (ref["scales"] == ub_scale).all(), "a row missed the scale_ub clamp"
 
 
 @pytest.mark.parametrize("rows", [16, 32, 48, 64, 96, 128, 256])
@@ -119,6 +120,35 @@ def test_variants_bitwise_identical_bf16(rrf):
             for v, k in ((1, 0), (2, 2), (2, 4), (2, 8), (2, 16))]
     for o in outs[1:]:
         assert np.array_equal(o["res_out"], outs[0]["res_out"])
+
+
+def test_programmatic_dependent_launch_flag(rrf):
+    """Launching without programmatic dependent launch gives the same bits,
+    and a chain of dependent calls (each reading the previous call's residual
+    output) matches the oracle: the wait for the previous grid keeps stream
+    order."""
+    c = dev_case("decode", 64)
+    a = parity.gpu_fused(c)
+    b = parity.gpu_fused(c, flags=rrf.RRF_FLAG_NO_PDL)
+    for k in a:
+        assert np.array_equal(a[k], b[k]), k
+    # chain: residual_out of call i is residual_in of call i + 1
+    res = c.residual.clone()
+    outs = []
+    for i in range(4):
+        nxt = torch.empty_like(res)
+        rrf.rrf_sum_rmsnorm_fp8(c.inputs, c.gamma, c.eps, c.weight_offset, c.scale_ub,
+                                residual_in=res, residual_out=nxt)
+        res = nxt
+        outs.append(nxt)
+    torch.cuda.synchronize()
+    expect = c.residual
+    for i in range(4):
+        step = workloads.Case(c.name, c.R, c.rows, c.cols, c.inputs, expect, c.gamma, c.eps,
+                              c.weight_offset, c.scale_ub)
+        ref = parity.oracle_fused(step)
+        assert np.array_equal(workloads.bits(outs[i]), ref["res_out"]), i
+        expect = outs[i]
 
 
 # --------------------------------------------------------------- edge cases ---
