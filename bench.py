@@ -80,10 +80,14 @@ def barrier(device=None):
             dist.barrier()
 
 
+ROWS_OVERRIDE = None  # --rows: a subset of the workload's row counts
+
+
 def workload_cases(name: str):
     """(rows, residual) of every call one step makes."""
     w = workloads.WORKLOADS[name]
-    return [(rows, w.residual) for rows in w.rows]
+    rows = ROWS_OVERRIDE if ROWS_OVERRIDE else w.rows
+    return [(r, w.residual) for r in rows]
 
 
 def step_bytes(name: str) -> int:
@@ -170,7 +174,7 @@ class DevicePool:
         import torch
         self.name = name
         w = workloads.WORKLOADS[name]
-        rows_list = list(w.rows) if rows_list is None else list(rows_list)
+        rows_list = [r for r, _ in workload_cases(name)] if rows_list is None else rows_list
         self.cases = [workloads.make_case(name, rows, device=device) for rows in rows_list]
         per_set = sum(workloads.fused_bytes(w.R, c.rows, c.cols, c.residual is not None)
                       for c in self.cases)
@@ -392,7 +396,7 @@ def run_rrf(args):
     # small call's sets hot in L2 when it runs alone)
     cases = []
     reps = max(args.steps, 100)
-    for c in pool.cases:
+    for c in ([] if args.no_breakdown else pool.cases):
         cp = DevicePool(name, device, L2_FLUSH_FACTOR * l2, rows_list=[c.rows])
         for i in range(3):
             cp.call(rrf, i, 0)
@@ -402,13 +406,14 @@ def run_rrf(args):
         tc = time_region(lambda _: gi.replay(), 1, device, stream)
         del gi, cp
         b = workloads.fused_bytes(w.R, c.rows, c.cols, c.residual is not None)
-        launch = rrf.rrf_plan_fused(w.R, c.rows, c.cols, props.multi_processor_count)
+        launch = rrf.rrf_plan_fused(w.R, c.rows, c.cols, props.multi_processor_count,
+                                    residual=c.residual is not None, rounds=True)
         cases.append({"rows": c.rows, "us_per_call": round(tc / reps * 1e6, 3),
                       "GB_s": round(b * reps / tc / 1e9, 1),
                       "frac": round(b * reps / tc / 1e9 / peak, 4),
                       "rows_per_s": round(c.rows * reps / tc, 1),
                       "launch": {"cluster": launch[0], "threads": launch[1],
-                                 "vecs_per_thread": launch[2]}})
+                                 "vecs_per_thread": launch[2], "stat_rounds": launch[3]}})
     torch.cuda.empty_cache()
 
     # ---- end to end through host buffers
@@ -457,9 +462,10 @@ def run_rrf(args):
             "io": "bf16 inputs/residual/gamma -> e4m3fn codes + f32 scales + bf16 residual",
             "data": "synthetic (seeded splitmix64 + Box-Muller, drawn on the GPU)",
             "impl": "rrf",
-            "config": {"workload": f"{name}: R={w.R}, cols={w.cols}, rows {list(w.rows)} "
-                                   f"per step, residual={'on' if w.residual else 'off'}",
-                       "R": w.R, "cols": w.cols, "rows": list(w.rows),
+            "config": {"workload": f"{name}: R={w.R}, cols={w.cols}, rows "
+                                   f"{[r for r, _ in workload_cases(name)]} per step, "
+                                   f"residual={'on' if w.residual else 'off'}",
+                       "R": w.R, "cols": w.cols, "rows": [r for r, _ in workload_cases(name)],
                        "bytes_per_step": per_step,
                        "l2": f"inputs larger than L2: {n_sets} rotating buffer sets, "
                              f"{n_sets * per_step >> 20} MiB of traffic > "
@@ -475,7 +481,7 @@ def run_rrf(args):
                          "traffic": None, "peak_kind": f"{peak_kind} hbm_gbs",
                          "kernel": "fused_kernel (rrf_fused.cu)",
                          "avg_launch_us": round(kernel_us, 3),
-                         "bytes_per_launch": round(per_step / len(w.rows))},
+                         "bytes_per_launch": round(per_step / len(workload_cases(name)))},
             "gpu_launches": launches,
             "clocks": clocks.summary(),
             "e2e": e2e,
@@ -543,10 +549,17 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["rrf", "reference"], default="rrf")
     ap.add_argument("--workload", choices=sorted(workloads.WORKLOADS), default="decode")
+    ap.add_argument("--rows", type=int, nargs="*", default=None,
+                    help="only these row counts of the workload (profiling runs)")
+    ap.add_argument("--no-breakdown", action="store_true",
+                    help="skip the per-call breakdown")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
     args = ap.parse_args(argv)
+    global ROWS_OVERRIDE
+    if args.rows:
+        ROWS_OVERRIDE = tuple(args.rows)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":

@@ -189,14 +189,29 @@ __device__ __forceinline__ bool stats_better(float key, float h, float g, const 
 }
 
 // Offer one element to a thread's statistics (the sum of squares is
-// accumulated separately, per 8-element vector).
+// accumulated separately, per 8-element vector).  A thread sees its elements
+// in a fixed order, so a strict comparison (the first of equal keys wins)
+// is deterministic; merges across threads use the total order.
 __device__ __forceinline__ void stats_offer(RowStats& s, float h, float g) {
     const float key = fabsf(__fmul_rn(h, g));
-    if (stats_better(key, h, g, s)) {
+    if (key > s.key) {
         s.key = key;
         s.h = h;
         s.g = g;
     }
+}
+
+// Block-wide maximum of one float, returned to every thread.
+__device__ __forceinline__ float block_max(float v, float* scratch) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, off));
+    if (lane == 0) scratch[warp] = v;
+    __syncthreads();
+    v = lane < nwarps ? scratch[lane] : 0.0f;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, off));
+    return v;
 }
 
 __device__ __forceinline__ RowStats stats_merge(RowStats a, const RowStats& b) {

@@ -40,6 +40,8 @@ struct FusedLaunch {
     int threads;          // threads per block
     int vecs_per_thread;  // 1, 2, 4 or 8
     bool pdl;             // launch with programmatic stream serialization
+    bool two_pass;        // single-block rows: reduce sum of squares and amax in
+                          // two rounds (bandwidth-bound batches)
 };
 
 // The fused kernel is compiled for input-count bounds RB in {2, 4, 8, 16}
@@ -74,6 +76,7 @@ cudaError_t launch_fused(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
                          bool residual, cudaStream_t stream);
 
 // The launch shape the library picks (pure host arithmetic).
-rrf_status plan_fused(int R, int64_t rows, int64_t cols, int sm_count, FusedLaunch* out);
+rrf_status plan_fused(int R, int64_t rows, int64_t cols, int sm_count, bool residual,
+                      FusedLaunch* out);
 
 }  // namespace rrf
