@@ -407,13 +407,13 @@ def run_rrf(args):
         del gi, cp
         b = workloads.fused_bytes(w.R, c.rows, c.cols, c.residual is not None)
         launch = rrf.rrf_plan_fused(w.R, c.rows, c.cols, props.multi_processor_count,
-                                    residual=c.residual is not None, rounds=True)
+                                    residual=c.residual is not None)
         cases.append({"rows": c.rows, "us_per_call": round(tc / reps * 1e6, 3),
                       "GB_s": round(b * reps / tc / 1e9, 1),
                       "frac": round(b * reps / tc / 1e9 / peak, 4),
                       "rows_per_s": round(c.rows * reps / tc, 1),
                       "launch": {"cluster": launch[0], "threads": launch[1],
-                                 "vecs_per_thread": launch[2], "stat_rounds": launch[3]}})
+                                 "vecs_per_thread": launch[2]}})
     torch.cuda.empty_cache()
 
     # ---- end to end through host buffers

@@ -29,10 +29,12 @@
  *   scale = max(min(max_j |y_j|, scale_ub), 1e-12) / 448
  *   q_j   = e4m3fn(y_j / scale), nearest even, saturating at +-448
  *   scales[i] = scale            (dequantise as y ~ e4m3fn_value(q) * scale)
- * The bf16 outputs (s, residual_out) are exact; the sum of squares is a
- * fixed-order fp32 tree, so scales agree with a float64 evaluation to about
- * 1e-6 relative, and a code may differ by one step from the float64 one only
- * where y / scale sits at an e4m3 rounding midpoint.
+ * The bf16 outputs (s, residual_out) are exact.  The kernels reduce the sum
+ * of squares as a fixed-order fp32 tree and take max_j |y_j| as
+ * r * max_j |h_j * (gamma_j + weight_offset)| (the same products rounded in
+ * the other order), so scales agree with the definition to about 1e-6
+ * relative, and a code may differ by one step only where y / scale sits at
+ * an e4m3 rounding midpoint.
  *
  * Conventions for every entry point
  *  - Layout: every 2-D array is contiguous row-major [rows, cols] (row stride
@@ -143,23 +145,14 @@ rrf_status rrf_sum_rmsnorm_fp8(const void* const* inputs, int num_inputs,
 
 /* Launch flags of rrf_sum_rmsnorm_fp8_ex. */
 #define RRF_FLAG_NO_PDL 1     /* launch without programmatic dependent launch     */
-#define RRF_FLAG_ONE_ROUND 2  /* reduce the row statistics in one round          */
-#define RRF_FLAG_TWO_ROUNDS 4 /* ... in two rounds (one-block rows only)         */
 
 /* rrf_sum_rmsnorm_fp8_ex -- rrf_sum_rmsnorm_fp8 with the launch forced, for
  * tests and benchmarks.  variant is one of RRF_VARIANT_*; cluster_size is
  * 2, 4, 8 or 16 for RRF_VARIANT_CLUSTER (0 = automatic) and ignored
  * otherwise; block_threads is a multiple of 32 in [32, 1024] or 0
- * (automatic); flags combines RRF_FLAG_NO_PDL with at most one of
- * RRF_FLAG_ONE_ROUND / RRF_FLAG_TWO_ROUNDS.  Results are bit-identical
+ * (automatic); flags is 0 or RRF_FLAG_NO_PDL.  Results are bit-identical
  * across variants for the bf16 outputs and agree within the stated tolerance
  * for scales and codes.
- *
- * Row statistics: the sum of squares and max |y| meet either in one round
- * (the element with the largest |h * (gamma + weight_offset)| is carried
- * with the sum of squares, and its y, computed once r is known, is max |y|)
- * or in two (sum of squares, then max |y| over every y); the library picks
- * two rounds for one-block rows of large batches only.
  *
  * Programmatic dependent launch: by default every kernel of this library is
  * launched so that it may start while the previous kernel in the stream is
@@ -178,13 +171,13 @@ rrf_status rrf_sum_rmsnorm_fp8_ex(const void* const* inputs, int num_inputs,
 /* rrf_plan_fused -- the launch rrf_sum_rmsnorm_fp8 would use on a GPU with
  * sm_count SMs for a call with (residual != 0) or without a residual,
  * without touching the GPU.  Writes the cluster size (1 = one
- * block per row), the threads per block, the 16-byte vectors each thread
- * holds and the rounds (1 or 2) in which the row statistics are reduced.
+ * block per row), the threads per block and the 16-byte vectors each thread
+ * holds.
  * Returns RRF_ERR_SHAPE / RRF_ERR_RANKS for shapes the library rejects and
  * RRF_ERR_NULL for a null output pointer. */
 rrf_status rrf_plan_fused(int num_inputs, int64_t rows, int64_t cols, int residual,
                           int sm_count, int* cluster_size, int* block_threads,
-                          int* vecs_per_thread, int* stat_rounds);
+                          int* vecs_per_thread);
 
 /* rrf_check_sum_args / rrf_check_fused_args -- the host-side validation of
  * rrf_sum / rrf_sum_rmsnorm_fp8 alone: the status those calls would return

@@ -22,8 +22,6 @@ from ._lib import (  # noqa: F401
     LIB_PATH,
     RRF_MAX_COLS,
     RRF_FLAG_NO_PDL,
-    RRF_FLAG_ONE_ROUND,
-    RRF_FLAG_TWO_ROUNDS,
     RRF_MAX_INPUTS,
     RRF_VARIANT_AUTO,
     RRF_VARIANT_CLUSTER,

@@ -14,8 +14,6 @@ RRF_VARIANT_AUTO = 0
 RRF_VARIANT_ROW = 1
 RRF_VARIANT_CLUSTER = 2
 RRF_FLAG_NO_PDL = 1
-RRF_FLAG_ONE_ROUND = 2
-RRF_FLAG_TWO_ROUNDS = 4
 
 
 class Status(enum.IntEnum):
@@ -64,7 +62,7 @@ lib.rrf_sum_rmsnorm_fp8_ex.restype = _int
 lib.rrf_sum_rmsnorm_fp8_ex.argtypes = _fused_args + [_int, _int, _int, _int, _vp]
 lib.rrf_plan_fused.restype = _int
 lib.rrf_plan_fused.argtypes = [_int, _i64, _i64, _int, _int, ctypes.POINTER(_int),
-                               ctypes.POINTER(_int), ctypes.POINTER(_int), ctypes.POINTER(_int)]
+                               ctypes.POINTER(_int), ctypes.POINTER(_int)]
 lib.rrf_check_sum_args.restype = _int
 lib.rrf_check_sum_args.argtypes = [_ptrs, _int, _i64, _i64, _vp]
 lib.rrf_check_fused_args.restype = _int
@@ -119,15 +117,13 @@ def rrf_check_fused_args(input_ptrs, rows, cols, residual_in, residual_out, gamm
                                     scales_out or None)
 
 
-def rrf_plan_fused(num_inputs: int, rows: int, cols: int, sm_count: int, residual=True,
-                   rounds=False):
+def rrf_plan_fused(num_inputs: int, rows: int, cols: int, sm_count: int, residual=True):
     """The launch the library would pick: (cluster_size, block_threads,
-    vecs_per_thread), plus the statistics rounds (1 or 2) if ``rounds``."""
-    c, t, v, s = _int(), _int(), _int(), _int()
+    vecs_per_thread)."""
+    c, t, v = _int(), _int(), _int()
     _raise_on(lib.rrf_plan_fused(num_inputs, rows, cols, int(bool(residual)), sm_count,
-                                 ctypes.byref(c),
-                                 ctypes.byref(t), ctypes.byref(v), ctypes.byref(s)))
-    return (c.value, t.value, v.value, s.value) if rounds else (c.value, t.value, v.value)
+                                 ctypes.byref(c), ctypes.byref(t), ctypes.byref(v)))
+    return c.value, t.value, v.value
 
 
 def rrf_sum_ptr(input_ptrs, rows, cols, out_ptr, stream=0) -> None:

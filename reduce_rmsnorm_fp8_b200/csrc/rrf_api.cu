@@ -116,18 +116,20 @@ static bool pick_block(int R, int64_t slice, int forced_threads, FusedLaunch* l)
     return false;
 }
 
-// Cost model of the cluster choice, fitted to launch-shape sweeps on B200
-// (1-256 rows of 4096-7168 columns, 4-8 inputs): a block streams its slice at
-// about kSmBytesPerNs, and a cluster round trip (barrier phase + distributed
-// shared-memory exchange) adds about kClusterNs.  Each SM carries at least
-// its share of the whole call's bytes once the grid covers the SMs.
-constexpr double kSmBytesPerNs = 80.0;
-constexpr double kClusterNs = 500.0;
+// The cluster choice, from launch-shape sweeps on B200 (148 SMs; 1-256 rows
+// of 4096-8192 columns, 4-8 inputs, with and without a residual; graph
+// replays over buffer sets larger than L2):
+//   * a batch of at least one row per SM, or rows under ~48 KB of traffic,
+//     runs best with one block per row (a block streams a 37 KB row in about
+//     the time a cluster round trip costs);
+//   * longer rows of smaller batches run best split over clusters of 8
+//     (150 KB rows: 2.53 us at 1 row vs 4.53 us unsplit), or of 4 once 4
+//     blocks per row already give two blocks per SM.
+constexpr double kSplitRowBytes = 48.0 * 1024.0;
 
-static double cluster_cost_ns(int64_t rows, double row_bytes, int c, int sm_count) {
-    const double per_block = row_bytes / c;
-    const double per_sm = (double)rows * row_bytes / sm_count;
-    return (per_block > per_sm ? per_block : per_sm) / kSmBytesPerNs + (c > 1 ? kClusterNs : 0.0);
+static int cluster_choice(int64_t rows, double row_bytes, int sm_count) {
+    if (rows >= sm_count || row_bytes < kSplitRowBytes) return 1;
+    return rows * 4 >= 2 * (int64_t)sm_count ? 4 : 8;
 }
 
 // Launch for a given cluster size (0 = the planner's choice) and block size
@@ -140,28 +142,17 @@ static rrf_status shape_launch(int R, int64_t rows, int64_t cols, int sm_count, 
     const int64_t vecs = cols / 8;
     int c = cluster;
     if (c == 0) {
-        // The cheapest cluster size up to 8 under the cost model (ties go to
-        // the smaller cluster), keeping at least 32 vectors per block; then
-        // split further, up to 16, while one block cannot hold its slice.
+        // The measured choice (see cluster_choice), at least 32 vectors per
+        // block; then split further, up to 16, while one block cannot hold
+        // its slice.
         const double row_bytes = (double)cols * (2.0 * R + (residual ? 4.0 : 0.0) + 1.0);
-        c = 1;
-        double best = cluster_cost_ns(rows, row_bytes, 1, sm_count);
-        for (int k = 2; k <= 8 && vecs / k >= 32; k *= 2) {
-            const double cost = cluster_cost_ns(rows, row_bytes, k, sm_count);
-            if (cost < best) {
-                best = cost;
-                c = k;
-            }
-        }
+        c = cluster_choice(rows, row_bytes, sm_count);
+        while (c > 1 && vecs / c < 32) c /= 2;
         while (c < 16 && !pick_block(R, (vecs + c - 1) / c, forced_threads, out)) c *= 2;
     }
     if (!pick_block(R, (vecs + c - 1) / c, forced_threads, out))
         return cluster == 0 && forced_threads == 0 ? RRF_ERR_SHAPE : RRF_ERR_UNSUPPORTED;
     out->cluster = c;
-    // Statistics in two block rounds for one-block rows once the grid fills
-    // the SMs (measured on B200: 8192 x 8192 prefill rows 215 us in two
-    // rounds vs 221 us in one; latency-bound calls favour one round).
-    out->two_pass = c == 1 && rows >= (int64_t)sm_count;
     out->pdl = true;
     return RRF_OK;
 }
@@ -276,9 +267,7 @@ extern "C" rrf_status rrf_sum_rmsnorm_fp8_ex(const void* const* inputs, int num_
                                          q_out, scales_out);
     if (st != RRF_OK) return st;
     if (variant < RRF_VARIANT_AUTO || variant > RRF_VARIANT_CLUSTER) return RRF_ERR_UNSUPPORTED;
-    if ((flags & ~(RRF_FLAG_NO_PDL | RRF_FLAG_ONE_ROUND | RRF_FLAG_TWO_ROUNDS)) != 0 ||
-        (flags & RRF_FLAG_ONE_ROUND && flags & RRF_FLAG_TWO_ROUNDS))
-        return RRF_ERR_UNSUPPORTED;
+    if ((flags & ~RRF_FLAG_NO_PDL) != 0) return RRF_ERR_UNSUPPORTED;
     if (block_threads != 0 && (block_threads < 32 || block_threads > 1024 || block_threads % 32))
         return RRF_ERR_UNSUPPORTED;
     if (variant == RRF_VARIANT_CLUSTER && cluster_size != 0 && cluster_size != 2 &&
@@ -306,11 +295,6 @@ extern "C" rrf_status rrf_sum_rmsnorm_fp8_ex(const void* const* inputs, int num_
         return st;
     const int64_t vecs = cols / 8;
     l.pdl = (flags & RRF_FLAG_NO_PDL) == 0;
-    if (flags & RRF_FLAG_ONE_ROUND) l.two_pass = false;
-    if (flags & RRF_FLAG_TWO_ROUNDS) {
-        if (l.cluster > 1) return RRF_ERR_UNSUPPORTED;
-        l.two_pass = true;
-    }
 
     FusedArgs a = {};
     for (int r = 0; r < num_inputs; ++r) a.in[r] = static_cast<const uint4*>(inputs[r]);
@@ -346,16 +330,14 @@ extern "C" rrf_status rrf_sum_rmsnorm_fp8(const void* const* inputs, int num_inp
 
 extern "C" rrf_status rrf_plan_fused(int num_inputs, int64_t rows, int64_t cols, int residual,
                                      int sm_count, int* cluster_size, int* block_threads,
-                                     int* vecs_per_thread, int* stat_rounds) {
-    if (!cluster_size || !block_threads || !vecs_per_thread || !stat_rounds)
-        return RRF_ERR_NULL;
+                                     int* vecs_per_thread) {
+    if (!cluster_size || !block_threads || !vecs_per_thread) return RRF_ERR_NULL;
     FusedLaunch l = {};
     rrf_status st = plan_fused(num_inputs, rows, cols, sm_count, residual != 0, &l);
     if (st != RRF_OK) return st;
     *cluster_size = l.cluster;
     *block_threads = l.threads;
     *vecs_per_thread = l.vecs_per_thread;
-    *stat_rounds = l.two_pass ? 2 : 1;
     return RRF_OK;
 }
 

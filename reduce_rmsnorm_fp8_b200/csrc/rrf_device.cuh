@@ -161,91 +161,61 @@ __device__ __forceinline__ void cluster_wait_acquire() {
 }
 
 // --------------------------------------------------------- row statistics --
-// Butterfly (xor) reductions: at every level lane i merges its value with
-// lane i ^ off's; the merge is commutative, so every lane ends with the same
-// bits and the result does not depend on which lane reads it.
+// What a row's norm needs from all of its elements, reduced in one round: the
+// sum of squares of h and the largest |h * g'| (g' = gamma + weight_offset).
+// max_j |y_j| with y_j = (h_j * r) * g'_j is then r * max_j |h_j g'_j| up to
+// the rounding of the two products (a couple of ulps).
 //
-// What a row's norm needs from all of its elements, reduced in one pass: the
-// sum of squares of h and the amax candidate, the element (h, g' = gamma +
-// weight_offset) with the largest key |h * g'|.  The merge keeps the larger
-// candidate under a total order (key, then the bits of h, then of g'), so it
-// is commutative and associative like the sum, and butterfly reductions
-// leave the same bits in every lane.
+// Butterfly (xor) reductions: at every level lane i merges its value with
+// lane i ^ off's; fp32 addition and fmaxf are commutative, so every lane ends
+// with the same bits, whichever lane reads the result.  A reduction over n
+// partials (n a power of two <= 32) runs log2(n) levels on lanes that hold
+// partial lane % n, so every lane of the warp ends with the total.
 
-struct __align__(16) RowStats {  // 16-byte aligned: one v4 store per peer
+struct __align__(8) RowStats {  // 8-byte aligned: one v2 store per peer
     float ss;   // sum of h^2
-    float key;  // |h * g'| of the candidate (-1: no element yet)
-    float h;
-    float g;
+    float key;  // max |h * g'|
 };
 
-__device__ __forceinline__ RowStats stats_empty() { return RowStats{0.0f, -1.0f, 0.0f, 0.0f}; }
+__device__ __forceinline__ RowStats stats_empty() { return RowStats{0.0f, 0.0f}; }
 
-__device__ __forceinline__ bool stats_better(float key, float h, float g, const RowStats& s) {
-    if (key != s.key) return key > s.key;  // NaN keys never win
-    const uint32_t hb = __float_as_uint(h), sh = __float_as_uint(s.h);
-    if (hb != sh) return hb > sh;
-    return __float_as_uint(g) > __float_as_uint(s.g);
-}
-
-// Offer one element to a thread's statistics (the sum of squares is
-// accumulated separately, per 8-element vector).  A thread sees its elements
-// in a fixed order, so a strict comparison (the first of equal keys wins)
-// is deterministic; merges across threads use the total order.
 __device__ __forceinline__ void stats_offer(RowStats& s, float h, float g) {
-    const float key = fabsf(__fmul_rn(h, g));
-    if (key > s.key) {
-        s.key = key;
-        s.h = h;
-        s.g = g;
-    }
-}
-
-// Block-wide maximum of one float, returned to every thread.
-__device__ __forceinline__ float block_max(float v, float* scratch) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, off));
-    if (lane == 0) scratch[warp] = v;
-    __syncthreads();
-    v = lane < nwarps ? scratch[lane] : 0.0f;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, off));
-    return v;
+    s.key = fmaxf(s.key, fabsf(__fmul_rn(h, g)));
 }
 
 __device__ __forceinline__ RowStats stats_merge(RowStats a, const RowStats& b) {
     a.ss = a.ss + b.ss;
-    if (stats_better(b.key, b.h, b.g, a)) {
-        a.key = b.key;
-        a.h = b.h;
-        a.g = b.g;
-    }
+    a.key = fmaxf(a.key, b.key);
     return a;
 }
 
-__device__ __forceinline__ RowStats shfl_xor_stats(const RowStats& s, int off) {
-    RowStats o;
-    o.ss = __shfl_xor_sync(0xFFFFFFFFu, s.ss, off);
-    o.key = __shfl_xor_sync(0xFFFFFFFFu, s.key, off);
-    o.h = __shfl_xor_sync(0xFFFFFFFFu, s.h, off);
-    o.g = __shfl_xor_sync(0xFFFFFFFFu, s.g, off);
-    return o;
+__device__ __forceinline__ RowStats stats_butterfly(RowStats s, int n) {
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        if (off >= n) break;
+        RowStats o;
+        o.ss = __shfl_xor_sync(0xFFFFFFFFu, s.ss, off);
+        o.key = __shfl_xor_sync(0xFFFFFFFFu, s.key, off);
+        s = stats_merge(s, o);
+    }
+    return s;
 }
 
-__device__ __forceinline__ RowStats warp_stats_reduce(RowStats s) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) s = stats_merge(s, shfl_xor_stats(s, off));
-    return s;
+__device__ __forceinline__ int pow2_ceil(int n) {
+    int p = 1;
+    while (p < n) p <<= 1;
+    return p;
 }
 
 // Block-wide statistics, returned to every thread (one __syncthreads).
 __device__ __forceinline__ RowStats block_stats(RowStats s, RowStats* scratch) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-    s = warp_stats_reduce(s);
+    s = stats_butterfly(s, 32);
     if (lane == 0) scratch[warp] = s;
     __syncthreads();
-    return warp_stats_reduce(lane < nwarps ? scratch[lane] : stats_empty());
+    const int n = pow2_ceil(nwarps);
+    const int i = lane & (n - 1);
+    return stats_butterfly(i < nwarps ? scratch[i] : stats_empty(), n);
 }
 
 // Store a block's statistics into slot `rank` of cluster block `peer`.
@@ -254,8 +224,8 @@ __device__ __forceinline__ void st_peer_stats(RowStats* slots, uint32_t rank, ui
     const uint32_t laddr = (uint32_t)__cvta_generic_to_shared(&slots[rank]);
     uint32_t raddr;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(raddr) : "r"(laddr), "r"(peer));
-    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};"
-                 :: "r"(raddr), "f"(s.ss), "f"(s.key), "f"(s.h), "f"(s.g)
+    asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" :: "r"(raddr), "f"(s.ss),
+                 "f"(s.key)
                  : "memory");
 }
 
@@ -263,14 +233,15 @@ __device__ __forceinline__ void st_peer_stats(RowStats* slots, uint32_t rank, ui
 // `rank` of every block of the cluster (threads 0..C-1 write one peer each),
 // one barrier phase publishes the writes, and every block reduces the C
 // slots with the same butterfly, so all blocks hold the same bits.  The
-// caller has completed barrier phase 0 (every block has started).
+// caller has completed barrier phase 0 (every block has started).  C is a
+// power of two.
 __device__ __forceinline__ RowStats cluster_stats_combine(const RowStats& block, RowStats* slots,
                                                           uint32_t rank, int C) {
     if ((int)threadIdx.x < C) st_peer_stats(slots, rank, threadIdx.x, block);
     cluster_arrive_release();
     cluster_wait_acquire();
     const int lane = threadIdx.x & 31;
-    return warp_stats_reduce(lane < C ? slots[lane] : stats_empty());
+    return stats_butterfly(slots[lane & (C - 1)], C);
 }
 
 }  // namespace rrf

@@ -8,10 +8,10 @@
 // the row's bf16 norm input h stays in registers between the two passes:
 //   1. load the R inputs, the residual and gamma; fp32 sum in rank order,
 //      round to bf16, add the residual and round again, store residual_out;
-//      accumulate the sum of squares and keep the element with the largest
-//      |h * (gamma + weight_offset)|, the amax candidate;
+//      accumulate the sum of squares and the largest |h * (gamma +
+//      weight_offset)|;
 //   2. after one reduction of both statistics (warp -> block -> cluster):
-//      r = 1 / sqrt(mean + eps), amax = |y| at the candidate,
+//      r = 1 / sqrt(mean + eps), amax = r * max |h * g'|,
 //      scale = max(min(amax, scale_ub), 1e-12) / 448, and the codes of
 //      y = (h * r) * (gamma + weight_offset) times 1 / scale.  Sources:
 // Modular docs `allreduce_rmsnorm_fp8` (one launch, no HBM round trip between
@@ -34,17 +34,10 @@ namespace {
 constexpr float kE4m3Max = 448.0f;
 constexpr float kScaleFloor = 1e-12f;
 
-// TWO_PASS (blocks of a single-block row only): the statistics are reduced
-// in two rounds, the sum of squares first and then max |y| from y itself.
-// It costs one more block barrier but keeps pass 1 free of the amax-candidate
-// arithmetic, which pays when many rows stream through each SM (prefill);
-// the one-round form wins when the call is latency-bound.
-template <int RB, int VPT, bool RES, bool CLUSTER, bool TWO_PASS>
+template <int RB, int VPT, bool RES, bool CLUSTER>
 __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const FusedArgs a) {
-    static_assert(!(CLUSTER && TWO_PASS), "cluster rows use the one-round statistics");
     __shared__ RowStats warp_stats[32];
     __shared__ RowStats cluster_stats[16];
-    __shared__ float warp_amax[32];
 
     // Phase 0 of the cluster barrier: announce that this block has started.
     // Its wait comes just before the first write into a peer's shared memory.
@@ -64,13 +57,13 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
     const int64_t row_base = row * (int64_t)a.vecs;
     // One vector per thread keeps gamma in registers between the passes;
     // longer slices re-read it (an L1 hit) to save registers.
-    constexpr bool KEEP_GAMMA = VPT == 1 && !TWO_PASS;
+    constexpr bool KEEP_GAMMA = VPT == 1;
 
     uint4 h[VPT];
     uint4 g[KEEP_GAMMA ? VPT : 1];
     RowStats st = stats_empty();
 
-    // ---- pass 1: sum, residual, sum of squares (and the amax candidate)
+    // ---- pass 1: sum, residual, sum of squares, max |h * g'|
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
         const int v = v_begin + tid + k * T;
@@ -81,8 +74,7 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
                 if (r < a.R) x[r] = ld_once(a.in[r] + row_base + v);
             uint4 res;
             if (RES) res = ld_once_coherent(a.res_in + row_base + v);
-            uint4 gv;
-            if (!TWO_PASS) gv = ld_shared_by_all(a.gamma + v);
+            const uint4 gv = ld_shared_by_all(a.gamma + v);
             if (KEEP_GAMMA) g[k] = gv;
 
             float acc[8];
@@ -96,18 +88,17 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
                 bf16x8_to_f32(s, t);
                 add_bf16x8(t, res);
                 s = f32_to_bf16x8(t);
-                st_once(a.res_out + row_base + v, s);
+                // With cluster statistics the store waits for the last pass:
+                // the barrier's release would otherwise wait for it to land.
+                if (!CLUSTER) st_once(a.res_out + row_base + v, s);
             }
             h[k] = s;
             st.ss += sumsq_bf16x8(s);
-            if (!TWO_PASS) {
-                float hf[8], gf[8];
-                bf16x8_to_f32(s, hf);
-                bf16x8_to_f32(gv, gf);
+            float hf[8], gf[8];
+            bf16x8_to_f32(s, hf);
+            bf16x8_to_f32(gv, gf);
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    stats_offer(st, hf[e], __fadd_rn(gf[e], a.weight_offset));
-            }
+            for (int e = 0; e < 8; ++e) stats_offer(st, hf[e], __fadd_rn(gf[e], a.weight_offset));
         }
     }
 
@@ -119,29 +110,9 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
     }
     const float ms = st.ss / a.cols_f;
     const float rinv = 1.0f / sqrtf(ms + a.eps);
-    float amax;
-    if (!TWO_PASS) {
-        // The largest |y_j| is reached at the element with the largest
-        // |h_j g'_j| (y = (h * r) * g' is monotone in |h g'| up to rounding);
-        // evaluating y there with the per-element formula gives max_j |y_j|.
-        amax = fabsf(__fmul_rn(__fmul_rn(st.h, rinv), st.g));
-    } else {
-        amax = 0.0f;
-#pragma unroll
-        for (int k = 0; k < VPT; ++k) {
-            const int v = v_begin + tid + k * T;
-            if (v < v_end) {
-                float hf[8], gf[8];
-                bf16x8_to_f32(h[k], hf);
-                bf16x8_to_f32(ld_shared_by_all(a.gamma + v), gf);
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    amax = fmaxf(amax, fabsf(__fmul_rn(__fmul_rn(hf[e], rinv),
-                                                       __fadd_rn(gf[e], a.weight_offset))));
-            }
-        }
-        amax = block_max(amax, warp_amax);
-    }
+    // max_j |y_j| = max_j |(h_j * r) * g'_j| = r * max_j |h_j * g'_j| up to the
+    // order of the two roundings.
+    const float amax = __fmul_rn(st.key, rinv);
     const float scale = fmaxf(fminf(amax, a.scale_ub), kScaleFloor) / kE4m3Max;
     const float inv_scale = 1.0f / scale;
 
@@ -159,15 +130,16 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
                 qv[e] = __fmul_rn(y, inv_scale);
             }
             st_once(a.q + row_base + v, f32_to_e4m3x8(qv));
+            if (RES && CLUSTER) st_once(a.res_out + row_base + v, h[k]);
         }
     }
     if (tid == 0 && rank == 0) a.scales[row] = scale;
 }
 
-template <int RB, int VPT, bool RES, bool CLUSTER, bool TWO_PASS>
+template <int RB, int VPT, bool RES, bool CLUSTER>
 cudaError_t launch_one(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
                        cudaStream_t stream) {
-    auto kernel = fused_kernel<RB, VPT, RES, CLUSTER, TWO_PASS>;
+    auto kernel = fused_kernel<RB, VPT, RES, CLUSTER>;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(rows * l.cluster), 1, 1);
     cfg.blockDim = dim3((unsigned)l.threads, 1, 1);
@@ -205,14 +177,14 @@ cudaError_t launch_one(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
     return cudaLaunchKernelEx(&cfg, kernel, a);
 }
 
-template <int RB, bool RES, bool CLUSTER, bool TWO_PASS>
+template <int RB, bool RES, bool CLUSTER>
 cudaError_t launch_vpt(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
                        cudaStream_t stream) {
     switch (l.vecs_per_thread) {
-        case 1: return launch_one<RB, 1, RES, CLUSTER, TWO_PASS>(a, rows, l, stream);
-        case 2: return launch_one<RB, 2, RES, CLUSTER, TWO_PASS>(a, rows, l, stream);
-        case 4: return launch_one<RB, 4, RES, CLUSTER, TWO_PASS>(a, rows, l, stream);
-        case 8: return launch_one<RB, 8, RES, CLUSTER, TWO_PASS>(a, rows, l, stream);
+        case 1: return launch_one<RB, 1, RES, CLUSTER>(a, rows, l, stream);
+        case 2: return launch_one<RB, 2, RES, CLUSTER>(a, rows, l, stream);
+        case 4: return launch_one<RB, 4, RES, CLUSTER>(a, rows, l, stream);
+        case 8: return launch_one<RB, 8, RES, CLUSTER>(a, rows, l, stream);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -220,9 +192,8 @@ cudaError_t launch_vpt(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
 template <int RB, bool RES>
 cudaError_t launch_shape(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
                          cudaStream_t stream) {
-    if (l.cluster > 1) return launch_vpt<RB, RES, true, false>(a, rows, l, stream);
-    return l.two_pass ? launch_vpt<RB, RES, false, true>(a, rows, l, stream)
-                      : launch_vpt<RB, RES, false, false>(a, rows, l, stream);
+    return l.cluster > 1 ? launch_vpt<RB, RES, true>(a, rows, l, stream)
+                         : launch_vpt<RB, RES, false>(a, rows, l, stream);
 }
 
 }  // namespace

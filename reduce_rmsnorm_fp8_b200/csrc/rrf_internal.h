@@ -40,8 +40,6 @@ struct FusedLaunch {
     int threads;          // threads per block
     int vecs_per_thread;  // 1, 2, 4 or 8
     bool pdl;             // launch with programmatic stream serialization
-    bool two_pass;        // single-block rows: reduce sum of squares and amax in
-                          // two rounds (bandwidth-bound batches)
 };
 
 // The fused kernel is compiled for input-count bounds RB in {2, 4, 8, 16}

@@ -56,7 +56,7 @@ def test_constants_match_header(rrf):
     expr = re.search(r"#define RRF_MAX_COLS \(([^)]*)\)", text).group(1)
     assert rrf.RRF_MAX_COLS == eval(expr)
     for name in ("RRF_VARIANT_AUTO", "RRF_VARIANT_ROW", "RRF_VARIANT_CLUSTER",
-                 "RRF_FLAG_NO_PDL", "RRF_FLAG_ONE_ROUND", "RRF_FLAG_TWO_ROUNDS"):
+                 "RRF_FLAG_NO_PDL"):
         assert getattr(rrf, name) == int(re.search(rf"#define {name} (\d+)", text).group(1))
     for st in rrf.Status:
         assert re.search(rf"RRF_{st.name} = {int(st)}\b", text), st
@@ -164,30 +164,24 @@ def test_sum_validation(rrf):
 # -------------------------------------------------------------- planner ---
 
 @pytest.mark.parametrize("R,rows,cols,res,want", [
-    (8, 8192, 8192, True, (1, 512, 2, 2)),   # prefill: one block per row, two rounds
-    (8, 1, 7168, True, (8, 128, 1, 1)),      # decode: clusters of 8 ...
-    (8, 8, 7168, True, (8, 128, 1, 1)),
-    (8, 32, 7168, True, (8, 128, 1, 1)),
-    (8, 64, 7168, True, (4, 224, 1, 1)),     # ... of 4 once 4 x rows covers the SMs
-    (4, 37, 7168, True, (4, 224, 1, 1)),
-    (4, 16, 4096, False, (1, 512, 1, 1)),    # 37 KB rows: one block streams it
-    (4, 64, 4096, False, (1, 512, 1, 1)),
-    (4, 256, 4096, False, (1, 512, 1, 2)),
-    (2, 4, 256, False, (1, 32, 1, 1)),       # too short to split
-    (4, 1, 8, False, (1, 32, 1, 1)),
-    (4, 4, 262144, True, (8, 512, 8, 1)),    # the longest row: 8 blocks of 512 x 8
-    (16, 1, 262144, True, (16, 512, 4, 1)),  # with 16 inputs: 16 blocks of 512 x 4
+    (8, 8192, 8192, True, (1, 512, 2)),   # prefill: one block per row
+    (8, 1, 7168, True, (8, 128, 1)),      # decode: clusters of 8
+    (8, 8, 7168, True, (8, 128, 1)),
+    (8, 32, 7168, True, (8, 128, 1)),
+    (8, 64, 7168, True, (8, 128, 1)),
+    (4, 37, 7168, True, (8, 128, 1)),
+    (4, 16, 4096, False, (1, 512, 1)),    # 37 KB rows: one block streams a row
+    (4, 64, 4096, False, (1, 512, 1)),
+    (4, 256, 4096, False, (1, 512, 1)),
+    (2, 4, 256, False, (1, 32, 1)),       # too short to split
+    (4, 1, 8, False, (1, 32, 1)),
+    (4, 4, 262144, True, (8, 512, 8)),    # the longest row: 8 blocks of 512 x 8
+    (16, 1, 262144, True, (16, 512, 4)),  # with 16 inputs: 16 blocks of 512 x 4
 ])
 def test_plan(rrf, R, rows, cols, res, want):
     """The planner's choices for the workloads' shapes: the fastest launch of
     the B200 sweeps that fitted its cost model."""
-    assert rrf.rrf_plan_fused(R, rows, cols, 148, residual=res, rounds=True) == want
-
-
-def test_plan_statistics_rounds(rrf):
-    """Two rounds only for one-block rows once the grid covers the SMs."""
-    assert rrf.rrf_plan_fused(8, 148, 8192, 148, rounds=True)[3] == 2
-    assert rrf.rrf_plan_fused(8, 147, 8192, 148, rounds=True)[3] == 1
+    assert rrf.rrf_plan_fused(R, rows, cols, 148, residual=res) == want
 
 
 def test_plan_covers_every_row(rrf):

@@ -114,24 +114,6 @@ def test_forced_block_sizes(rrf, threads):
         parity.assert_fused_parity(gpu, ref, f"threads={threads} C={cluster}")
 
 
-@pytest.mark.parametrize("name,rows", [("decode", 64), ("odd", 37), ("sweep", 256), ("tiny", 4)])
-@pytest.mark.parametrize("rounds", ["one", "two"])
-def test_statistics_rounds(rrf, name, rows, rounds):
-    """Both ways of reducing the row statistics match the oracle on one-block
-    rows (the one-round amax candidate and the two-round max over y)."""
-    c = dev_case(name, rows)
-    flags = rrf.RRF_FLAG_ONE_ROUND if rounds == "one" else rrf.RRF_FLAG_TWO_ROUNDS
-    gpu = parity.gpu_fused(c, variant=1, flags=flags)
-    parity.assert_fused_parity(gpu, parity.oracle_fused(c), f"{name} {rows} {rounds}")
-
-
-def test_two_rounds_needs_one_block_rows(rrf):
-    c = dev_case("decode", 8)
-    with pytest.raises(rrf.RrfError) as e:
-        parity.gpu_fused(c, variant=2, cluster_size=4, flags=rrf.RRF_FLAG_TWO_ROUNDS)
-    assert e.value.status == rrf.Status.ERR_UNSUPPORTED
-
-
 def test_variants_bitwise_identical_bf16(rrf):
     c = dev_case("decode", 32)
     outs = [parity.gpu_fused(c, variant=v, cluster_size=k)
