@@ -144,15 +144,35 @@ rrf_status rrf_sum_rmsnorm_fp8(const void* const* inputs, int num_inputs,
                                  arrive / wait per thread per barrier phase)      */
 
 /* Launch flags of rrf_sum_rmsnorm_fp8_ex. */
-#define RRF_FLAG_NO_PDL 1     /* launch without programmatic dependent launch     */
+#define RRF_FLAG_NO_PDL 1            /* launch without programmatic dependent launch */
+#define RRF_FLAG_BARRIER_EXCHANGE 2  /* clusters meet at a cluster barrier phase
+                                        instead of the transaction-counted exchange */
+#define RRF_FLAG_DEBUG_STARVE_EXCHANGE 0x100 /* test hook: every block of a cluster
+                                        waits for one value more than its peers
+                                        send, so its bounded wait runs out (about
+                                        2 ms), the kernel sets
+                                        RRF_DEVICE_ERROR_EXCHANGE_TIMEOUT and
+                                        finishes with meaningless codes and
+                                        scales; needs a cluster launch with the
+                                        transaction-counted exchange            */
 
 /* rrf_sum_rmsnorm_fp8_ex -- rrf_sum_rmsnorm_fp8 with the launch forced, for
  * tests and benchmarks.  variant is one of RRF_VARIANT_*; cluster_size is
  * 2, 4, 8 or 16 for RRF_VARIANT_CLUSTER (0 = automatic) and ignored
  * otherwise; block_threads is a multiple of 32 in [32, 1024] or 0
- * (automatic); flags is 0 or RRF_FLAG_NO_PDL.  Results are bit-identical
- * across variants for the bf16 outputs and agree within the stated tolerance
- * for scales and codes.
+ * (automatic); flags combines RRF_FLAG_*.  Results are bit-identical across
+ * variants for the bf16 outputs and agree within the stated tolerance for
+ * scales and codes.
+ *
+ * Cluster exchange: the blocks of a row's cluster share their statistics
+ * either through st.async stores into each other's shared memory, counted
+ * on an mbarrier that each block waits on (the library's choice from 32 rows
+ * on), or at a cluster barrier phase (its choice below 32 rows, and always
+ * with RRF_FLAG_BARRIER_EXCHANGE), following the rules of the TensorRT-LLM
+ * PR #19836 write-up: a completed phase before any remote write, one arrive
+ * and one wait per thread per phase.  The mbarrier waits are bounded (about 2 ms):
+ * a wait that runs out sets RRF_DEVICE_ERROR_EXCHANGE_TIMEOUT in the device
+ * error word (rrf_device_error) instead of hanging the GPU.
  *
  * Programmatic dependent launch: by default every kernel of this library is
  * launched so that it may start while the previous kernel in the stream is
@@ -189,6 +209,17 @@ rrf_status rrf_check_fused_args(const void* const* inputs, int num_inputs, int64
                                 const void* residual_out, const void* gamma, float eps,
                                 float weight_offset, float scale_ub, const void* q_out,
                                 const void* scales_out);
+
+/* Device error bits. */
+#define RRF_DEVICE_ERROR_EXCHANGE_TIMEOUT 1u /* a cluster block's bounded wait for its
+                                               peers' statistics ran out          */
+
+/* rrf_device_error -- the device error word of the current device: the OR
+ * of RRF_DEVICE_ERROR_* bits that kernels of this library have set since it
+ * was last cleared.  Synchronises the device first (all streams), so call it
+ * between steps, not inside stream capture.  clear != 0 resets the word.
+ * Errors: RRF_ERR_NULL, RRF_ERR_CUDA. */
+rrf_status rrf_device_error(unsigned int* flags, int clear);
 
 /* Text for a status code (static storage, never NULL). */
 const char* rrf_status_string(rrf_status status);

@@ -14,6 +14,9 @@ RRF_VARIANT_AUTO = 0
 RRF_VARIANT_ROW = 1
 RRF_VARIANT_CLUSTER = 2
 RRF_FLAG_NO_PDL = 1
+RRF_FLAG_BARRIER_EXCHANGE = 2
+RRF_FLAG_DEBUG_STARVE_EXCHANGE = 0x100
+RRF_DEVICE_ERROR_EXCHANGE_TIMEOUT = 1
 
 
 class Status(enum.IntEnum):
@@ -73,6 +76,8 @@ lib.rrf_last_cuda_error.restype = _int
 lib.rrf_last_cuda_error.argtypes = []
 lib.rrf_debug_fail_next_launch.restype = None
 lib.rrf_debug_fail_next_launch.argtypes = [_int]
+lib.rrf_device_error.restype = _int
+lib.rrf_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), _int]
 lib.rrf_version.restype = ctypes.c_char_p
 lib.rrf_version.argtypes = []
 
@@ -87,6 +92,14 @@ def rrf_last_cuda_error() -> int:
 
 def rrf_debug_fail_next_launch(cuda_error: int) -> None:
     lib.rrf_debug_fail_next_launch(int(cuda_error))
+
+
+def rrf_device_error(clear: bool = False) -> int:
+    """The device error word of the current device (RRF_DEVICE_ERROR_* bits);
+    synchronises the device."""
+    v = ctypes.c_uint(0)
+    _raise_on(lib.rrf_device_error(ctypes.byref(v), int(bool(clear))))
+    return v.value
 
 
 def rrf_version() -> str:

@@ -18,6 +18,12 @@ namespace {
 thread_local int t_last_cuda_error = 0;
 thread_local int t_fail_next_launch = 0;
 
+// The library's device error word: kernels set bits in it (a wait that ran
+// out); rrf_device_error reads and clears it.  Static device memory, one per
+// device; its address is looked up once per device.
+__device__ unsigned int g_device_error;
+std::atomic<uintptr_t> g_device_error_addr[64];
+
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_sm_count[kMaxDevices];
 
@@ -43,6 +49,27 @@ rrf_status current_sm_count(int* sm_count) {
     if (e != cudaSuccess) return cuda_fail(e);
     if (dev >= 0 && dev < kMaxDevices) g_sm_count[dev].store(n, std::memory_order_relaxed);
     *sm_count = n;
+    return RRF_OK;
+}
+
+// Address of the device error word on the current device.
+rrf_status device_error_word(unsigned int** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev >= 0 && dev < kMaxDevices) {
+        uintptr_t cached = g_device_error_addr[dev].load(std::memory_order_relaxed);
+        if (cached != 0) {
+            *out = (unsigned int*)cached;
+            return RRF_OK;
+        }
+    }
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_device_error);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev >= 0 && dev < kMaxDevices)
+        g_device_error_addr[dev].store((uintptr_t)p, std::memory_order_relaxed);
+    *out = (unsigned int*)p;
     return RRF_OK;
 }
 
@@ -154,6 +181,11 @@ static rrf_status shape_launch(int R, int64_t rows, int64_t cols, int sm_count, 
         return cluster == 0 && forced_threads == 0 ? RRF_ERR_SHAPE : RRF_ERR_UNSUPPORTED;
     out->cluster = c;
     out->pdl = true;
+    // Exchange: measured on B200, the cluster barrier phase is quicker for
+    // 1-8 rows (2.50 vs 2.73 us at one 7168-column row), the st.async +
+    // mbarrier exchange from 32 rows on (4.19 vs 4.36 us at 64 rows; 0.3 us
+    // less at 37 and 64 rows of 4 inputs).
+    out->async_exchange = rows >= 32;
     return RRF_OK;
 }
 
@@ -267,7 +299,9 @@ extern "C" rrf_status rrf_sum_rmsnorm_fp8_ex(const void* const* inputs, int num_
                                          q_out, scales_out);
     if (st != RRF_OK) return st;
     if (variant < RRF_VARIANT_AUTO || variant > RRF_VARIANT_CLUSTER) return RRF_ERR_UNSUPPORTED;
-    if ((flags & ~RRF_FLAG_NO_PDL) != 0) return RRF_ERR_UNSUPPORTED;
+    if ((flags & ~(RRF_FLAG_NO_PDL | RRF_FLAG_BARRIER_EXCHANGE | RRF_FLAG_DEBUG_STARVE_EXCHANGE)) !=
+        0)
+        return RRF_ERR_UNSUPPORTED;
     if (block_threads != 0 && (block_threads < 32 || block_threads > 1024 || block_threads % 32))
         return RRF_ERR_UNSUPPORTED;
     if (variant == RRF_VARIANT_CLUSTER && cluster_size != 0 && cluster_size != 2 &&
@@ -295,6 +329,11 @@ extern "C" rrf_status rrf_sum_rmsnorm_fp8_ex(const void* const* inputs, int num_
         return st;
     const int64_t vecs = cols / 8;
     l.pdl = (flags & RRF_FLAG_NO_PDL) == 0;
+    if (flags & RRF_FLAG_BARRIER_EXCHANGE) l.async_exchange = false;
+    if ((flags & RRF_FLAG_DEBUG_STARVE_EXCHANGE) && !(l.cluster > 1 && l.async_exchange))
+        return RRF_ERR_UNSUPPORTED;
+    unsigned int* err = nullptr;
+    if ((st = device_error_word(&err)) != RRF_OK) return st;
 
     FusedArgs a = {};
     for (int r = 0; r < num_inputs; ++r) a.in[r] = static_cast<const uint4*>(inputs[r]);
@@ -311,6 +350,8 @@ extern "C" rrf_status rrf_sum_rmsnorm_fp8_ex(const void* const* inputs, int num_
     a.eps = eps;
     a.weight_offset = weight_offset;
     a.scale_ub = scale_ub;
+    a.err = err;
+    a.starve = (flags & RRF_FLAG_DEBUG_STARVE_EXCHANGE) ? 1 : 0;
     cudaError_t e;
     if (!take_injected_failure(&e))
         e = launch_fused(a, rows, l, residual_in != nullptr, (cudaStream_t)stream);
@@ -357,6 +398,18 @@ extern "C" const char* rrf_status_string(rrf_status status) {
 }
 
 extern "C" int rrf_last_cuda_error(void) { return t_last_cuda_error; }
+
+extern "C" rrf_status rrf_device_error(unsigned int* flags, int clear) {
+    if (flags == nullptr) return RRF_ERR_NULL;
+    unsigned int* word = nullptr;
+    rrf_status st = device_error_word(&word);
+    if (st != RRF_OK) return st;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaMemcpy(flags, word, sizeof *flags, cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && clear) e = cudaMemset(word, 0, sizeof *word);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    return e == cudaSuccess ? RRF_OK : cuda_fail(e);
+}
 
 extern "C" void rrf_debug_fail_next_launch(int cuda_error) { t_fail_next_launch = cuda_error; }
 

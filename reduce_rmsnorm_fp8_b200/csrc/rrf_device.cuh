@@ -9,6 +9,12 @@
 
 namespace rrf {
 
+// Device error bits (the library's device error word; see rrf_device_error).
+constexpr unsigned int kDeviceErrorExchangeTimeout = 1u;
+// Bound on a wait for the cluster's statistics: far above the microsecond a
+// healthy exchange takes, far below anything that would look like a hang.
+constexpr unsigned long long kExchangeWaitLimitNs = 2000000ull;  // 2 ms
+
 // ------------------------------------------------------------------ memory --
 
 // Streamed 16-byte load of data read exactly once: read-only path, no L1
@@ -160,6 +166,81 @@ __device__ __forceinline__ void cluster_wait_acquire() {
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// ------------------------------------------ transaction-counted exchange --
+// The other way for a cluster's blocks to meet: each block pushes its value
+// into every peer's shared memory with st.async, which counts the bytes on
+// the peer's mbarrier, and waits on its own mbarrier until all C values have
+// landed.  No thread waits for the cluster's other threads, and no release
+// fence waits for this thread's global stores.  Every wait is bounded in
+// time: a wait that runs out sets a bit in the library's device error word
+// and the kernel finishes without the missing values instead of hanging.
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t arrivals) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(smem_u32(bar)), "r"(arrivals)
+                 : "memory");
+}
+
+// Make this thread's mbarrier initialisations visible to the cluster (for the
+// peers' st.async) before the next cluster barrier arrival.
+__device__ __forceinline__ void fence_mbar_init_cluster() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// One arrival that also announces `bytes` of incoming transactions.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                 :: "r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait until phase `parity` of `bar` completes, for at most limit_ns
+// nanoseconds; returns false if the wait ran out.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  uint64_t limit_ns) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait_cluster(bar, parity))
+        if (global_timer_ns() - t0 > limit_ns) return false;
+    return true;
+}
+
+// Store two floats into shared-memory word pair `local` of cluster block
+// `peer` and count 8 bytes on that block's mbarrier `bar` (same offsets in
+// every block).
+__device__ __forceinline__ void st_async_peer_f32x2(void* local, uint64_t* bar, uint32_t peer,
+                                                    float x, float y) {
+    uint32_t raddr, rbar;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(raddr) : "r"(smem_u32(local)),
+                 "r"(peer));
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rbar) : "r"(smem_u32(bar)),
+                 "r"(peer));
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];"
+                 :: "r"(raddr), "f"(x), "f"(y), "r"(rbar)
+                 : "memory");
+}
+
 // --------------------------------------------------------- row statistics --
 // What a row's norm needs from all of its elements, reduced in one round: the
 // sum of squares of h and the largest |h * g'| (g' = gamma + weight_offset).
@@ -227,6 +308,23 @@ __device__ __forceinline__ void st_peer_stats(RowStats* slots, uint32_t rank, ui
     asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" :: "r"(raddr), "f"(s.ss),
                  "f"(s.key)
                  : "memory");
+}
+
+// Cluster-wide statistics through the transaction-counted exchange: thread p
+// (p < C) pushes the block's statistics into slot `rank` of block p; every
+// thread then waits (bounded) for this block's C slots and reduces them with
+// the same butterfly in every block.  The caller has completed barrier phase
+// 0 (every block has started and initialised `bar`, which expects C * 8
+// bytes).  On a timeout the error bit is set and the slots are used as they
+// are.
+__device__ __forceinline__ RowStats cluster_stats_async(const RowStats& block, RowStats* slots,
+                                                        uint64_t* bar, uint32_t rank, int C,
+                                                        unsigned int* err) {
+    if ((int)threadIdx.x < C)
+        st_async_peer_f32x2(&slots[rank], bar, threadIdx.x, block.ss, block.key);
+    if (!mbar_wait_bounded(bar, 0, kExchangeWaitLimitNs)) atomicOr(err, kDeviceErrorExchangeTimeout);
+    const int lane = threadIdx.x & 31;
+    return stats_butterfly(slots[lane & (C - 1)], C);
 }
 
 // Cluster-wide statistics: block `rank` writes its statistics into slot

@@ -34,14 +34,28 @@ namespace {
 constexpr float kE4m3Max = 448.0f;
 constexpr float kScaleFloor = 1e-12f;
 
-template <int RB, int VPT, bool RES, bool CLUSTER>
+// ASYNC (cluster rows only): the blocks of a cluster meet through the
+// transaction-counted exchange (st.async into the peers' shared memory,
+// bounded mbarrier waits) instead of a cluster barrier phase.
+template <int RB, int VPT, bool RES, bool CLUSTER, bool ASYNC>
 __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const FusedArgs a) {
+    static_assert(CLUSTER || !ASYNC, "the exchange is between the blocks of a cluster");
     __shared__ RowStats warp_stats[32];
     __shared__ RowStats cluster_stats[16];
+    __shared__ uint64_t exchange_bar;
 
-    // Phase 0 of the cluster barrier: announce that this block has started.
-    // Its wait comes just before the first write into a peer's shared memory.
-    if (CLUSTER) cluster_arrive_relaxed();
+    if (CLUSTER) {
+        if (ASYNC && threadIdx.x == 0) {
+            // one arrival (this one) and C blocks' 8 bytes of statistics
+            mbar_init(&exchange_bar, 1);
+            mbar_arrive_expect_tx(&exchange_bar, 8u * (uint32_t)(a.cluster + a.starve));
+            fence_mbar_init_cluster();
+        }
+        // Phase 0 of the cluster barrier: this block has started (and set up
+        // its exchange barrier).  Its wait comes just before the first write
+        // into a peer's shared memory.
+        cluster_arrive_relaxed();
+    }
     // With programmatic dependent launch this block may run ahead of the
     // previous kernel: wait for it before any global access, then let the
     // next kernel launch early (it waits for this grid the same way).
@@ -88,9 +102,10 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
                 bf16x8_to_f32(s, t);
                 add_bf16x8(t, res);
                 s = f32_to_bf16x8(t);
-                // With cluster statistics the store waits for the last pass:
-                // the barrier's release would otherwise wait for it to land.
-                if (!CLUSTER) st_once(a.res_out + row_base + v, s);
+                // With the cluster barrier exchange the store waits for the
+                // last pass: the barrier's release would otherwise wait for it
+                // to land.
+                if (!CLUSTER || ASYNC) st_once(a.res_out + row_base + v, s);
             }
             h[k] = s;
             st.ss += sumsq_bf16x8(s);
@@ -106,7 +121,8 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
     st = block_stats(st, warp_stats);
     if (CLUSTER) {
         cluster_wait_acquire();  // phase 0 done: every block of the cluster runs
-        st = cluster_stats_combine(st, cluster_stats, rank, a.cluster);
+        st = ASYNC ? cluster_stats_async(st, cluster_stats, &exchange_bar, rank, a.cluster, a.err)
+                   : cluster_stats_combine(st, cluster_stats, rank, a.cluster);
     }
     const float ms = st.ss / a.cols_f;
     const float rinv = 1.0f / sqrtf(ms + a.eps);
@@ -130,16 +146,16 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
                 qv[e] = __fmul_rn(y, inv_scale);
             }
             st_once(a.q + row_base + v, f32_to_e4m3x8(qv));
-            if (RES && CLUSTER) st_once(a.res_out + row_base + v, h[k]);
+            if (RES && CLUSTER && !ASYNC) st_once(a.res_out + row_base + v, h[k]);
         }
     }
     if (tid == 0 && rank == 0) a.scales[row] = scale;
 }
 
-template <int RB, int VPT, bool RES, bool CLUSTER>
+template <int RB, int VPT, bool RES, bool CLUSTER, bool ASYNC>
 cudaError_t launch_one(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
                        cudaStream_t stream) {
-    auto kernel = fused_kernel<RB, VPT, RES, CLUSTER>;
+    auto kernel = fused_kernel<RB, VPT, RES, CLUSTER, ASYNC>;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(rows * l.cluster), 1, 1);
     cfg.blockDim = dim3((unsigned)l.threads, 1, 1);
@@ -177,14 +193,14 @@ cudaError_t launch_one(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
     return cudaLaunchKernelEx(&cfg, kernel, a);
 }
 
-template <int RB, bool RES, bool CLUSTER>
+template <int RB, bool RES, bool CLUSTER, bool ASYNC>
 cudaError_t launch_vpt(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
                        cudaStream_t stream) {
     switch (l.vecs_per_thread) {
-        case 1: return launch_one<RB, 1, RES, CLUSTER>(a, rows, l, stream);
-        case 2: return launch_one<RB, 2, RES, CLUSTER>(a, rows, l, stream);
-        case 4: return launch_one<RB, 4, RES, CLUSTER>(a, rows, l, stream);
-        case 8: return launch_one<RB, 8, RES, CLUSTER>(a, rows, l, stream);
+        case 1: return launch_one<RB, 1, RES, CLUSTER, ASYNC>(a, rows, l, stream);
+        case 2: return launch_one<RB, 2, RES, CLUSTER, ASYNC>(a, rows, l, stream);
+        case 4: return launch_one<RB, 4, RES, CLUSTER, ASYNC>(a, rows, l, stream);
+        case 8: return launch_one<RB, 8, RES, CLUSTER, ASYNC>(a, rows, l, stream);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -192,8 +208,9 @@ cudaError_t launch_vpt(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
 template <int RB, bool RES>
 cudaError_t launch_shape(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
                          cudaStream_t stream) {
-    return l.cluster > 1 ? launch_vpt<RB, RES, true>(a, rows, l, stream)
-                         : launch_vpt<RB, RES, false>(a, rows, l, stream);
+    if (l.cluster == 1) return launch_vpt<RB, RES, false, false>(a, rows, l, stream);
+    return l.async_exchange ? launch_vpt<RB, RES, true, true>(a, rows, l, stream)
+                            : launch_vpt<RB, RES, true, false>(a, rows, l, stream);
 }
 
 }  // namespace

@@ -33,6 +33,8 @@ struct FusedArgs {
     float eps;
     float weight_offset;
     float scale_ub;
+    unsigned int* err;     // the library's device error word
+    int starve;            // test hook: exchange values a block waits for beyond C
 };
 
 struct FusedLaunch {
@@ -40,6 +42,7 @@ struct FusedLaunch {
     int threads;          // threads per block
     int vecs_per_thread;  // 1, 2, 4 or 8
     bool pdl;             // launch with programmatic stream serialization
+    bool async_exchange;  // clusters meet through st.async + mbarrier waits
 };
 
 // The fused kernel is compiled for input-count bounds RB in {2, 4, 8, 16}

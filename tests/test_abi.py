@@ -56,8 +56,10 @@ def test_constants_match_header(rrf):
     expr = re.search(r"#define RRF_MAX_COLS \(([^)]*)\)", text).group(1)
     assert rrf.RRF_MAX_COLS == eval(expr)
     for name in ("RRF_VARIANT_AUTO", "RRF_VARIANT_ROW", "RRF_VARIANT_CLUSTER",
-                 "RRF_FLAG_NO_PDL"):
-        assert getattr(rrf, name) == int(re.search(rf"#define {name} (\d+)", text).group(1))
+                 "RRF_FLAG_NO_PDL", "RRF_FLAG_BARRIER_EXCHANGE",
+                 "RRF_FLAG_DEBUG_STARVE_EXCHANGE", "RRF_DEVICE_ERROR_EXCHANGE_TIMEOUT"):
+        assert getattr(rrf, name) == int(
+            re.search(rf"#define {name} (0x[0-9a-fA-F]+|\d+)u?", text).group(1), 0)
     for st in rrf.Status:
         assert re.search(rf"RRF_{st.name} = {int(st)}\b", text), st
 
@@ -202,12 +204,18 @@ def test_plan_rejects(rrf):
         rrf.rrf_plan_fused(0, 1, 64, 148)
 
 
-def test_import_fails_loudly_without_library(tmp_path):
-    """Without librrf.so the package refuses to import: there is no fallback."""
+def test_use_fails_loudly_without_library(tmp_path):
+    """Without librrf.so the first use of the package raises ImportError:
+    there is no fallback.  (The bare import succeeds so that the build step
+    can run from a fresh checkout.)"""
     import shutil
     pkg = tmp_path / "reduce_rmsnorm_fp8_b200"
     shutil.copytree(os.path.join(ROOT, "reduce_rmsnorm_fp8_b200"), pkg,
                     ignore=shutil.ignore_patterns("*.so", "_build", "__pycache__"))
-    r = subprocess.run([sys.executable, "-c", "import reduce_rmsnorm_fp8_b200"],
-                       cwd=tmp_path, capture_output=True, text=True)
-    assert r.returncode != 0 and "librrf.so is missing" in r.stderr
+    code = ("import reduce_rmsnorm_fp8_b200 as r, reduce_rmsnorm_fp8_b200.build as b\n"
+            "assert b.LIB.endswith('librrf.so')\n"
+            "r.rrf_sum\n")
+    res = subprocess.run([sys.executable, "-c", code], cwd=tmp_path, capture_output=True,
+                         text=True)
+    assert res.returncode != 0 and "librrf.so is missing" in res.stderr
+    assert "ImportError" in res.stderr

@@ -114,6 +114,38 @@ def test_forced_block_sizes(rrf, threads):
         parity.assert_fused_parity(gpu, ref, f"threads={threads} C={cluster}")
 
 
+@pytest.mark.parametrize("cluster", [2, 4, 8, 16])
+@pytest.mark.parametrize("exchange", ["async", "barrier"])
+def test_cluster_exchanges(rrf, cluster, exchange):
+    """Both ways for a cluster's blocks to share their statistics -- st.async
+    into the peers' shared memory counted on mbarriers, or a cluster barrier
+    phase -- match the oracle, and leave the device error word clear."""
+    rrf.rrf_device_error(clear=True)
+    flags = 0 if exchange == "async" else rrf.RRF_FLAG_BARRIER_EXCHANGE
+    for name, rows in (("decode", 8), ("odd", 37)):
+        c = dev_case(name, rows)
+        gpu = parity.gpu_fused(c, variant=2, cluster_size=cluster, flags=flags)
+        parity.assert_fused_parity(gpu, parity.oracle_fused(c), f"{name} C={cluster} {exchange}")
+    assert rrf.rrf_device_error() == 0
+
+
+def test_starved_exchange_times_out_and_reports(rrf):
+    """Failure detection without a GPU fault: every block waits for one value
+    that no peer sends; the bounded wait runs out (about 2 ms), the kernel
+    sets the timeout bit and finishes; the context stays usable and the next
+    call is correct."""
+    c = dev_case("decode", 8)
+    rrf.rrf_device_error(clear=True)
+    parity.gpu_fused(c, variant=2, cluster_size=8, flags=rrf.RRF_FLAG_DEBUG_STARVE_EXCHANGE)
+    assert rrf.rrf_device_error(clear=True) & rrf.RRF_DEVICE_ERROR_EXCHANGE_TIMEOUT
+    assert rrf.rrf_device_error() == 0
+    parity.assert_fused_parity(parity.gpu_fused(c), parity.oracle_fused(c), "after timeout")
+    assert rrf.rrf_device_error() == 0
+    with pytest.raises(rrf.RrfError) as e:  # the hook needs a clustered launch
+        parity.gpu_fused(c, variant=1, flags=rrf.RRF_FLAG_DEBUG_STARVE_EXCHANGE)
+    assert e.value.status == rrf.Status.ERR_UNSUPPORTED
+
+
 def test_variants_bitwise_identical_bf16(rrf):
     c = dev_case("decode", 32)
     outs = [parity.gpu_fused(c, variant=v, cluster_size=k)
