@@ -138,7 +138,7 @@ class ClockSampler:
                 self.reasons |= int(n.nvmlDeviceGetCurrentClocksEventReasons(self._h))
             except Exception:
                 break
-            time.sleep(0.002)
+            time.sleep(0.0005)
 
     def __enter__(self):
         if self._nvml is not None:
@@ -545,7 +545,7 @@ def run_reference(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description="fused sum + RMSNorm + FP8 benchmark")
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["rrf", "reference"], default="rrf")
     ap.add_argument("--workload", choices=sorted(workloads.WORKLOADS), default="decode")
