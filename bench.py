@@ -30,7 +30,6 @@ import math
 import os
 import statistics
 import sys
-import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -96,6 +95,37 @@ def step_bytes(name: str) -> int:
                workload_cases(name))
 
 
+def kernel_source_hash() -> str:
+    """sha256 of the fused kernel's sources: a recorded ncu traffic figure is
+    valid only for the kernel it was taken from."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("rrf_fused.cu", "rrf_device.cuh"):
+        with open(os.path.join(ROOT, "reduce_rmsnorm_fp8_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum)
+    of the fused kernel on `workload`, from profiles/fused_kernel_traffic.txt,
+    or None if none is recorded for the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "fused_kernel_traffic.txt")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    src = None
+    for line in lines:
+        if line.startswith("kernel_source_sha256:"):
+            src = line.split(":", 1)[1].strip()
+        elif line and not line.startswith("#") and src == kernel_source_hash():
+            parts = line.split()
+            if parts[0] == workload:
+                return int(parts[1])
+    return None
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -107,8 +137,9 @@ def measured_peaks():
 
 
 class ClockSampler:
-    """Polls NVML for the SM clock and the active clock-event reasons of one
-    GPU on a background thread while the timed region runs."""
+    """Samples NVML for the SM clock and the active clock-event reasons of one
+    GPU; time_region calls sample() until the timed region's end event has
+    completed."""
 
     REASONS = {  # NVML clocks-event-reason bits
         0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
@@ -119,37 +150,39 @@ class ClockSampler:
     def __init__(self, index: int):
         self.samples, self.reasons = [], 0
         self.max_mhz = None
-        self._stop = threading.Event()
-        self._thread = None
         try:
             import pynvml
             pynvml.nvmlInit()
             self._nvml = pynvml
-            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self._h = None
+            try:  # the NVML handle of the CUDA device, by PCI bus id
+                import torch
+                pr = torch.cuda.get_device_properties(index)
+                bus = "%08X:%02X:%02X.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
         except Exception:
             self._nvml = None
 
-    def _run(self):
+    def sample(self):
+        """Take one sample now (called from the timing loop while the device
+        works through the timed region)."""
+        if self._nvml is None:
+            return
         n = self._nvml
-        while not self._stop.is_set():
-            try:
-                self.samples.append(n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM))
-                self.reasons |= int(n.nvmlDeviceGetCurrentClocksEventReasons(self._h))
-            except Exception:
-                break
-            time.sleep(0.0005)
+        try:
+            self.samples.append(n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM))
+            self.reasons |= int(n.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+        except Exception:
+            pass
 
     def __enter__(self):
-        if self._nvml is not None:
-            self._thread = threading.Thread(target=self._run, daemon=True)
-            self._thread.start()
         return self
 
     def __exit__(self, *exc):
-        if self._thread is not None:
-            self._stop.set()
-            self._thread.join()
+        return False
 
     def summary(self):
         if self._nvml is None:
@@ -210,9 +243,10 @@ class DevicePool:
         return sum(self.call(rrf, k, i) for i in range(len(self.cases)))
 
 
-def time_region(fn, k_steps: int, device, stream):
+def time_region(fn, k_steps: int, device, stream, clocks=None):
     """Device time of k_steps calls of fn(i), CUDA events on `stream`, with a
-    barrier and a synchronisation on both sides; max over ranks, seconds."""
+    barrier and a synchronisation on both sides; max over ranks, seconds.
+    With a ClockSampler, samples the clocks until the end event completes."""
     import torch
     barrier(device)
     torch.cuda.synchronize(device)
@@ -222,6 +256,9 @@ def time_region(fn, k_steps: int, device, stream):
     for i in range(k_steps):
         fn(i)
     end.record(stream)
+    if clocks is not None:
+        while not end.query():
+            clocks.sample()
     torch.cuda.synchronize(device)
     barrier(device)
     return max_over_ranks(start.elapsed_time(end) / 1e3, device)
@@ -383,8 +420,8 @@ def run_rrf(args):
                                     args.steps, device)
     graph.replay()  # one untimed replay: graph upload
     torch.cuda.synchronize(device)
-    with ClockSampler(device.index) as clocks:
-        t = time_region(lambda _: graph.replay(), 1, device, stream)
+    clocks = ClockSampler(device.index)
+    t = time_region(lambda _: graph.replay(), 1, device, stream, clocks)
     del graph
     n_sets = pool.n_sets
     per_step = step_bytes(name)
@@ -478,7 +515,12 @@ def run_rrf(args):
             "cases": cases,
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
-                         "traffic": None, "peak_kind": f"{peak_kind} hbm_gbs",
+                         "traffic": recorded_traffic(name),
+                         "traffic_note": "ncu dram__bytes_read.sum + dram__bytes_write.sum "
+                                         "per launch, averaged over the step's launches "
+                                         "(profiles/fused_kernel_traffic.txt); null when "
+                                         "not recorded for these kernel sources",
+                         "peak_kind": f"{peak_kind} hbm_gbs",
                          "kernel": "fused_kernel (rrf_fused.cu)",
                          "avg_launch_us": round(kernel_us, 3),
                          "bytes_per_launch": round(per_step / len(workload_cases(name)))},

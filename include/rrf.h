@@ -153,8 +153,8 @@ rrf_status rrf_sum_rmsnorm_fp8(const void* const* inputs, int num_inputs,
                                         2 ms), the kernel sets
                                         RRF_DEVICE_ERROR_EXCHANGE_TIMEOUT and
                                         finishes with meaningless codes and
-                                        scales; needs a cluster launch with the
-                                        transaction-counted exchange            */
+                                        scales; selects the transaction-counted
+                                        exchange and needs a cluster launch     */
 
 /* rrf_sum_rmsnorm_fp8_ex -- rrf_sum_rmsnorm_fp8 with the launch forced, for
  * tests and benchmarks.  variant is one of RRF_VARIANT_*; cluster_size is

@@ -330,8 +330,11 @@ extern "C" rrf_status rrf_sum_rmsnorm_fp8_ex(const void* const* inputs, int num_
     const int64_t vecs = cols / 8;
     l.pdl = (flags & RRF_FLAG_NO_PDL) == 0;
     if (flags & RRF_FLAG_BARRIER_EXCHANGE) l.async_exchange = false;
-    if ((flags & RRF_FLAG_DEBUG_STARVE_EXCHANGE) && !(l.cluster > 1 && l.async_exchange))
-        return RRF_ERR_UNSUPPORTED;
+    if (flags & RRF_FLAG_DEBUG_STARVE_EXCHANGE) {
+        // the hook exercises the bounded wait of the transaction-counted exchange
+        if (l.cluster == 1 || (flags & RRF_FLAG_BARRIER_EXCHANGE)) return RRF_ERR_UNSUPPORTED;
+        l.async_exchange = true;
+    }
     unsigned int* err = nullptr;
     if ((st = device_error_word(&err)) != RRF_OK) return st;
 

@@ -141,9 +141,12 @@ def test_starved_exchange_times_out_and_reports(rrf):
     assert rrf.rrf_device_error() == 0
     parity.assert_fused_parity(parity.gpu_fused(c), parity.oracle_fused(c), "after timeout")
     assert rrf.rrf_device_error() == 0
-    with pytest.raises(rrf.RrfError) as e:  # the hook needs a clustered launch
-        parity.gpu_fused(c, variant=1, flags=rrf.RRF_FLAG_DEBUG_STARVE_EXCHANGE)
-    assert e.value.status == rrf.Status.ERR_UNSUPPORTED
+    for variant, flags in ((1, 0), (2, rrf.RRF_FLAG_BARRIER_EXCHANGE)):
+        # the hook needs a clustered launch with the transaction-counted exchange
+        with pytest.raises(rrf.RrfError) as e:
+            parity.gpu_fused(c, variant=variant, cluster_size=0 if variant == 1 else 8,
+                             flags=flags | rrf.RRF_FLAG_DEBUG_STARVE_EXCHANGE)
+        assert e.value.status == rrf.Status.ERR_UNSUPPORTED
 
 
 def test_variants_bitwise_identical_bf16(rrf):
