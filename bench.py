@@ -136,10 +136,30 @@ def measured_peaks():
         return 6650.0, "fallback"
 
 
+_CLOCK_POLL = r"""
+import sys, time
+import pynvml
+pynvml.nvmlInit()
+bus = sys.argv[1]
+try:
+    h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+except Exception:
+    h = pynvml.nvmlDeviceGetHandleByIndex(int(sys.argv[2]))
+print("max", pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM), flush=True)
+while True:
+    t = time.monotonic()
+    c = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+    r = int(pynvml.nvmlDeviceGetCurrentClocksEventReasons(h))
+    print(f"{t:.6f} {c} {r}", flush=True)
+    time.sleep(0.0002)
+"""
+
+
 class ClockSampler:
-    """Samples NVML for the SM clock and the active clock-event reasons of one
-    GPU; time_region calls sample() until the timed region's end event has
-    completed."""
+    """Samples the SM clock and the active clock-event reasons of one GPU
+    through NVML in a separate process (so no Python lock of this process
+    can starve it), every ~0.2 ms; summary() keeps the samples taken between
+    mark_start() and mark_end(), the timed region."""
 
     REASONS = {  # NVML clocks-event-reason bits
         0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
@@ -148,50 +168,56 @@ class ClockSampler:
         0x100: "display_clock_setting"}
 
     def __init__(self, index: int):
-        self.samples, self.reasons = [], 0
-        self.max_mhz = None
+        import subprocess
+        import tempfile
+        import torch
+        self.t0 = self.t1 = None
+        bus = ""
         try:
-            import pynvml
-            pynvml.nvmlInit()
-            self._nvml = pynvml
-            self._h = None
-            try:  # the NVML handle of the CUDA device, by PCI bus id
-                import torch
-                pr = torch.cuda.get_device_properties(index)
-                bus = "%08X:%02X:%02X.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
-                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
-            except Exception:
-                self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
-        except Exception:
-            self._nvml = None
-
-    def sample(self):
-        """Take one sample now (called from the timing loop while the device
-        works through the timed region)."""
-        if self._nvml is None:
-            return
-        n = self._nvml
-        try:
-            self.samples.append(n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM))
-            self.reasons |= int(n.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+            pr = torch.cuda.get_device_properties(index)
+            bus = "%08X:%02X:%02X.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
         except Exception:
             pass
+        self._out = tempfile.TemporaryFile(mode="w+")
+        try:
+            self._proc = subprocess.Popen([sys.executable, "-c", _CLOCK_POLL, bus, str(index)],
+                                          stdout=self._out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self._proc = None
+        # wait (briefly) for the poller's first sample
+        deadline = time.monotonic() + 20.0
+        while self._proc is not None and time.monotonic() < deadline:
+            self._out.seek(0)
+            if self._out.read().count("\n") >= 2 or self._proc.poll() is not None:
+                break
+            time.sleep(0.05)
 
-    def __enter__(self):
-        return self
+    def mark_start(self):
+        self.t0 = time.monotonic()
 
-    def __exit__(self, *exc):
-        return False
+    def mark_end(self):
+        self.t1 = time.monotonic()
 
     def summary(self):
-        if self._nvml is None:
+        if self._proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
-        reasons = [name for bit, name in self.REASONS.items()
-                   if self.reasons & bit and name != "gpu_idle"]
-        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
-                "sm_max_mhz": self.max_mhz, "reasons": reasons,
-                "samples": len(self.samples)}
+        self._proc.terminate()
+        self._proc.wait()
+        self._out.seek(0)
+        max_mhz, samples, reasons = None, [], 0
+        for line in self._out.read().splitlines():
+            parts = line.split()
+            if parts and parts[0] == "max":
+                max_mhz = int(parts[1])
+            elif len(parts) == 3:
+                t, c, r = float(parts[0]), int(parts[1]), int(parts[2])
+                if self.t0 is not None and self.t0 <= t <= self.t1:
+                    samples.append(c)
+                    reasons |= r
+        names = [n for bit, n in self.REASONS.items() if reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(samples) if samples else None,
+                "sm_max_mhz": max_mhz, "reasons": names, "samples": len(samples),
+                "source": "NVML, sampled every ~0.2 ms during the timed region"}
 
 
 # -------------------------------------------------------------- CUDA arm ---
@@ -203,7 +229,7 @@ class DevicePool:
     tensor kind.  n_sets is chosen so the sets together exceed min_bytes of
     algorithmic traffic, so a set is cold in L2 when its turn comes again."""
 
-    def __init__(self, name: str, device, min_bytes: int, rows_list=None):
+    def __init__(self, name: str, device, min_bytes: int, rows_list=None, with_sum=False):
         import torch
         self.name = name
         w = workloads.WORKLOADS[name]
@@ -224,6 +250,8 @@ class DevicePool:
             if c.residual is not None:
                 b["residual"] = c.residual.unsqueeze(0).expand(shape).contiguous()
                 b["res_out"] = torch.empty(shape, dtype=torch.bfloat16, device=device)
+            if with_sum:
+                b["sum_out"] = torch.empty(shape, dtype=torch.bfloat16, device=device)
             self.big.append(b)
         self.eps, self.wo, self.ub = w.eps, w.weight_offset, w.scale_ub
 
@@ -237,6 +265,12 @@ class DevicePool:
             q_out=b["q"][s], scales_out=b["scales"][s])
         return 1
 
+    def call_sum(self, rrf, k: int, i: int) -> int:
+        """Enqueue the sum-only call i on set k mod n_sets; returns 1."""
+        b, s = self.big[i], k % self.n_sets
+        rrf.rrf_sum([x[s] for x in b["inputs"]], out=b["sum_out"][s])
+        return 1
+
     def run_step(self, rrf, k: int) -> int:
         """Enqueue step k: every call of the workload on set k mod n_sets;
         returns the number of kernels launched."""
@@ -246,20 +280,21 @@ class DevicePool:
 def time_region(fn, k_steps: int, device, stream, clocks=None):
     """Device time of k_steps calls of fn(i), CUDA events on `stream`, with a
     barrier and a synchronisation on both sides; max over ranks, seconds.
-    With a ClockSampler, samples the clocks until the end event completes."""
+    A ClockSampler is told when the region starts and ends."""
     import torch
     barrier(device)
     torch.cuda.synchronize(device)
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
+    if clocks is not None:
+        clocks.mark_start()
     start.record(stream)
     for i in range(k_steps):
         fn(i)
     end.record(stream)
-    if clocks is not None:
-        while not end.query():
-            clocks.sample()
     torch.cuda.synchronize(device)
+    if clocks is not None:
+        clocks.mark_end()
     barrier(device)
     return max_over_ranks(start.elapsed_time(end) / 1e3, device)
 
@@ -418,10 +453,11 @@ def run_rrf(args):
     torch.cuda.synchronize(device)
     graph, launches = capture_steps(lambda i: pool.run_step(rrf, args.warmup + i),
                                     args.steps, device)
+    clocks = ClockSampler(device.index)
     graph.replay()  # one untimed replay: graph upload
     torch.cuda.synchronize(device)
-    clocks = ClockSampler(device.index)
     t = time_region(lambda _: graph.replay(), 1, device, stream, clocks)
+    clock_info = clocks.summary()  # stops the poller
     del graph
     n_sets = pool.n_sets
     per_step = step_bytes(name)
@@ -485,6 +521,32 @@ def run_rrf(args):
         del pf
         torch.cuda.empty_cache()
 
+    # ---- the sum-only / fused sweep over the b12x payload sizes (R=4, 4096 cols)
+    sweep = None
+    if not args.no_secondary and name != "sweep":
+        sweep = []
+        ws = workloads.WORKLOADS["sweep"]
+        for rows in ws.rows:
+            sp = DevicePool("sweep", device, L2_FLUSH_FACTOR * l2, rows_list=[rows],
+                            with_sum=True)
+            rec = {"rows": rows, "payload_KiB": rows * ws.cols * 2 // 1024}
+            for op, fn, nbytes in (
+                    ("sum", sp.call_sum, workloads.sum_bytes(ws.R, rows, ws.cols)),
+                    ("fused", sp.call, workloads.fused_bytes(ws.R, rows, ws.cols, False))):
+                for i in range(3):
+                    fn(rrf, i, 0)
+                reps = 200
+                gs, _ = capture_steps(lambda k, fn=fn: fn(rrf, 3 + k, 0), reps, device)
+                gs.replay()
+                torch.cuda.synchronize(device)
+                ts = time_region(lambda _: gs.replay(), 1, device, stream)
+                del gs
+                rec[f"{op}_us"] = round(ts / reps * 1e6, 3)
+                rec[f"{op}_GB_s"] = round(nbytes * reps / ts / 1e9, 1)
+            sweep.append(rec)
+            del sp
+        torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(name)
@@ -525,9 +587,10 @@ def run_rrf(args):
                          "avg_launch_us": round(kernel_us, 3),
                          "bytes_per_launch": round(per_step / len(workload_cases(name)))},
             "gpu_launches": launches,
-            "clocks": clocks.summary(),
+            "clocks": clock_info,
             "e2e": e2e,
             "prefill": secondary,
+            "sweep": sweep,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
