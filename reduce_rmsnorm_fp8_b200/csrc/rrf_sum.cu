@@ -34,15 +34,21 @@ __global__ void __launch_bounds__(256) sum_kernel(const SumArgs a) {
 
 template <int RB>
 cudaError_t launch_rb(const SumArgs& a, int sm_count, bool pdl, cudaStream_t stream) {
-    constexpr int kThreads = 256;
-    // Enough blocks for every vector, capped at a few resident waves; the
-    // grid-stride loop covers the rest.
-    const int64_t need = (a.n_vecs + kThreads - 1) / kThreads;
+    // Large calls: 256-thread blocks, at most 8 resident waves' worth, the
+    // grid-stride loop covers the rest.  Small calls (fewer vectors than 256
+    // per SM) are latency-bound: smaller blocks spread them over every SM.
+    int threads = 256;
+    if (a.n_vecs < (int64_t)sm_count * 256) {
+        const int64_t per_sm = (a.n_vecs + sm_count - 1) / sm_count;
+        threads = (int)((per_sm + 31) / 32 * 32);
+        if (threads < 32) threads = 32;
+    }
+    const int64_t need = (a.n_vecs + threads - 1) / threads;
     const int64_t cap = (int64_t)sm_count * 8;
     const unsigned blocks = (unsigned)(need < cap ? need : cap);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(blocks, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.blockDim = dim3((unsigned)threads, 1, 1);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
