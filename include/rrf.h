@@ -165,12 +165,11 @@ rrf_status rrf_sum_rmsnorm_fp8(const void* const* inputs, int num_inputs,
  * scales and codes.
  *
  * Cluster exchange: the blocks of a row's cluster share their statistics
- * either through st.async stores into each other's shared memory, counted
- * on an mbarrier that each block waits on (the library's choice from 32 rows
- * on), or at a cluster barrier phase (its choice below 32 rows, and always
- * with RRF_FLAG_BARRIER_EXCHANGE), following the rules of the TensorRT-LLM
- * PR #19836 write-up: a completed phase before any remote write, one arrive
- * and one wait per thread per phase.  The mbarrier waits are bounded (about 2 ms):
+ * through st.async stores into each other's shared memory, counted on an
+ * mbarrier that each block waits on (the default), or, with
+ * RRF_FLAG_BARRIER_EXCHANGE, at a cluster barrier phase following the rules
+ * of the TensorRT-LLM PR #19836 write-up: a completed phase before any
+ * remote write, one arrive and one wait per thread per phase.  The mbarrier waits are bounded (about 2 ms):
  * a wait that runs out sets RRF_DEVICE_ERROR_EXCHANGE_TIMEOUT in the device
  * error word (rrf_device_error) instead of hanging the GPU.
  *

@@ -181,11 +181,11 @@ static rrf_status shape_launch(int R, int64_t rows, int64_t cols, int sm_count, 
         return cluster == 0 && forced_threads == 0 ? RRF_ERR_SHAPE : RRF_ERR_UNSUPPORTED;
     out->cluster = c;
     out->pdl = true;
-    // Exchange: measured on B200, the cluster barrier phase is quicker for
-    // 1-8 rows (2.50 vs 2.73 us at one 7168-column row), the st.async +
-    // mbarrier exchange from 32 rows on (4.19 vs 4.36 us at 64 rows; 0.3 us
-    // less at 37 and 64 rows of 4 inputs).
-    out->async_exchange = rows >= 32;
+    // Exchange: measured on B200 (residual stores after the exchange in both
+    // forms), the st.async + mbarrier exchange ties the cluster barrier at 1-8
+    // rows and beats it from 32 rows on (4.03 vs 4.39 us at 64 rows of 7168
+    // columns; 0.3 us less at 37 and 64 rows of 4 inputs).
+    out->async_exchange = true;
     return RRF_OK;
 }
 

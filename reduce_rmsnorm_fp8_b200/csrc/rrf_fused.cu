@@ -102,10 +102,12 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
                 bf16x8_to_f32(s, t);
                 add_bf16x8(t, res);
                 s = f32_to_bf16x8(t);
-                // With the cluster barrier exchange the store waits for the
-                // last pass: the barrier's release would otherwise wait for it
-                // to land.
-                if (!CLUSTER || ASYNC) st_once(a.res_out + row_base + v, s);
+                // Cluster rows store the residual in the last pass, after the
+                // exchange: with the barrier exchange its release would
+                // otherwise wait for the store to land, and with either
+                // exchange the early stores measured slower on B200 (0.1-0.2 us
+                // at 32-64 rows of 7168 columns).
+                if (!CLUSTER) st_once(a.res_out + row_base + v, s);
             }
             h[k] = s;
             st.ss += sumsq_bf16x8(s);
@@ -146,7 +148,7 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
                 qv[e] = __fmul_rn(y, inv_scale);
             }
             st_once(a.q + row_base + v, f32_to_e4m3x8(qv));
-            if (RES && CLUSTER && !ASYNC) st_once(a.res_out + row_base + v, h[k]);
+            if (RES && CLUSTER) st_once(a.res_out + row_base + v, h[k]);
         }
     }
     if (tid == 0 && rank == 0) a.scales[row] = scale;
