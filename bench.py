@@ -332,11 +332,13 @@ class _Arena:
 
 
 def e2e_measure(rrf, name: str, k_steps: int, warmup: int, device, stream):
-    """The same metric through the public call with HOST buffers: every step
+    """The same metric through the public call with HOST buffers.  Every step
     copies its inputs (all calls' inputs, residuals and gammas, packed in one
     pinned host buffer) to the device in one copy, runs the calls, and reads
-    all results (codes, scales, residual outputs) back in one copy; both
-    copies are inside the timed region."""
+    all results (codes, scales, residual outputs) back to pinned host memory
+    in one copy; all copies are inside the timed region.  Steps are
+    double-buffered over three streams (H2D, compute, D2H), as a serving loop
+    would run them, so one step's copies overlap the neighbouring steps'."""
     import torch
     w = workloads.WORKLOADS[name]
     cases = [workloads.make_case(name, rows) for rows, _ in workload_cases(name)]
@@ -352,10 +354,12 @@ def e2e_measure(rrf, name: str, k_steps: int, warmup: int, device, stream):
                 "res_out": outs.add(shape, torch.bfloat16) if c.residual is not None else None}
         slots.append(slot)
     h_in = torch.empty(ins.size, dtype=torch.uint8).pin_memory()
-    h_out = torch.empty(outs.size, dtype=torch.uint8).pin_memory()
-    d_in = torch.empty(ins.size, dtype=torch.uint8, device=device)
-    d_out = torch.empty(outs.size, dtype=torch.uint8, device=device)
-    hv, dv, ov = ins.views(h_in), ins.views(d_in), outs.views(d_out)
+    h_out = [torch.empty(outs.size, dtype=torch.uint8).pin_memory() for _ in range(2)]
+    d_in = [torch.empty(ins.size, dtype=torch.uint8, device=device) for _ in range(2)]
+    d_out = [torch.empty(outs.size, dtype=torch.uint8, device=device) for _ in range(2)]
+    hv = ins.views(h_in)
+    dv = [ins.views(b) for b in d_in]
+    ov = [outs.views(b) for b in d_out]
     for c, slot in zip(cases, slots):  # the host data of the step
         for x, i in zip(c.inputs, slot["inputs"]):
             hv[i].copy_(x)
@@ -365,21 +369,51 @@ def e2e_measure(rrf, name: str, k_steps: int, warmup: int, device, stream):
     h2d = sum(n for _, n, _, _ in ins.items)
     d2h = sum(n for _, n, _, _ in outs.items)
 
-    def step(_):
-        d_in.copy_(h_in, non_blocking=True)
-        for slot in slots:
-            rrf.rrf_sum_rmsnorm_fp8(
-                [dv[i] for i in slot["inputs"]], dv[slot["gamma"]], w.eps, w.weight_offset,
-                w.scale_ub,
-                residual_in=None if slot["residual"] is None else dv[slot["residual"]],
-                residual_out=None if slot["res_out"] is None else ov[slot["res_out"]],
-                q_out=ov[slot["q"]].view(torch.float8_e4m3fn), scales_out=ov[slot["scales"]])
-        h_out.copy_(d_out, non_blocking=True)
+    s_in, s_cmp, s_out = (torch.cuda.Stream(device) for _ in range(3))
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
+    copied_out = [torch.cuda.Event() for _ in range(2)]
+    used = [False, False]
 
-    with torch.cuda.stream(stream):
-        for i in range(warmup):
-            step(i)
-        t = time_region(step, k_steps, device, stream)
+    def step(k):
+        b = k % 2
+        with torch.cuda.stream(s_in):
+            if used[b]:
+                s_in.wait_event(computed[b])  # slot b's inputs are free again
+            d_in[b].copy_(h_in, non_blocking=True)
+            in_ready[b].record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(in_ready[b])
+            if used[b]:
+                s_cmp.wait_event(copied_out[b])  # slot b's outputs were read
+            for slot in slots:
+                rrf.rrf_sum_rmsnorm_fp8(
+                    [dv[b][i] for i in slot["inputs"]], dv[b][slot["gamma"]], w.eps,
+                    w.weight_offset, w.scale_ub,
+                    residual_in=None if slot["residual"] is None else dv[b][slot["residual"]],
+                    residual_out=None if slot["res_out"] is None else ov[b][slot["res_out"]],
+                    q_out=ov[b][slot["q"]].view(torch.float8_e4m3fn),
+                    scales_out=ov[b][slot["scales"]])
+            computed[b].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(computed[b])
+            h_out[b].copy_(d_out[b], non_blocking=True)
+            copied_out[b].record(s_out)
+        used[b] = True
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(s_in)
+    for i in range(k_steps):
+        step(warmup + i)
+    s_in.wait_stream(s_out)
+    end.record(s_in)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    t = max_over_ranks(start.elapsed_time(end) / 1e3, device)
     return t, h2d, d2h
 
 
@@ -497,7 +531,9 @@ def run_rrf(args):
         ke = max(10, args.steps // 10)
         e2e = {"value": round(world * per_step * ke / te / 1e9, 3), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": round(te / ke * 1e3, 4)}
+               "ms_per_step": round(te / ke * 1e3, 4),
+               "how": "rrf_sum_rmsnorm_fp8 on device copies of pinned host buffers: one "
+                      "H2D and one D2H copy per step, double-buffered over three streams"}
 
     # ---- secondary: the prefill-size call, where the kernel can reach HBM speed
     secondary = None
@@ -519,6 +555,47 @@ def run_rrf(args):
                      "GB_s": round(bp * kp / tp / 1e9, 1),
                      "frac": round(bp * kp / tp / 1e9 / peak, 4), "calls": kp}
         del pf
+        torch.cuda.empty_cache()
+        # the sum alone at the same size (8 inputs of 8192 x 8192)
+        pf = DevicePool("prefill", device, 2 * l2, with_sum=True)
+        for i in range(3):
+            pf.call_sum(rrf, i, 0)
+        gs, _ = capture_steps(lambda k: pf.call_sum(rrf, k, 0), kp, device)
+        gs.replay()
+        torch.cuda.synchronize(device)
+        ts = time_region(lambda _: gs.replay(), 1, device, stream)
+        del gs, pf
+        torch.cuda.empty_cache()
+        bs = workloads.sum_bytes(8, 8192, 8192)
+        secondary.update({"sum_us_per_call": round(ts / kp * 1e6, 2),
+                          "sum_GB_s": round(bs * kp / ts / 1e9, 1),
+                          "sum_frac": round(bs * kp / ts / 1e9 / peak, 4)})
+
+    # ---- the other configurations, each call alone over its own pool
+    others = None
+    if not args.no_secondary:
+        others = {}
+        for oname in ("tiny", "odd"):
+            if oname == name:
+                continue
+            recs = []
+            wo = workloads.WORKLOADS[oname]
+            for rows in wo.rows:
+                op = DevicePool(oname, device, L2_FLUSH_FACTOR * l2, rows_list=[rows])
+                for i in range(3):
+                    op.call(rrf, i, 0)
+                reps = 200
+                go, _ = capture_steps(lambda k: op.call(rrf, 3 + k, 0), reps, device)
+                go.replay()
+                torch.cuda.synchronize(device)
+                to = time_region(lambda _: go.replay(), 1, device, stream)
+                del go, op
+                bo = workloads.fused_bytes(wo.R, rows, wo.cols, wo.residual)
+                recs.append({"rows": rows, "us_per_call": round(to / reps * 1e6, 3),
+                             "GB_s": round(bo * reps / to / 1e9, 1),
+                             "frac": round(bo * reps / to / 1e9 / peak, 4)})
+            others[oname] = {"R": wo.R, "cols": wo.cols, "residual": wo.residual,
+                             "calls": recs}
         torch.cuda.empty_cache()
 
     # ---- the sum-only / fused sweep over the b12x payload sizes (R=4, 4096 cols)
@@ -591,6 +668,7 @@ def run_rrf(args):
             "e2e": e2e,
             "prefill": secondary,
             "sweep": sweep,
+            "other_configs": others,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

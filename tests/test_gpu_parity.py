@@ -186,6 +186,41 @@ def test_programmatic_dependent_launch_flag(rrf):
         expect = outs[i]
 
 
+# --------------------------------------------------------------- random shapes ---
+
+def test_random_shapes_and_launches(rrf):
+    """60 seeded random problems: R, rows, cols (multiples of 8, many ragged),
+    residual on/off (in place or not), scalars, and a random forced launch
+    (automatic, one block per row, or a cluster of 2-16 with either
+    exchange, a random block size); every one matches the oracle."""
+    rng = np.random.default_rng(2026)
+    checked = 0
+    for _ in range(60):
+        R = int(rng.integers(1, 17))
+        rows = int(rng.choice([1, 2, 3, 5, 7, 16, 33, 64, 150, 300]))
+        cols = int(8 * rng.integers(1, 1200))
+        c = dev_case("decode", rows, cols=cols, R=R, residual=bool(rng.integers(0, 2)))
+        c.eps = float(rng.choice([0.0, 1e-6, 1e-5, 0.1]))
+        c.weight_offset = float(rng.choice([0.0, 1.0, -0.5]))
+        c.scale_ub = float(rng.choice([1200.0, 8.0, 0.5, float("inf")]))
+        variant = int(rng.choice([0, 1, 2]))
+        cluster = int(rng.choice([2, 4, 8, 16])) if variant == 2 else 0
+        threads = int(rng.choice([0, 0, 32, 64, 128, 256, 512]))
+        flags = int(rng.choice([0, rrf.RRF_FLAG_BARRIER_EXCHANGE, rrf.RRF_FLAG_NO_PDL]))
+        in_place = c.residual is not None and bool(rng.integers(0, 2))
+        try:
+            gpu = parity.gpu_fused(c, variant=variant, cluster_size=cluster,
+                                   block_threads=threads, flags=flags, in_place=in_place)
+        except rrf.RrfError as e:
+            assert e.status == rrf.Status.ERR_UNSUPPORTED  # the forced launch cannot cover it
+            continue
+        parity.assert_fused_parity(gpu, parity.oracle_fused(c),
+                                   f"R={R} {rows}x{cols} v{variant} C{cluster} T{threads} f{flags}")
+        checked += 1
+    assert checked >= 40
+    assert rrf.rrf_device_error() == 0
+
+
 # --------------------------------------------------------------- edge cases ---
 
 @pytest.mark.parametrize("cols", [8, 16, 264, 2880, 7176, 8200, 16384, 131072, 262144])
