@@ -34,9 +34,10 @@ __global__ void __launch_bounds__(256) sum_kernel(const SumArgs a) {
 
 template <int RB>
 cudaError_t launch_rb(const SumArgs& a, int sm_count, bool pdl, cudaStream_t stream) {
-    // Large calls: 256-thread blocks, at most 8 resident waves' worth, the
-    // grid-stride loop covers the rest.  Small calls (fewer vectors than 256
-    // per SM) are latency-bound: smaller blocks spread them over every SM.
+    // Large calls: 256-thread blocks, 16 per SM (two full residencies; a
+    // streaming probe of the same 8:1 read/write mix peaked there on B200),
+    // the grid-stride loop covers the rest.  Small calls (fewer vectors than
+    // 256 per SM) are latency-bound: smaller blocks spread them over every SM.
     int threads = 256;
     if (a.n_vecs < (int64_t)sm_count * 256) {
         const int64_t per_sm = (a.n_vecs + sm_count - 1) / sm_count;
@@ -44,7 +45,7 @@ cudaError_t launch_rb(const SumArgs& a, int sm_count, bool pdl, cudaStream_t str
         if (threads < 32) threads = 32;
     }
     const int64_t need = (a.n_vecs + threads - 1) / threads;
-    const int64_t cap = (int64_t)sm_count * 8;
+    const int64_t cap = (int64_t)sm_count * 16;
     const unsigned blocks = (unsigned)(need < cap ? need : cap);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(blocks, 1, 1);
