@@ -187,6 +187,73 @@ rrf_status rrf_sum_rmsnorm_fp8_ex(const void* const* inputs, int num_inputs,
                                   float* scales_out, int variant, int cluster_size,
                                   int block_threads, int flags, rrf_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * The sharded form: a row's hidden dimension split across devices.
+ *
+ * Tenstorrent rmsnorm_2d.py (RMSNorm2D, decode_forward / prefill_forward)
+ * splits the norm into a pre-all-gather pass that computes per-device row
+ * statistics, an all-gather of those statistics, and a post-all-gather pass
+ * that normalises each device's shard.  Here the statistics are the pair
+ * (sum_j h_j^2, max_j |h_j * (gamma_j + weight_offset)|) over the shard's
+ * columns, so the one exchange also carries what the FP8 scale needs: the
+ * post pass combines the pairs of every shard in a fixed order (every shard
+ * derives the same scale) and quantises its own columns.  The exchange itself
+ * (an all-gather of rows * 8 bytes per shard) is the caller's (e.g. NCCL);
+ * the result equals rrf_sum_rmsnorm_fp8 on the whole rows up to the order of
+ * the fp32 sum of squares.
+ * ---------------------------------------------------------------------- */
+
+/* At most this many shards of a row. */
+#define RRF_MAX_SHARDS 64
+
+/* rrf_sum_rmsnorm_fp8_pre -- phase 1 on this device's column shard
+ * [rows, cols]: the bf16 sum of the inputs, the optional residual (written
+ * back), and per row the shard statistics.
+ * inputs, num_inputs, rows, cols, residual_in, residual_out  as for
+ *               rrf_sum_rmsnorm_fp8 (cols: this shard's columns)
+ * h_out         bf16 [rows, cols], 16-byte aligned: receives the norm input
+ *               h when there is no residual; must be NULL with a residual
+ *               (residual_out then holds h)
+ * gamma         bf16 [cols], this shard's gamma
+ * weight_offset added to gamma (as for rrf_sum_rmsnorm_fp8)
+ * stats_out     float [rows][2], 8-byte aligned: (sum of h^2, max |h * g'|)
+ * Errors: RRF_ERR_NULL, RRF_ERR_RANKS, RRF_ERR_SHAPE, RRF_ERR_ALIGN,
+ *         RRF_ERR_ALIAS, RRF_ERR_VALUE, RRF_ERR_CUDA. */
+rrf_status rrf_sum_rmsnorm_fp8_pre(const void* const* inputs, int num_inputs, int64_t rows,
+                                   int64_t cols, const void* residual_in, void* residual_out,
+                                   void* h_out, const void* gamma, float weight_offset,
+                                   float* stats_out, rrf_stream_t stream);
+
+/* rrf_rmsnorm_fp8_post -- phase 2 on this device's column shard: codes and
+ * scales from the norm input and the gathered statistics of all shards.
+ * h             bf16 [rows, cols], this shard's norm input (phase 1's h_out
+ *               or residual_out), 16-byte aligned
+ * stats         float [shards][rows][2]: every shard's phase-1 statistics,
+ *               in shard order, 8-byte aligned
+ * shards        1..RRF_MAX_SHARDS
+ * total_cols    the whole row's columns (the mean's divisor), >= cols
+ * gamma         bf16 [cols], this shard's gamma
+ * eps, weight_offset, scale_ub  as for rrf_sum_rmsnorm_fp8
+ * q_out         fp8 e4m3fn codes [rows, cols], 16-byte aligned
+ * scales_out    float [rows] or NULL (every shard derives the same scales,
+ *               so one of them may write them)
+ * Errors: RRF_ERR_NULL, RRF_ERR_SHAPE, RRF_ERR_ALIGN, RRF_ERR_ALIAS,
+ *         RRF_ERR_VALUE, RRF_ERR_CUDA. */
+rrf_status rrf_rmsnorm_fp8_post(const void* h, int64_t rows, int64_t cols, const float* stats,
+                                int shards, int64_t total_cols, const void* gamma, float eps,
+                                float weight_offset, float scale_ub, void* q_out,
+                                float* scales_out, rrf_stream_t stream);
+
+/* The host validation of the two phases alone (no GPU needed). */
+rrf_status rrf_check_pre_args(const void* const* inputs, int num_inputs, int64_t rows,
+                              int64_t cols, const void* residual_in, const void* residual_out,
+                              const void* h_out, const void* gamma, float weight_offset,
+                              const void* stats_out);
+rrf_status rrf_check_post_args(const void* h, int64_t rows, int64_t cols, const float* stats,
+                               int shards, int64_t total_cols, const void* gamma, float eps,
+                               float weight_offset, float scale_ub, const void* q_out,
+                               const void* scales_out);
+
 /* rrf_plan_fused -- the launch rrf_sum_rmsnorm_fp8 would use on a GPU with
  * sm_count SMs for a call with (residual != 0) or without a residual,
  * without touching the GPU.  Writes the cluster size (1 = one

@@ -19,6 +19,9 @@ Functions, named after the C entry points:
   rrf_plan_fused(num_inputs, rows, cols, sm_count) -> (cluster, threads, vpt)
   rrf_check_sum_args / rrf_check_fused_args (raw pointers, host only)
   rrf_device_error(clear=False) -> RRF_DEVICE_ERROR_* bits
+  rrf_sum_rmsnorm_fp8_pre / rrf_rmsnorm_fp8_post: the two phases of the
+      sharded form (a row's hidden dimension split across devices); the
+      torch.distributed glue between them is in ``sharded.py``
 """
 from __future__ import annotations
 
@@ -29,7 +32,9 @@ _EXPORTS = (
     "Status", "lib", "rrf_check_fused_args", "rrf_check_sum_args",
     "rrf_debug_fail_next_launch", "rrf_device_error", "rrf_last_cuda_error", "rrf_plan_fused",
     "rrf_status_string", "rrf_sum", "rrf_sum_ptr", "rrf_sum_rmsnorm_fp8",
-    "rrf_sum_rmsnorm_fp8_ex", "rrf_sum_rmsnorm_fp8_ptr", "rrf_version",
+    "rrf_sum_rmsnorm_fp8_ex", "rrf_sum_rmsnorm_fp8_ptr", "rrf_version", "RRF_MAX_SHARDS",
+    "rrf_sum_rmsnorm_fp8_pre", "rrf_rmsnorm_fp8_post", "rrf_check_pre_args",
+    "rrf_check_post_args",
 )
 
 __all__ = list(_EXPORTS)

@@ -17,6 +17,7 @@ RRF_FLAG_NO_PDL = 1
 RRF_FLAG_BARRIER_EXCHANGE = 2
 RRF_FLAG_DEBUG_STARVE_EXCHANGE = 0x100
 RRF_DEVICE_ERROR_EXCHANGE_TIMEOUT = 1
+RRF_MAX_SHARDS = 64
 
 
 class Status(enum.IntEnum):
@@ -76,6 +77,17 @@ lib.rrf_last_cuda_error.restype = _int
 lib.rrf_last_cuda_error.argtypes = []
 lib.rrf_debug_fail_next_launch.restype = None
 lib.rrf_debug_fail_next_launch.argtypes = [_int]
+lib.rrf_sum_rmsnorm_fp8_pre.restype = _int
+lib.rrf_sum_rmsnorm_fp8_pre.argtypes = [_ptrs, _int, _i64, _i64, _vp, _vp, _vp, _vp, _f32, _vp,
+                                        _vp]
+lib.rrf_rmsnorm_fp8_post.restype = _int
+lib.rrf_rmsnorm_fp8_post.argtypes = [_vp, _i64, _i64, _vp, _int, _i64, _vp, _f32, _f32, _f32,
+                                     _vp, _vp, _vp]
+lib.rrf_check_pre_args.restype = _int
+lib.rrf_check_pre_args.argtypes = [_ptrs, _int, _i64, _i64, _vp, _vp, _vp, _vp, _f32, _vp]
+lib.rrf_check_post_args.restype = _int
+lib.rrf_check_post_args.argtypes = [_vp, _i64, _i64, _vp, _int, _i64, _vp, _f32, _f32, _f32,
+                                    _vp, _vp]
 lib.rrf_device_error.restype = _int
 lib.rrf_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), _int]
 lib.rrf_version.restype = ctypes.c_char_p
@@ -238,3 +250,76 @@ def rrf_sum_rmsnorm_fp8(inputs, gamma, eps, weight_offset, scale_ub, residual_in
     float32 [..., 1], residual_out or None)."""
     return rrf_sum_rmsnorm_fp8_ex(inputs, gamma, eps, weight_offset, scale_ub, residual_in,
                                   residual_out, q_out, scales_out)
+
+
+# ------------------------------------------------------------ sharded norm ---
+
+def rrf_check_pre_args(input_ptrs, rows, cols, residual_in, residual_out, h_out, gamma,
+                       weight_offset, stats_out) -> int:
+    return lib.rrf_check_pre_args(_ptr_table(input_ptrs), len(input_ptrs), rows, cols,
+                                  residual_in or None, residual_out or None, h_out or None,
+                                  gamma or None, weight_offset, stats_out or None)
+
+
+def rrf_check_post_args(h, rows, cols, stats, shards, total_cols, gamma, eps, weight_offset,
+                        scale_ub, q_out, scales_out) -> int:
+    return lib.rrf_check_post_args(h or None, rows, cols, stats or None, shards, total_cols,
+                                   gamma or None, eps, weight_offset, scale_ub, q_out or None,
+                                   scales_out or None)
+
+
+def rrf_sum_rmsnorm_fp8_pre(inputs, gamma, weight_offset, residual_in=None, residual_out=None,
+                            h_out=None, stats_out=None):
+    """Phase 1 of the sharded norm on this device's column shard.  Returns
+    (stats float32 [rows, 2], h) where h is residual_out (with a residual) or
+    h_out (without)."""
+    torch = _torch()
+    rows, cols = _rows_cols(inputs)
+    x0 = inputs[0]
+    dev = x0.device
+    if gamma.dtype != torch.bfloat16 or gamma.numel() != cols or gamma.device != dev:
+        raise ValueError("gamma must be a bf16 tensor of length cols on the inputs' device")
+    if residual_in is not None:
+        if residual_out is None:
+            residual_out = torch.empty_like(residual_in)
+        h = residual_out
+    else:
+        if h_out is None:
+            h_out = torch.empty_like(x0)
+        h = h_out
+    if stats_out is None:
+        stats_out = torch.empty((rows, 2), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _raise_on(lib.rrf_sum_rmsnorm_fp8_pre(
+            _ptr_table([x.data_ptr() for x in inputs]), len(inputs), rows, cols,
+            residual_in.data_ptr() if residual_in is not None else None,
+            residual_out.data_ptr() if residual_out is not None else None,
+            h_out.data_ptr() if h_out is not None else None, gamma.data_ptr(), weight_offset,
+            stats_out.data_ptr(), _stream(dev)))
+    return stats_out, h
+
+
+def rrf_rmsnorm_fp8_post(h, gamma, stats, total_cols, eps, weight_offset, scale_ub, q_out=None,
+                         scales_out=None, write_scales=True):
+    """Phase 2 of the sharded norm: ``stats`` float32 [shards, rows, 2] (all
+    shards' phase-1 statistics, in shard order).  Returns (q, scales or None)."""
+    torch = _torch()
+    if h.dtype != torch.bfloat16 or not h.is_contiguous() or h.device.type != "cuda":
+        raise ValueError("h must be a contiguous bf16 CUDA tensor")
+    cols = h.shape[-1]
+    rows = h.numel() // cols if cols else 0
+    dev = h.device
+    shards = stats.shape[0]
+    if stats.dtype != torch.float32 or tuple(stats.shape) != (shards, rows, 2) or \
+            not stats.is_contiguous():
+        raise ValueError("stats must be a contiguous float32 [shards, rows, 2] tensor")
+    if q_out is None:
+        q_out = torch.empty(h.shape, dtype=torch.float8_e4m3fn, device=dev)
+    if scales_out is None and write_scales:
+        scales_out = torch.empty(tuple(h.shape[:-1]) + (1,), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _raise_on(lib.rrf_rmsnorm_fp8_post(
+            h.data_ptr(), rows, cols, stats.data_ptr(), shards, total_cols, gamma.data_ptr(),
+            eps, weight_offset, scale_ub, q_out.data_ptr(),
+            scales_out.data_ptr() if scales_out is not None else None, _stream(dev)))
+    return q_out, scales_out

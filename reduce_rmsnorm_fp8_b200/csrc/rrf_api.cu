@@ -372,6 +372,145 @@ extern "C" rrf_status rrf_sum_rmsnorm_fp8(const void* const* inputs, int num_inp
                                   RRF_VARIANT_AUTO, 0, 0, 0, stream);
 }
 
+// -------------------------------------------------------- sharded norm ---
+
+extern "C" rrf_status rrf_check_pre_args(const void* const* inputs, int num_inputs, int64_t rows,
+                                         int64_t cols, const void* residual_in,
+                                         const void* residual_out, const void* h_out,
+                                         const void* gamma, float weight_offset,
+                                         const void* stats_out) {
+    rrf_status st = check_shape(num_inputs, rows, cols, RRF_MAX_COLS);
+    if (st != RRF_OK) return st;
+    if (!std::isfinite(weight_offset)) return RRF_ERR_VALUE;
+    if (rows == 0) return RRF_OK;
+    if ((st = check_inputs(inputs, num_inputs)) != RRF_OK) return st;
+    if ((residual_in == nullptr) != (residual_out == nullptr)) return RRF_ERR_NULL;
+    // the norm input goes to residual_out with a residual, to h_out without
+    if ((residual_in == nullptr) == (h_out == nullptr)) return RRF_ERR_NULL;
+    if (gamma == nullptr || stats_out == nullptr) return RRF_ERR_NULL;
+    if (!aligned(gamma, 16) || !aligned(stats_out, 8)) return RRF_ERR_ALIGN;
+    if (residual_in != nullptr && (!aligned(residual_in, 16) || !aligned(residual_out, 16)))
+        return RRF_ERR_ALIGN;
+    if (h_out != nullptr && !aligned(h_out, 16)) return RRF_ERR_ALIGN;
+    const int64_t bf16_bytes = rows * cols * 2;
+    Range reads[RRF_MAX_INPUTS + 2];
+    int n_reads = 0;
+    for (int r = 0; r < num_inputs; ++r) reads[n_reads++] = range_of(inputs[r], bf16_bytes);
+    reads[n_reads++] = range_of(gamma, cols * 2);
+    if (residual_in != nullptr && residual_in != residual_out)
+        reads[n_reads++] = range_of(residual_in, bf16_bytes);
+    Range writes[2];
+    int n_writes = 0;
+    writes[n_writes++] = range_of(residual_out != nullptr ? residual_out : h_out, bf16_bytes);
+    writes[n_writes++] = range_of(stats_out, rows * 8);
+    for (int w = 0; w < n_writes; ++w) {
+        for (int r = 0; r < n_reads; ++r)
+            if (overlap(writes[w], reads[r])) return RRF_ERR_ALIAS;
+        for (int w2 = w + 1; w2 < n_writes; ++w2)
+            if (overlap(writes[w], writes[w2])) return RRF_ERR_ALIAS;
+    }
+    return RRF_OK;
+}
+
+extern "C" rrf_status rrf_sum_rmsnorm_fp8_pre(const void* const* inputs, int num_inputs,
+                                              int64_t rows, int64_t cols,
+                                              const void* residual_in, void* residual_out,
+                                              void* h_out, const void* gamma,
+                                              float weight_offset, float* stats_out,
+                                              rrf_stream_t stream) {
+    rrf_status st = rrf_check_pre_args(inputs, num_inputs, rows, cols, residual_in,
+                                       residual_out, h_out, gamma, weight_offset, stats_out);
+    if (st != RRF_OK || rows == 0) return st;
+    int sm_count = 0;
+    if ((st = current_sm_count(&sm_count)) != RRF_OK) return st;
+    FusedLaunch l = {};
+    if ((st = shape_launch(num_inputs, rows, cols, sm_count, 0, 0, residual_in != nullptr,
+                           &l)) != RRF_OK)
+        return st;
+    unsigned int* err = nullptr;
+    if ((st = device_error_word(&err)) != RRF_OK) return st;
+    const int64_t vecs = cols / 8;
+    FusedArgs a = {};
+    for (int r = 0; r < num_inputs; ++r) a.in[r] = static_cast<const uint4*>(inputs[r]);
+    a.res_in = static_cast<const uint4*>(residual_in);
+    a.res_out = static_cast<uint4*>(residual_out);
+    a.gamma = static_cast<const uint4*>(gamma);
+    a.R = num_inputs;
+    a.vecs = (int)vecs;
+    a.cluster = l.cluster;
+    a.slice_vecs = (int)((vecs + l.cluster - 1) / l.cluster);
+    a.cols_f = (float)cols;
+    a.weight_offset = weight_offset;
+    a.scale_ub = 1.0f;
+    a.err = err;
+    a.stats_only = 1;
+    a.stats = reinterpret_cast<float2*>(stats_out);
+    a.h_out = static_cast<uint4*>(h_out);
+    cudaError_t e;
+    if (!take_injected_failure(&e))
+        e = launch_fused(a, rows, l, residual_in != nullptr, (cudaStream_t)stream);
+    return e == cudaSuccess ? RRF_OK : cuda_fail(e);
+}
+
+extern "C" rrf_status rrf_check_post_args(const void* h, int64_t rows, int64_t cols,
+                                          const float* stats, int shards, int64_t total_cols,
+                                          const void* gamma, float eps, float weight_offset,
+                                          float scale_ub, const void* q_out,
+                                          const void* scales_out) {
+    if (shards < 1 || shards > RRF_MAX_SHARDS) return RRF_ERR_SHAPE;
+    if (rows < 0 || cols <= 0 || cols % 8 != 0 || total_cols < cols) return RRF_ERR_SHAPE;
+    if (rows > 0 && rows > (INT64_MAX / 2) / cols) return RRF_ERR_SHAPE;
+    if (rows * ((cols / 8 + 127) / 128) > (int64_t)INT32_MAX) return RRF_ERR_SHAPE;
+    if (!(std::isfinite(eps) && eps >= 0.0f)) return RRF_ERR_VALUE;
+    if (!std::isfinite(weight_offset)) return RRF_ERR_VALUE;
+    if (std::isnan(scale_ub) || !(scale_ub > 0.0f)) return RRF_ERR_VALUE;
+    if (rows == 0) return RRF_OK;
+    if (h == nullptr || stats == nullptr || gamma == nullptr || q_out == nullptr)
+        return RRF_ERR_NULL;
+    if (!aligned(h, 16) || !aligned(gamma, 16) || !aligned(q_out, 16) || !aligned(stats, 8))
+        return RRF_ERR_ALIGN;
+    if (scales_out != nullptr && !aligned(scales_out, 4)) return RRF_ERR_ALIGN;
+    const Range reads[3] = {range_of(h, rows * cols * 2), range_of(gamma, cols * 2),
+                            range_of(stats, (int64_t)shards * rows * 8)};
+    Range writes[2];
+    int n_writes = 0;
+    writes[n_writes++] = range_of(q_out, rows * cols);
+    if (scales_out != nullptr) writes[n_writes++] = range_of(scales_out, rows * 4);
+    for (int w = 0; w < n_writes; ++w) {
+        for (int r = 0; r < 3; ++r)
+            if (overlap(writes[w], reads[r])) return RRF_ERR_ALIAS;
+        for (int w2 = w + 1; w2 < n_writes; ++w2)
+            if (overlap(writes[w], writes[w2])) return RRF_ERR_ALIAS;
+    }
+    return RRF_OK;
+}
+
+extern "C" rrf_status rrf_rmsnorm_fp8_post(const void* h, int64_t rows, int64_t cols,
+                                           const float* stats, int shards, int64_t total_cols,
+                                           const void* gamma, float eps, float weight_offset,
+                                           float scale_ub, void* q_out, float* scales_out,
+                                           rrf_stream_t stream) {
+    rrf_status st = rrf_check_post_args(h, rows, cols, stats, shards, total_cols, gamma, eps,
+                                        weight_offset, scale_ub, q_out, scales_out);
+    if (st != RRF_OK || rows == 0) return st;
+    PostArgs a = {};
+    a.h = static_cast<const uint4*>(h);
+    a.gamma = static_cast<const uint4*>(gamma);
+    a.stats = reinterpret_cast<const float2*>(stats);
+    a.q = static_cast<uint2*>(q_out);
+    a.scales = scales_out;
+    a.rows = rows;
+    a.vecs = (int)(cols / 8);
+    a.shards = shards;
+    a.total_cols_f = (float)total_cols;
+    a.eps = eps;
+    a.weight_offset = weight_offset;
+    a.scale_ub = scale_ub;
+    cudaError_t e;
+    if (!take_injected_failure(&e)) e = launch_post(a, true, (cudaStream_t)stream);
+    return e == cudaSuccess ? RRF_OK : cuda_fail(e);
+}
+
 extern "C" rrf_status rrf_plan_fused(int num_inputs, int64_t rows, int64_t cols, int residual,
                                      int sm_count, int* cluster_size, int* block_threads,
                                      int* vecs_per_thread) {

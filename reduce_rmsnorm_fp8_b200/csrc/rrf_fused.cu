@@ -106,8 +106,11 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
                 // exchange: with the barrier exchange its release would
                 // otherwise wait for the store to land, and with either
                 // exchange the early stores measured slower on B200 (0.1-0.2 us
-                // at 32-64 rows of 7168 columns).
-                if (!CLUSTER) st_once(a.res_out + row_base + v, s);
+                // at 32-64 rows of 7168 columns).  The statistics-only form
+                // has no last pass.
+                if (!CLUSTER || a.stats_only) st_once(a.res_out + row_base + v, s);
+            } else if (a.stats_only) {
+                st_once(a.h_out + row_base + v, s);
             }
             h[k] = s;
             st.ss += sumsq_bf16x8(s);
@@ -125,6 +128,11 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
         cluster_wait_acquire();  // phase 0 done: every block of the cluster runs
         st = ASYNC ? cluster_stats_async(st, cluster_stats, &exchange_bar, rank, a.cluster, a.err)
                    : cluster_stats_combine(st, cluster_stats, rank, a.cluster);
+    }
+    if (a.stats_only) {
+        // first phase of the sharded norm: this shard's row statistics
+        if (tid == 0 && rank == 0) a.stats[row] = make_float2(st.ss, st.key);
+        return;
     }
     const float ms = st.ss / a.cols_f;
     const float rinv = 1.0f / sqrtf(ms + a.eps);

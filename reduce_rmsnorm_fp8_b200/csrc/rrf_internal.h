@@ -35,6 +35,29 @@ struct FusedArgs {
     float scale_ub;
     unsigned int* err;     // the library's device error word
     int starve;            // test hook: exchange values a block waits for beyond C
+    // Statistics-only form (the first phase of the sharded norm): instead of
+    // codes and scales the kernel writes each row's (sum h^2, max |h g'|) and,
+    // without a residual, the bf16 norm input h itself.
+    int stats_only;
+    float2* stats;         // [rows]
+    uint4* h_out;          // [rows, cols] or null (with a residual, res_out holds h)
+};
+
+// The second phase of the sharded norm: quantise one column shard from the
+// statistics of every shard.
+struct PostArgs {
+    const uint4* h;        // bf16 norm input of this shard [rows, cols]
+    const uint4* gamma;    // this shard's gamma [cols]
+    const float2* stats;   // [shards, rows]: (sum h^2, max |h g'|) per shard
+    uint2* q;              // [rows, cols] codes
+    float* scales;         // [rows] or null (another shard writes them)
+    int64_t rows;
+    int vecs;              // cols / 8
+    int shards;
+    float total_cols_f;    // columns of the whole row (all shards), the mean's divisor
+    float eps;
+    float weight_offset;
+    float scale_ub;
 };
 
 struct FusedLaunch {
@@ -75,6 +98,8 @@ cudaError_t launch_fused_rb16(const FusedArgs& a, int64_t rows, const FusedLaunc
                               bool residual, cudaStream_t stream);
 cudaError_t launch_fused(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
                          bool residual, cudaStream_t stream);
+
+cudaError_t launch_post(const PostArgs& a, bool pdl, cudaStream_t stream);
 
 // The launch shape the library picks (pure host arithmetic).
 rrf_status plan_fused(int R, int64_t rows, int64_t cols, int sm_count, bool residual,

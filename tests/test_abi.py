@@ -219,3 +219,44 @@ def test_use_fails_loudly_without_library(tmp_path):
                          text=True)
     assert res.returncode != 0 and "librrf.so is missing" in res.stderr
     assert "ImportError" in res.stderr
+
+
+# ------------------------------------------------------------ sharded form ---
+
+def test_pre_validation(rrf):
+    ins = [A, 2 * A]
+    ok = dict(input_ptrs=ins, rows=8, cols=64, residual_in=0, residual_out=0, h_out=8 * A,
+              gamma=9 * A, weight_offset=0.0, stats_out=10 * A)
+    assert rrf.rrf_check_pre_args(**ok) == rrf.Status.OK
+    res = dict(ok, residual_in=11 * A, residual_out=12 * A, h_out=0)
+    assert rrf.rrf_check_pre_args(**res) == rrf.Status.OK
+    for change, status in [
+            (dict(h_out=0), "ERR_NULL"),                               # nowhere to put h
+            (dict(res, h_out=8 * A), "ERR_NULL"),                      # h twice
+            (dict(stats_out=0), "ERR_NULL"),
+            (dict(stats_out=10 * A + 4), "ERR_ALIGN"),
+            (dict(h_out=8 * A + 8), "ERR_ALIGN"),
+            (dict(h_out=A + 64), "ERR_ALIAS"),                        # over an input
+            (dict(stats_out=8 * A + 16), "ERR_ALIAS"),                # over h
+            (dict(cols=12), "ERR_SHAPE"),
+            (dict(weight_offset=float("nan")), "ERR_VALUE")]:
+        kw = dict(ok)
+        kw.update(change)
+        assert rrf.rrf_check_pre_args(**kw) == rrf.Status[status], change
+
+
+def test_post_validation(rrf):
+    ok = dict(h=A, rows=8, cols=64, stats=2 * A, shards=4, total_cols=256, gamma=3 * A,
+              eps=1e-5, weight_offset=0.0, scale_ub=1200.0, q_out=4 * A, scales_out=5 * A)
+    assert rrf.rrf_check_post_args(**ok) == rrf.Status.OK
+    assert rrf.rrf_check_post_args(**dict(ok, scales_out=0)) == rrf.Status.OK
+    for change, status in [
+            (dict(shards=0), "ERR_SHAPE"), (dict(shards=65), "ERR_SHAPE"),
+            (dict(total_cols=56), "ERR_SHAPE"), (dict(cols=60), "ERR_SHAPE"),
+            (dict(h=0), "ERR_NULL"), (dict(stats=0), "ERR_NULL"), (dict(q_out=0), "ERR_NULL"),
+            (dict(stats=2 * A + 4), "ERR_ALIGN"), (dict(q_out=4 * A + 8), "ERR_ALIGN"),
+            (dict(q_out=A + 16), "ERR_ALIAS"), (dict(scales_out=2 * A + 8), "ERR_ALIAS"),
+            (dict(eps=-1.0), "ERR_VALUE"), (dict(scale_ub=0.0), "ERR_VALUE")]:
+        kw = dict(ok)
+        kw.update(change)
+        assert rrf.rrf_check_post_args(**kw) == rrf.Status[status], change
