@@ -299,6 +299,56 @@ def time_region(fn, k_steps: int, device, stream, clocks=None):
     return max_over_ranks(start.elapsed_time(end) / 1e3, device)
 
 
+def time_sharded(rrf, label, rows, cols, shards, device, stream, l2, peak):
+    """Both phases of the sharded form on one shard [rows, cols] of a row
+    split into `shards` (R = 8, residual), each over rotating buffer sets
+    larger than 3 x L2; the gathered statistics are synthetic (the other
+    shards' are copies of this one's)."""
+    import torch
+    c = workloads.make_case(label, rows, cols=cols, device=device)
+    R = c.R
+    pre_b = R * rows * cols * 2 + 4 * rows * cols + 2 * cols + 8 * rows
+    post_b = 2 * rows * cols + 2 * cols + 8 * shards * rows + rows * cols + 4 * rows
+    n = max(2, math.ceil(L2_FLUSH_FACTOR * l2 / (pre_b + post_b)))
+    shape = (n, rows, cols)
+    xs = [x.unsqueeze(0).expand(shape).contiguous() for x in c.inputs]
+    res = c.residual.unsqueeze(0).expand(shape).contiguous()
+    h = torch.empty(shape, dtype=torch.bfloat16, device=device)
+    st = torch.empty((n, rows, 2), dtype=torch.float32, device=device)
+    gathered = torch.empty((n, shards, rows, 2), dtype=torch.float32, device=device)
+    q = torch.empty(shape, dtype=torch.float8_e4m3fn, device=device)
+    sc = torch.empty((n, rows, 1), dtype=torch.float32, device=device)
+
+    def pre(k):
+        s = k % n
+        rrf.rrf_sum_rmsnorm_fp8_pre([x[s] for x in xs], c.gamma, c.weight_offset,
+                                    residual_in=res[s], residual_out=h[s], stats_out=st[s])
+        return 1
+
+    def post(k):
+        s = k % n
+        rrf.rrf_rmsnorm_fp8_post(h[s], c.gamma, gathered[s], cols * shards, c.eps,
+                                 c.weight_offset, c.scale_ub, q_out=q[s], scales_out=sc[s])
+        return 1
+
+    for k in range(n):
+        pre(k)
+    torch.cuda.synchronize(device)
+    gathered.copy_(st.unsqueeze(1).expand(n, shards, rows, 2))
+    rec = {"shard": f"{label} {rows} x {cols} (1 of {shards})", "R": R}
+    for name, fn, nbytes in (("pre", pre, pre_b), ("post", post, post_b)):
+        reps = 100 if rows < 1024 else 10
+        g, _ = capture_steps(fn, reps, device)
+        g.replay()
+        torch.cuda.synchronize(device)
+        t = time_region(lambda _: g.replay(), 1, device, stream)
+        del g
+        rec[f"{name}_us"] = round(t / reps * 1e6, 3)
+        rec[f"{name}_GB_s"] = round(nbytes * reps / t / 1e9, 1)
+        rec[f"{name}_frac"] = round(nbytes * reps / t / 1e9 / peak, 4)
+    return rec
+
+
 def capture_steps(fn, n: int, device):
     """Capture fn(0) .. fn(n-1) into one CUDA graph; returns (graph, number
     of kernels fn launched)."""
@@ -624,6 +674,16 @@ def run_rrf(args):
             del sp
         torch.cuda.empty_cache()
 
+    # ---- the sharded form, one shard of 8 (the all-gather between the phases
+    # is not on one GPU): decode 32 x 7168 -> 896 columns, prefill 8192 x 8192
+    # -> 1024 columns, R = 8 with residual
+    sharded = None
+    if not args.no_secondary:
+        sharded = []
+        for label, rows, cols in (("decode", 32, 896), ("prefill", 8192, 1024)):
+            sharded.append(time_sharded(rrf, label, rows, cols, 8, device, stream, l2, peak))
+        torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(name)
@@ -669,6 +729,7 @@ def run_rrf(args):
             "prefill": secondary,
             "sweep": sweep,
             "other_configs": others,
+            "sharded": sharded,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

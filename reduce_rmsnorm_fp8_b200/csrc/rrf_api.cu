@@ -460,7 +460,7 @@ extern "C" rrf_status rrf_check_post_args(const void* h, int64_t rows, int64_t c
     if (shards < 1 || shards > RRF_MAX_SHARDS) return RRF_ERR_SHAPE;
     if (rows < 0 || cols <= 0 || cols % 8 != 0 || total_cols < cols) return RRF_ERR_SHAPE;
     if (rows > 0 && rows > (INT64_MAX / 2) / cols) return RRF_ERR_SHAPE;
-    if (rows * ((cols / 8 + 127) / 128) > (int64_t)INT32_MAX) return RRF_ERR_SHAPE;
+    if ((rows + 3) / 4 * ((cols / 8 + 63) / 64) > (int64_t)INT32_MAX) return RRF_ERR_SHAPE;
     if (!(std::isfinite(eps) && eps >= 0.0f)) return RRF_ERR_VALUE;
     if (!std::isfinite(weight_offset)) return RRF_ERR_VALUE;
     if (std::isnan(scale_ub) || !(scale_ub > 0.0f)) return RRF_ERR_VALUE;
@@ -493,6 +493,8 @@ extern "C" rrf_status rrf_rmsnorm_fp8_post(const void* h, int64_t rows, int64_t 
     rrf_status st = rrf_check_post_args(h, rows, cols, stats, shards, total_cols, gamma, eps,
                                         weight_offset, scale_ub, q_out, scales_out);
     if (st != RRF_OK || rows == 0) return st;
+    int sm_count = 0;
+    if ((st = current_sm_count(&sm_count)) != RRF_OK) return st;
     PostArgs a = {};
     a.h = static_cast<const uint4*>(h);
     a.gamma = static_cast<const uint4*>(gamma);
@@ -507,7 +509,7 @@ extern "C" rrf_status rrf_rmsnorm_fp8_post(const void* h, int64_t rows, int64_t 
     a.weight_offset = weight_offset;
     a.scale_ub = scale_ub;
     cudaError_t e;
-    if (!take_injected_failure(&e)) e = launch_post(a, true, (cudaStream_t)stream);
+    if (!take_injected_failure(&e)) e = launch_post(a, sm_count, true, (cudaStream_t)stream);
     return e == cudaSuccess ? RRF_OK : cuda_fail(e);
 }
 

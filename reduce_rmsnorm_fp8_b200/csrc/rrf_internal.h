@@ -99,7 +99,7 @@ cudaError_t launch_fused_rb16(const FusedArgs& a, int64_t rows, const FusedLaunc
 cudaError_t launch_fused(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
                          bool residual, cudaStream_t stream);
 
-cudaError_t launch_post(const PostArgs& a, bool pdl, cudaStream_t stream);
+cudaError_t launch_post(const PostArgs& a, int sm_count, bool pdl, cudaStream_t stream);
 
 // The launch shape the library picks (pure host arithmetic).
 rrf_status plan_fused(int R, int64_t rows, int64_t cols, int sm_count, bool residual,

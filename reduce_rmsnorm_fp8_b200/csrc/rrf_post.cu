@@ -18,51 +18,100 @@
 namespace rrf {
 namespace {
 
-constexpr int kPostThreads = 128;
+constexpr int kPostThreads = 128;         // 4 warps per block
+constexpr int kPostVecsPerLane = 2;       // a block's chunk: 64 vectors of each row
+constexpr int kPostChunkVecs = 32 * kPostVecsPerLane;
 
-__global__ void __launch_bounds__(kPostThreads) post_kernel(const PostArgs a) {
+// A block takes 4 * RPW consecutive rows (RPW per warp) and one 64-vector
+// chunk of them.  The gathered statistics are shard-major ([shards][rows]
+// [2]), so the block's rows are contiguous within each shard: every thread
+// stages some of them in shared memory with coalesced loads, then one thread
+// per row merges the row's shards in shard order (the same order in every
+// block of every shard, so every shard derives the same scale) and derives
+// the row's 1/r, scale and 1/scale once; the warps then quantise their rows.
+// (Per-row scale work in every thread, and scattered per-row statistics
+// reads, measured as the bottlenecks of earlier forms on B200.)
+template <int RPW>
+__global__ void __launch_bounds__(kPostThreads) post_kernel(const PostArgs a, int chunks) {
+    constexpr int RB = 4 * RPW;  // rows per block
+    __shared__ float2 stage[RRF_MAX_SHARDS * RB];  // [shard][row]
+    __shared__ float3 rowval[RB];                  // (1/r, scale, 1/scale)
     wait_for_previous_grid();  // see rrf_device.cuh: programmatic dependent launch
     allow_next_grid();
 
-    const int64_t blocks_per_row = (a.vecs + kPostThreads - 1) / kPostThreads;
-    const int64_t row = (int64_t)blockIdx.x / blocks_per_row;
-    const int v = (int)((int64_t)blockIdx.x % blocks_per_row) * kPostThreads + threadIdx.x;
-    const int lane = threadIdx.x & 31;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t row0 = (int64_t)(blockIdx.x / chunks) * RB;
+    const int v0 = (int)(blockIdx.x % chunks) * kPostChunkVecs;
+    const int64_t left = a.rows - row0;
+    const int nrows = left < RB ? (int)left : RB;
 
-    // The row's statistics over all shards: lane s (+32k) takes shard s, then a
-    // full butterfly -- every warp of every shard reduces the same values in
-    // the same order.
-    RowStats st = stats_empty();
-    for (int s = lane; s < a.shards; s += 32) {
-        const float2 p = a.stats[(int64_t)s * a.rows + row];
-        st = stats_merge(st, RowStats{p.x, p.y});
-    }
-    st = stats_butterfly(st, 32);
-    const float ms = st.ss / a.total_cols_f;
-    const float rinv = 1.0f / sqrtf(ms + a.eps);
-    const float amax = __fmul_rn(st.key, rinv);
-    const float scale = fmaxf(fminf(amax, a.scale_ub), 1e-12f) / 448.0f;
-    const float inv_scale = 1.0f / scale;
-
-    if (v < a.vecs) {
-        const int64_t i = row * (int64_t)a.vecs + v;
-        float hf[8], gf[8], qv[8];
-        bf16x8_to_f32(ld_once(a.h + i), hf);
-        bf16x8_to_f32(ld_shared_by_all(a.gamma + v), gf);
+    // the data of this warp's rows first
+    uint4 hv[RPW][kPostVecsPerLane];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const float y = __fmul_rn(__fmul_rn(hf[e], rinv), __fadd_rn(gf[e], a.weight_offset));
-            qv[e] = __fmul_rn(y, inv_scale);
+    for (int k = 0; k < RPW; ++k) {
+        const int r = warp + 4 * k;
+#pragma unroll
+        for (int j = 0; j < kPostVecsPerLane; ++j) {
+            const int v = v0 + lane + 32 * j;
+            if (r < nrows && v < a.vecs) hv[k][j] = ld_once(a.h + (row0 + r) * a.vecs + v);
         }
-        st_once(a.q + i, f32_to_e4m3x8(qv));
     }
-    if (v == 0 && a.scales != nullptr) a.scales[row] = scale;
+    // the statistics of the block's rows, coalesced per shard
+    for (int i = tid; i < a.shards * RB; i += kPostThreads) {
+        const int s = i / RB, r = i % RB;
+        stage[i] = r < nrows ? a.stats[(int64_t)s * a.rows + row0 + r] : make_float2(0.0f, 0.0f);
+    }
+    __syncthreads();
+    if (tid < nrows) {
+        float ss = 0.0f, key = 0.0f;
+        for (int s = 0; s < a.shards; ++s) {
+            const float2 p = stage[s * RB + tid];
+            ss = ss + p.x;
+            key = fmaxf(key, p.y);
+        }
+        const float ms = ss / a.total_cols_f;
+        const float rinv = 1.0f / sqrtf(ms + a.eps);
+        const float amax = __fmul_rn(key, rinv);
+        const float scale = fmaxf(fminf(amax, a.scale_ub), 1e-12f) / 448.0f;
+        rowval[tid] = make_float3(rinv, scale, 1.0f / scale);
+        if (v0 == 0 && a.scales != nullptr) a.scales[row0 + tid] = scale;
+    }
+    __syncthreads();
+
+    uint4 gv[kPostVecsPerLane];
+#pragma unroll
+    for (int j = 0; j < kPostVecsPerLane; ++j) {
+        const int v = v0 + lane + 32 * j;
+        gv[j] = v < a.vecs ? ld_shared_by_all(a.gamma + v) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int k = 0; k < RPW; ++k) {
+        const int r = warp + 4 * k;
+        if (r >= nrows) break;  // uniform across the warp
+        const float3 rv = rowval[r];
+#pragma unroll
+        for (int j = 0; j < kPostVecsPerLane; ++j) {
+            const int v = v0 + lane + 32 * j;
+            if (v < a.vecs) {
+                float hf[8], gf[8], qv[8];
+                bf16x8_to_f32(hv[k][j], hf);
+                bf16x8_to_f32(gv[j], gf);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float y =
+                        __fmul_rn(__fmul_rn(hf[e], rv.x), __fadd_rn(gf[e], a.weight_offset));
+                    qv[e] = __fmul_rn(y, rv.z);
+                }
+                st_once(a.q + (row0 + r) * a.vecs + v, f32_to_e4m3x8(qv));
+            }
+        }
+    }
 }
 
-}  // namespace
-
-cudaError_t launch_post(const PostArgs& a, bool pdl, cudaStream_t stream) {
-    const int64_t blocks = a.rows * ((a.vecs + kPostThreads - 1) / kPostThreads);
+template <int RPW>
+cudaError_t launch_rpw(const PostArgs& a, int chunks, bool pdl, cudaStream_t stream) {
+    constexpr int RB = 4 * RPW;
+    const int64_t blocks = (a.rows + RB - 1) / RB * chunks;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)blocks, 1, 1);
     cfg.blockDim = dim3(kPostThreads, 1, 1);
@@ -72,7 +121,18 @@ cudaError_t launch_post(const PostArgs& a, bool pdl, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, post_kernel, a);
+    return cudaLaunchKernelEx(&cfg, post_kernel<RPW>, a, chunks);
+}
+
+}  // namespace
+
+cudaError_t launch_post(const PostArgs& a, int sm_count, bool pdl, cudaStream_t stream) {
+    const int chunks = (a.vecs + kPostChunkVecs - 1) / kPostChunkVecs;
+    // Four rows per warp once that still gives every SM several blocks; one
+    // row per warp for small calls, which are latency-bound.
+    if ((a.rows + 15) / 16 * chunks >= 4 * (int64_t)sm_count)
+        return launch_rpw<4>(a, chunks, pdl, stream);
+    return launch_rpw<1>(a, chunks, pdl, stream);
 }
 
 }  // namespace rrf
