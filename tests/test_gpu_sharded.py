@@ -68,6 +68,18 @@ def test_sharded_matches_whole_rows(rrf, name, rows, S):
     assert np.array_equal(h_all, ref["h"])
 
 
+@pytest.mark.parametrize("name,rows", [("decode", 64), ("odd", 37), ("sweep", 16)])
+def test_one_shard_equals_fused_call(rrf, name, rows):
+    """With one shard the two phases reproduce the fused call bit for bit:
+    the same launch computes the same statistics, and merging one shard's
+    pair changes nothing."""
+    c = parity.to_device(workloads.make_case(name, rows))
+    out, _, _, _ = run_sharded(rrf, c, 1)
+    fused = parity.gpu_fused(c)
+    for k in fused:
+        assert np.array_equal(out[k], fused[k]), k
+
+
 def test_shard_statistics_pinned(rrf):
     """Phase 1's statistics: max |h * g'| equals the fp32 products' maximum
     computed from the oracle's h (exactly: a max does not depend on order);
