@@ -349,6 +349,58 @@ def time_sharded(rrf, label, rows, cols, shards, device, stream, l2, peak):
     return rec
 
 
+def time_allreduce(rrf, label, rows, world, mode, device, stream, l2):
+    """The multi-GPU call with all `world` ranks in one launch on this GPU
+    (LocalGroup): one CUDA graph of `reps` calls numbered 1..reps after a
+    reset of the signal pads, cycling through buffer sets larger than 3 x L2
+    (the residual updated in place);
+    microseconds per call.  This GPU's memory stands in for the links, so the
+    number bounds the kernel's own cost, not a multi-GPU call's."""
+    import torch
+
+    from reduce_rmsnorm_fp8_b200 import allreduce
+    c = workloads.make_case(label, rows, R=world, device=device)
+    cols = c.cols
+    set_bytes = world * rows * cols * 2 * 3 + world * rows * cols
+    n = max(1, math.ceil(L2_FLUSH_FACTOR * l2 / set_bytes))
+    rep = lambda t: t.unsqueeze(0).repeat(n, 1, 1)  # a copy, also for n == 1
+    xs = [rep(x) for x in c.inputs]                # [n, rows, cols] per rank
+    rs = [rep(c.residual) for _ in range(world)]
+    qs = [torch.empty((n, rows, cols), dtype=torch.float8_e4m3fn, device=device)
+          for _ in range(world)]
+    ss = [torch.empty((n, rows, 1), dtype=torch.float32, device=device) for _ in range(world)]
+    g = allreduce.LocalGroup(world, device)
+
+    def call(k):
+        i = k % n
+        g([x[i] for x in xs], c.gamma, c.eps, c.weight_offset, c.scale_ub,
+          residual_in=[r[i] for r in rs], residual_out=[r[i] for r in rs],
+          q_out=[q[i] for q in qs], scales_out=[s[i] for s in ss], mode=mode, epoch=k + 1)
+        return 1
+
+    reps = max(50, n) if rows < 1024 else 5
+    for k in range(reps):  # warm-up, eager
+        call(k)
+    torch.cuda.synchronize(device)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for p in g.pads:
+            p.zero_()
+        for k in range(reps):
+            call(k)
+    graph.replay()
+    torch.cuda.synchronize(device)
+    t = time_region(lambda _: graph.replay(), 1, device, stream)
+    del graph
+    sm = torch.cuda.get_device_properties(device).multi_processor_count
+    m, cl, th, vpt = rrf.rrf_plan_allreduce(world, rows, cols, sm, True, mode)
+    flags = rrf.rrf_device_error(clear=True)
+    return {"case": f"{label} {rows} x {cols}, {world} ranks",
+            "mode": "two-shot" if m == 2 else "one-shot",
+            "launch": {"cluster": cl, "threads": th, "vecs_per_thread": vpt},
+            "us_per_call": round(t / reps * 1e6, 3), "device_error": flags}
+
+
 def capture_steps(fn, n: int, device):
     """Capture fn(0) .. fn(n-1) into one CUDA graph; returns (graph, number
     of kernels fn launched)."""
@@ -684,6 +736,15 @@ def run_rrf(args):
             sharded.append(time_sharded(rrf, label, rows, cols, 8, device, stream, l2, peak))
         torch.cuda.empty_cache()
 
+    # ---- the multi-GPU call, all ranks emulated in one launch on this GPU
+    emulated = None
+    if not args.no_secondary:
+        emulated = [time_allreduce(rrf, label, rows, ranks, mode, device, stream, l2)
+                    for label, rows, ranks, mode in (("decode", 1, 8, 0), ("decode", 8, 8, 0),
+                                                     ("decode", 64, 8, 0), ("decode", 64, 8, 1),
+                                                     ("prefill", 8192, 8, 0))]
+        torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(name)
@@ -730,6 +791,7 @@ def run_rrf(args):
             "sweep": sweep,
             "other_configs": others,
             "sharded": sharded,
+            "allreduce_emulated": emulated,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

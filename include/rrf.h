@@ -254,6 +254,102 @@ rrf_status rrf_check_post_args(const void* h, int64_t rows, int64_t cols, const 
                                float weight_offset, float scale_ub, const void* q_out,
                                const void* scales_out);
 
+/* ------------------------------------------------------------------------
+ * The multi-GPU form: the `world` partials live on `world` GPUs.
+ *
+ * Modular docs, `allreduce_rmsnorm_fp8` (its description and the paragraph
+ * on signal buffer sizing): one kernel launch does the all-reduce over peer
+ * memory and the norm; below a payload threshold every GPU reduces all rows
+ * itself (1-stage), above it every GPU reduces ceil(rows / ngpus) rows and
+ * the FP8 rows and scales are then gathered (2-stage).  b12x PR #283: a rank
+ * takes its rows from every peer and accumulates them in fp32 in fixed rank
+ * order, rounding once.  TensorRT-LLM PR #19836: arrivals are counted per
+ * CTA.
+ *
+ * One call is one kernel per rank that reads and writes the other ranks'
+ * buffers directly (peer loads and stores over NVLink / NVSwitch):
+ *  - start barrier: block b of every rank tells block b of every rank that
+ *    it runs (the rank's input, produced earlier in its stream, is ready)
+ *    and waits for the same word from every rank;
+ *  - one-shot (RRF_AR_ONE_SHOT): every rank computes every row from all
+ *    ranks' partials and writes its own outputs;  two-shot
+ *    (RRF_AR_TWO_SHOT): rank k computes rows [k*P, min((k+1)*P, rows)),
+ *    P = ceil(rows / world), and stores their codes, scales and residual
+ *    into every rank's outputs;
+ *  - end barrier: the same words again after the stores; when the call has
+ *    completed on a rank (stream order) its outputs are whole and no peer
+ *    reads its input any more, so the caller may overwrite it.
+ * A row's arithmetic is that of rrf_sum_rmsnorm_fp8 with the partials as
+ * inputs in rank order: the bf16 sum and residual are the same bits, scales
+ * and codes agree within that call's tolerance (the same bits for the same
+ * launch shape).
+ *
+ * Buffers: every pointer array has `world` entries, entry j being rank j's
+ * buffer as this GPU addresses it: a peer mapping in a job with one process
+ * per GPU (every rank passes the same buffers, each through its own
+ * mappings), or another buffer of this GPU when one launch runs all ranks
+ * (local_ranks == world, used to run the whole exchange on one GPU).
+ * Signal pads: RRF_AR_SIGNAL_WORDS 32-bit words per rank, zeroed once before
+ * the first call; `epoch` numbers the calls 1, 2, 3, ... (the same number on
+ * every rank for the same call, never 0).  After RRF_DEVICE_ERROR_PEER_TIMEOUT
+ * the pads must be zeroed again and the numbering restarted.
+ * ---------------------------------------------------------------------- */
+
+#define RRF_AR_MAX_WORLD 8
+#define RRF_AR_MAX_BLOCKS 1024 /* blocks per rank of one launch */
+#define RRF_AR_SIGNAL_WORDS (2 * RRF_AR_MAX_WORLD * RRF_AR_MAX_BLOCKS)
+#define RRF_AR_AUTO 0     /* two-shot when every rank gets a row, else one-shot */
+#define RRF_AR_ONE_SHOT 1
+#define RRF_AR_TWO_SHOT 2
+
+/* rrf_allreduce_rmsnorm_fp8 -- one call of the multi-GPU form.
+ * inputs        [world] bf16 [rows, cols] partials, 16-byte aligned
+ * residual_in   [world] bf16 [rows, cols] residuals (rank j reads entry j;
+ *               all ranks hold the same residual), or NULL for none
+ * residual_out  [world] bf16 [rows, cols], NULL exactly when residual_in is;
+ *               entry j may equal residual_in[j] (in place)
+ * q_out         [world] fp8 e4m3fn codes [rows, cols], 16-byte aligned
+ * scales_out    [world] float [rows], 4-byte aligned
+ * signals       [world] pads of RRF_AR_SIGNAL_WORDS words, 16-byte aligned
+ * world         1..RRF_AR_MAX_WORLD;  rank: this process's rank (0 when
+ *               local_ranks == world);  local_ranks: 1 or world
+ * rows, cols, gamma, eps, weight_offset, scale_ub  as for rrf_sum_rmsnorm_fp8
+ *               (gamma: this GPU's copy); cols <= 8 * 8 * 512 * 4
+ * epoch         the call's number (see above);  mode: RRF_AR_*
+ * timeout_ns    bound on each barrier wait (0 = one second)
+ * Every rank must make the same call (same shape, mode and epoch).
+ * Errors: RRF_ERR_NULL, RRF_ERR_RANKS (world or rank out of range),
+ *         RRF_ERR_SHAPE, RRF_ERR_ALIGN, RRF_ERR_ALIAS, RRF_ERR_VALUE
+ *         (epoch 0 included), RRF_ERR_UNSUPPORTED (mode or local_ranks out of
+ *         range, or all ranks' blocks cannot be resident on this GPU at
+ *         once), RRF_ERR_CUDA. */
+rrf_status rrf_allreduce_rmsnorm_fp8(const void* const* inputs, const void* const* residual_in,
+                                     void* const* residual_out, void* const* q_out,
+                                     float* const* scales_out, unsigned int* const* signals,
+                                     int world, int rank, int local_ranks, int64_t rows,
+                                     int64_t cols, const void* gamma, float eps,
+                                     float weight_offset, float scale_ub, unsigned int epoch,
+                                     int mode, uint64_t timeout_ns, rrf_stream_t stream);
+
+/* The host validation of rrf_allreduce_rmsnorm_fp8 alone (no GPU needed). */
+rrf_status rrf_check_allreduce_args(const void* const* inputs, const void* const* residual_in,
+                                    void* const* residual_out, void* const* q_out,
+                                    float* const* scales_out, unsigned int* const* signals,
+                                    int world, int rank, int local_ranks, int64_t rows,
+                                    int64_t cols, const void* gamma, float eps,
+                                    float weight_offset, float scale_ub, unsigned int epoch,
+                                    int mode);
+
+/* rrf_plan_allreduce -- the mode and row shape rrf_allreduce_rmsnorm_fp8
+ * picks on a GPU with sm_count SMs, without touching the GPU: the mode
+ * (RRF_AR_ONE_SHOT / RRF_AR_TWO_SHOT), blocks per row, threads per block and
+ * 16-byte vectors per thread.  (The blocks per rank also depend on the
+ * occupancy of the compiled kernel, known only on the device.)
+ * Errors: RRF_ERR_NULL, RRF_ERR_RANKS, RRF_ERR_SHAPE, RRF_ERR_UNSUPPORTED. */
+rrf_status rrf_plan_allreduce(int world, int64_t rows, int64_t cols, int residual, int mode,
+                              int sm_count, int* mode_out, int* cluster_size,
+                              int* block_threads, int* vecs_per_thread);
+
 /* rrf_plan_fused -- the launch rrf_sum_rmsnorm_fp8 would use on a GPU with
  * sm_count SMs for a call with (residual != 0) or without a residual,
  * without touching the GPU.  Writes the cluster size (1 = one
@@ -279,6 +375,8 @@ rrf_status rrf_check_fused_args(const void* const* inputs, int num_inputs, int64
 /* Device error bits. */
 #define RRF_DEVICE_ERROR_EXCHANGE_TIMEOUT 1u /* a cluster block's bounded wait for its
                                                peers' statistics ran out          */
+#define RRF_DEVICE_ERROR_PEER_TIMEOUT 2u /* a multi-GPU barrier wait for a peer
+                                            rank ran out                      */
 
 /* rrf_device_error -- the device error word of the current device: the OR
  * of RRF_DEVICE_ERROR_* bits that kernels of this library have set since it

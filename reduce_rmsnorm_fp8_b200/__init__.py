@@ -34,7 +34,10 @@ _EXPORTS = (
     "rrf_status_string", "rrf_sum", "rrf_sum_ptr", "rrf_sum_rmsnorm_fp8",
     "rrf_sum_rmsnorm_fp8_ex", "rrf_sum_rmsnorm_fp8_ptr", "rrf_version", "RRF_MAX_SHARDS",
     "rrf_sum_rmsnorm_fp8_pre", "rrf_rmsnorm_fp8_post", "rrf_check_pre_args",
-    "rrf_check_post_args",
+    "rrf_check_post_args", "RRF_DEVICE_ERROR_PEER_TIMEOUT", "RRF_AR_MAX_WORLD",
+    "RRF_AR_MAX_BLOCKS", "RRF_AR_SIGNAL_WORDS", "RRF_AR_AUTO", "RRF_AR_ONE_SHOT",
+    "RRF_AR_TWO_SHOT", "rrf_check_allreduce_args", "rrf_plan_allreduce",
+    "rrf_allreduce_rmsnorm_fp8_ptr",
 )
 
 __all__ = list(_EXPORTS)

@@ -18,6 +18,13 @@ RRF_FLAG_BARRIER_EXCHANGE = 2
 RRF_FLAG_DEBUG_STARVE_EXCHANGE = 0x100
 RRF_DEVICE_ERROR_EXCHANGE_TIMEOUT = 1
 RRF_MAX_SHARDS = 64
+RRF_DEVICE_ERROR_PEER_TIMEOUT = 2
+RRF_AR_MAX_WORLD = 8
+RRF_AR_MAX_BLOCKS = 1024
+RRF_AR_SIGNAL_WORDS = 2 * RRF_AR_MAX_WORLD * RRF_AR_MAX_BLOCKS
+RRF_AR_AUTO = 0
+RRF_AR_ONE_SHOT = 1
+RRF_AR_TWO_SHOT = 2
 
 
 class Status(enum.IntEnum):
@@ -88,6 +95,14 @@ lib.rrf_check_pre_args.argtypes = [_ptrs, _int, _i64, _i64, _vp, _vp, _vp, _vp, 
 lib.rrf_check_post_args.restype = _int
 lib.rrf_check_post_args.argtypes = [_vp, _i64, _i64, _vp, _int, _i64, _vp, _f32, _f32, _f32,
                                     _vp, _vp]
+_ar_args = [_ptrs, _ptrs, _ptrs, _ptrs, _ptrs, _ptrs, _int, _int, _int, _i64, _i64, _vp, _f32,
+            _f32, _f32, ctypes.c_uint, _int]
+lib.rrf_allreduce_rmsnorm_fp8.restype = _int
+lib.rrf_allreduce_rmsnorm_fp8.argtypes = _ar_args + [ctypes.c_uint64, _vp]
+lib.rrf_check_allreduce_args.restype = _int
+lib.rrf_check_allreduce_args.argtypes = _ar_args
+lib.rrf_plan_allreduce.restype = _int
+lib.rrf_plan_allreduce.argtypes = [_int, _i64, _i64, _int, _int, _int] + [ctypes.POINTER(_int)] * 4
 lib.rrf_device_error.restype = _int
 lib.rrf_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), _int]
 lib.rrf_version.restype = ctypes.c_char_p
@@ -149,6 +164,43 @@ def rrf_plan_fused(num_inputs: int, rows: int, cols: int, sm_count: int, residua
     _raise_on(lib.rrf_plan_fused(num_inputs, rows, cols, int(bool(residual)), sm_count,
                                  ctypes.byref(c), ctypes.byref(t), ctypes.byref(v)))
     return c.value, t.value, v.value
+
+
+def _ar_tables(inputs, residual_in, residual_out, q_out, scales_out, signals):
+    opt = (lambda t: None if t is None else _ptr_table(t))
+    return tuple(opt(t) for t in (inputs, residual_in, residual_out, q_out, scales_out, signals))
+
+
+def rrf_check_allreduce_args(inputs, residual_in, residual_out, q_out, scales_out, signals,
+                             rank, local_ranks, rows, cols, gamma, eps, weight_offset, scale_ub,
+                             epoch, mode, world=None) -> int:
+    """Host validation of the multi-GPU call on raw pointers (lists of
+    ``world`` ints; residual lists may be None)."""
+    world = len(inputs) if world is None else world
+    return lib.rrf_check_allreduce_args(
+        *_ar_tables(inputs, residual_in, residual_out, q_out, scales_out, signals), world,
+        rank, local_ranks, rows, cols, gamma or None, eps, weight_offset, scale_ub, epoch, mode)
+
+
+def rrf_plan_allreduce(world: int, rows: int, cols: int, sm_count: int, residual=True,
+                       mode: int = 0):
+    """The multi-GPU call's choice: (mode, cluster_size, block_threads,
+    vecs_per_thread)."""
+    out = [_int() for _ in range(4)]
+    _raise_on(lib.rrf_plan_allreduce(world, rows, cols, int(bool(residual)), mode, sm_count,
+                                     *[ctypes.byref(o) for o in out]))
+    return tuple(o.value for o in out)
+
+
+def rrf_allreduce_rmsnorm_fp8_ptr(inputs, residual_in, residual_out, q_out, scales_out, signals,
+                                  rank, local_ranks, rows, cols, gamma, eps, weight_offset,
+                                  scale_ub, epoch, mode=0, timeout_ns=0, stream=0) -> None:
+    """rrf_allreduce_rmsnorm_fp8 on raw pointers: every list holds one device
+    address per rank, as this GPU addresses that rank's buffer."""
+    _raise_on(lib.rrf_allreduce_rmsnorm_fp8(
+        *_ar_tables(inputs, residual_in, residual_out, q_out, scales_out, signals), len(inputs),
+        rank, local_ranks, rows, cols, gamma or None, eps, weight_offset, scale_ub, epoch, mode,
+        timeout_ns, stream or None))
 
 
 def rrf_sum_ptr(input_ptrs, rows, cols, out_ptr, stream=0) -> None:

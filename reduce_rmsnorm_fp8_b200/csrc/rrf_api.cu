@@ -513,6 +513,203 @@ extern "C" rrf_status rrf_rmsnorm_fp8_post(const void* h, int64_t rows, int64_t 
     return e == cudaSuccess ? RRF_OK : cuda_fail(e);
 }
 
+// ------------------------------------------------------ multi-GPU form ---
+
+namespace rrf {
+namespace {
+
+constexpr int64_t kArMaxCols = (int64_t)8 * 8 * kArMaxThreads * 4;  // C * 8 * T * VPT
+constexpr uint64_t kArDefaultTimeoutNs = 1000000000ull;             // 1 s
+
+// Two-shot splits the rows over the ranks, so it needs a row per rank; it
+// moves (world - 1) / world of the partials over the links where one-shot
+// moves world - 1 times them, and both take the same two barriers.
+int ar_mode(int world, int64_t rows, int mode) {
+    if (mode != RRF_AR_AUTO) return mode;
+    return rows >= world ? RRF_AR_TWO_SHOT : RRF_AR_ONE_SHOT;
+}
+
+// The row shape for the rows one rank computes, chosen as for the single-GPU
+// kernel (cluster_choice), then the fewest vectors per thread (at most 4)
+// that keep a block at <= 512 threads, splitting the row further (up to
+// clusters of 8) while none does.
+rrf_status plan_allreduce(int world, int64_t rows, int64_t cols, bool residual, int mode,
+                          int sm_count, ArLaunch* l) {
+    if (world < 1 || world > RRF_AR_MAX_WORLD) return RRF_ERR_RANKS;
+    rrf_status st = check_shape(world, rows, cols, kArMaxCols);
+    if (st != RRF_OK) return st;
+    if (mode < RRF_AR_AUTO || mode > RRF_AR_TWO_SHOT) return RRF_ERR_UNSUPPORTED;
+    if (sm_count < 1) sm_count = 1;
+    l->two_shot = ar_mode(world, rows, mode) == RRF_AR_TWO_SHOT;
+    const int64_t mine = l->two_shot ? (rows + world - 1) / world : rows;
+    const int64_t vecs = cols / 8;
+    const double row_bytes = (double)cols * (2.0 * world + (residual ? 4.0 : 0.0) + 1.0);
+    int c = cluster_choice(mine, row_bytes, sm_count);
+    while (c > 1 && vecs / c < 32) c /= 2;
+    for (;;) {
+        const int64_t slice = (vecs + c - 1) / c;
+        int vpt = 1;
+        while (vpt < 4 && slice > (int64_t)kArMaxThreads * vpt) vpt *= 2;
+        if (slice <= (int64_t)kArMaxThreads * vpt) {
+            l->cluster = c;
+            l->vecs_per_thread = vpt;
+            l->threads = round_up32((slice + vpt - 1) / vpt);
+            break;
+        }
+        if (c >= 8) return RRF_ERR_SHAPE;
+        c *= 2;
+    }
+    l->residual = residual;
+    l->local_ranks = 1;
+    l->blocks = 0;
+    return RRF_OK;
+}
+
+}  // namespace
+}  // namespace rrf
+
+extern "C" rrf_status rrf_check_allreduce_args(
+    const void* const* inputs, const void* const* residual_in, void* const* residual_out,
+    void* const* q_out, float* const* scales_out, unsigned int* const* signals, int world,
+    int rank, int local_ranks, int64_t rows, int64_t cols, const void* gamma, float eps,
+    float weight_offset, float scale_ub, unsigned int epoch, int mode) {
+    if (world < 1 || world > RRF_AR_MAX_WORLD) return RRF_ERR_RANKS;
+    if (local_ranks != 1 && local_ranks != world) return RRF_ERR_UNSUPPORTED;
+    if (rank < 0 || rank >= world || (local_ranks > 1 && rank != 0)) return RRF_ERR_RANKS;
+    if (mode < RRF_AR_AUTO || mode > RRF_AR_TWO_SHOT) return RRF_ERR_UNSUPPORTED;
+    rrf_status st = check_shape(world, rows, cols, kArMaxCols);
+    if (st != RRF_OK) return st;
+    if (!(std::isfinite(eps) && eps >= 0.0f)) return RRF_ERR_VALUE;
+    if (!std::isfinite(weight_offset)) return RRF_ERR_VALUE;
+    if (std::isnan(scale_ub) || !(scale_ub > 0.0f)) return RRF_ERR_VALUE;
+    if (epoch == 0) return RRF_ERR_VALUE;
+    if (rows == 0) return RRF_OK;
+    if (!inputs || !q_out || !scales_out || !signals || !gamma) return RRF_ERR_NULL;
+    if ((residual_in == nullptr) != (residual_out == nullptr)) return RRF_ERR_NULL;
+    if (!aligned(gamma, 16)) return RRF_ERR_ALIGN;
+    const bool res = residual_in != nullptr;
+    for (int j = 0; j < world; ++j) {
+        if (!inputs[j] || !q_out[j] || !scales_out[j] || !signals[j]) return RRF_ERR_NULL;
+        if (res && (!residual_in[j] || !residual_out[j])) return RRF_ERR_NULL;
+        if (!aligned(inputs[j], 16) || !aligned(q_out[j], 16) || !aligned(scales_out[j], 4) ||
+            !aligned(signals[j], 16))
+            return RRF_ERR_ALIGN;
+        if (res && (!aligned(residual_in[j], 16) || !aligned(residual_out[j], 16)))
+            return RRF_ERR_ALIGN;
+    }
+    // No write may overlap a read or another write, except residual_out[j]
+    // == residual_in[j] exactly (every rank's buffers, as this GPU sees them).
+    const int64_t bf16_bytes = rows * cols * 2;
+    Range reads[2 * RRF_AR_MAX_WORLD + 1];
+    Range writes[4 * RRF_AR_MAX_WORLD];
+    int n_reads = 0, n_writes = 0;
+    reads[n_reads++] = range_of(gamma, cols * 2);
+    for (int j = 0; j < world; ++j) {
+        reads[n_reads++] = range_of(inputs[j], bf16_bytes);
+        if (res && residual_in[j] != residual_out[j])
+            reads[n_reads++] = range_of(residual_in[j], bf16_bytes);
+        writes[n_writes++] = range_of(q_out[j], rows * cols);
+        writes[n_writes++] = range_of(scales_out[j], rows * 4);
+        writes[n_writes++] = range_of(signals[j], (int64_t)RRF_AR_SIGNAL_WORDS * 4);
+        if (res) writes[n_writes++] = range_of(residual_out[j], bf16_bytes);
+    }
+    for (int w = 0; w < n_writes; ++w) {
+        for (int r = 0; r < n_reads; ++r)
+            if (overlap(writes[w], reads[r])) return RRF_ERR_ALIAS;
+        for (int w2 = w + 1; w2 < n_writes; ++w2)
+            if (overlap(writes[w], writes[w2])) return RRF_ERR_ALIAS;
+    }
+    if (res) {  // an in-place residual may serve only its own rank
+        for (int j = 0; j < world; ++j)
+            for (int i = 0; i < world; ++i)
+                if (i != j && overlap(range_of(residual_out[j], bf16_bytes),
+                                      range_of(residual_in[i], bf16_bytes)))
+                    return RRF_ERR_ALIAS;
+    }
+    return RRF_OK;
+}
+
+extern "C" rrf_status rrf_allreduce_rmsnorm_fp8(
+    const void* const* inputs, const void* const* residual_in, void* const* residual_out,
+    void* const* q_out, float* const* scales_out, unsigned int* const* signals, int world,
+    int rank, int local_ranks, int64_t rows, int64_t cols, const void* gamma, float eps,
+    float weight_offset, float scale_ub, unsigned int epoch, int mode, uint64_t timeout_ns,
+    rrf_stream_t stream) {
+    rrf_status st = rrf_check_allreduce_args(inputs, residual_in, residual_out, q_out,
+                                             scales_out, signals, world, rank, local_ranks,
+                                             rows, cols, gamma, eps, weight_offset, scale_ub,
+                                             epoch, mode);
+    if (st != RRF_OK || rows == 0) return st;
+    int sm_count = 0;
+    if ((st = current_sm_count(&sm_count)) != RRF_OK) return st;
+    ArLaunch l = {};
+    if ((st = plan_allreduce(world, rows, cols, residual_in != nullptr, mode, sm_count, &l)) !=
+        RRF_OK)
+        return st;
+    l.local_ranks = local_ranks;
+    // A persistent grid: every block of every rank in this launch resident
+    // at once (the barriers pair block b of every rank), at most one cluster
+    // per row of the rank's range.
+    int resident = 0;
+    cudaError_t e = allreduce_resident_blocks(l, &resident);
+    if (e != cudaSuccess) return cuda_fail(e);
+    int64_t cap = resident / local_ranks;
+    if (cap > RRF_AR_MAX_BLOCKS) cap = RRF_AR_MAX_BLOCKS;
+    cap = cap / l.cluster * l.cluster;
+    if (cap < l.cluster) return RRF_ERR_UNSUPPORTED;
+    const int64_t mine = l.two_shot ? (rows + world - 1) / world : rows;
+    const int64_t want = mine * l.cluster;
+    l.blocks = (int)(want < cap ? want : cap);
+    unsigned int* err = nullptr;
+    if ((st = device_error_word(&err)) != RRF_OK) return st;
+
+    ArArgs a = {};
+    for (int j = 0; j < world; ++j) {
+        a.in[j] = static_cast<const uint4*>(inputs[j]);
+        if (residual_in != nullptr) {
+            a.res_in[j] = static_cast<const uint4*>(residual_in[j]);
+            a.res_out[j] = static_cast<uint4*>(residual_out[j]);
+        }
+        a.q[j] = static_cast<uint2*>(q_out[j]);
+        a.scales[j] = scales_out[j];
+        a.sig[j] = signals[j];
+    }
+    a.gamma = static_cast<const uint4*>(gamma);
+    a.world = world;
+    a.rank0 = rank;
+    a.blocks = l.blocks;
+    a.two_shot = l.two_shot;
+    a.rows = rows;
+    a.rows_per_rank = mine;
+    a.vecs = (int)(cols / 8);
+    a.cluster = l.cluster;
+    a.slice_vecs = (int)((cols / 8 + l.cluster - 1) / l.cluster);
+    a.cols_f = (float)cols;
+    a.eps = eps;
+    a.weight_offset = weight_offset;
+    a.scale_ub = scale_ub;
+    a.epoch = epoch;
+    a.timeout_ns = timeout_ns != 0 ? timeout_ns : kArDefaultTimeoutNs;
+    a.err = err;
+    if (!take_injected_failure(&e)) e = launch_allreduce(a, l, (cudaStream_t)stream);
+    return e == cudaSuccess ? RRF_OK : cuda_fail(e);
+}
+
+extern "C" rrf_status rrf_plan_allreduce(int world, int64_t rows, int64_t cols, int residual,
+                                         int mode, int sm_count, int* mode_out,
+                                         int* cluster_size, int* block_threads,
+                                         int* vecs_per_thread) {
+    if (!mode_out || !cluster_size || !block_threads || !vecs_per_thread) return RRF_ERR_NULL;
+    ArLaunch l = {};
+    rrf_status st = plan_allreduce(world, rows, cols, residual != 0, mode, sm_count, &l);
+    if (st != RRF_OK) return st;
+    *mode_out = l.two_shot ? RRF_AR_TWO_SHOT : RRF_AR_ONE_SHOT;
+    *cluster_size = l.cluster;
+    *block_threads = l.threads;
+    *vecs_per_thread = l.vecs_per_thread;
+    return RRF_OK;
+}
+
 extern "C" rrf_status rrf_plan_fused(int num_inputs, int64_t rows, int64_t cols, int residual,
                                      int sm_count, int* cluster_size, int* block_threads,
                                      int* vecs_per_thread) {

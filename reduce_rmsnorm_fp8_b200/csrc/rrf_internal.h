@@ -60,6 +60,49 @@ struct PostArgs {
     float scale_ub;
 };
 
+// The multi-GPU form (rrf_allreduce.cu).  Pointer arrays are indexed by rank
+// and hold each rank's buffer as this GPU addresses it (a peer mapping, or,
+// with several ranks in one launch, another buffer of this GPU).
+struct ArArgs {
+    const uint4* in[RRF_AR_MAX_WORLD];      // partials [rows, cols]
+    const uint4* res_in[RRF_AR_MAX_WORLD];  // residuals, or null
+    uint4* res_out[RRF_AR_MAX_WORLD];
+    uint2* q[RRF_AR_MAX_WORLD];             // codes [rows, cols]
+    float* scales[RRF_AR_MAX_WORLD];        // [rows]
+    unsigned int* sig[RRF_AR_MAX_WORLD];    // signal pads
+    const uint4* gamma;
+    int world;
+    int rank0;             // first rank this launch runs
+    int blocks;            // blocks per rank (G, a multiple of the cluster size)
+    int two_shot;
+    int64_t rows;
+    int64_t rows_per_rank; // two-shot: ceil(rows / world)
+    int vecs;
+    int slice_vecs;
+    int cluster;
+    float cols_f;
+    float eps;
+    float weight_offset;
+    float scale_ub;
+    unsigned int epoch;
+    unsigned long long timeout_ns;
+    unsigned int* err;
+};
+
+struct ArLaunch {
+    int two_shot;
+    int cluster;          // blocks per row (1, 2, 4 or 8)
+    int threads;
+    int vecs_per_thread;  // 1, 2 or 4
+    int blocks;           // per rank
+    int local_ranks;      // ranks in one launch
+    bool residual;
+};
+
+// Largest block of the multi-GPU kernel (RRF_AR_MAX_WORLD loads in flight
+// and up to 4 vectors per thread fit the register budget of 512 threads).
+constexpr int kArMaxThreads = 512;
+
 struct FusedLaunch {
     int cluster;          // blocks per row
     int threads;          // threads per block
@@ -100,6 +143,11 @@ cudaError_t launch_fused(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
                          bool residual, cudaStream_t stream);
 
 cudaError_t launch_post(const PostArgs& a, int sm_count, bool pdl, cudaStream_t stream);
+
+cudaError_t launch_allreduce(const ArArgs& a, const ArLaunch& l, cudaStream_t stream);
+// Blocks of the launch shape `l` that can be resident on the current device
+// at once (the occupancy query; nothing is launched).
+cudaError_t allreduce_resident_blocks(const ArLaunch& l, int* resident);
 
 // The launch shape the library picks (pure host arithmetic).
 rrf_status plan_fused(int R, int64_t rows, int64_t cols, int sm_count, bool residual,

@@ -82,8 +82,14 @@ def select_rows(gpu: dict, rows) -> dict:
     return out
 
 
-def assert_fused_parity(gpu: dict, ref: dict, label: str = "") -> dict:
-    """Compare one call's outputs; returns a summary of the comparison."""
+def assert_fused_parity(gpu: dict, ref: dict, label: str = "", cap_at_ties: bool = False) -> dict:
+    """Compare one call's outputs; returns a summary of the comparison.
+
+    cap_at_ties: for problems outside the workloads' own input counts, where
+    the bf16 inputs can put many y / scale values exactly on an e4m3 midpoint
+    (ratios of short-mantissa products), the cap on differing codes is the
+    larger of 0.1% and the number of oracle values within 1e-6 of a midpoint;
+    every differing code must still sit at a midpoint and differ by one step."""
     if "res_out" in ref:
         assert np.array_equal(gpu["res_out"], ref["res_out"]), f"{label}: residual_out differs"
     rel = np.abs(gpu["scales"].astype(np.float64) - ref["scales"]) / ref["scales"]
@@ -92,8 +98,11 @@ def assert_fused_parity(gpu: dict, ref: dict, label: str = "") -> dict:
     diff = qg != qr
     n_diff = int(diff.sum())
     if n_diff:
-        assert n_diff <= CODE_MISMATCH_FRACTION * qr.size, f"{label}: {n_diff} codes differ"
         near = midpoint_distance(ref["v"]) <= CODE_MIDPOINT_RTOL
+        cap = CODE_MISMATCH_FRACTION * qr.size
+        if cap_at_ties:
+            cap = max(cap, int(near.sum()))
+        assert n_diff <= cap, f"{label}: {n_diff} codes differ"
         assert near[diff].all(), f"{label}: a code differs away from a rounding midpoint"
         same_sign = (qg[diff] & 0x80) == (qr[diff] & 0x80)
         step = np.abs((qg[diff] & 0x7F).astype(int) - (qr[diff] & 0x7F).astype(int))

@@ -57,9 +57,17 @@ def test_constants_match_header(rrf):
     assert rrf.RRF_MAX_COLS == eval(expr)
     for name in ("RRF_VARIANT_AUTO", "RRF_VARIANT_ROW", "RRF_VARIANT_CLUSTER",
                  "RRF_FLAG_NO_PDL", "RRF_FLAG_BARRIER_EXCHANGE",
-                 "RRF_FLAG_DEBUG_STARVE_EXCHANGE", "RRF_DEVICE_ERROR_EXCHANGE_TIMEOUT"):
+                 "RRF_FLAG_DEBUG_STARVE_EXCHANGE", "RRF_DEVICE_ERROR_EXCHANGE_TIMEOUT",
+                 "RRF_DEVICE_ERROR_PEER_TIMEOUT", "RRF_AR_MAX_WORLD", "RRF_AR_MAX_BLOCKS",
+                 "RRF_AR_AUTO", "RRF_AR_ONE_SHOT", "RRF_AR_TWO_SHOT", "RRF_MAX_SHARDS"):
         assert getattr(rrf, name) == int(
             re.search(rf"#define {name} (0x[0-9a-fA-F]+|\d+)u?", text).group(1), 0)
+    expr = re.search(r"#define RRF_AR_SIGNAL_WORDS \(([^)]*)\)", text).group(1)
+    assert rrf.RRF_AR_SIGNAL_WORDS == eval(expr, {"RRF_AR_MAX_WORLD": rrf.RRF_AR_MAX_WORLD,
+                                                  "RRF_AR_MAX_BLOCKS": rrf.RRF_AR_MAX_BLOCKS})
+    from reduce_rmsnorm_fp8_b200 import allreduce
+    assert (allreduce.RRF_AR_SIGNAL_WORDS, allreduce.RRF_AR_MAX_WORLD, allreduce.RRF_AR_AUTO) == \
+        (rrf.RRF_AR_SIGNAL_WORDS, rrf.RRF_AR_MAX_WORLD, rrf.RRF_AR_AUTO)
     for st in rrf.Status:
         assert re.search(rf"RRF_{st.name} = {int(st)}\b", text), st
 
@@ -260,3 +268,117 @@ def test_post_validation(rrf):
         kw = dict(ok)
         kw.update(change)
         assert rrf.rrf_check_post_args(**kw) == rrf.Status[status], change
+
+
+def _ar_ok(world=4, residual=True):
+    """Valid fake arguments of the multi-GPU call: rank j's buffers at
+    distinct aligned addresses (rows 8, cols 64)."""
+    at = lambda k: [(k * 16 + j) * A for j in range(world)]
+    return dict(inputs=at(1), residual_in=at(2) if residual else None,
+                residual_out=at(3) if residual else None, q_out=at(4), scales_out=at(5),
+                signals=at(6), rank=0, local_ranks=1, rows=8, cols=64, gamma=A // 2, eps=1e-5,
+                weight_offset=0.0, scale_ub=1200.0, epoch=1, mode=0)
+
+
+def test_allreduce_validation_accepts_valid(rrf):
+    for world in (1, 2, 8):
+        for res in (True, False):
+            assert rrf.rrf_check_allreduce_args(**_ar_ok(world, res)) == rrf.Status.OK
+    ok = _ar_ok()
+    assert rrf.rrf_check_allreduce_args(**dict(ok, local_ranks=4)) == rrf.Status.OK
+    assert rrf.rrf_check_allreduce_args(**dict(ok, rank=3)) == rrf.Status.OK
+    in_place = dict(ok, residual_out=ok["residual_in"])
+    assert rrf.rrf_check_allreduce_args(**in_place) == rrf.Status.OK
+    # rows == 0 is a no-op that looks at no pointer
+    empty = {k: (None if isinstance(v, list) else v) for k, v in ok.items()}
+    assert rrf.rrf_check_allreduce_args(**dict(empty, rows=0, gamma=0), world=4) == \
+        rrf.Status.OK
+
+
+def _swap(lst, j, value):
+    out = list(lst)
+    out[j] = value
+    return out
+
+
+@pytest.mark.parametrize("change,status", [
+    (lambda o: dict(o, rank=4), "ERR_RANKS"),
+    (lambda o: dict(o, rank=-1), "ERR_RANKS"),
+    (lambda o: dict(o, rank=1, local_ranks=4), "ERR_RANKS"),
+    (lambda o: dict(o, local_ranks=2), "ERR_UNSUPPORTED"),
+    (lambda o: dict(o, mode=3), "ERR_UNSUPPORTED"),
+    (lambda o: dict(o, epoch=0), "ERR_VALUE"),
+    (lambda o: dict(o, eps=-1.0), "ERR_VALUE"),
+    (lambda o: dict(o, scale_ub=float("nan")), "ERR_VALUE"),
+    (lambda o: dict(o, cols=60), "ERR_SHAPE"),
+    (lambda o: dict(o, cols=8 * 8 * 512 * 4 + 8), "ERR_SHAPE"),
+    (lambda o: dict(o, rows=-1), "ERR_SHAPE"),
+    (lambda o: dict(o, gamma=0), "ERR_NULL"),
+    (lambda o: dict(o, residual_out=None), "ERR_NULL"),
+    (lambda o: dict(o, q_out=_swap(o["q_out"], 2, 0)), "ERR_NULL"),
+    (lambda o: dict(o, signals=_swap(o["signals"], 3, 0)), "ERR_NULL"),
+    (lambda o: dict(o, inputs=_swap(o["inputs"], 1, o["inputs"][1] + 8)), "ERR_ALIGN"),
+    (lambda o: dict(o, scales_out=_swap(o["scales_out"], 1, o["scales_out"][1] + 2)),
+     "ERR_ALIGN"),
+    (lambda o: dict(o, signals=_swap(o["signals"], 0, o["signals"][0] + 4)), "ERR_ALIGN"),
+    # a rank's codes over another rank's partial
+    (lambda o: dict(o, q_out=_swap(o["q_out"], 2, o["inputs"][0] + 64)), "ERR_ALIAS"),
+    # two ranks' scales in one buffer
+    (lambda o: dict(o, scales_out=_swap(o["scales_out"], 1, o["scales_out"][0])), "ERR_ALIAS"),
+    # a pad over another rank's residual
+    (lambda o: dict(o, signals=_swap(o["signals"], 1, o["residual_out"][2])), "ERR_ALIAS"),
+    # an in-place residual that serves another rank's input
+    (lambda o: dict(o, residual_out=_swap(o["residual_out"], 1, o["residual_in"][2])),
+     "ERR_ALIAS"),
+])
+def test_allreduce_validation_rejects(rrf, change, status):
+    assert rrf.rrf_check_allreduce_args(**change(_ar_ok())) == rrf.Status[status]
+
+
+def test_allreduce_world_bounds(rrf):
+    ok = _ar_ok(8)
+    assert rrf.rrf_check_allreduce_args(**ok, world=9) == rrf.Status.ERR_RANKS
+    assert rrf.rrf_check_allreduce_args(**ok, world=0) == rrf.Status.ERR_RANKS
+
+
+@pytest.mark.parametrize("world,rows,cols,res,mode,want", [
+    (8, 64, 7168, True, 0, (2, 8, 128, 1)),     # 8 rows per rank, rows split in clusters of 8
+    (8, 1, 7168, True, 0, (1, 8, 128, 1)),      # fewer rows than ranks: one-shot
+    (8, 8192, 8192, True, 0, (2, 1, 512, 2)),   # prefill: 1024 rows per rank, a block per row
+    (4, 37, 7168, True, 0, (2, 8, 128, 1)),
+    (8, 64, 7168, True, 1, (1, 8, 128, 1)),     # forced one-shot: 64 rows per rank
+    (2, 4, 256, False, 0, (2, 1, 32, 1)),       # short rows: one block of one warp
+    (8, 16, 131072, False, 2, (2, 8, 512, 4)),  # the widest row
+])
+def test_allreduce_plan(rrf, world, rows, cols, res, mode, want):
+    assert rrf.rrf_plan_allreduce(world, rows, cols, 148, res, mode) == want
+
+
+def test_allreduce_plan_rejects(rrf):
+    with pytest.raises(rrf.RrfError) as e:
+        rrf.rrf_plan_allreduce(9, 8, 64, 148)
+    assert e.value.status == rrf.Status.ERR_RANKS
+    with pytest.raises(rrf.RrfError) as e:
+        rrf.rrf_plan_allreduce(8, 8, 131072 + 8, 148)
+    assert e.value.status == rrf.Status.ERR_SHAPE
+
+
+def test_two_shot_rows_tile_the_batch():
+    from reduce_rmsnorm_fp8_b200 import allreduce
+    for rows in (0, 1, 7, 37, 64, 8192):
+        for world in (1, 2, 3, 8):
+            spans = [allreduce.two_shot_rows(rows, world, k) for k in range(world)]
+            assert spans[0][0] == 0 and spans[-1][1] == rows
+            assert all(a[1] == b[0] for a, b in zip(spans, spans[1:]))
+            assert all(b - a <= -(-rows // world) for a, b in spans)
+
+
+def test_peer_layout_is_aligned_and_disjoint():
+    from reduce_rmsnorm_fp8_b200 import allreduce
+    for res in (True, False):
+        regions, total = allreduce.peer_layout(37, 7168, res)
+        spans = sorted(regions.values())
+        assert all(off % 256 == 0 for off, _ in spans)
+        assert all(a[0] + a[1] <= b[0] for a, b in zip(spans, spans[1:]))
+        assert spans[-1][0] + spans[-1][1] <= total
+        assert ("residual" in regions) == res

@@ -92,3 +92,64 @@ def test_weak_scaling_value_formula():
         __import__("workloads").fused_bytes(8, r, 7168, True) for r in (1, 8, 32, 64))
     value = world * per_step * steps / t / 1e9
     assert value == pytest.approx(4 * 15863204 * 100 / 2e-3 / 1e9)
+
+
+def _two_shot_worker(rank, world, port, out_dir):
+    """The two-shot data flow of the multi-GPU call with gloo as the
+    transport: rank k holds partial k only; it fetches the partials of its
+    row block from every rank (an all-gather here, peer loads on GPUs),
+    computes those rows, and every rank gathers all blocks' codes, scales and
+    residual rows."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import oracle
+    import workloads
+    from reduce_rmsnorm_fp8_b200.allreduce import two_shot_rows
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    try:
+        c = workloads.make_case("odd", 37, R=world)
+        bits = workloads.bits
+        mine = torch.from_numpy(bits(c.inputs[rank]).view(np.uint8).copy())  # bytes: gloo has no 16-bit ints
+        parts = [torch.empty_like(mine) for _ in range(world)]
+        dist.all_gather(parts, mine)
+        start, stop = two_shot_rows(c.rows, world, rank)
+        per = -(-c.rows // world)
+        blk = oracle.sum_rmsnorm_fp8([p.numpy().view(np.uint16) for p in parts], c.rows, c.cols,
+                                     bits(c.gamma), c.eps, c.weight_offset, c.scale_ub,
+                                     residual=bits(c.residual), row_start=start,
+                                     row_count=stop - start)
+        gathered = {}
+        for key, width in (("q", c.cols), ("res_out", c.cols), ("scales", 1)):
+            pad = np.zeros((per, width), dtype=blk[key].dtype)
+            pad[:stop - start] = blk[key].reshape(stop - start, width)
+            t = torch.from_numpy(pad.view(np.uint8).copy())
+            out = [torch.empty_like(t) for _ in range(world)]
+            dist.all_gather(out, t)
+            whole = np.concatenate([o.numpy().view(blk[key].dtype).reshape(per, width)
+                                    for o in out])[:c.rows]
+            gathered[key] = whole.reshape((c.rows,) + blk[key].shape[1:])
+        np.savez(os.path.join(out_dir, f"ts{rank}.npz"), **gathered)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_shot_flow_on_gloo(tmp_path):
+    world, port = 2, free_port()
+    mp.start_processes(_two_shot_worker, args=(world, port, str(tmp_path)), nprocs=world,
+                       start_method="spawn", join=True)
+    import oracle
+    import workloads
+    c = workloads.make_case("odd", 37, R=world)
+    bits = workloads.bits
+    whole = oracle.sum_rmsnorm_fp8([bits(x) for x in c.inputs], c.rows, c.cols, bits(c.gamma),
+                                   c.eps, c.weight_offset, c.scale_ub,
+                                   residual=bits(c.residual))
+    for r in range(world):
+        got = np.load(tmp_path / f"ts{r}.npz")
+        for key in ("q", "scales", "res_out"):
+            assert np.array_equal(got[key], whole[key]), (r, key)
