@@ -82,6 +82,10 @@ class Oracle:
         lib.oracle_sum_rmsnorm_fp8_rows.argtypes = [
             ctypes.POINTER(u16p), ctypes.c_int, i64, i64, i64, vp, vp, vp,
             ctypes.c_float, ctypes.c_float, ctypes.c_float, vp, vp, vp, vp]
+        lib.oracle_bf16_round_double.restype = ctypes.c_uint16
+        lib.oracle_bf16_round_double.argtypes = [ctypes.c_double]
+        lib.oracle_scaled_mm.restype = None
+        lib.oracle_scaled_mm.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp, vp]
         self.lib = lib
         self.path = lib_path
 
@@ -163,6 +167,33 @@ class Oracle:
         return out
 
 
+    def bf16_round_double(self, values) -> np.ndarray:
+        """float64 -> nearest bf16 (ties to even) in one rounding, as uint16."""
+        v = np.asarray(values, dtype=np.float64)
+        return np.array([self.lib.oracle_bf16_round_double(float(x)) for x in v.ravel()],
+                        dtype=np.uint16).reshape(v.shape)
+
+    def scaled_mm(self, a, a_scale, b, b_scale, bias=None, exact: bool = False):
+        """The FP8 GEMM: a uint8 e4m3fn codes [M, K], b [N, K], scales float32
+        [M] and [N], bias bf16 bits [N] or None.  Returns out (bf16 bits
+        [M, N]) and, with ``exact``, also the float64 values before the
+        rounding."""
+        a = np.ascontiguousarray(a, dtype=np.uint8)
+        b = np.ascontiguousarray(b, dtype=np.uint8)
+        M, K = a.shape
+        N = b.shape[0]
+        if b.shape[1] != K:
+            raise ValueError("a and b need the same K")
+        sa = np.ascontiguousarray(a_scale, dtype=np.float32).reshape(M)
+        sb = np.ascontiguousarray(b_scale, dtype=np.float32).reshape(N)
+        bi = None if bias is None else np.ascontiguousarray(bias, dtype=np.uint16).reshape(N)
+        out = np.empty((M, N), dtype=np.uint16)
+        ex = np.empty((M, N), dtype=np.float64) if exact else None
+        self.lib.oracle_scaled_mm(_ptr(a), _ptr(sa), _ptr(b), _ptr(sb), _ptr(bi), M, N, K,
+                                  _ptr(out), _ptr(ex))
+        return (out, ex) if exact else out
+
+
 def default() -> Oracle:
     """The oracle built from ``rrf_oracle.c`` (compiled on first use)."""
     global _default
@@ -190,3 +221,11 @@ def sum_bf16(inputs, rows, cols):
 
 def sum_rmsnorm_fp8(*args, **kwargs):
     return default().sum_rmsnorm_fp8(*args, **kwargs)
+
+
+def bf16_round_double(values):
+    return default().bf16_round_double(values)
+
+
+def scaled_mm(*args, **kwargs):
+    return default().scaled_mm(*args, **kwargs)

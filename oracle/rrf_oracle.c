@@ -44,6 +44,12 @@
  *
  * Build with -ffp-contract=off (no FMA contraction) and without fast-math, so
  * every fp32 operation above is one IEEE-rounded operation.
+ *
+ * The FP8 GEMM that consumes the per-row scales (oracle_scaled_mm, at the
+ * end) follows the Huawei Ascend aclnnAlltoAllQuantMatmul page, the formula
+ * of its per-token dynamic quantisation scenario: out = (x1_q @ x2) *
+ * x1Scale * x2Scale + bias, one x1Scale per row of x1 and one x2Scale per
+ * output column.
  */
 #include <math.h>
 #include <stddef.h>
@@ -219,4 +225,56 @@ void oracle_sum_rmsnorm_fp8(const uint16_t* const* x, int R, int64_t rows, int64
                             float scale_ub, uint8_t* q, float* scales) {
     oracle_sum_rmsnorm_fp8_rows(x, R, 0, rows, cols, res_in, res_out, gamma, eps,
                                 weight_offset, scale_ub, q, scales, NULL, NULL);
+}
+
+/* ------------------------------------------------------- the FP8 GEMM --- */
+
+/* Round a float64 value to the nearest bf16 (ties to the even encoding),
+ * without passing through fp32 (which would round twice).  bf16 holds 8
+ * significant bits; below 2^-126 the spacing stays 2^-133 (subnormals).
+ * Magnitudes that round to 2^128 or beyond become infinity. */
+uint16_t oracle_bf16_round_double(double x) {
+    if (isnan(x)) return 0x7FC0;
+    uint16_t sign = signbit(x) ? 0x8000 : 0x0000;
+    double a = fabs(x);
+    if (a == 0.0) return sign;
+    int e;
+    frexp(a, &e); /* a = f * 2^e, 0.5 <= f < 1 */
+    int q_exp = e - 8; /* spacing of the 8-bit significands in [2^(e-1), 2^e) */
+    if (q_exp < -133) q_exp = -133;
+    double quantum = ldexp(1.0, q_exp);
+    double k = floor(a / quantum); /* a / quantum is exact: a power-of-two scaling */
+    double lo = k * quantum, hi = (k + 1.0) * quantum;
+    double pick;
+    if (a - lo < hi - a) pick = lo;
+    else if (hi - a < a - lo) pick = hi;
+    else pick = (fmod(k, 2.0) == 0.0) ? lo : hi;
+    if (pick >= ldexp(1.0, 128)) return (uint16_t)(sign | 0x7F80);
+    float f = (float)pick; /* exact: 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(sign | ((u >> 16) & 0x7FFF));
+}
+
+/* out[m][n] = RN_bf16(S * a_scale[m] * b_scale[n] + bias[n]) with
+ * S = sum_k e4m3(a[m][k]) * e4m3(b[n][k]).  a is [M, K] and b is [N, K], both
+ * row-major e4m3fn codes; bias (bf16 [N]) may be NULL.  Everything is float64:
+ * each product of two e4m3 values is an integer multiple of 2^-18 below
+ * 2^18, so for K below 2^17 the sum S is exact; the scaling and the bias add
+ * two float64 roundings (relative 2^-53) before the one rounding to bf16.
+ * exact (may be NULL) receives that float64 value. */
+void oracle_scaled_mm(const uint8_t* a, const float* a_scale, const uint8_t* b,
+                      const float* b_scale, const uint16_t* bias, int64_t M, int64_t N,
+                      int64_t K, uint16_t* out, double* exact) {
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double S = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                S += oracle_e4m3_decode(a[m * K + k]) * oracle_e4m3_decode(b[n * K + k]);
+            double y = S * (double)a_scale[m] * (double)b_scale[n];
+            if (bias != NULL) y += (double)oracle_bf16_to_float(bias[n]);
+            if (exact != NULL) exact[m * N + n] = y;
+            out[m * N + n] = oracle_bf16_round_double(y);
+        }
+    }
 }

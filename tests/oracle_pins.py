@@ -471,4 +471,130 @@ def pin_row_independence(o):
         assert np.array_equal(whole[k], np.concatenate([p[k] for p in parts])), k
 
 
+# --------------------------------------------------------------- FP8 GEMM ---
+# The consumer of the per-row scales (Ascend aclnnAlltoAllQuantMatmul,
+# per-token dynamic quantisation): out = RN_bf16((a_q @ b_q^T) * a_scale *
+# b_scale + bias).
+
+def _bf16_table():
+    """Every finite non-negative bf16 value, ascending, and its bit pattern."""
+    bits = np.arange(0, 0x7F80, dtype=np.uint16)
+    return f32(bits).astype(np.float64), bits
+
+
+def brute_bf16_round_double(values) -> np.ndarray:
+    """Nearest bf16 of float64 values by search in the table of all finite
+    bf16 values; ties to the even pattern; beyond the midpoint between the
+    largest finite value and 2^128, infinity."""
+    vals, bits = _bf16_table()
+    top = np.append(vals, 2.0 ** 128)
+    v = np.asarray(values, dtype=np.float64).reshape(-1)
+    out = np.empty(v.size, dtype=np.uint16)
+    for i, x in enumerate(v):
+        a = abs(x)
+        j = int(np.searchsorted(top, a, side="right")) - 1  # top[j] <= a < top[j + 1]
+        lo, hi = top[j], top[min(j + 1, len(top) - 1)]
+        if a - lo < hi - a or a == lo:
+            k = j
+        elif hi - a < a - lo:
+            k = j + 1
+        else:
+            k = j if j % 2 == 0 else j + 1
+        b = 0x7F80 if k >= len(vals) else int(bits[k])
+        out[i] = b | (0x8000 if math.copysign(1.0, x) < 0 else 0)
+    return out.reshape(np.shape(values))
+
+
+def rand_e4m3(seed: int, shape, std: float = 1.0) -> np.ndarray:
+    """e4m3fn codes of normal samples (torch's conversion, clamped)."""
+    rng = np.random.default_rng(seed)
+    return lib_e4m3_torch(rng.normal(0.0, std, size=shape).astype(np.float32))
+
+
+def pin_bf16_round_double_brute_force(o):
+    rng = np.random.default_rng(31)
+    x = np.concatenate([
+        rng.normal(0, 1, 400) * np.exp2(rng.integers(-140, 128, 400)),
+        # exact midpoints (ties), and one float64 ulp either side of them
+        (np.arange(256, 512) + 0.5) * 2.0 ** -8,
+        np.nextafter((np.arange(256, 320) + 0.5) * 2.0 ** -8, np.inf),
+        np.nextafter((np.arange(256, 320) + 0.5) * 2.0 ** -8, -np.inf),
+        [0.0, -0.0, 2.0 ** -134, 2.0 ** -133 * 1.5, 3.3895313892515355e38,
+         2.0 ** 128 - 2.0 ** 119, np.nextafter(2.0 ** 128 - 2.0 ** 119, 0), 1e300]])
+    x = np.concatenate([x, -x])
+    assert np.array_equal(o.bf16_round_double(x), brute_bf16_round_double(x))
+
+
+def pin_bf16_round_double_agrees_on_floats(o):
+    """On values that are fp32 numbers the one rounding equals the pinned
+    float32 rounding (torch's)."""
+    rng = np.random.default_rng(32)
+    v = (rng.normal(0, 1, 2000) * np.exp2(rng.integers(-100, 100, 2000))).astype(np.float32)
+    assert np.array_equal(o.bf16_round_double(v.astype(np.float64)), lib_bf16(v))
+
+
+def pin_scaled_mm_vs_float64_matmul(o):
+    """Sum, scales and bias against numpy's float64 matmul of the codes'
+    values (ml_dtypes' decoding); the sum of exact products is exact, so the
+    float64 values agree bit for bit."""
+    M, N, K = 5, 7, 96
+    a, b = rand_e4m3(33, (M, K), 2.0), rand_e4m3(34, (N, K), 0.5)
+    rng = np.random.default_rng(35)
+    sa = rng.uniform(0.5, 2.0, M).astype(np.float32)
+    sb = rng.uniform(0.01, 0.1, N).astype(np.float32)
+    bias = lib_bf16(rng.normal(0, 1, N).astype(np.float32))
+    S = lib_e4m3_decode(a) @ lib_e4m3_decode(b).T
+    want = S * sa.astype(np.float64)[:, None] * sb.astype(np.float64)[None, :] + \
+        f32(bias).astype(np.float64)[None, :]
+    out, ex = o.scaled_mm(a, sa, b, sb, bias, exact=True)
+    assert np.array_equal(ex, want)
+    assert np.array_equal(out, brute_bf16_round_double(want))
+    out0 = o.scaled_mm(a, sa, b, sb, None)
+    assert np.array_equal(out0, brute_bf16_round_double(want - f32(bias)[None, :]))
+
+
+def pin_scaled_mm_closed_forms(o):
+    """All-ones codes give K * a_scale * b_scale; negating a row of a
+    negates that row of the output; zero codes give +0."""
+    M, N, K = 3, 4, 160
+    ones = np.full((M, K), 0x38, np.uint8)  # e4m3fn 1.0
+    sa = np.array([1.0, 0.5, 3.0], np.float32)
+    sb = np.array([1.0, 2.0, 0.25, 0.125], np.float32)
+    out, ex = o.scaled_mm(ones, sa, np.full((N, K), 0x38, np.uint8), sb, exact=True)
+    assert np.array_equal(ex, K * sa[:, None].astype(np.float64) * sb[None, :])
+    a, b = rand_e4m3(36, (M, K)), rand_e4m3(37, (N, K))
+    pos = o.scaled_mm(a, sa, b, sb)
+    neg_a = a.copy()
+    neg_a[1] ^= 0x80
+    neg = o.scaled_mm(neg_a, sa, b, sb)
+    assert np.array_equal(neg[0], pos[0]) and np.array_equal(neg[2], pos[2])
+    nz = pos[1] & 0x7FFF != 0
+    assert np.array_equal(neg[1][nz], pos[1][nz] ^ 0x8000)
+    zero = o.scaled_mm(np.zeros((M, K), np.uint8), sa, b, sb)
+    assert np.all(zero == 0)
+
+
+def pin_scaled_mm_rounds_once(o):
+    """y = 1 * 1 * (1 + 2^-8) + 2^-40: just above the bf16 midpoint between 1
+    and 1 + 2^-7, so one rounding gives 1 + 2^-7 (0x3F81); rounding to fp32
+    first would land on the midpoint and then tie to 1.0 (0x3F80)."""
+    one = np.full((1, 16), 0, np.uint8)
+    one[0, 0] = 0x38
+    sb = np.array([1.0 + 2.0 ** -8], np.float32)
+    up = o.scaled_mm(one, np.ones(1, np.float32), one, sb, bf16_of([2.0 ** -40]))
+    down = o.scaled_mm(one, np.ones(1, np.float32), one, sb, bf16_of([-2.0 ** -40]))
+    assert up[0, 0] == 0x3F81 and down[0, 0] == 0x3F80
+
+
+def pin_scaled_mm_k_split(o):
+    """The sum over K is the sum of the sums over two halves (exactly)."""
+    M, N, K = 4, 5, 256
+    a, b = rand_e4m3(38, (M, K), 3.0), rand_e4m3(39, (N, K), 3.0)
+    one_m, one_n = np.ones(M, np.float32), np.ones(N, np.float32)
+    _, whole = o.scaled_mm(a, one_m, b, one_n, exact=True)
+    _, lo = o.scaled_mm(a[:, :100], one_m, b[:, :100], one_n, exact=True)
+    _, hi = o.scaled_mm(a[:, 100:], one_m, b[:, 100:], one_n, exact=True)
+    assert np.array_equal(whole, lo + hi)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

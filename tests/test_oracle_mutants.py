@@ -48,6 +48,18 @@ MUTANTS = [
      "ldexp((double)(8 + m), e - 11)"),
     ("bf16 ties away from zero", "return (lo & 1) ? hi : lo;", "return hi;"),
     ("bf16 truncation", "if (dhi < dlo) return hi;", "if (0) return hi;"),
+    ("GEMM last k dropped", "for (int64_t k = 0; k < K; ++k)\n                S +=",
+     "for (int64_t k = 0; k < K - 1; ++k)\n                S +="),
+    ("GEMM b read transposed", "oracle_e4m3_decode(b[n * K + k])",
+     "oracle_e4m3_decode(b[(k * N + n) % (N * K)])"),
+    ("GEMM one scale for all rows", "S * (double)a_scale[m] * (double)b_scale[n]",
+     "S * (double)a_scale[0] * (double)b_scale[n]"),
+    ("GEMM bias dropped", "if (bias != NULL) y += (double)oracle_bf16_to_float(bias[n]);", ""),
+    ("GEMM rounds through fp32", "out[m * N + n] = oracle_bf16_round_double(y);",
+     "out[m * N + n] = oracle_bf16_round((float)y);"),
+    ("double rounding ties up", "pick = (fmod(k, 2.0) == 0.0) ? lo : hi;", "pick = hi;"),
+    ("double rounding truncates", "else if (hi - a < a - lo) pick = hi;", "else if (0) pick = hi;"),
+    ("double rounding 7 significant bits", "int q_exp = e - 8;", "int q_exp = e - 7;"),
 ]
 
 
