@@ -350,6 +350,45 @@ rrf_status rrf_plan_allreduce(int world, int64_t rows, int64_t cols, int residua
                               int sm_count, int* mode_out, int* cluster_size,
                               int* block_threads, int* vecs_per_thread);
 
+/* ------------------------------------------------------------------------
+ * A consumer of the per-row scales: the FP8 GEMM that follows the
+ * quantisation in a transformer layer.
+ *
+ * Ascend CANN docs, aclnnAlltoAllQuantMatmul (the formulas of its K-C and
+ * per-token dynamic quantisation scenarios): after the activations x1 are
+ * quantised per token (row) with scale x1Scale, the product is
+ * out = (x1_q @ x2) * x1Scale * x2Scale (+ bias), x2Scale one per output
+ * column.  Here x1_q and x1Scale are exactly the codes and scales that
+ * rrf_sum_rmsnorm_fp8 writes, and x2 is a weight stored like a linear
+ * layer's, one row of K codes per output column:
+ *
+ *   out[m][n] = RN_bf16( (sum_k e4m3(a[m][k]) * e4m3(b[n][k])) * a_scale[m]
+ *                        * b_scale[n] + bias[n] )
+ *
+ * The products of two e4m3 values are exact; the tensor cores sum them in
+ * fp32 (in an order of their own), then the epilogue multiplies by the two
+ * scales, adds bias and rounds once to bf16.
+ * ---------------------------------------------------------------------- */
+
+/* rrf_scaled_mm_fp8 -- the GEMM above on the tensor cores (sm_100a).
+ * a         e4m3fn codes [M, K] row-major (K contiguous), 16-byte aligned
+ * a_scale   float [M] (per row: rrf_sum_rmsnorm_fp8's scales_out), 4-byte aligned
+ * b         e4m3fn codes [N, K] row-major (K contiguous), 16-byte aligned
+ * b_scale   float [N] (per output column), 4-byte aligned
+ * bias      bf16 [N] or NULL, 2-byte aligned
+ * out       bf16 [M, N] row-major, 16-byte aligned
+ * M, N, K   M >= 0 (M == 0 is a no-op); N, K >= 16 and multiples of 16
+ * Errors: RRF_ERR_NULL, RRF_ERR_SHAPE, RRF_ERR_ALIGN, RRF_ERR_ALIAS (out
+ *         overlapping an operand), RRF_ERR_CUDA. */
+rrf_status rrf_scaled_mm_fp8(const void* a, const float* a_scale, const void* b,
+                             const float* b_scale, const void* bias, void* out, int64_t M,
+                             int64_t N, int64_t K, rrf_stream_t stream);
+
+/* The host validation of rrf_scaled_mm_fp8 alone (no GPU needed). */
+rrf_status rrf_check_scaled_mm_args(const void* a, const float* a_scale, const void* b,
+                                    const float* b_scale, const void* bias, const void* out,
+                                    int64_t M, int64_t N, int64_t K);
+
 /* rrf_plan_fused -- the launch rrf_sum_rmsnorm_fp8 would use on a GPU with
  * sm_count SMs for a call with (residual != 0) or without a residual,
  * without touching the GPU.  Writes the cluster size (1 = one
@@ -377,6 +416,8 @@ rrf_status rrf_check_fused_args(const void* const* inputs, int num_inputs, int64
                                                peers' statistics ran out          */
 #define RRF_DEVICE_ERROR_PEER_TIMEOUT 2u /* a multi-GPU barrier wait for a peer
                                             rank ran out                      */
+#define RRF_DEVICE_ERROR_GEMM_TIMEOUT 4u /* a wait of the FP8 GEMM's operand
+                                            pipeline ran out                  */
 
 /* rrf_device_error -- the device error word of the current device: the OR
  * of RRF_DEVICE_ERROR_* bits that kernels of this library have set since it

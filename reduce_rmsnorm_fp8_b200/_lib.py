@@ -25,6 +25,7 @@ RRF_AR_SIGNAL_WORDS = 2 * RRF_AR_MAX_WORLD * RRF_AR_MAX_BLOCKS
 RRF_AR_AUTO = 0
 RRF_AR_ONE_SHOT = 1
 RRF_AR_TWO_SHOT = 2
+RRF_DEVICE_ERROR_GEMM_TIMEOUT = 4
 
 
 class Status(enum.IntEnum):
@@ -103,6 +104,10 @@ lib.rrf_check_allreduce_args.restype = _int
 lib.rrf_check_allreduce_args.argtypes = _ar_args
 lib.rrf_plan_allreduce.restype = _int
 lib.rrf_plan_allreduce.argtypes = [_int, _i64, _i64, _int, _int, _int] + [ctypes.POINTER(_int)] * 4
+lib.rrf_scaled_mm_fp8.restype = _int
+lib.rrf_scaled_mm_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]
+lib.rrf_check_scaled_mm_args.restype = _int
+lib.rrf_check_scaled_mm_args.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64]
 lib.rrf_device_error.restype = _int
 lib.rrf_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), _int]
 lib.rrf_version.restype = ctypes.c_char_p
@@ -375,3 +380,41 @@ def rrf_rmsnorm_fp8_post(h, gamma, stats, total_cols, eps, weight_offset, scale_
             eps, weight_offset, scale_ub, q_out.data_ptr(),
             scales_out.data_ptr() if scales_out is not None else None, _stream(dev)))
     return q_out, scales_out
+
+
+def rrf_check_scaled_mm_args(a, a_scale, b, b_scale, bias, out, M, N, K) -> int:
+    """Host validation of the FP8 GEMM on raw pointers."""
+    return lib.rrf_check_scaled_mm_args(a or None, a_scale or None, b or None, b_scale or None,
+                                        bias or None, out or None, M, N, K)
+
+
+def rrf_scaled_mm_fp8(a, a_scale, b, b_scale, bias=None, out=None):
+    """out = RN_bf16((a @ b^T) * a_scale * b_scale + bias) on the tensor
+    cores.  a: float8_e4m3fn [M, K] (e.g. rrf_sum_rmsnorm_fp8's codes), a_scale
+    float32 [M] or [M, 1] (its scales), b: float8_e4m3fn [N, K] (a weight
+    stored like a linear layer's), b_scale float32 [N], bias bf16 [N] or None.
+    Returns out, bf16 [M, N]."""
+    torch = _torch()
+    for t, name in ((a, "a"), (b, "b")):
+        if t.dtype != torch.float8_e4m3fn or t.dim() != 2 or not t.is_contiguous() or \
+                t.device.type != "cuda":
+            raise ValueError(f"{name} must be a contiguous 2-D float8_e4m3fn CUDA tensor")
+    M, K = a.shape
+    N = b.shape[0]
+    if b.shape[1] != K:
+        raise ValueError("a and b need the same K")
+    dev = a.device
+    for t, n, name in ((a_scale, M, "a_scale"), (b_scale, N, "b_scale")):
+        if t.dtype != torch.float32 or t.numel() != n or not t.is_contiguous() or t.device != dev:
+            raise ValueError(f"{name} must be a contiguous float32 tensor of {n} values")
+    if bias is not None and (bias.dtype != torch.bfloat16 or bias.numel() != N or
+                             bias.device != dev):
+        raise ValueError("bias must be a bf16 tensor of N values")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    with torch.cuda.device(dev):
+        _raise_on(lib.rrf_scaled_mm_fp8(
+            a.data_ptr(), a_scale.data_ptr(), b.data_ptr(), b_scale.data_ptr(),
+            bias.data_ptr() if bias is not None else None, out.data_ptr(), M, N, K,
+            _stream(dev)))
+    return out

@@ -710,6 +710,54 @@ extern "C" rrf_status rrf_plan_allreduce(int world, int64_t rows, int64_t cols, 
     return RRF_OK;
 }
 
+// ---------------------------------------------------------- FP8 GEMM ---
+
+extern "C" rrf_status rrf_check_scaled_mm_args(const void* a, const float* a_scale,
+                                               const void* b, const float* b_scale,
+                                               const void* bias, const void* out, int64_t M,
+                                               int64_t N, int64_t K) {
+    // N and K: multiples of 16 (16-byte rows for the tensor maps and the
+    // stores); M: the grid's second dimension counts 128-row tiles
+    if (M < 0 || N < 16 || K < 16 || N % 16 != 0 || K % 16 != 0) return RRF_ERR_SHAPE;
+    if (M > 65535LL * 128 || N > (int64_t)INT32_MAX / 2 || K > (int64_t)INT32_MAX / 2)
+        return RRF_ERR_SHAPE;
+    if (M == 0) return RRF_OK;
+    if (!a || !a_scale || !b || !b_scale || !out) return RRF_ERR_NULL;
+    if (!aligned(a, 16) || !aligned(b, 16) || !aligned(out, 16) || !aligned(a_scale, 4) ||
+        !aligned(b_scale, 4) || (bias != nullptr && !aligned(bias, 2)))
+        return RRF_ERR_ALIGN;
+    const Range o = range_of(out, M * N * 2);
+    const Range reads[5] = {range_of(a, M * K), range_of(b, N * K), range_of(a_scale, M * 4),
+                            range_of(b_scale, N * 4),
+                            bias != nullptr ? range_of(bias, N * 2) : Range{0, 0}};
+    for (const Range& r : reads)
+        if (overlap(o, r)) return RRF_ERR_ALIAS;
+    return RRF_OK;
+}
+
+extern "C" rrf_status rrf_scaled_mm_fp8(const void* a, const float* a_scale, const void* b,
+                                        const float* b_scale, const void* bias, void* out,
+                                        int64_t M, int64_t N, int64_t K, rrf_stream_t stream) {
+    rrf_status st = rrf_check_scaled_mm_args(a, a_scale, b, b_scale, bias, out, M, N, K);
+    if (st != RRF_OK || M == 0) return st;
+    int sm_count = 0;
+    if ((st = current_sm_count(&sm_count)) != RRF_OK) return st;
+    unsigned int* err = nullptr;
+    if ((st = device_error_word(&err)) != RRF_OK) return st;
+    GemmArgs g = {};
+    g.a_scale = a_scale;
+    g.b_scale = b_scale;
+    g.bias = static_cast<const uint16_t*>(bias);
+    g.out = static_cast<uint16_t*>(out);
+    g.M = (int)M;
+    g.N = (int)N;
+    g.K = (int)K;
+    g.err = err;
+    cudaError_t e;
+    if (!take_injected_failure(&e)) e = launch_scaled_mm(g, a, b, sm_count, (cudaStream_t)stream);
+    return e == cudaSuccess ? RRF_OK : cuda_fail(e);
+}
+
 extern "C" rrf_status rrf_plan_fused(int num_inputs, int64_t rows, int64_t cols, int residual,
                                      int sm_count, int* cluster_size, int* block_threads,
                                      int* vecs_per_thread) {

@@ -1,0 +1,367 @@
+// rrf_gemm.cu -- the FP8 GEMM that consumes the per-row scales:
+//   out[m][n] = RN_bf16((sum_k a[m][k] * b[n][k]) * a_scale[m] * b_scale[n] + bias[n])
+// on the 5th-generation tensor cores (Ascend CANN docs,
+// aclnnAlltoAllQuantMatmul: per-token dynamic quantisation of the
+// activations, then (x1_q @ x2) * x1Scale * x2Scale + bias).
+//
+// One CTA computes a 128 x BN tile of out.  Warp roles:
+//   warp 0   one thread issues the TMA loads of the A (128 x 128 bytes) and
+//            B (BN x 128 bytes) k-tiles into a ring of kStages shared-memory
+//            stages (128-byte swizzle, the layout the MMA descriptors name);
+//   warp 1   allocates the fp32 accumulator in tensor memory (BN columns of
+//            128 lanes) and one thread issues tcgen05.mma (kind::f8f6f4,
+//            M = 128, N = BN, K = 32 per instruction, 4 per k-tile); a
+//            tcgen05.commit per k-tile hands the stage back to the producer;
+//   warps 2-5 the epilogue: tcgen05.ld of its 32 accumulator lanes (rows),
+//            the two scales and bias, one rounding to bf16, 64-byte stores.
+// Every mbarrier wait is bounded in time; a wait that runs out sets
+// RRF_DEVICE_ERROR_GEMM_TIMEOUT, and the CTA still waits (bounded) for its
+// own loads and MMAs and frees its tensor memory before it returns.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "rrf_device.cuh"
+#include "rrf_internal.h"
+
+namespace rrf {
+namespace {
+
+constexpr int kBM = 128;             // rows of a tile (the MMA's M)
+constexpr int kBK = 128;             // k per stage: 128 one-byte codes = one swizzle row
+constexpr int kStages = 4;
+constexpr int kThreads = 192;        // 6 warps
+constexpr int kMmaK = 32;            // k of one kind::f8f6f4 instruction
+constexpr unsigned long long kGemmWaitLimitNs = 100000000ull;  // 100 ms
+
+// ---------------------------------------------------------------- mbarrier --
+
+__device__ __forceinline__ bool mbar_try_wait_cta(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Wait for phase `parity` of `bar`; false (and the error bit) if the wait ran
+// out.
+__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, unsigned int* err) {
+    if (mbar_try_wait_cta(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait_cta(bar, parity)) {
+        if (global_timer_ns() - t0 > kGemmWaitLimitNs) {
+            atomicOr(err, RRF_DEVICE_ERROR_GEMM_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+// ---------------------------------------------------------------------- TMA --
+
+// 2-D tiled load of box {x, y} at coordinates (x, y) into shared memory,
+// completing `bytes` on `bar` (no multicast).
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];"
+        :
+        : "r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+
+// ----------------------------------------------------------------- tcgen05 --
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t cols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(smem_u32(dst_smem)), "r"(cols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(taddr), "r"(cols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before_sync() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after_sync() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, both K-major e4m3, fp32 D.
+__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+        :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive once on `bar` when every tcgen05 operation this thread issued so
+// far has completed.
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 :: "r"(smem_u32(bar))
+                 : "memory");
+}
+
+// 32 consecutive fp32 accumulator columns of this thread's lane.
+__device__ __forceinline__ void tmem_load_32(uint32_t taddr, float v[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, "
+        "[%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor of a K-major tile stored as rows of 128
+// bytes in 128-byte-swizzled 1024-byte atoms (8 rows each), the layout a
+// TMA load with CU_TENSOR_MAP_SWIZZLE_128B writes: start address >> 4,
+// leading-dimension offset 1 (unused within a swizzle row), stride between
+// 8-row groups 1024 bytes, descriptor version 1, layout SWIZZLE_128B (2).
+__device__ __forceinline__ uint64_t kmajor_sw128_desc(const void* tile) {
+    const uint64_t addr = smem_u32(tile);
+    return ((addr >> 4) & 0x3FFFull) | (1ull << 16) | ((1024ull >> 4) << 32) | (1ull << 46) |
+           (2ull << 61);
+}
+
+// Instruction descriptor of kind::f8f6f4: fp32 accumulator, A and B e4m3,
+// both K-major, N = bn, M = 128.
+__host__ __device__ constexpr uint32_t f8_idesc(int bn) {
+    return (1u << 4) | ((uint32_t)(bn >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+}
+
+// ------------------------------------------------------------------ kernel --
+
+template <int BN>
+struct Tile {
+    static constexpr int kABytes = kBM * kBK;            // 16 KB
+    static constexpr int kBBytes = BN * kBK;
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    // stages, then the barriers and the tensor-memory address; 1 KB of slack
+    // to align the stages to the 1024-byte swizzle atom
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + (2 * kStages + 1) * 8 + 16;
+};
+
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+    scaled_mm_kernel(const __grid_constant__ CUtensorMap tma_a,
+                     const __grid_constant__ CUtensorMap tma_b, const GemmArgs g) {
+    using T = Tile<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * T::kStageBytes);
+    uint64_t* empty = full + kStages;
+    uint64_t* accum = empty + kStages;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * BN, m0 = blockIdx.y * kBM;
+    const int ktiles = (g.K + kBK - 1) / kBK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(accum, 1);
+        fence_mbar_init_cluster();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, BN);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---- producer: TMA loads of the k-tiles into the stage ring
+        if (lane == 0) {
+            int issued = 0;
+            for (int kt = 0; kt < ktiles; ++kt) {
+                const int s = kt % kStages;
+                // a fresh barrier counts as having completed the phase before
+                // phase 0, so the first pass over the ring does not wait
+                if (!wait_phase(&empty[s], ((kt / kStages) & 1) ^ 1, g.err)) break;
+                uint8_t* dst = smem + s * T::kStageBytes;
+                mbar_arrive_expect_tx(&full[s], T::kStageBytes);
+                tma_load_2d(dst, &tma_a, &full[s], kt * kBK, m0);
+                tma_load_2d(dst + T::kABytes, &tma_b, &full[s], kt * kBK, n0);
+                ++issued;
+            }
+            // the loads still in flight land before the CTA may exit
+            for (int kt = issued > kStages ? issued - kStages : 0; kt < issued; ++kt)
+                wait_phase(&full[kt % kStages], (kt / kStages) & 1, g.err);
+        }
+    } else if (warp == 1) {
+        // ---- MMA issue: 4 instructions of K = 32 per k-tile
+        if (lane == 0) {
+            constexpr uint32_t idesc = f8_idesc(BN);
+            for (int kt = 0; kt < ktiles; ++kt) {
+                const int s = kt % kStages;
+                if (!wait_phase(&full[s], (kt / kStages) & 1, g.err)) break;
+                tc_fence_after_sync();
+                const uint8_t* tile = smem + s * T::kStageBytes;
+                const uint64_t ad = kmajor_sw128_desc(tile);
+                const uint64_t bd = kmajor_sw128_desc(tile + T::kABytes);
+#pragma unroll
+                for (int k = 0; k < kBK / kMmaK; ++k) {
+                    // advance the start address by k * 32 bytes inside the swizzle row
+                    const uint64_t step = (uint64_t)(k * kMmaK) >> 4;
+                    mma_f8(tmem, ad + step, bd + step, idesc, (kt | k) != 0);
+                }
+                mma_commit(&empty[s]);  // the stage is free once these MMAs are done
+            }
+            mma_commit(accum);  // every MMA issued above has completed
+        }
+        __syncwarp();
+    } else {
+        // ---- epilogue: warp w reads accumulator lanes 32 * (w % 4) ...
+        const int quarter = warp & 3;
+        const int row = m0 + quarter * 32 + lane;
+        bool have = wait_phase(accum, 0, g.err);
+        have = __all_sync(0xFFFFFFFFu, have);
+        tc_fence_after_sync();
+        if (have) {
+            const float sa = row < g.M ? g.a_scale[row] : 0.0f;
+            for (int c = 0; c < BN; c += 32) {
+                float v[32];
+                tmem_load_32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c, v);
+                const int n = n0 + c;
+                if (row >= g.M || n >= g.N) continue;
+                const int valid = g.N - n < 32 ? g.N - n : 32;  // 16 or 32 (N % 16 == 0)
+                uint32_t packed[16];
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                    float y0 = __fmul_rn(__fmul_rn(v[i], sa), i < valid ? g.b_scale[n + i] : 0.0f);
+                    float y1 = __fmul_rn(__fmul_rn(v[i + 1], sa),
+                                         i + 1 < valid ? g.b_scale[n + i + 1] : 0.0f);
+                    if (g.bias != nullptr && i < valid) {
+                        y0 = __fadd_rn(y0, __uint_as_float((uint32_t)g.bias[n + i] << 16));
+                        y1 = __fadd_rn(y1, __uint_as_float((uint32_t)g.bias[n + i + 1] << 16));
+                    }
+                    packed[i / 2] = f32x2_to_bf16x2(y0, y1);
+                }
+                uint4* dst = reinterpret_cast<uint4*>(g.out + (int64_t)row * g.N + n);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (j * 8 < valid)
+                        dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2],
+                                            packed[4 * j + 3]);
+            }
+        }
+    }
+
+    // ---- teardown: tensor memory is freed after the last MMA and load
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        wait_phase(accum, 0, g.err);  // at once unless a wait above ran out
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, BN);
+    }
+}
+
+// ------------------------------------------------------------------- host --
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The driver's tensor-map encoder, through the runtime's entry-point query
+// (the library links only the runtime).
+EncodeTiled encode_tiled() {
+    static EncodeTiled fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiled>(p);
+    });
+    return fn;
+}
+
+// A [rows, K] byte matrix, box of 128 bytes x box_rows rows, 128-byte swizzle;
+// rows and columns past the matrix read as zero.
+bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int box_rows) {
+    EncodeTiled fn = encode_tiled();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)K};
+    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
+    const cuuint32_t elem[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+              elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+template <int BN>
+cudaError_t launch_bn(const GemmArgs& g, const void* a, const void* b, cudaStream_t stream) {
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, a, g.M, g.K, kBM) || !make_map(&mb, b, g.N, g.K, BN))
+        return cudaErrorInvalidValue;
+    auto kernel = scaled_mm_kernel<BN>;
+    // the dynamic shared memory above 48 KB is enabled once per device
+    static std::atomic<uint64_t> enabled_on{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
+    if (bit == 0 || (enabled_on.load(std::memory_order_relaxed) & bit) == 0) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Tile<BN>::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        enabled_on.fetch_or(bit, std::memory_order_relaxed);
+    }
+    const dim3 grid((unsigned)((g.N + BN - 1) / BN), (unsigned)((g.M + kBM - 1) / kBM), 1);
+    kernel<<<grid, kThreads, Tile<BN>::kSmemBytes, stream>>>(ma, mb, g);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_scaled_mm(const GemmArgs& g, const void* a, const void* b, int sm_count,
+                             cudaStream_t stream) {
+    // 128 x 256 tiles once they fill the SMs, else 128 x 128 (twice the CTAs)
+    const int64_t tiles256 = ((g.M + kBM - 1) / kBM) * ((g.N + 255) / 256);
+    if (tiles256 >= sm_count) return launch_bn<256>(g, a, b, stream);
+    return launch_bn<128>(g, a, b, stream);
+}
+
+}  // namespace rrf

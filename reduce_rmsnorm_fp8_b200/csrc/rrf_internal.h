@@ -103,6 +103,17 @@ struct ArLaunch {
 // and up to 4 vectors per thread fit the register budget of 512 threads).
 constexpr int kArMaxThreads = 512;
 
+// The FP8 GEMM (rrf_gemm.cu); the operands themselves reach the kernel as
+// tensor maps.
+struct GemmArgs {
+    const float* a_scale;  // [M]
+    const float* b_scale;  // [N]
+    const uint16_t* bias;  // bf16 [N] or null
+    uint16_t* out;         // bf16 [M, N]
+    int M, N, K;
+    unsigned int* err;
+};
+
 struct FusedLaunch {
     int cluster;          // blocks per row
     int threads;          // threads per block
@@ -145,6 +156,8 @@ cudaError_t launch_fused(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
 cudaError_t launch_post(const PostArgs& a, int sm_count, bool pdl, cudaStream_t stream);
 
 cudaError_t launch_allreduce(const ArArgs& a, const ArLaunch& l, cudaStream_t stream);
+cudaError_t launch_scaled_mm(const GemmArgs& g, const void* a, const void* b, int sm_count,
+                             cudaStream_t stream);
 // Blocks of the launch shape `l` that can be resident on the current device
 // at once (the occupancy query; nothing is launched).
 cudaError_t allreduce_resident_blocks(const ArLaunch& l, int* resident);

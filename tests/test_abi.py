@@ -58,7 +58,8 @@ def test_constants_match_header(rrf):
     for name in ("RRF_VARIANT_AUTO", "RRF_VARIANT_ROW", "RRF_VARIANT_CLUSTER",
                  "RRF_FLAG_NO_PDL", "RRF_FLAG_BARRIER_EXCHANGE",
                  "RRF_FLAG_DEBUG_STARVE_EXCHANGE", "RRF_DEVICE_ERROR_EXCHANGE_TIMEOUT",
-                 "RRF_DEVICE_ERROR_PEER_TIMEOUT", "RRF_AR_MAX_WORLD", "RRF_AR_MAX_BLOCKS",
+                 "RRF_DEVICE_ERROR_PEER_TIMEOUT", "RRF_DEVICE_ERROR_GEMM_TIMEOUT",
+                 "RRF_AR_MAX_WORLD", "RRF_AR_MAX_BLOCKS",
                  "RRF_AR_AUTO", "RRF_AR_ONE_SHOT", "RRF_AR_TWO_SHOT", "RRF_MAX_SHARDS"):
         assert getattr(rrf, name) == int(
             re.search(rf"#define {name} (0x[0-9a-fA-F]+|\d+)u?", text).group(1), 0)
@@ -382,3 +383,25 @@ def test_peer_layout_is_aligned_and_disjoint():
         assert all(a[0] + a[1] <= b[0] for a, b in zip(spans, spans[1:]))
         assert spans[-1][0] + spans[-1][1] <= total
         assert ("residual" in regions) == res
+
+
+def test_scaled_mm_validation(rrf):
+    ok = dict(a=A, a_scale=2 * A, b=3 * A, b_scale=4 * A, bias=5 * A, out=6 * A, M=64, N=256,
+              K=512)
+    assert rrf.rrf_check_scaled_mm_args(**ok) == rrf.Status.OK
+    assert rrf.rrf_check_scaled_mm_args(**dict(ok, bias=0)) == rrf.Status.OK
+    # M == 0 is a no-op that looks at no pointer
+    assert rrf.rrf_check_scaled_mm_args(0, 0, 0, 0, 0, 0, 0, 256, 512) == rrf.Status.OK
+    for change, status in [
+            (dict(N=8), "ERR_SHAPE"), (dict(K=8), "ERR_SHAPE"), (dict(N=264), "ERR_SHAPE"),
+            (dict(K=520), "ERR_SHAPE"), (dict(M=-1), "ERR_SHAPE"),
+            (dict(M=65535 * 128 + 1), "ERR_SHAPE"),
+            (dict(a=0), "ERR_NULL"), (dict(b_scale=0), "ERR_NULL"), (dict(out=0), "ERR_NULL"),
+            (dict(a=A + 8), "ERR_ALIGN"), (dict(out=6 * A + 4), "ERR_ALIGN"),
+            (dict(a_scale=2 * A + 2), "ERR_ALIGN"), (dict(bias=5 * A + 1), "ERR_ALIGN"),
+            (dict(out=A + 16), "ERR_ALIAS"),                     # over a
+            (dict(b_scale=6 * A + 1024), "ERR_ALIAS"),           # a scale inside out
+            (dict(bias=6 * A + 64 * 256 * 2 - 2), "ERR_ALIAS")]:  # bias at out's end
+        kw = dict(ok)
+        kw.update(change)
+        assert rrf.rrf_check_scaled_mm_args(**kw) == rrf.Status[status], change

@@ -204,3 +204,59 @@ def fused_bytes(R: int, rows: int, cols: int, residual: bool) -> int:
 def sum_bytes(R: int, rows: int, cols: int) -> int:
     """Algorithmic HBM bytes of one sum-only call: R reads and one write."""
     return (R + 1) * rows * cols * 2
+
+
+# ------------------------------------------------------------ FP8 GEMM ---
+# Operands of the GEMM that consumes the per-row scales.  The activation
+# codes and scales normally come from the fused call; these stand-alone
+# operands are codes of N(0, 1) samples (torch's saturating float8_e4m3fn
+# conversion: input preparation, not the GEMM's arithmetic), per-row scales
+# U(0.001, 0.01), weight codes of N(0, 1), per-column scales U(0.0005, 0.002)
+# (a weight of magnitude ~1e-3 quantised per output column) and a bf16 bias
+# N(0, 0.1).  Seeds: 9000 + 10 * sub + tensor.
+
+GEMM_SHAPES = {
+    # decode: the decode batch sizes against a 7168 x 7168 projection
+    "gemm_decode": dict(Ms=(1, 8, 32, 64), N=7168, K=7168),
+    # prefill: 8192 rows of the 8192-wide prefill hidden state, 8192 outputs
+    "gemm_prefill": dict(Ms=(8192,), N=8192, K=8192),
+}
+
+
+@dataclasses.dataclass
+class GemmCase:
+    M: int
+    N: int
+    K: int
+    a: "torch.Tensor"        # float8_e4m3fn [M, K]
+    a_scale: "torch.Tensor"  # float32 [M]
+    b: "torch.Tensor"        # float8_e4m3fn [N, K]
+    b_scale: "torch.Tensor"  # float32 [N]
+    bias: "torch.Tensor | None"  # bf16 [N]
+
+
+def _e4m3_codes(seed: int, n: int, device):
+    import torch
+    x = normal(seed, n, 0.0, 1.0, device).float()
+    return x.clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
+
+
+def make_gemm_case(M: int, N: int, K: int, sub: int = 0, bias: bool = True,
+                   device="cpu") -> GemmCase:
+    s = lambda t: 9000 + 10 * sub + t
+    a = _e4m3_codes(s(0), M * K, device).reshape(M, K)
+    b = _e4m3_codes(s(1), N * K, device).reshape(N, K)
+    sa = (0.001 + 0.009 * uniform(s(2), M, device)).float()
+    sb = (0.0005 + 0.0015 * uniform(s(3), N, device)).float()
+    bi = to_bf16(normal(s(4), N, 0.0, 0.1, device)) if bias else None
+    return GemmCase(M, N, K, a, sa, b, sb, bi)
+
+
+def gemm_bytes(M: int, N: int, K: int, bias: bool = True) -> int:
+    """Algorithmic HBM bytes of one GEMM call: each operand read once, the
+    bf16 output written once."""
+    return M * K + N * K + 4 * M + 4 * N + (2 * N if bias else 0) + 2 * M * N
+
+
+def gemm_flops(M: int, N: int, K: int) -> int:
+    return 2 * M * N * K
