@@ -136,6 +136,17 @@ def measured_peaks():
         return 6650.0, "fallback"
 
 
+def fp8_peak_tflops():
+    """Dense fp8 tensor peak: the measured cuBLAS bf16 burst figure times the
+    nominal fp8 / bf16 ratio (4.5 / 2.25 PFLOP/s), else the fallback 1.59
+    PFLOP/s bf16 times the same ratio."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            return 2.0 * float(json.load(fh)["bf16_tflops"]), "measured bf16_tflops x 2"
+    except Exception:
+        return 2.0 * 1590.0, "fallback bf16 x 2"
+
+
 _CLOCK_POLL = r"""
 import sys, time
 import pynvml
@@ -399,6 +410,39 @@ def time_allreduce(rrf, label, rows, world, mode, device, stream, l2):
             "mode": "two-shot" if m == 2 else "one-shot",
             "launch": {"cluster": cl, "threads": th, "vecs_per_thread": vpt},
             "us_per_call": round(t / reps * 1e6, 3), "device_error": flags}
+
+
+def time_gemm(rrf, M, N, K, device, stream, l2, hbm_peak):
+    """The FP8 GEMM that consumes the per-row scales (rrf_scaled_mm_fp8), one
+    CUDA graph of calls cycling through operand sets larger than 3 x L2;
+    TFLOP/s against the fp8 tensor peak and algorithmic GB/s against HBM."""
+    import torch
+    sets_bytes = workloads.gemm_bytes(M, N, K)
+    n = max(1, math.ceil(L2_FLUSH_FACTOR * l2 / sets_bytes))
+    cases = [workloads.make_gemm_case(M, N, K, sub=i, device=device) for i in range(n)]
+    outs = [torch.empty((M, N), dtype=torch.bfloat16, device=device) for _ in range(n)]
+
+    def call(k):
+        c = cases[k % n]
+        rrf.rrf_scaled_mm_fp8(c.a, c.a_scale, c.b, c.b_scale, c.bias, out=outs[k % n])
+        return 1
+
+    for k in range(3):
+        call(k)
+    reps = max(n, 20 if M * N * K >= 2 ** 36 else 100)
+    g, _ = capture_steps(call, reps, device)
+    g.replay()
+    torch.cuda.synchronize(device)
+    t = time_region(lambda _: g.replay(), 1, device, stream) / reps
+    del g, cases, outs
+    tf = workloads.gemm_flops(M, N, K) / t / 1e12
+    gbs = workloads.gemm_bytes(M, N, K) / t / 1e9
+    fp8_peak, fp8_kind = fp8_peak_tflops()
+    return {"shape": f"{M} x {N} x {K}", "us_per_call": round(t * 1e6, 3),
+            "TFLOP_s": round(tf, 1), "tensor_frac": round(tf / fp8_peak, 4),
+            "GB_s": round(gbs, 1), "hbm_frac": round(gbs / hbm_peak, 4),
+            "fp8_peak_TFLOP_s": round(fp8_peak, 1), "fp8_peak_kind": fp8_kind,
+            "operand_sets": n, "device_error": rrf.rrf_device_error(clear=True)}
 
 
 def capture_steps(fn, n: int, device):
@@ -745,6 +789,13 @@ def run_rrf(args):
                                                      ("prefill", 8192, 8, 0))]
         torch.cuda.empty_cache()
 
+    # ---- the FP8 GEMM that consumes the per-row scales
+    gemm = None
+    if not args.no_secondary:
+        gemm = [time_gemm(rrf, M, 7168, 7168, device, stream, l2, peak) for M in (1, 8, 32, 64)]
+        gemm.append(time_gemm(rrf, 8192, 8192, 8192, device, stream, l2, peak))
+        torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(name)
@@ -792,6 +843,7 @@ def run_rrf(args):
             "other_configs": others,
             "sharded": sharded,
             "allreduce_emulated": emulated,
+            "gemm_fp8": gemm,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
@@ -848,6 +900,19 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_gemm_only(M: int, N: int, K: int):
+    """One GEMM shape through time_gemm (3 eager calls, then graph replays),
+    for profiling; prints its record."""
+    import torch
+
+    import reduce_rmsnorm_fp8_b200 as rrf
+    device = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(device)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    rec = time_gemm(rrf, M, N, K, device, stream, l2, measured_peaks()[0])
+    print(json.dumps({"gemm_fp8": rec}), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description="fused sum + RMSNorm + FP8 benchmark")
     ap.add_argument("--gpus", type=int, default=1)
@@ -862,13 +927,17 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--gemm", type=int, nargs=3, metavar=("M", "N", "K"), default=None,
+                    help="time only the FP8 GEMM of this shape (profiling runs)")
     args = ap.parse_args(argv)
     global ROWS_OVERRIDE
     if args.rows:
         ROWS_OVERRIDE = tuple(args.rows)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.impl == "reference":
+    if args.gemm is not None:
+        run_gemm_only(*args.gemm)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_rrf(args)

@@ -4,16 +4,19 @@
 // aclnnAlltoAllQuantMatmul: per-token dynamic quantisation of the
 // activations, then (x1_q @ x2) * x1Scale * x2Scale + bias).
 //
-// One CTA computes a 128 x BN tile of out.  Warp roles:
+// A persistent CTA per SM walks 128 x BN tiles of out (BN 256, 128 or 64).
+// Warp roles:
 //   warp 0   one thread issues the TMA loads of the A (128 x 128 bytes) and
-//            B (BN x 128 bytes) k-tiles into a ring of kStages shared-memory
-//            stages (128-byte swizzle, the layout the MMA descriptors name);
-//   warp 1   allocates the fp32 accumulator in tensor memory (BN columns of
-//            128 lanes) and one thread issues tcgen05.mma (kind::f8f6f4,
+//            B (BN x 128 bytes) k-tiles into a ring of shared-memory stages
+//            (128-byte swizzle, the layout the MMA descriptors name);
+//   warp 1   allocates two fp32 accumulators in tensor memory (BN columns of
+//            128 lanes each) and one thread issues tcgen05.mma (kind::f8f6f4,
 //            M = 128, N = BN, K = 32 per instruction, 4 per k-tile); a
-//            tcgen05.commit per k-tile hands the stage back to the producer;
+//            tcgen05.commit per k-tile hands the stage back to the producer,
+//            one per tile hands the accumulator to the epilogue;
 //   warps 2-5 the epilogue: tcgen05.ld of its 32 accumulator lanes (rows),
-//            the two scales and bias, one rounding to bf16, 64-byte stores.
+//            the two scales and bias, one rounding to bf16, 64-byte stores,
+//            while the MMAs of the next tile fill the other accumulator.
 // Every mbarrier wait is bounded in time; a wait that runs out sets
 // RRF_DEVICE_ERROR_GEMM_TIMEOUT, and the CTA still waits (bounded) for its
 // own loads and MMAs and frees its tensor memory before it returns.
@@ -31,7 +34,6 @@ namespace {
 
 constexpr int kBM = 128;             // rows of a tile (the MMA's M)
 constexpr int kBK = 128;             // k per stage: 128 one-byte codes = one swizzle row
-constexpr int kStages = 4;
 constexpr int kThreads = 192;        // 6 warps
 constexpr int kMmaK = 32;            // k of one kind::f8f6f4 instruction
 constexpr unsigned long long kGemmWaitLimitNs = 100000000ull;  // 100 ms
@@ -161,43 +163,71 @@ __host__ __device__ constexpr uint32_t f8_idesc(int bn) {
 
 // ------------------------------------------------------------------ kernel --
 
-template <int BN>
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_u32(bar)) : "memory");
+}
+
+// AROWS: rows of A loaded per stage.  128 normally; 64 for calls of at most
+// 64 rows, which halves the A stage and so deepens the ring (the MMA still
+// reads 128 rows: rows 64-127 come from the B half of the same stage, whose
+// 8 KB follow, and land in accumulator rows that are never stored).
+template <int BN, int AROWS>
 struct Tile {
-    static constexpr int kABytes = kBM * kBK;            // 16 KB
+    static_assert(AROWS == kBM || (AROWS == 64 && BN == 64),
+                  "the MMA's 128 rows of A must stay inside the stage");
+    static constexpr int kABytes = AROWS * kBK;
     static constexpr int kBBytes = BN * kBK;
     static constexpr int kStageBytes = kABytes + kBBytes;
-    // stages, then the barriers and the tensor-memory address; 1 KB of slack
-    // to align the stages to the 1024-byte swizzle atom
-    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + (2 * kStages + 1) * 8 + 16;
+    // as many stages as fit in 200 KB, at most 12: 4 at BN 256, 6 at 128,
+    // 8 at 64, 12 with 64-row A stages
+    static constexpr int kStages =
+        (200 * 1024) / kStageBytes > 12 ? 12 : (200 * 1024) / kStageBytes;
+    static constexpr int kTmemCols = 2 * BN;  // two accumulators
+    // full / empty per stage, full / empty per accumulator, one for the drain
+    static constexpr int kBarriers = 2 * kStages + 4 + 1;
+    // 1 KB of slack aligns the stages to the 1024-byte swizzle atom
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarriers * 8 + 16;
 };
 
-template <int BN>
+// A persistent grid: CTA c takes tiles c, c + gridDim.x, ... (row-major over
+// the 128 x BN tiles, so the CTAs working at one time share A rows and B
+// columns in L2).  The accumulator is double-buffered in tensor memory: the
+// MMAs of a CTA's next tile run while the epilogue warps drain this one.
+template <int BN, int AROWS>
 __global__ void __launch_bounds__(kThreads, 1)
     scaled_mm_kernel(const __grid_constant__ CUtensorMap tma_a,
                      const __grid_constant__ CUtensorMap tma_b, const GemmArgs g) {
-    using T = Tile<BN>;
+    using T = Tile<BN, AROWS>;
+    constexpr int S = T::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * T::kStageBytes);
-    uint64_t* empty = full + kStages;
-    uint64_t* accum = empty + kStages;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * T::kStageBytes);
+    uint64_t* empty = full + S;
+    uint64_t* acc_full = empty + S;       // [2]: the tile's MMAs are done
+    uint64_t* acc_empty = acc_full + 2;   // [2]: the epilogue has read the tile
+    uint64_t* drained = acc_empty + 2;    // every MMA of the CTA is done
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * BN, m0 = blockIdx.y * kBM;
+    const int tiles_n = (g.N + BN - 1) / BN;
+    const int tiles = tiles_n * ((g.M + kBM - 1) / kBM);
     const int ktiles = (g.K + kBK - 1) / kBK;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(accum, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 4);  // one arrival per epilogue warp
+        }
+        mbar_init(drained, 1);
         fence_mbar_init_cluster();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, BN);
+        tmem_alloc(tmem_slot, T::kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before_sync();
@@ -206,58 +236,81 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ---- producer: TMA loads of the k-tiles into the stage ring
+        // ---- producer: TMA loads of every k-tile of every tile of this CTA
         if (lane == 0) {
-            int issued = 0;
-            for (int kt = 0; kt < ktiles; ++kt) {
-                const int s = kt % kStages;
-                // a fresh barrier counts as having completed the phase before
-                // phase 0, so the first pass over the ring does not wait
-                if (!wait_phase(&empty[s], ((kt / kStages) & 1) ^ 1, g.err)) break;
-                uint8_t* dst = smem + s * T::kStageBytes;
-                mbar_arrive_expect_tx(&full[s], T::kStageBytes);
-                tma_load_2d(dst, &tma_a, &full[s], kt * kBK, m0);
-                tma_load_2d(dst + T::kABytes, &tma_b, &full[s], kt * kBK, n0);
-                ++issued;
+            int it = 0;  // k-tiles issued, over all tiles
+            bool ok = true;
+            for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+                const int m0 = (t / tiles_n) * kBM, n0 = (t % tiles_n) * BN;
+                for (int kt = 0; kt < ktiles; ++kt, ++it) {
+                    const int s = it % S;
+                    // a fresh barrier counts as having completed the phase
+                    // before phase 0: the first pass over the ring does not wait
+                    if (!wait_phase(&empty[s], ((it / S) & 1) ^ 1, g.err)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* dst = smem + s * T::kStageBytes;
+                    mbar_arrive_expect_tx(&full[s], T::kStageBytes);
+                    tma_load_2d(dst, &tma_a, &full[s], kt * kBK, m0);
+                    tma_load_2d(dst + T::kABytes, &tma_b, &full[s], kt * kBK, n0);
+                }
             }
             // the loads still in flight land before the CTA may exit
-            for (int kt = issued > kStages ? issued - kStages : 0; kt < issued; ++kt)
-                wait_phase(&full[kt % kStages], (kt / kStages) & 1, g.err);
+            for (int i = it > S ? it - S : 0; i < it; ++i)
+                wait_phase(&full[i % S], (i / S) & 1, g.err);
         }
     } else if (warp == 1) {
         // ---- MMA issue: 4 instructions of K = 32 per k-tile
         if (lane == 0) {
             constexpr uint32_t idesc = f8_idesc(BN);
-            for (int kt = 0; kt < ktiles; ++kt) {
-                const int s = kt % kStages;
-                if (!wait_phase(&full[s], (kt / kStages) & 1, g.err)) break;
+            int it = 0, j = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++j) {
+                const int buf = j & 1;
+                // the epilogue has drained this accumulator's previous tile
+                if (!wait_phase(&acc_empty[buf], ((j >> 1) & 1) ^ 1, g.err)) break;
                 tc_fence_after_sync();
-                const uint8_t* tile = smem + s * T::kStageBytes;
-                const uint64_t ad = kmajor_sw128_desc(tile);
-                const uint64_t bd = kmajor_sw128_desc(tile + T::kABytes);
+                const uint32_t d = tmem + (uint32_t)(buf * BN);
+                for (int kt = 0; kt < ktiles; ++kt, ++it) {
+                    const int s = it % S;
+                    if (!wait_phase(&full[s], (it / S) & 1, g.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint8_t* tile = smem + s * T::kStageBytes;
+                    const uint64_t ad = kmajor_sw128_desc(tile);
+                    const uint64_t bd = kmajor_sw128_desc(tile + T::kABytes);
 #pragma unroll
-                for (int k = 0; k < kBK / kMmaK; ++k) {
-                    // advance the start address by k * 32 bytes inside the swizzle row
-                    const uint64_t step = (uint64_t)(k * kMmaK) >> 4;
-                    mma_f8(tmem, ad + step, bd + step, idesc, (kt | k) != 0);
+                    for (int k = 0; k < kBK / kMmaK; ++k) {
+                        // advance the start address by k * 32 bytes in the swizzle row
+                        const uint64_t step = (uint64_t)(k * kMmaK) >> 4;
+                        mma_f8(d, ad + step, bd + step, idesc, (kt | k) != 0);
+                    }
+                    mma_commit(&empty[s]);  // the stage is free once these are done
                 }
-                mma_commit(&empty[s]);  // the stage is free once these MMAs are done
+                mma_commit(&acc_full[buf]);
             }
-            mma_commit(accum);  // every MMA issued above has completed
+            mma_commit(drained);
         }
         __syncwarp();
     } else {
         // ---- epilogue: warp w reads accumulator lanes 32 * (w % 4) ...
         const int quarter = warp & 3;
-        const int row = m0 + quarter * 32 + lane;
-        bool have = wait_phase(accum, 0, g.err);
-        have = __all_sync(0xFFFFFFFFu, have);
-        tc_fence_after_sync();
-        if (have) {
+        int j = 0;
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
+            const int buf = j & 1;
+            const int m0 = (t / tiles_n) * kBM, n0 = (t % tiles_n) * BN;
+            bool have = wait_phase(&acc_full[buf], (j >> 1) & 1, g.err);
+            if (!__all_sync(0xFFFFFFFFu, have)) break;
+            tc_fence_after_sync();
+            const int row = m0 + quarter * 32 + lane;
             const float sa = row < g.M ? g.a_scale[row] : 0.0f;
+            const uint32_t base = tmem + (uint32_t)(buf * BN) + ((uint32_t)(quarter * 32) << 16);
             for (int c = 0; c < BN; c += 32) {
                 float v[32];
-                tmem_load_32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c, v);
+                tmem_load_32(base + (uint32_t)c, v);
                 const int n = n0 + c;
                 if (row >= g.M || n >= g.N) continue;
                 const int valid = g.N - n < 32 ? g.N - n : 32;  // 16 or 32 (N % 16 == 0)
@@ -275,21 +328,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 uint4* dst = reinterpret_cast<uint4*>(g.out + (int64_t)row * g.N + n);
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    if (j * 8 < valid)
-                        dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2],
-                                            packed[4 * j + 3]);
+                for (int q = 0; q < 4; ++q)
+                    if (q * 8 < valid)
+                        dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2],
+                                            packed[4 * q + 3]);
             }
+            // this warp's reads of the accumulator are done: hand it back
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
         }
     }
 
-    // ---- teardown: tensor memory is freed after the last MMA and load
+    // ---- teardown: tensor memory is freed after the CTA's last MMA and load
     tc_fence_before_sync();
     __syncthreads();
     if (warp == 1) {
-        wait_phase(accum, 0, g.err);  // at once unless a wait above ran out
+        wait_phase(drained, 0, g.err);
         tc_fence_after_sync();
-        tmem_dealloc(tmem, BN);
+        tmem_dealloc(tmem, T::kTmemCols);
     }
 }
 
@@ -331,12 +388,14 @@ bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int b
            CUDA_SUCCESS;
 }
 
-template <int BN>
-cudaError_t launch_bn(const GemmArgs& g, const void* a, const void* b, cudaStream_t stream) {
+template <int BN, int AROWS>
+cudaError_t launch_bn(const GemmArgs& g, const void* a, const void* b, int sm_count,
+                      cudaStream_t stream) {
+    using T = Tile<BN, AROWS>;
     CUtensorMap ma, mb;
-    if (!make_map(&ma, a, g.M, g.K, kBM) || !make_map(&mb, b, g.N, g.K, BN))
+    if (!make_map(&ma, a, g.M, g.K, AROWS) || !make_map(&mb, b, g.N, g.K, BN))
         return cudaErrorInvalidValue;
-    auto kernel = scaled_mm_kernel<BN>;
+    auto kernel = scaled_mm_kernel<BN, AROWS>;
     // the dynamic shared memory above 48 KB is enabled once per device
     static std::atomic<uint64_t> enabled_on{0};
     int dev = 0;
@@ -345,12 +404,13 @@ cudaError_t launch_bn(const GemmArgs& g, const void* a, const void* b, cudaStrea
     const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
     if (bit == 0 || (enabled_on.load(std::memory_order_relaxed) & bit) == 0) {
         e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Tile<BN>::kSmemBytes);
+                                 T::kSmemBytes);
         if (e != cudaSuccess) return e;
         enabled_on.fetch_or(bit, std::memory_order_relaxed);
     }
-    const dim3 grid((unsigned)((g.N + BN - 1) / BN), (unsigned)((g.M + kBM - 1) / kBM), 1);
-    kernel<<<grid, kThreads, Tile<BN>::kSmemBytes, stream>>>(ma, mb, g);
+    const int64_t tiles = (int64_t)((g.N + BN - 1) / BN) * ((g.M + kBM - 1) / kBM);
+    const unsigned grid = (unsigned)(tiles < sm_count ? tiles : sm_count);  // one CTA per SM
+    kernel<<<grid, kThreads, T::kSmemBytes, stream>>>(ma, mb, g);
     return cudaGetLastError();
 }
 
@@ -358,10 +418,16 @@ cudaError_t launch_bn(const GemmArgs& g, const void* a, const void* b, cudaStrea
 
 cudaError_t launch_scaled_mm(const GemmArgs& g, const void* a, const void* b, int sm_count,
                              cudaStream_t stream) {
-    // 128 x 256 tiles once they fill the SMs, else 128 x 128 (twice the CTAs)
-    const int64_t tiles256 = ((g.M + kBM - 1) / kBM) * ((g.N + 255) / 256);
-    if (tiles256 >= sm_count) return launch_bn<256>(g, a, b, stream);
-    return launch_bn<128>(g, a, b, stream);
+    // The widest tile that still gives every SM a tile; short, wide
+    // problems (decode batches against a weight) take 128 x 64 tiles, the
+    // most CTAs streaming the weight.
+    const int64_t row_tiles = (g.M + kBM - 1) / kBM;
+    if (row_tiles * ((g.N + 255) / 256) >= sm_count)
+        return launch_bn<256, kBM>(g, a, b, sm_count, stream);
+    if (row_tiles * ((g.N + 127) / 128) >= sm_count)
+        return launch_bn<128, kBM>(g, a, b, sm_count, stream);
+    if (g.M <= 64) return launch_bn<64, 64>(g, a, b, sm_count, stream);
+    return launch_bn<64, kBM>(g, a, b, sm_count, stream);
 }
 
 }  // namespace rrf
