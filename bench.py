@@ -362,9 +362,8 @@ def time_sharded(rrf, label, rows, cols, shards, device, stream, l2, peak):
 
 def time_allreduce(rrf, label, rows, world, mode, device, stream, l2):
     """The multi-GPU call with all `world` ranks in one launch on this GPU
-    (LocalGroup): one CUDA graph of `reps` calls numbered 1..reps after a
-    reset of the signal pads, cycling through buffer sets larger than 3 x L2
-    (the residual updated in place);
+    (LocalGroup): one CUDA graph of `reps` calls, cycling through buffer sets
+    larger than 3 x L2 (the residual updated in place);
     microseconds per call.  This GPU's memory stands in for the links, so the
     number bounds the kernel's own cost, not a multi-GPU call's."""
     import torch
@@ -386,7 +385,7 @@ def time_allreduce(rrf, label, rows, world, mode, device, stream, l2):
         i = k % n
         g([x[i] for x in xs], c.gamma, c.eps, c.weight_offset, c.scale_ub,
           residual_in=[r[i] for r in rs], residual_out=[r[i] for r in rs],
-          q_out=[q[i] for q in qs], scales_out=[s[i] for s in ss], mode=mode, epoch=k + 1)
+          q_out=[q[i] for q in qs], scales_out=[s[i] for s in ss], mode=mode)
         return 1
 
     reps = max(50, n) if rows < 1024 else 5
@@ -394,9 +393,7 @@ def time_allreduce(rrf, label, rows, world, mode, device, stream, l2):
         call(k)
     torch.cuda.synchronize(device)
     graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        for p in g.pads:
-            p.zero_()
+    with torch.cuda.graph(graph):  # the pads number the replayed calls themselves
         for k in range(reps):
             call(k)
     graph.replay()

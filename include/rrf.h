@@ -290,14 +290,16 @@ rrf_status rrf_check_post_args(const void* h, int64_t rows, int64_t cols, const 
  * mappings), or another buffer of this GPU when one launch runs all ranks
  * (local_ranks == world, used to run the whole exchange on one GPU).
  * Signal pads: RRF_AR_SIGNAL_WORDS 32-bit words per rank, zeroed once before
- * the first call; `epoch` numbers the calls 1, 2, 3, ... (the same number on
- * every rank for the same call, never 0).  After RRF_DEVICE_ERROR_PEER_TIMEOUT
- * the pads must be zeroed again and the numbering restarted.
+ * the first call.  Besides the barrier words a pad holds one call counter
+ * per block, which the kernel itself advances, so the calls need no number
+ * from the host and a call captured in a CUDA graph stays correct when the
+ * graph is replayed.  Every rank must make the same sequence of calls on its
+ * pads.  After RRF_DEVICE_ERROR_PEER_TIMEOUT the pads must be zeroed again.
  * ---------------------------------------------------------------------- */
 
 #define RRF_AR_MAX_WORLD 8
 #define RRF_AR_MAX_BLOCKS 1024 /* blocks per rank of one launch */
-#define RRF_AR_SIGNAL_WORDS (2 * RRF_AR_MAX_WORLD * RRF_AR_MAX_BLOCKS)
+#define RRF_AR_SIGNAL_WORDS ((2 * RRF_AR_MAX_WORLD + 1) * RRF_AR_MAX_BLOCKS)
 #define RRF_AR_AUTO 0     /* two-shot when every rank gets a row, else one-shot */
 #define RRF_AR_ONE_SHOT 1
 #define RRF_AR_TWO_SHOT 2
@@ -315,12 +317,12 @@ rrf_status rrf_check_post_args(const void* h, int64_t rows, int64_t cols, const 
  *               local_ranks == world);  local_ranks: 1 or world
  * rows, cols, gamma, eps, weight_offset, scale_ub  as for rrf_sum_rmsnorm_fp8
  *               (gamma: this GPU's copy); cols <= 8 * 8 * 512 * 4
- * epoch         the call's number (see above);  mode: RRF_AR_*
+ * mode          RRF_AR_*
  * timeout_ns    bound on each barrier wait (0 = one second)
- * Every rank must make the same call (same shape, mode and epoch).
+ * Every rank must make the same call (same shape and mode).
  * Errors: RRF_ERR_NULL, RRF_ERR_RANKS (world or rank out of range),
- *         RRF_ERR_SHAPE, RRF_ERR_ALIGN, RRF_ERR_ALIAS, RRF_ERR_VALUE
- *         (epoch 0 included), RRF_ERR_UNSUPPORTED (mode or local_ranks out of
+ *         RRF_ERR_SHAPE, RRF_ERR_ALIGN, RRF_ERR_ALIAS, RRF_ERR_VALUE,
+ *         RRF_ERR_UNSUPPORTED (mode or local_ranks out of
  *         range, or all ranks' blocks cannot be resident on this GPU at
  *         once), RRF_ERR_CUDA. */
 rrf_status rrf_allreduce_rmsnorm_fp8(const void* const* inputs, const void* const* residual_in,
@@ -328,8 +330,8 @@ rrf_status rrf_allreduce_rmsnorm_fp8(const void* const* inputs, const void* cons
                                      float* const* scales_out, unsigned int* const* signals,
                                      int world, int rank, int local_ranks, int64_t rows,
                                      int64_t cols, const void* gamma, float eps,
-                                     float weight_offset, float scale_ub, unsigned int epoch,
-                                     int mode, uint64_t timeout_ns, rrf_stream_t stream);
+                                     float weight_offset, float scale_ub, int mode,
+                                     uint64_t timeout_ns, rrf_stream_t stream);
 
 /* The host validation of rrf_allreduce_rmsnorm_fp8 alone (no GPU needed). */
 rrf_status rrf_check_allreduce_args(const void* const* inputs, const void* const* residual_in,
@@ -337,8 +339,7 @@ rrf_status rrf_check_allreduce_args(const void* const* inputs, const void* const
                                     float* const* scales_out, unsigned int* const* signals,
                                     int world, int rank, int local_ranks, int64_t rows,
                                     int64_t cols, const void* gamma, float eps,
-                                    float weight_offset, float scale_ub, unsigned int epoch,
-                                    int mode);
+                                    float weight_offset, float scale_ub, int mode);
 
 /* rrf_plan_allreduce -- the mode and row shape rrf_allreduce_rmsnorm_fp8
  * picks on a GPU with sm_count SMs, without touching the GPU: the mode

@@ -21,7 +21,7 @@ RRF_MAX_SHARDS = 64
 RRF_DEVICE_ERROR_PEER_TIMEOUT = 2
 RRF_AR_MAX_WORLD = 8
 RRF_AR_MAX_BLOCKS = 1024
-RRF_AR_SIGNAL_WORDS = 2 * RRF_AR_MAX_WORLD * RRF_AR_MAX_BLOCKS
+RRF_AR_SIGNAL_WORDS = (2 * RRF_AR_MAX_WORLD + 1) * RRF_AR_MAX_BLOCKS
 RRF_AR_AUTO = 0
 RRF_AR_ONE_SHOT = 1
 RRF_AR_TWO_SHOT = 2
@@ -97,7 +97,7 @@ lib.rrf_check_post_args.restype = _int
 lib.rrf_check_post_args.argtypes = [_vp, _i64, _i64, _vp, _int, _i64, _vp, _f32, _f32, _f32,
                                     _vp, _vp]
 _ar_args = [_ptrs, _ptrs, _ptrs, _ptrs, _ptrs, _ptrs, _int, _int, _int, _i64, _i64, _vp, _f32,
-            _f32, _f32, ctypes.c_uint, _int]
+            _f32, _f32, _int]
 lib.rrf_allreduce_rmsnorm_fp8.restype = _int
 lib.rrf_allreduce_rmsnorm_fp8.argtypes = _ar_args + [ctypes.c_uint64, _vp]
 lib.rrf_check_allreduce_args.restype = _int
@@ -178,13 +178,13 @@ def _ar_tables(inputs, residual_in, residual_out, q_out, scales_out, signals):
 
 def rrf_check_allreduce_args(inputs, residual_in, residual_out, q_out, scales_out, signals,
                              rank, local_ranks, rows, cols, gamma, eps, weight_offset, scale_ub,
-                             epoch, mode, world=None) -> int:
+                             mode, world=None) -> int:
     """Host validation of the multi-GPU call on raw pointers (lists of
     ``world`` ints; residual lists may be None)."""
     world = len(inputs) if world is None else world
     return lib.rrf_check_allreduce_args(
         *_ar_tables(inputs, residual_in, residual_out, q_out, scales_out, signals), world,
-        rank, local_ranks, rows, cols, gamma or None, eps, weight_offset, scale_ub, epoch, mode)
+        rank, local_ranks, rows, cols, gamma or None, eps, weight_offset, scale_ub, mode)
 
 
 def rrf_plan_allreduce(world: int, rows: int, cols: int, sm_count: int, residual=True,
@@ -199,12 +199,12 @@ def rrf_plan_allreduce(world: int, rows: int, cols: int, sm_count: int, residual
 
 def rrf_allreduce_rmsnorm_fp8_ptr(inputs, residual_in, residual_out, q_out, scales_out, signals,
                                   rank, local_ranks, rows, cols, gamma, eps, weight_offset,
-                                  scale_ub, epoch, mode=0, timeout_ns=0, stream=0) -> None:
+                                  scale_ub, mode=0, timeout_ns=0, stream=0) -> None:
     """rrf_allreduce_rmsnorm_fp8 on raw pointers: every list holds one device
     address per rank, as this GPU addresses that rank's buffer."""
     _raise_on(lib.rrf_allreduce_rmsnorm_fp8(
         *_ar_tables(inputs, residual_in, residual_out, q_out, scales_out, signals), len(inputs),
-        rank, local_ranks, rows, cols, gamma or None, eps, weight_offset, scale_ub, epoch, mode,
+        rank, local_ranks, rows, cols, gamma or None, eps, weight_offset, scale_ub, mode,
         timeout_ns, stream or None))
 
 

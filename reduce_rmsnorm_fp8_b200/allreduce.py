@@ -19,7 +19,7 @@ from __future__ import annotations
 
 # Entries of the C header, for the helpers below that need no library.
 RRF_AR_MAX_WORLD = 8
-RRF_AR_SIGNAL_WORDS = 2 * RRF_AR_MAX_WORLD * 1024
+RRF_AR_SIGNAL_WORDS = (2 * RRF_AR_MAX_WORLD + 1) * 1024
 RRF_AR_AUTO = 0
 
 
@@ -57,8 +57,9 @@ def _check_rank_tensors(ts, like, what, dtype=None):
 class LocalGroup:
     """``world`` ranks whose buffers all live on one GPU; every call runs all
     of them in one launch (each rank's blocks meet the others' at the same
-    barriers as in a multi-GPU job).  Keeps the ranks' signal pads and the
-    call counter."""
+    barriers as in a multi-GPU job).  Keeps the ranks' signal pads (which
+    carry the calls' numbering themselves, so calls may be captured in a
+    CUDA graph and replayed)."""
 
     def __init__(self, world: int, device=None):
         torch = _torch()
@@ -69,22 +70,15 @@ class LocalGroup:
             else torch.device(device)
         self.pads = [torch.zeros(RRF_AR_SIGNAL_WORDS, dtype=torch.int32, device=self.device)
                      for _ in range(world)]
-        self.epoch = 0
 
     def reset(self):
-        """Zero the pads and restart the call numbering (needed after a
-        barrier wait ran out)."""
+        """Zero the pads (needed after a barrier wait ran out)."""
         for p in self.pads:
             p.zero_()
-        self.epoch = 0
-
-    def next_epoch(self) -> int:
-        self.epoch = self.epoch % 0xFFFFFFFF + 1
-        return self.epoch
 
     def __call__(self, partials, gamma, eps, weight_offset, scale_ub, residual_in=None,
                  residual_out=None, q_out=None, scales_out=None, mode=RRF_AR_AUTO,
-                 timeout_ns=0, epoch=None):
+                 timeout_ns=0):
         """One call over the ranks' partials (``world`` bf16 tensors of one
         shape).  residual_in: one tensor per rank (the same values on every
         rank) or None; residual_out defaults to new tensors (pass residual_in
@@ -112,14 +106,12 @@ class LocalGroup:
                                       device=x0.device) for _ in range(self.world)]
         _check_rank_tensors(q_out, partials, "q_out", torch.float8_e4m3fn)
         _check_rank_tensors(scales_out, partials, "scales_out", torch.float32)
-        e = self.next_epoch() if epoch is None else epoch
         ptrs = (lambda ts: None if ts is None else [t.data_ptr() for t in ts])
         with torch.cuda.device(x0.device):
             _lib().rrf_allreduce_rmsnorm_fp8_ptr(
                 ptrs(partials), ptrs(residual_in), ptrs(residual_out), ptrs(q_out),
                 ptrs(scales_out), ptrs(self.pads), 0, self.world, rows, cols, gamma.data_ptr(),
-                eps, weight_offset, scale_ub, e, mode, timeout_ns,
-                _lib()._stream(x0.device))
+                eps, weight_offset, scale_ub, mode, timeout_ns, _lib()._stream(x0.device))
         return q_out, scales_out, residual_out
 
 
@@ -174,7 +166,6 @@ class PeerGroup:
         self.buf[off:off + nbytes].zero_()
         torch.cuda.synchronize(self.device)
         dist.barrier(group)
-        self.epoch = 0
 
     def _view(self, name, rows, dtype, shape):
         off, _ = self.layout[name]
@@ -206,14 +197,12 @@ class PeerGroup:
         if gamma.dtype != torch.bfloat16 or gamma.numel() != self.cols or \
                 gamma.device != self.device:
             raise ValueError("gamma must be a bf16 tensor of length cols on the group's device")
-        self.epoch = self.epoch % 0xFFFFFFFF + 1
         res = self.ptrs["residual"] if self.has_residual else None
         with torch.cuda.device(self.device):
             _lib().rrf_allreduce_rmsnorm_fp8_ptr(
                 self.ptrs["input"], res, res, self.ptrs["q"], self.ptrs["scales"],
                 self.ptrs["pad"], self.rank, 1, rows, self.cols, gamma.data_ptr(), eps,
-                weight_offset, scale_ub, self.epoch, mode, timeout_ns,
-                _lib()._stream(self.device))
+                weight_offset, scale_ub, mode, timeout_ns, _lib()._stream(self.device))
         q = self._view("q", rows, torch.float8_e4m3fn, (rows, self.cols))
         scales = self._view("scales", rows, torch.float32, (rows, 1))
         return q, scales, (self.residual(rows) if self.has_residual else None)

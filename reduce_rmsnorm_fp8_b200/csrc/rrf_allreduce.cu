@@ -22,8 +22,12 @@
 //   end barrier    the same after the stores: when every block of rank k has
 //                  passed it, every peer block has finished its stores into
 //                  k's outputs and its reads of k's input.
-// A flag word holds the call's epoch (the caller numbers its calls 1, 2, ...),
-// so the pads are zeroed once, not per call.  Every wait is bounded in time;
+// A flag word holds the call's number, which each block keeps in a counter
+// word of its own rank's pad and advances at the end of the call: the pads
+// are zeroed once, the host passes no number, and a call replayed from a
+// CUDA graph is numbered afresh.  Block b's counter has the same history on
+// every rank (every rank makes the same calls with the same grid), so block
+// b of every rank uses the same number.  Every wait is bounded in time;
 // one that runs out sets a bit in the device error word and the kernel goes
 // on with the same control flow (no block of a cluster may skip a phase that
 // its peers take), so it always finishes.
@@ -47,12 +51,23 @@ __device__ __forceinline__ unsigned int* flag_word(unsigned int* pad, int phase,
     return pad + ((size_t)(phase * RRF_AR_MAX_WORLD + src) * RRF_AR_MAX_BLOCKS + block);
 }
 
+// The calls block `block` of this rank has completed on this pad.
+__device__ __forceinline__ unsigned int* counter_word(unsigned int* pad, int block) {
+    return pad + (size_t)2 * RRF_AR_MAX_WORLD * RRF_AR_MAX_BLOCKS + block;
+}
+
 __device__ __forceinline__ void st_release_sys(unsigned int* p, unsigned int v) {
     asm volatile("st.release.sys.global.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
 }
 
 __device__ __forceinline__ void st_relaxed_sys(unsigned int* p, unsigned int v) {
     asm volatile("st.relaxed.sys.global.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned int ld_relaxed_gpu(const unsigned int* p) {
+    unsigned int v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
 }
 
 __device__ __forceinline__ unsigned int ld_acquire_sys(const unsigned int* p) {
@@ -72,17 +87,18 @@ __device__ __forceinline__ unsigned int ld_acquire_sys(const unsigned int* p) {
 // began.  (On B200 each system-scope release costs about 3 us even with
 // nothing to drain, measured with all ranks in one launch; a separate
 // __threadfence_system before the release added as much again.)
-__device__ void peer_barrier(const ArArgs& a, int phase, int rank, int block) {
+__device__ void peer_barrier(const ArArgs& a, int phase, int rank, int block,
+                             unsigned int call) {
     __syncthreads();
     const int t = threadIdx.x;
     if (t < a.world) {
         unsigned int* theirs = flag_word(a.sig[t], phase, rank, block);
-        if (phase == 0) st_relaxed_sys(theirs, a.epoch);
-        else st_release_sys(theirs, a.epoch);
+        if (phase == 0) st_relaxed_sys(theirs, call);
+        else st_release_sys(theirs, call);
         const unsigned int* mine = flag_word(a.sig[rank], phase, t, block);
-        if (ld_acquire_sys(mine) != a.epoch) {
+        if (ld_acquire_sys(mine) != call) {
             const uint64_t t0 = global_timer_ns();
-            while (ld_acquire_sys(mine) != a.epoch) {
+            while (ld_acquire_sys(mine) != call) {
                 if (global_timer_ns() - t0 > a.timeout_ns) {
                     atomicOr(a.err, RRF_DEVICE_ERROR_PEER_TIMEOUT);
                     break;
@@ -130,10 +146,18 @@ __global__ void __launch_bounds__(kArMaxThreads, VPT <= 2 ? 2 : 1) ar_kernel(con
     const int v_begin = (int)crank * a.slice_vecs;
     const int v_end = min(v_begin + a.slice_vecs, a.vecs);
 
+    // This call's number: one more than the calls this block has completed
+    // on its rank's pad (written by this block at the end of the previous
+    // call, an earlier kernel of the stream).
+    __shared__ unsigned int call_s;
+    if (tid == 0) call_s = ld_relaxed_gpu(counter_word(a.sig[rank], block)) + 1u;
+    __syncthreads();
+    const unsigned int call = call_s;
+
     // Cluster phase 0 (every block of the cluster has started) overlaps the
     // start barrier; its wait comes before the first remote shared store.
     if (CLUSTER) cluster_arrive_relaxed();
-    peer_barrier(a, 0, rank, block);
+    peer_barrier(a, 0, rank, block, call);
     if (CLUSTER) cluster_wait_acquire();
 
     const int64_t first = a.two_shot ? (int64_t)rank * a.rows_per_rank : 0;
@@ -234,7 +258,8 @@ __global__ void __launch_bounds__(kArMaxThreads, VPT <= 2 ? 2 : 1) ar_kernel(con
             }
         }
     }
-    peer_barrier(a, 1, rank, block);
+    peer_barrier(a, 1, rank, block, call);
+    if (tid == 0) *counter_word(a.sig[rank], block) = call;
 }
 
 // Clusters of up to 8 (the portable size) only.

@@ -572,7 +572,7 @@ extern "C" rrf_status rrf_check_allreduce_args(
     const void* const* inputs, const void* const* residual_in, void* const* residual_out,
     void* const* q_out, float* const* scales_out, unsigned int* const* signals, int world,
     int rank, int local_ranks, int64_t rows, int64_t cols, const void* gamma, float eps,
-    float weight_offset, float scale_ub, unsigned int epoch, int mode) {
+    float weight_offset, float scale_ub, int mode) {
     if (world < 1 || world > RRF_AR_MAX_WORLD) return RRF_ERR_RANKS;
     if (local_ranks != 1 && local_ranks != world) return RRF_ERR_UNSUPPORTED;
     if (rank < 0 || rank >= world || (local_ranks > 1 && rank != 0)) return RRF_ERR_RANKS;
@@ -582,7 +582,6 @@ extern "C" rrf_status rrf_check_allreduce_args(
     if (!(std::isfinite(eps) && eps >= 0.0f)) return RRF_ERR_VALUE;
     if (!std::isfinite(weight_offset)) return RRF_ERR_VALUE;
     if (std::isnan(scale_ub) || !(scale_ub > 0.0f)) return RRF_ERR_VALUE;
-    if (epoch == 0) return RRF_ERR_VALUE;
     if (rows == 0) return RRF_OK;
     if (!inputs || !q_out || !scales_out || !signals || !gamma) return RRF_ERR_NULL;
     if ((residual_in == nullptr) != (residual_out == nullptr)) return RRF_ERR_NULL;
@@ -633,12 +632,11 @@ extern "C" rrf_status rrf_allreduce_rmsnorm_fp8(
     const void* const* inputs, const void* const* residual_in, void* const* residual_out,
     void* const* q_out, float* const* scales_out, unsigned int* const* signals, int world,
     int rank, int local_ranks, int64_t rows, int64_t cols, const void* gamma, float eps,
-    float weight_offset, float scale_ub, unsigned int epoch, int mode, uint64_t timeout_ns,
-    rrf_stream_t stream) {
+    float weight_offset, float scale_ub, int mode, uint64_t timeout_ns, rrf_stream_t stream) {
     rrf_status st = rrf_check_allreduce_args(inputs, residual_in, residual_out, q_out,
                                              scales_out, signals, world, rank, local_ranks,
                                              rows, cols, gamma, eps, weight_offset, scale_ub,
-                                             epoch, mode);
+                                             mode);
     if (st != RRF_OK || rows == 0) return st;
     int sm_count = 0;
     if ((st = current_sm_count(&sm_count)) != RRF_OK) return st;
@@ -688,7 +686,6 @@ extern "C" rrf_status rrf_allreduce_rmsnorm_fp8(
     a.eps = eps;
     a.weight_offset = weight_offset;
     a.scale_ub = scale_ub;
-    a.epoch = epoch;
     a.timeout_ns = timeout_ns != 0 ? timeout_ns : kArDefaultTimeoutNs;
     a.err = err;
     if (!take_injected_failure(&e)) e = launch_allreduce(a, l, (cudaStream_t)stream);

@@ -84,7 +84,6 @@ struct ArArgs {
     float eps;
     float weight_offset;
     float scale_ub;
-    unsigned int epoch;
     unsigned long long timeout_ns;
     unsigned int* err;
 };

@@ -63,7 +63,7 @@ def test_constants_match_header(rrf):
                  "RRF_AR_AUTO", "RRF_AR_ONE_SHOT", "RRF_AR_TWO_SHOT", "RRF_MAX_SHARDS"):
         assert getattr(rrf, name) == int(
             re.search(rf"#define {name} (0x[0-9a-fA-F]+|\d+)u?", text).group(1), 0)
-    expr = re.search(r"#define RRF_AR_SIGNAL_WORDS \(([^)]*)\)", text).group(1)
+    expr = re.search(r"#define RRF_AR_SIGNAL_WORDS (\(.*\))\s*$", text, flags=re.M).group(1)
     assert rrf.RRF_AR_SIGNAL_WORDS == eval(expr, {"RRF_AR_MAX_WORLD": rrf.RRF_AR_MAX_WORLD,
                                                   "RRF_AR_MAX_BLOCKS": rrf.RRF_AR_MAX_BLOCKS})
     from reduce_rmsnorm_fp8_b200 import allreduce
@@ -278,7 +278,7 @@ def _ar_ok(world=4, residual=True):
     return dict(inputs=at(1), residual_in=at(2) if residual else None,
                 residual_out=at(3) if residual else None, q_out=at(4), scales_out=at(5),
                 signals=at(6), rank=0, local_ranks=1, rows=8, cols=64, gamma=A // 2, eps=1e-5,
-                weight_offset=0.0, scale_ub=1200.0, epoch=1, mode=0)
+                weight_offset=0.0, scale_ub=1200.0, mode=0)
 
 
 def test_allreduce_validation_accepts_valid(rrf):
@@ -308,7 +308,6 @@ def _swap(lst, j, value):
     (lambda o: dict(o, rank=1, local_ranks=4), "ERR_RANKS"),
     (lambda o: dict(o, local_ranks=2), "ERR_UNSUPPORTED"),
     (lambda o: dict(o, mode=3), "ERR_UNSUPPORTED"),
-    (lambda o: dict(o, epoch=0), "ERR_VALUE"),
     (lambda o: dict(o, eps=-1.0), "ERR_VALUE"),
     (lambda o: dict(o, scale_ub=float("nan")), "ERR_VALUE"),
     (lambda o: dict(o, cols=60), "ERR_SHAPE"),

@@ -7,6 +7,8 @@ Every rank's outputs must equal the oracle's on the whole problem (the
 partials as the inputs, in rank order) within the fused call's tolerances,
 and every rank must hold the same bits.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -105,16 +107,51 @@ def test_in_place_residual(allreduce, mode):
     parity.assert_fused_parity(outs[0], ref, "in place")
 
 
-def test_repeated_calls_on_one_group(allreduce):
-    """Calls 1..6 on the same pads (the epoch protocol), new data each time,
-    alternating modes."""
+def test_repeated_calls_on_one_group(rrf, allreduce):
+    """Six calls on the same pads (the blocks' call counters), new data and
+    shapes each time, alternating modes."""
     g = allreduce.LocalGroup(4)
     for i in range(6):
-        c = rank_case("odd", 37, 4, sub=20 + i)
+        c = rank_case("odd", 37 if i % 3 else 64, 4, sub=20 + i)
         outs = run_local(allreduce, c, ONE if i % 2 else TWO, group=g)
         assert_ranks_agree(outs)
         parity.assert_fused_parity(outs[0], parity.oracle_fused(c), f"call {i + 1}")
-    assert g.epoch == 6
+    assert rrf.rrf_device_error() == 0
+
+
+def test_graph_replay(rrf, allreduce):
+    """A call captured in a CUDA graph and replayed three times over new
+    inputs copied into the captured buffers: every replay synchronises the
+    ranks afresh and is correct."""
+    world = 8
+    g = allreduce.LocalGroup(world)
+    c0 = rank_case("decode", 32, world, sub=40)
+    xs = [x.clone() for x in c0.inputs]
+    res = [c0.residual.clone() for _ in range(world)]
+    q = [torch.empty(x.shape, dtype=torch.float8_e4m3fn, device="cuda") for x in xs]
+    sc = [torch.empty((x.shape[0], 1), dtype=torch.float32, device="cuda") for x in xs]
+    call = lambda: g(xs, c0.gamma, c0.eps, c0.weight_offset, c0.scale_ub, residual_in=res,
+                     residual_out=res, q_out=q, scales_out=sc, mode=TWO)
+    call()  # warm-up outside the capture
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    for i in range(3):
+        # new partials and residual; gamma stays the captured one
+        c = dataclasses.replace(rank_case("decode", 32, world, sub=41 + i), gamma=c0.gamma)
+        for x, src in zip(xs, c.inputs):
+            x.copy_(src)
+        for r in res:
+            r.copy_(c.residual)
+        graph.replay()
+        torch.cuda.synchronize()
+        outs = [{"q": q[k].view(torch.uint8).cpu().numpy(),
+                 "scales": sc[k].reshape(-1).cpu().numpy(),
+                 "res_out": workloads.bits(res[k])} for k in range(world)]
+        assert_ranks_agree(outs)
+        parity.assert_fused_parity(outs[0], parity.oracle_fused(c), f"replay {i}")
+    assert rrf.rrf_device_error() == 0
 
 
 def test_two_shot_full_prefill(allreduce):
@@ -151,7 +188,7 @@ def test_missing_peer_times_out(rrf, allreduce):
     gamma = torch.ones(cols, dtype=torch.bfloat16, device="cuda")
     ptr = lambda ts: [t.data_ptr() for t in ts]
     rrf.rrf_allreduce_rmsnorm_fp8_ptr(ptr(xs), None, None, ptr(qs), ptr(scales), ptr(pads), 0, 1,
-                                      rows, cols, gamma.data_ptr(), 1e-6, 0.0, 1.0, 1,
+                                      rows, cols, gamma.data_ptr(), 1e-6, 0.0, 1.0,
                                       mode=TWO, timeout_ns=1_000_000,
                                       stream=torch.cuda.current_stream().cuda_stream)
     torch.cuda.synchronize()
