@@ -163,6 +163,31 @@ __host__ __device__ constexpr uint32_t f8_idesc(int bn) {
 
 // ------------------------------------------------------------------ kernel --
 
+// The epilogue of 32 accumulator columns [n, n + 32) of one output row: both
+// scales and the bias in fp32, one rounding to bf16, 64-byte stores (16 or
+// 32 columns valid: N % 16 == 0).
+__device__ __forceinline__ void store_row_chunk(const GemmArgs& g, const float v[32], float sa,
+                                                int row, int n) {
+    const int valid = g.N - n < 32 ? g.N - n : 32;
+    uint32_t packed[16];
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+        float y0 = __fmul_rn(__fmul_rn(v[i], sa), i < valid ? g.b_scale[n + i] : 0.0f);
+        float y1 = __fmul_rn(__fmul_rn(v[i + 1], sa), i + 1 < valid ? g.b_scale[n + i + 1] : 0.0f);
+        if (g.bias != nullptr && i < valid) {
+            y0 = __fadd_rn(y0, __uint_as_float((uint32_t)g.bias[n + i] << 16));
+            y1 = __fadd_rn(y1, __uint_as_float((uint32_t)g.bias[n + i + 1] << 16));
+        }
+        packed[i / 2] = f32x2_to_bf16x2(y0, y1);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(g.out + (int64_t)row * g.N + n);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        if (q * 8 < valid)
+            dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2],
+                                packed[4 * q + 3]);
+}
+
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_u32(bar)) : "memory");
 }
@@ -313,25 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_load_32(base + (uint32_t)c, v);
                 const int n = n0 + c;
                 if (row >= g.M || n >= g.N) continue;
-                const int valid = g.N - n < 32 ? g.N - n : 32;  // 16 or 32 (N % 16 == 0)
-                uint32_t packed[16];
-#pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    float y0 = __fmul_rn(__fmul_rn(v[i], sa), i < valid ? g.b_scale[n + i] : 0.0f);
-                    float y1 = __fmul_rn(__fmul_rn(v[i + 1], sa),
-                                         i + 1 < valid ? g.b_scale[n + i + 1] : 0.0f);
-                    if (g.bias != nullptr && i < valid) {
-                        y0 = __fadd_rn(y0, __uint_as_float((uint32_t)g.bias[n + i] << 16));
-                        y1 = __fadd_rn(y1, __uint_as_float((uint32_t)g.bias[n + i + 1] << 16));
-                    }
-                    packed[i / 2] = f32x2_to_bf16x2(y0, y1);
-                }
-                uint4* dst = reinterpret_cast<uint4*>(g.out + (int64_t)row * g.N + n);
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    if (q * 8 < valid)
-                        dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2],
-                                            packed[4 * q + 3]);
+                store_row_chunk(g, v, sa, row, n);
             }
             // this warp's reads of the accumulator are done: hand it back
             tc_fence_before_sync();
@@ -348,6 +355,241 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after_sync();
         tmem_dealloc(tmem, T::kTmemCols);
     }
+}
+
+// ------------------------------------------------- two-CTA (pair) kernel --
+// A cluster of two CTAs on neighbouring SMs computes a 256 x 256 tile with
+// tcgen05.mma.cta_group::2 (M = 256, N = 256): each CTA loads 128 rows of A
+// and 128 rows of B per k-tile (32 KB instead of the one-CTA kernel's 48 KB
+// for the same MMA work per SM) and holds 128 accumulator rows x 256 columns
+// of the tile, twice (double buffer).  The even CTA of the pair (the
+// leader) arms the stage barriers and issues the MMAs, which read both CTAs'
+// shared memory; both CTAs' loads complete on the leader's barriers.
+
+// Shared::cluster address of the same shared-memory location in CTA `rank`
+// of the cluster.
+__device__ __forceinline__ uint32_t peer_smem(const void* local, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(local)),
+                 "r"(rank));
+    return r;
+}
+
+// One arrival on an mbarrier given by its shared::cluster address.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" :: "r"(bar)
+                 : "memory");
+}
+
+// A load of the pair: lands in this CTA's shared memory and completes its
+// bytes on the barrier at the same offset in the pair's even CTA.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                                 int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];"
+        :
+        : "r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar) & 0xFEFFFFFFu), "r"(x), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t cols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(smem_u32(dst_smem)), "r"(cols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t cols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" :: "r"(taddr), "r"(cols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mma_f8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+        :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive once on the barrier at shared::cluster address `bar` when the
+// pair's tcgen05 operations issued so far by this thread have completed.
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 :: "r"(bar)
+                 : "memory");
+}
+
+// Instruction descriptor of the pair's MMA: as f8_idesc with M = 256.
+__host__ __device__ constexpr uint32_t f8_idesc_pair(int bn) {
+    return (1u << 4) | ((uint32_t)(bn >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+}
+
+struct PairTile {
+    static constexpr int kHalfBytes = 128 * kBK;            // 16 KB: 128 rows of A or of B
+    static constexpr int kStageBytes = 2 * kHalfBytes;      // this CTA's A half and B half
+    static constexpr int kStages = 6;                       // 192 KB
+    static constexpr int kTmemCols = 512;                   // two 256-column accumulators
+    static constexpr int kBarriers = 2 * kStages + 4 + 1;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarriers * 8 + 16;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    scaled_mm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
+                          const __grid_constant__ CUtensorMap tma_b, const GemmArgs g) {
+    using T = PairTile;
+    constexpr int S = T::kStages;
+    constexpr int BN = 256;  // the pair tile is 256 x 256
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * T::kStageBytes);  // leader's are used
+    uint64_t* empty = full + S;
+    uint64_t* acc_full = empty + S;       // [2]
+    uint64_t* acc_empty = acc_full + 2;   // [2], the leader's: both CTAs' epilogue warps
+    uint64_t* drained = acc_empty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();  // 0: the leader
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int tiles_n = (g.N + 255) / 256;
+    const int tiles = tiles_n * ((g.M + 255) / 256);
+    const int ktiles = (g.K + kBK - 1) / kBK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 8);  // 4 epilogue warps in each CTA of the pair
+        }
+        mbar_init(drained, 1);
+        fence_mbar_init_cluster();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, T::kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before_sync();
+    // both CTAs' barriers and tensor memory exist before either signals the other
+    cluster_arrive_release();
+    cluster_wait_acquire();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---- producer (each CTA): its 128 rows of A and of B per k-tile
+        if (lane == 0) {
+            int it = 0;
+            bool ok = true;
+            for (int t = pair; t < tiles && ok; t += npairs) {
+                const int m0 = (t / tiles_n) * 256 + (int)rank * 128;
+                const int n0 = (t % tiles_n) * 256 + (int)rank * 128;
+                for (int kt = 0; kt < ktiles; ++kt, ++it) {
+                    const int s = it % S;
+                    if (!wait_phase(&empty[s], ((it / S) & 1) ^ 1, g.err)) {
+                        ok = false;
+                        break;
+                    }
+                    // the leader arms its barrier for both CTAs' bytes; the
+                    // odd CTA's loads may land first (the count goes negative)
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * T::kStageBytes);
+                    uint8_t* dst = smem + s * T::kStageBytes;
+                    tma_load_2d_pair(dst, &tma_a, &full[s], kt * kBK, m0);
+                    tma_load_2d_pair(dst + T::kHalfBytes, &tma_b, &full[s], kt * kBK, n0);
+                }
+            }
+            // this CTA's loads in flight have landed once the MMAs released
+            // their stages (the empty barriers are this CTA's own)
+            for (int i = it > S ? it - S : 0; i < it; ++i)
+                wait_phase(&empty[i % S], (i / S) & 1, g.err);
+        }
+    } else if (warp == 1) {
+        // ---- MMA issue (the leader only)
+        if (rank == 0 && lane == 0) {
+            constexpr uint32_t idesc = f8_idesc_pair(BN);
+            const uint32_t peer = 1;
+            int it = 0, j = 0;
+            bool ok = true;
+            for (int t = pair; t < tiles && ok; t += npairs, ++j) {
+                const int buf = j & 1;
+                if (!wait_phase(&acc_empty[buf], ((j >> 1) & 1) ^ 1, g.err)) break;
+                tc_fence_after_sync();
+                const uint32_t d = tmem + (uint32_t)(buf * BN);
+                for (int kt = 0; kt < ktiles; ++kt, ++it) {
+                    const int s = it % S;
+                    if (!wait_phase(&full[s], (it / S) & 1, g.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint8_t* tile = smem + s * T::kStageBytes;
+                    const uint64_t ad = kmajor_sw128_desc(tile);
+                    const uint64_t bd = kmajor_sw128_desc(tile + T::kHalfBytes);
+#pragma unroll
+                    for (int k = 0; k < kBK / kMmaK; ++k) {
+                        const uint64_t step = (uint64_t)(k * kMmaK) >> 4;
+                        mma_f8_pair(d, ad + step, bd + step, idesc, (kt | k) != 0);
+                    }
+                    // both CTAs' stage s is free once these MMAs are done
+                    mma_commit_pair(smem_u32(&empty[s]));
+                    mma_commit_pair(peer_smem(&empty[s], peer));
+                }
+                mma_commit_pair(smem_u32(&acc_full[buf]));
+                mma_commit_pair(peer_smem(&acc_full[buf], peer));
+            }
+            mma_commit_pair(smem_u32(drained));
+            mma_commit_pair(peer_smem(drained, peer));
+        }
+        __syncwarp();
+    } else {
+        // ---- epilogue (each CTA): its 128 accumulator rows of the tile
+        const int quarter = warp & 3;
+        const uint32_t leader_acc_empty[2] = {peer_smem(&acc_empty[0], 0),
+                                              peer_smem(&acc_empty[1], 0)};
+        int j = 0;
+        for (int t = pair; t < tiles; t += npairs, ++j) {
+            const int buf = j & 1;
+            const int m0 = (t / tiles_n) * 256 + (int)rank * 128, n0 = (t % tiles_n) * 256;
+            bool have = wait_phase(&acc_full[buf], (j >> 1) & 1, g.err);
+            if (!__all_sync(0xFFFFFFFFu, have)) break;
+            tc_fence_after_sync();
+            const int row = m0 + quarter * 32 + lane;
+            const float sa = row < g.M ? g.a_scale[row] : 0.0f;
+            const uint32_t base = tmem + (uint32_t)(buf * BN) + ((uint32_t)(quarter * 32) << 16);
+            for (int c = 0; c < BN; c += 32) {
+                float v[32];
+                tmem_load_32(base + (uint32_t)c, v);
+                const int n = n0 + c;
+                if (row >= g.M || n >= g.N) continue;
+                store_row_chunk(g, v, sa, row, n);
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(leader_acc_empty[buf]);
+        }
+    }
+
+    // ---- teardown: every MMA of the pair is done before tensor memory is
+    // freed, and neither CTA leaves while the other may still use it
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        wait_phase(drained, 0, g.err);
+        tc_fence_after_sync();
+        tmem_dealloc_pair(tmem, T::kTmemCols);
+    }
+    cluster_arrive_release();
+    cluster_wait_acquire();
 }
 
 // ------------------------------------------------------------------- host --
@@ -414,6 +656,40 @@ cudaError_t launch_bn(const GemmArgs& g, const void* a, const void* b, int sm_co
     return cudaGetLastError();
 }
 
+cudaError_t launch_pair(const GemmArgs& g, const void* a, const void* b, int sm_count,
+                        cudaStream_t stream) {
+    using T = PairTile;
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, a, g.M, g.K, 128) || !make_map(&mb, b, g.N, g.K, 128))
+        return cudaErrorInvalidValue;
+    static std::atomic<uint64_t> enabled_on{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
+    if (bit == 0 || (enabled_on.load(std::memory_order_relaxed) & bit) == 0) {
+        e = cudaFuncSetAttribute(scaled_mm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 T::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        enabled_on.fetch_or(bit, std::memory_order_relaxed);
+    }
+    const int64_t tiles = (int64_t)((g.N + 255) / 256) * ((g.M + 255) / 256);
+    const int64_t pairs = tiles < sm_count / 2 ? tiles : sm_count / 2;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = T::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, scaled_mm_pair_kernel, ma, mb, g);
+}
+
 }  // namespace
 
 cudaError_t launch_scaled_mm(const GemmArgs& g, const void* a, const void* b, int sm_count,
@@ -422,6 +698,9 @@ cudaError_t launch_scaled_mm(const GemmArgs& g, const void* a, const void* b, in
     // problems (decode batches against a weight) take 128 x 64 tiles, the
     // most CTAs streaming the weight.
     const int64_t row_tiles = (g.M + kBM - 1) / kBM;
+    // large products: 256 x 256 tiles on SM pairs once they fill every pair
+    if (((g.M + 255) / 256) * ((g.N + 255) / 256) >= sm_count / 2)
+        return launch_pair(g, a, b, sm_count, stream);
     if (row_tiles * ((g.N + 255) / 256) >= sm_count)
         return launch_bn<256, kBM>(g, a, b, sm_count, stream);
     if (row_tiles * ((g.N + 127) / 128) >= sm_count)
