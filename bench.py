@@ -910,6 +910,21 @@ def run_gemm_only(M: int, N: int, K: int):
     print(json.dumps({"gemm_fp8": rec}), flush=True)
 
 
+def run_one_secondary(key, fn, *args):
+    """One secondary measurement alone (profiling runs); prints its record."""
+    import torch
+
+    import reduce_rmsnorm_fp8_b200 as rrf
+    device = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(device)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    if fn is time_sharded:
+        rec = fn(rrf, *args, device, stream, l2, measured_peaks()[0])
+    else:
+        rec = fn(rrf, *args, device, stream, l2)
+    print(json.dumps({key: rec}), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description="fused sum + RMSNorm + FP8 benchmark")
     ap.add_argument("--gpus", type=int, default=1)
@@ -926,6 +941,12 @@ def main(argv=None):
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--gemm", type=int, nargs=3, metavar=("M", "N", "K"), default=None,
                     help="time only the FP8 GEMM of this shape (profiling runs)")
+    ap.add_argument("--allreduce", nargs=4, metavar=("WORKLOAD", "ROWS", "RANKS", "MODE"),
+                    default=None, help="time only the multi-GPU call, all ranks in one launch "
+                                       "(MODE 0 auto, 1 one-shot, 2 two-shot; profiling runs)")
+    ap.add_argument("--sharded", nargs=4, metavar=("WORKLOAD", "ROWS", "COLS", "SHARDS"),
+                    default=None, help="time only the two phases of the sharded form on one "
+                                       "shard (profiling runs)")
     args = ap.parse_args(argv)
     global ROWS_OVERRIDE
     if args.rows:
@@ -934,6 +955,13 @@ def main(argv=None):
         ap.error("--warmup must be at least 3")
     if args.gemm is not None:
         run_gemm_only(*args.gemm)
+    elif args.allreduce is not None:
+        w, rows, ranks, mode = args.allreduce
+        run_one_secondary("allreduce_emulated", time_allreduce, w, int(rows), int(ranks),
+                          int(mode))
+    elif args.sharded is not None:
+        w, rows, cols, shards = args.sharded
+        run_one_secondary("sharded", time_sharded, w, int(rows), int(cols), int(shards))
     elif args.impl == "reference":
         run_reference(args)
     else:

@@ -45,7 +45,14 @@ __global__ void __launch_bounds__(kPostThreads) post_kernel(const PostArgs a, in
     const int64_t left = a.rows - row0;
     const int nrows = left < RB ? (int)left : RB;
 
-    // the data of this warp's rows first
+    // the data of this warp's rows and the chunk's gamma first: every global
+    // load of the block is in flight before its first barrier
+    uint4 gv[kPostVecsPerLane];
+#pragma unroll
+    for (int j = 0; j < kPostVecsPerLane; ++j) {
+        const int v = v0 + lane + 32 * j;
+        gv[j] = v < a.vecs ? ld_shared_by_all(a.gamma + v) : make_uint4(0, 0, 0, 0);
+    }
     uint4 hv[RPW][kPostVecsPerLane];
 #pragma unroll
     for (int k = 0; k < RPW; ++k) {
@@ -78,12 +85,6 @@ __global__ void __launch_bounds__(kPostThreads) post_kernel(const PostArgs a, in
     }
     __syncthreads();
 
-    uint4 gv[kPostVecsPerLane];
-#pragma unroll
-    for (int j = 0; j < kPostVecsPerLane; ++j) {
-        const int v = v0 + lane + 32 * j;
-        gv[j] = v < a.vecs ? ld_shared_by_all(a.gamma + v) : make_uint4(0, 0, 0, 0);
-    }
 #pragma unroll
     for (int k = 0; k < RPW; ++k) {
         const int r = warp + 4 * k;
