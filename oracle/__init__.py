@@ -82,6 +82,12 @@ class Oracle:
         lib.oracle_sum_rmsnorm_fp8_rows.argtypes = [
             ctypes.POINTER(u16p), ctypes.c_int, i64, i64, i64, vp, vp, vp,
             ctypes.c_float, ctypes.c_float, ctypes.c_float, vp, vp, vp, vp]
+        lib.oracle_mx_scale_code.restype = ctypes.c_uint8
+        lib.oracle_mx_scale_code.argtypes = [ctypes.c_float]
+        lib.oracle_sum_rmsnorm_mxfp8_rows.restype = None
+        lib.oracle_sum_rmsnorm_mxfp8_rows.argtypes = [
+            ctypes.POINTER(u16p), ctypes.c_int, i64, i64, i64, vp, vp, vp, ctypes.c_float,
+            ctypes.c_float, vp, vp, vp, vp]
         lib.oracle_bf16_round_double.restype = ctypes.c_uint16
         lib.oracle_bf16_round_double.argtypes = [ctypes.c_double]
         lib.oracle_scaled_mm.restype = None
@@ -167,6 +173,45 @@ class Oracle:
         return out
 
 
+    def mx_scale_code(self, amax: float) -> int:
+        """E8M0 code of a block's shared scale from its max |V| (OCP MX)."""
+        return int(self.lib.oracle_mx_scale_code(float(amax)))
+
+    def sum_rmsnorm_mxfp8(self, inputs, rows: int, cols: int, gamma, eps: float,
+                          weight_offset: float, residual=None, row_start: int = 0,
+                          row_count: int | None = None, detail: bool = False) -> dict:
+        """The norm with MX output on rows [row_start, row_start + row_count):
+        ``q`` (uint8 [n, cols]), ``scales_mx`` (uint8 E8M0 codes
+        [n, cols / 32]), ``res_out`` with a residual; ``detail`` adds ``h``
+        and ``v`` (float32 y * 2^(127 - code))."""
+        if cols % 32:
+            raise ValueError("cols must be a multiple of 32")
+        if row_count is None:
+            row_count = rows - row_start
+        if not (0 <= row_start and row_start + row_count <= rows):
+            raise ValueError("row range out of bounds")
+        arrs, table = self._table(inputs, rows, cols)
+        g = np.ascontiguousarray(gamma, dtype=np.uint16).reshape(cols)
+        q = np.zeros((rows, cols), dtype=np.uint8)
+        sc = np.zeros((rows, cols // 32), dtype=np.uint8)
+        res_in = res_out = None
+        if residual is not None:
+            res_in = _bf16_rows(residual, rows, cols)
+            res_out = np.zeros((rows, cols), dtype=np.uint16)
+        h = np.zeros((rows, cols), dtype=np.uint16)
+        v = np.zeros((rows, cols), dtype=np.float32) if detail else None
+        self.lib.oracle_sum_rmsnorm_mxfp8_rows(
+            table, len(arrs), row_start, row_count, cols, _ptr(res_in), _ptr(res_out), _ptr(g),
+            eps, weight_offset, _ptr(q), _ptr(sc), _ptr(h), _ptr(v))
+        sl = slice(row_start, row_start + row_count)
+        out = {"q": q[sl].copy(), "scales_mx": sc[sl].copy()}
+        if res_out is not None:
+            out["res_out"] = res_out[sl].copy()
+        if detail:
+            out["h"] = h[sl].copy()
+            out["v"] = v[sl].copy()
+        return out
+
     def bf16_round_double(self, values) -> np.ndarray:
         """float64 -> nearest bf16 (ties to even) in one rounding, as uint16."""
         v = np.asarray(values, dtype=np.float64)
@@ -229,3 +274,7 @@ def bf16_round_double(values):
 
 def scaled_mm(*args, **kwargs):
     return default().scaled_mm(*args, **kwargs)
+
+
+def sum_rmsnorm_mxfp8(*args, **kwargs):
+    return default().sum_rmsnorm_mxfp8(*args, **kwargs)

@@ -50,6 +50,15 @@
  * of its per-token dynamic quantisation scenario: out = (x1_q @ x2) *
  * x1Scale * x2Scale + bias, one x1Scale per row of x1 and one x2Scale per
  * output column.
+ *
+ * The same page's mx scenario carries x1Scale of shape (BS, ceil(H/64), 2):
+ * one scale per 32 elements of a row.  oracle_sum_rmsnorm_mxfp8_rows gives
+ * the norm's output in that form, following the OCP Microscaling Formats
+ * (MX) v1.0 specification (conversion to MX, section 6.3): a block of 32
+ * elements shares the scale X = 2^(floor(log2(max |V|)) - 8), 8 being the
+ * exponent of e4m3's largest normal (448 = 1.75 * 2^8), stored as an E8M0
+ * code (the exponent biased by 127); each element is V / X rounded to
+ * e4m3fn, nearest even, saturating.
  */
 #include <math.h>
 #include <stddef.h>
@@ -275,6 +284,73 @@ void oracle_scaled_mm(const uint8_t* a, const float* a_scale, const uint8_t* b,
             if (bias != NULL) y += (double)oracle_bf16_to_float(bias[n]);
             if (exact != NULL) exact[m * N + n] = y;
             out[m * N + n] = oracle_bf16_round_double(y);
+        }
+    }
+}
+
+/* ------------------------------------------- MX (block-scaled) output --- */
+
+#define MX_BLOCK 32
+
+/* E8M0 code of a block's shared scale from the block's max |V|: the biased
+ * exponent of 2^(floor(log2(amax)) - 8), clamped to the codes of finite
+ * scales (0..254).  An all-zero block takes code 0 (a reading: the
+ * specification leaves the scale of a zero block free). */
+uint8_t oracle_mx_scale_code(float amax) {
+    if (!(amax > 0.0f)) return 0;
+    int e;
+    frexp((double)amax, &e); /* amax = f * 2^e with 0.5 <= f < 1: floor(log2(amax)) = e - 1 */
+    int c = (e - 1) - 8 + 127;
+    if (c < 0) c = 0;
+    if (c > 254) c = 254;
+    return (uint8_t)c;
+}
+
+/* Steps 1-4 of the fused operation (the sum, the residual, r and y = (h *
+ * r) * g'), then per block of 32 columns: the E8M0 scale code from the
+ * block's max |y| and the codes e4m3fn(y * 2^(127 - code)) (a power-of-two
+ * scaling, exact in fp32 here).  scales_mx is [rows][cols / 32]; cols is a
+ * multiple of 32.  v_out (may be NULL) receives y * 2^(127 - code). */
+void oracle_sum_rmsnorm_mxfp8_rows(const uint16_t* const* x, int R, int64_t row0,
+                                   int64_t nrows, int64_t cols, const uint16_t* res_in,
+                                   uint16_t* res_out, const uint16_t* gamma, float eps,
+                                   float weight_offset, uint8_t* q, uint8_t* scales_mx,
+                                   uint16_t* h_out, float* v_out) {
+    const int64_t nblocks = cols / MX_BLOCK;
+    for (int64_t i = row0; i < row0 + nrows; ++i) {
+        const int64_t base = i * cols;
+        double ss = 0.0;
+        for (int64_t j = 0; j < cols; ++j) {
+            uint16_t h = sum_element(x, R, base + j);
+            if (res_in != NULL) {
+                float t = oracle_bf16_to_float(h) + oracle_bf16_to_float(res_in[base + j]);
+                h = oracle_bf16_round(t);
+                res_out[base + j] = h;
+            }
+            h_out[base + j] = h;
+            double hd = (double)oracle_bf16_to_float(h);
+            ss += hd * hd;
+        }
+        float ms = (float)ss / (float)cols;
+        float r = 1.0f / sqrtf(ms + eps);
+
+        for (int64_t b = 0; b < nblocks; ++b) {
+            float y[MX_BLOCK];
+            float amax = 0.0f;
+            for (int k = 0; k < MX_BLOCK; ++k) {
+                const int64_t j = b * MX_BLOCK + k;
+                float g = oracle_bf16_to_float(gamma[j]) + weight_offset;
+                y[k] = (oracle_bf16_to_float(h_out[base + j]) * r) * g;
+                if (fabsf(y[k]) > amax) amax = fabsf(y[k]);
+            }
+            uint8_t c = oracle_mx_scale_code(amax);
+            scales_mx[i * nblocks + b] = c;
+            float inv_x = ldexpf(1.0f, 127 - (int)c);
+            for (int k = 0; k < MX_BLOCK; ++k) {
+                float v = y[k] * inv_x;
+                if (v_out != NULL) v_out[base + b * MX_BLOCK + k] = v;
+                q[base + b * MX_BLOCK + k] = oracle_e4m3_encode(v);
+            }
         }
     }
 }

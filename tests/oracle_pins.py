@@ -471,6 +471,75 @@ def pin_row_independence(o):
         assert np.array_equal(whole[k], np.concatenate([p[k] for p in parts])), k
 
 
+# ------------------------------------------------------------- MX output ---
+# The OCP MX v1.0 conversion: a block of 32 elements shares X = 2^(floor(
+# log2(max |V|)) - 8) (e4m3's largest normal is 1.75 * 2^8), an E8M0 code;
+# elements are V / X rounded to e4m3fn, nearest even, saturating.
+
+def e8m0_value(codes) -> np.ndarray:
+    """E8M0 codes -> values by ml_dtypes' float8_e8m0fnu decoding."""
+    return np.asarray(codes, dtype=np.uint8).view(ml_dtypes.float8_e8m0fnu).astype(np.float64)
+
+
+def pin_mx_scale_code(o):
+    """The code's scale X is the power of two with 256 <= amax / X < 512."""
+    rng = np.random.default_rng(41)
+    amax = np.concatenate([np.exp2(np.arange(-100.0, 120.0)),
+                           rng.uniform(0.5, 2.0, 300) * np.exp2(rng.integers(-110, 110, 300))])
+    for a in amax.astype(np.float32):
+        x = e8m0_value(o.mx_scale_code(float(a)))
+        assert 256.0 <= float(a) / x < 512.0, (a, x)
+    assert o.mx_scale_code(0.0) == 0
+
+
+def pin_mx_blocks_vs_row_scaled_oracle(o):
+    """On a random problem: every block's largest |v| lies in [256, 512);
+    the codes are torch's saturating conversion of v; v * X is the same y as
+    the row-scaled (pinned) path's v * scale; h and the residual agree."""
+    R, rows, cols = 3, 4, 256
+    xs = [rand_bf16(43 + r, (rows, cols)) for r in range(R)]
+    res = rand_bf16(50, (rows, cols))
+    gamma = rand_bf16(51, cols, 0.1, 1.0)
+    mx = o.sum_rmsnorm_mxfp8(xs, rows, cols, gamma, 1e-5, 0.0, residual=res, detail=True)
+    ref = o.sum_rmsnorm_fp8(xs, rows, cols, gamma, 1e-5, 0.0, 1e30, residual=res, detail=True)
+    v = mx["v"].reshape(rows, cols // 32, 32)
+    m = np.abs(v).max(axis=2)
+    assert np.all((m >= 256.0) & (m < 512.0))
+    assert np.array_equal(mx["q"], lib_e4m3_torch(mx["v"]))
+    X = np.repeat(e8m0_value(mx["scales_mx"]), 32, axis=1)
+    y_mx = mx["v"].astype(np.float64) * X
+    y_row = ref["v"].astype(np.float64) * ref["scales"].astype(np.float64)[:, None]
+    assert np.all(np.abs(y_mx - y_row) <= 2.0 ** -22 * np.abs(y_row) + 1e-30)
+    assert np.array_equal(mx["h"], ref["h"]) and np.array_equal(mx["res_out"], ref["res_out"])
+
+
+def pin_mx_block_isolation(o):
+    """Row of ones with one 64 at column 52 (R = 1, gamma 1, no residual):
+    r = 1 / sqrt((127 + 4096) / 128 + eps); the 64 raises only block 1's
+    scale: codes floor(log2(64 r)) + 119 there, floor(log2(r)) + 119 elsewhere."""
+    cols = 128
+    row = np.ones((1, cols), np.float32)
+    row[0, 52] = 64.0
+    eps = 1e-6
+    mx = o.sum_rmsnorm_mxfp8([bf16_of(row)], 1, cols, bf16_of(np.ones(cols, np.float32)), eps,
+                             0.0, detail=True)
+    r = 1.0 / math.sqrt((127.0 + 4096.0) / cols + eps)
+    want = [math.floor(math.log2(r)) + 119] * 4
+    want[1] = math.floor(math.log2(64.0 * r)) + 119
+    assert mx["scales_mx"][0].tolist() == want
+
+
+def pin_mx_zero_block(o):
+    """A block of zeros: code 0 and zero codes; the other blocks unaffected."""
+    cols = 96
+    row = rand_bf16(52, (1, cols))
+    row[0, 32:64] = 0
+    gamma = bf16_of(np.ones(cols, np.float32))
+    mx = o.sum_rmsnorm_mxfp8([row], 1, cols, gamma, 1e-6, 0.0)
+    assert mx["scales_mx"][0, 1] == 0 and np.all(mx["q"][0, 32:64] == 0)
+    assert mx["scales_mx"][0, 0] > 0 and mx["scales_mx"][0, 2] > 0
+
+
 # --------------------------------------------------------------- FP8 GEMM ---
 # The consumer of the per-row scales (Ascend aclnnAlltoAllQuantMatmul,
 # per-token dynamic quantisation): out = RN_bf16((a_q @ b_q^T) * a_scale *

@@ -60,6 +60,12 @@ MUTANTS = [
     ("double rounding ties up", "pick = (fmod(k, 2.0) == 0.0) ? lo : hi;", "pick = hi;"),
     ("double rounding truncates", "else if (hi - a < a - lo) pick = hi;", "else if (0) pick = hi;"),
     ("double rounding 7 significant bits", "int q_exp = e - 8;", "int q_exp = e - 7;"),
+    ("MX scale rounded up", "int c = (e - 1) - 8 + 127;", "int c = e - 8 + 127;"),
+    ("MX e4m3 exponent 7", "int c = (e - 1) - 8 + 127;", "int c = (e - 1) - 7 + 127;"),
+    ("MX amax over half a block", "if (fabsf(y[k]) > amax) amax = fabsf(y[k]);",
+     "if (k < 16 && fabsf(y[k]) > amax) amax = fabsf(y[k]);"),
+    ("MX zero block scale 1", "if (!(amax > 0.0f)) return 0;", "if (!(amax > 0.0f)) return 127;"),
+    ("MX scale applied as a multiplier", "float v = y[k] * inv_x;", "float v = y[k] / inv_x;"),
 ]
 
 
