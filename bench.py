@@ -442,6 +442,45 @@ def time_gemm(rrf, M, N, K, device, stream, l2, hbm_peak):
             "operand_sets": n, "device_error": rrf.rrf_device_error(clear=True)}
 
 
+def mx_bytes(R: int, rows: int, cols: int, residual: bool) -> int:
+    """Algorithmic HBM bytes of one MX call: as the row-scaled call, with one
+    E8M0 byte per 32 elements in place of one float per row."""
+    return R * rows * cols * 2 + (4 * rows * cols if residual else 0) + cols * 2 \
+        + rows * cols + rows * cols // 32
+
+
+def time_mx(rrf, label, rows, device, stream, l2, peak):
+    """The MX output (rrf_sum_rmsnorm_mxfp8) on one configuration, one CUDA
+    graph of calls cycling through buffer sets larger than 3 x L2."""
+    import torch
+    c = workloads.make_case(label, rows, device=device)
+    nbytes = mx_bytes(c.R, rows, c.cols, c.residual is not None)
+    n = max(2, math.ceil(L2_FLUSH_FACTOR * l2 / nbytes))
+    rep = lambda t: t.unsqueeze(0).repeat(n, *([1] * t.dim()))
+    xs = [rep(x) for x in c.inputs]
+    res = None if c.residual is None else rep(c.residual)
+    q = torch.empty((n, rows, c.cols), dtype=torch.float8_e4m3fn, device=device)
+    sc = torch.empty((n, rows, c.cols // 32), dtype=torch.uint8, device=device)
+
+    def call(k):
+        i = k % n
+        r = None if res is None else res[i]
+        rrf.rrf_sum_rmsnorm_mxfp8([x[i] for x in xs], c.gamma, c.eps, c.weight_offset,
+                                  residual_in=r, residual_out=r, q_out=q[i], scales_mx_out=sc[i])
+        return 1
+
+    for k in range(3):
+        call(k)
+    reps = max(n, 100) if rows < 1024 else 10
+    g, _ = capture_steps(call, reps, device)
+    g.replay()
+    torch.cuda.synchronize(device)
+    t = time_region(lambda _: g.replay(), 1, device, stream) / reps
+    del g, xs, res, q, sc
+    return {"case": f"{label} {rows} x {c.cols}", "R": c.R, "us_per_call": round(t * 1e6, 3),
+            "GB_s": round(nbytes / t / 1e9, 1), "frac": round(nbytes / t / 1e9 / peak, 4)}
+
+
 def capture_steps(fn, n: int, device):
     """Capture fn(0) .. fn(n-1) into one CUDA graph; returns (graph, number
     of kernels fn launched)."""
@@ -786,6 +825,14 @@ def run_rrf(args):
                                                      ("prefill", 8192, 8, 0))]
         torch.cuda.empty_cache()
 
+    # ---- the MX output (per-32-element scales)
+    mx = None
+    if not args.no_secondary:
+        mx = [time_mx(rrf, label, rows, device, stream, l2, peak)
+              for label, rows in (("decode", 1), ("decode", 8), ("decode", 32), ("decode", 64),
+                                  ("prefill", 8192))]
+        torch.cuda.empty_cache()
+
     # ---- the FP8 GEMM that consumes the per-row scales
     gemm = None
     if not args.no_secondary:
@@ -840,6 +887,7 @@ def run_rrf(args):
             "other_configs": others,
             "sharded": sharded,
             "allreduce_emulated": emulated,
+            "mx": mx,
             "gemm_fp8": gemm,
             "cpu_baseline": cpu,
         }

@@ -188,6 +188,39 @@ rrf_status rrf_sum_rmsnorm_fp8_ex(const void* const* inputs, int num_inputs,
                                   int block_threads, int flags, rrf_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * MX output: per-block instead of per-row scales.
+ *
+ * Ascend CANN docs, aclnnAlltoAllQuantMatmul, mx scenario: the activations'
+ * x1Scale has shape (BS, ceil(H/64), 2), one scale per 32 elements of a row.
+ * OCP Microscaling Formats (MX) v1.0, conversion to MX: a block of 32
+ * elements shares X = 2^(floor(log2(max |V|)) - 8) (8 being the exponent of
+ * e4m3's largest normal, 448 = 1.75 * 2^8), stored as an E8M0 code (the
+ * exponent biased by 127); each element becomes e4m3fn(V / X), nearest even,
+ * saturating.
+ *
+ * rrf_sum_rmsnorm_mxfp8 -- the sum, the residual and the norm as in
+ * rrf_sum_rmsnorm_fp8, then per block of 32 columns of y the E8M0 code of the
+ * block's scale and the codes of y / X (no scale_ub: the scale follows the
+ * block).  An all-zero block takes code 0.
+ * inputs, num_inputs, rows, residual_in, residual_out, gamma, eps,
+ * weight_offset   as for rrf_sum_rmsnorm_fp8
+ * cols            a multiple of 32
+ * q_out           fp8 e4m3fn codes [rows, cols], 16-byte aligned
+ * scales_mx_out   E8M0 codes [rows, cols / 32] (one byte each)
+ * Errors: RRF_ERR_NULL, RRF_ERR_RANKS, RRF_ERR_SHAPE, RRF_ERR_ALIGN,
+ *         RRF_ERR_ALIAS, RRF_ERR_VALUE, RRF_ERR_CUDA. */
+rrf_status rrf_sum_rmsnorm_mxfp8(const void* const* inputs, int num_inputs, int64_t rows,
+                                 int64_t cols, const void* residual_in, void* residual_out,
+                                 const void* gamma, float eps, float weight_offset, void* q_out,
+                                 void* scales_mx_out, rrf_stream_t stream);
+
+/* The host validation of rrf_sum_rmsnorm_mxfp8 alone (no GPU needed). */
+rrf_status rrf_check_mxfp8_args(const void* const* inputs, int num_inputs, int64_t rows,
+                                int64_t cols, const void* residual_in, const void* residual_out,
+                                const void* gamma, float eps, float weight_offset,
+                                const void* q_out, const void* scales_mx_out);
+
+/* ------------------------------------------------------------------------
  * The sharded form: a row's hidden dimension split across devices.
  *
  * Tenstorrent rmsnorm_2d.py (RMSNorm2D, decode_forward / prefill_forward)

@@ -104,6 +104,12 @@ lib.rrf_check_allreduce_args.restype = _int
 lib.rrf_check_allreduce_args.argtypes = _ar_args
 lib.rrf_plan_allreduce.restype = _int
 lib.rrf_plan_allreduce.argtypes = [_int, _i64, _i64, _int, _int, _int] + [ctypes.POINTER(_int)] * 4
+lib.rrf_sum_rmsnorm_mxfp8.restype = _int
+lib.rrf_sum_rmsnorm_mxfp8.argtypes = [_ptrs, _int, _i64, _i64, _vp, _vp, _vp, _f32, _f32, _vp,
+                                      _vp, _vp]
+lib.rrf_check_mxfp8_args.restype = _int
+lib.rrf_check_mxfp8_args.argtypes = [_ptrs, _int, _i64, _i64, _vp, _vp, _vp, _f32, _f32, _vp,
+                                     _vp]
 lib.rrf_scaled_mm_fp8.restype = _int
 lib.rrf_scaled_mm_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]
 lib.rrf_check_scaled_mm_args.restype = _int
@@ -307,6 +313,42 @@ def rrf_sum_rmsnorm_fp8(inputs, gamma, eps, weight_offset, scale_ub, residual_in
     float32 [..., 1], residual_out or None)."""
     return rrf_sum_rmsnorm_fp8_ex(inputs, gamma, eps, weight_offset, scale_ub, residual_in,
                                   residual_out, q_out, scales_out)
+
+
+def rrf_check_mxfp8_args(input_ptrs, rows, cols, residual_in, residual_out, gamma, eps,
+                         weight_offset, q_out, scales_mx_out) -> int:
+    return lib.rrf_check_mxfp8_args(_ptr_table(input_ptrs), len(input_ptrs), rows, cols,
+                                    residual_in or None, residual_out or None, gamma or None,
+                                    eps, weight_offset, q_out or None, scales_mx_out or None)
+
+
+def rrf_sum_rmsnorm_mxfp8(inputs, gamma, eps, weight_offset, residual_in=None,
+                          residual_out=None, q_out=None, scales_mx_out=None):
+    """The fused operation with MX output: one E8M0 scale code per 32
+    elements.  Returns (q: float8_e4m3fn like the inputs, scales_mx: uint8
+    [..., cols / 32], residual_out or None)."""
+    torch = _torch()
+    rows, cols = _rows_cols(inputs)
+    x0 = inputs[0]
+    dev = x0.device
+    if gamma.dtype != torch.bfloat16 or gamma.numel() != cols or gamma.device != dev:
+        raise ValueError("gamma must be a bf16 tensor of length cols on the inputs' device")
+    if cols % 32:
+        raise ValueError("cols must be a multiple of 32")
+    if residual_in is not None and residual_out is None:
+        residual_out = torch.empty_like(residual_in)
+    if q_out is None:
+        q_out = torch.empty(x0.shape, dtype=torch.float8_e4m3fn, device=dev)
+    if scales_mx_out is None:
+        scales_mx_out = torch.empty(tuple(x0.shape[:-1]) + (cols // 32,), dtype=torch.uint8,
+                                    device=dev)
+    with torch.cuda.device(dev):
+        _raise_on(lib.rrf_sum_rmsnorm_mxfp8(
+            _ptr_table([x.data_ptr() for x in inputs]), len(inputs), rows, cols,
+            residual_in.data_ptr() if residual_in is not None else None,
+            residual_out.data_ptr() if residual_out is not None else None, gamma.data_ptr(),
+            eps, weight_offset, q_out.data_ptr(), scales_mx_out.data_ptr(), _stream(dev)))
+    return q_out, scales_mx_out, residual_out
 
 
 # ------------------------------------------------------------ sharded norm ---

@@ -372,6 +372,89 @@ extern "C" rrf_status rrf_sum_rmsnorm_fp8(const void* const* inputs, int num_inp
                                   RRF_VARIANT_AUTO, 0, 0, 0, stream);
 }
 
+// ------------------------------------------------------------ MX output ---
+
+extern "C" rrf_status rrf_check_mxfp8_args(const void* const* inputs, int num_inputs,
+                                           int64_t rows, int64_t cols, const void* residual_in,
+                                           const void* residual_out, const void* gamma,
+                                           float eps, float weight_offset, const void* q_out,
+                                           const void* scales_mx_out) {
+    rrf_status st = check_shape(num_inputs, rows, cols, RRF_MAX_COLS);
+    if (st != RRF_OK) return st;
+    if (cols % 32 != 0) return RRF_ERR_SHAPE;
+    if (!(std::isfinite(eps) && eps >= 0.0f)) return RRF_ERR_VALUE;
+    if (!std::isfinite(weight_offset)) return RRF_ERR_VALUE;
+    if (rows == 0) return RRF_OK;
+    if ((st = check_inputs(inputs, num_inputs)) != RRF_OK) return st;
+    if ((residual_in == nullptr) != (residual_out == nullptr)) return RRF_ERR_NULL;
+    if (gamma == nullptr || q_out == nullptr || scales_mx_out == nullptr) return RRF_ERR_NULL;
+    if (!aligned(gamma, 16) || !aligned(q_out, 16)) return RRF_ERR_ALIGN;
+    if (residual_in != nullptr && (!aligned(residual_in, 16) || !aligned(residual_out, 16)))
+        return RRF_ERR_ALIGN;
+    const int64_t bf16_bytes = rows * cols * 2;
+    Range reads[RRF_MAX_INPUTS + 2];
+    int n_reads = 0;
+    for (int r = 0; r < num_inputs; ++r) reads[n_reads++] = range_of(inputs[r], bf16_bytes);
+    reads[n_reads++] = range_of(gamma, cols * 2);
+    if (residual_in != nullptr && residual_in != residual_out)
+        reads[n_reads++] = range_of(residual_in, bf16_bytes);
+    Range writes[3];
+    int n_writes = 0;
+    writes[n_writes++] = range_of(q_out, rows * cols);
+    writes[n_writes++] = range_of(scales_mx_out, rows * (cols / 32));
+    if (residual_out != nullptr) writes[n_writes++] = range_of(residual_out, bf16_bytes);
+    for (int w = 0; w < n_writes; ++w) {
+        for (int r = 0; r < n_reads; ++r)
+            if (overlap(writes[w], reads[r])) return RRF_ERR_ALIAS;
+        for (int w2 = w + 1; w2 < n_writes; ++w2)
+            if (overlap(writes[w], writes[w2])) return RRF_ERR_ALIAS;
+    }
+    return RRF_OK;
+}
+
+extern "C" rrf_status rrf_sum_rmsnorm_mxfp8(const void* const* inputs, int num_inputs,
+                                            int64_t rows, int64_t cols, const void* residual_in,
+                                            void* residual_out, const void* gamma, float eps,
+                                            float weight_offset, void* q_out,
+                                            void* scales_mx_out, rrf_stream_t stream) {
+    rrf_status st = rrf_check_mxfp8_args(inputs, num_inputs, rows, cols, residual_in,
+                                         residual_out, gamma, eps, weight_offset, q_out,
+                                         scales_mx_out);
+    if (st != RRF_OK || rows == 0) return st;
+    int sm_count = 0;
+    if ((st = current_sm_count(&sm_count)) != RRF_OK) return st;
+    FusedLaunch l = {};
+    if ((st = shape_launch(num_inputs, rows, cols, sm_count, 0, 0, residual_in != nullptr,
+                           &l)) != RRF_OK)
+        return st;
+    l.mx = true;
+    unsigned int* err = nullptr;
+    if ((st = device_error_word(&err)) != RRF_OK) return st;
+    const int64_t vecs = cols / 8;
+    FusedArgs a = {};
+    for (int r = 0; r < num_inputs; ++r) a.in[r] = static_cast<const uint4*>(inputs[r]);
+    a.res_in = static_cast<const uint4*>(residual_in);
+    a.res_out = static_cast<uint4*>(residual_out);
+    a.gamma = static_cast<const uint4*>(gamma);
+    a.q = static_cast<uint2*>(q_out);
+    a.scales_mx = static_cast<uint8_t*>(scales_mx_out);
+    a.R = num_inputs;
+    a.vecs = (int)vecs;
+    a.cluster = l.cluster;
+    // a cluster block's slice starts on a 32-element block (4 vectors); the
+    // block's threads (a multiple of 32) x vectors per thread still cover it
+    a.slice_vecs = (int)(((vecs + l.cluster - 1) / l.cluster + 3) / 4 * 4);
+    a.cols_f = (float)cols;
+    a.eps = eps;
+    a.weight_offset = weight_offset;
+    a.scale_ub = 1.0f;
+    a.err = err;
+    cudaError_t e;
+    if (!take_injected_failure(&e))
+        e = launch_fused(a, rows, l, residual_in != nullptr, (cudaStream_t)stream);
+    return e == cudaSuccess ? RRF_OK : cuda_fail(e);
+}
+
 // -------------------------------------------------------- sharded norm ---
 
 extern "C" rrf_status rrf_check_pre_args(const void* const* inputs, int num_inputs, int64_t rows,

@@ -34,10 +34,20 @@ namespace {
 constexpr float kE4m3Max = 448.0f;
 constexpr float kScaleFloor = 1e-12f;
 
+// E8M0 code of an MX block's shared scale 2^(floor(log2(amax)) - 8) (OCP MX
+// v1.0, e4m3 elements: 448 = 1.75 * 2^8): the biased exponent field of
+// amax minus 8, clamped at 0 (zero, subnormal and tiny maxima).
+__device__ __forceinline__ uint32_t mx_scale_code(float amax) {
+    const int e = (int)((__float_as_uint(amax) >> 23) & 0xFFu);
+    return e > 8 ? (uint32_t)(e - 8) : 0u;
+}
+
 // ASYNC (cluster rows only): the blocks of a cluster meet through the
 // transaction-counted exchange (st.async into the peers' shared memory,
 // bounded mbarrier waits) instead of a cluster barrier phase.
-template <int RB, int VPT, bool RES, bool CLUSTER, bool ASYNC>
+// MX: the output takes one E8M0 scale per 32 elements (4 vectors held by 4
+// consecutive lanes) instead of one scale per row.
+template <int RB, int VPT, bool RES, bool CLUSTER, bool ASYNC, bool MX = false>
 __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const FusedArgs a) {
     static_assert(CLUSTER || !ASYNC, "the exchange is between the blocks of a cluster");
     __shared__ RowStats warp_stats[32];
@@ -143,29 +153,65 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
     const float inv_scale = 1.0f / scale;
 
     // ---- last pass: quantise
+    if constexpr (MX) {
+        // A block of 32 elements is the vectors of lanes 4i .. 4i+3 (slices
+        // and block sizes are multiples of 4 vectors): its max |y| by two
+        // shuffles, which every lane executes.
 #pragma unroll
-    for (int k = 0; k < VPT; ++k) {
-        const int v = v_begin + tid + k * T;
-        if (v < v_end) {
-            float hf[8], gf[8], qv[8];
-            bf16x8_to_f32(h[k], hf);
-            bf16x8_to_f32(KEEP_GAMMA ? g[k] : ld_shared_by_all(a.gamma + v), gf);
+        for (int k = 0; k < VPT; ++k) {
+            const int v = v_begin + tid + k * T;
+            const bool live = v < v_end;  // the same for the 4 lanes of a block
+            float y[8];
+            float bmax = 0.0f;
+            if (live) {
+                float hf[8], gf[8];
+                bf16x8_to_f32(h[k], hf);
+                bf16x8_to_f32(KEEP_GAMMA ? g[k] : ld_shared_by_all(a.gamma + v), gf);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float y = __fmul_rn(__fmul_rn(hf[e], rinv), __fadd_rn(gf[e], a.weight_offset));
-                qv[e] = __fmul_rn(y, inv_scale);
+                for (int e = 0; e < 8; ++e) {
+                    y[e] = __fmul_rn(__fmul_rn(hf[e], rinv), __fadd_rn(gf[e], a.weight_offset));
+                    bmax = fmaxf(bmax, fabsf(y[e]));
+                }
             }
-            st_once(a.q + row_base + v, f32_to_e4m3x8(qv));
-            if (RES && CLUSTER) st_once(a.res_out + row_base + v, h[k]);
+            bmax = fmaxf(bmax, __shfl_xor_sync(0xFFFFFFFFu, bmax, 1));
+            bmax = fmaxf(bmax, __shfl_xor_sync(0xFFFFFFFFu, bmax, 2));
+            if (live) {
+                const uint32_t code = mx_scale_code(bmax);
+                const float inv_x = __uint_as_float((254u - code) << 23);  // 2^(127 - code)
+                float qv[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) qv[e] = __fmul_rn(y[e], inv_x);
+                st_once(a.q + row_base + v, f32_to_e4m3x8(qv));
+                if ((v & 3) == 0) a.scales_mx[(row_base + v) >> 2] = (uint8_t)code;
+                if (RES && CLUSTER) st_once(a.res_out + row_base + v, h[k]);
+            }
         }
+    } else {
+#pragma unroll
+        for (int k = 0; k < VPT; ++k) {
+            const int v = v_begin + tid + k * T;
+            if (v < v_end) {
+                float hf[8], gf[8], qv[8];
+                bf16x8_to_f32(h[k], hf);
+                bf16x8_to_f32(KEEP_GAMMA ? g[k] : ld_shared_by_all(a.gamma + v), gf);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float y =
+                        __fmul_rn(__fmul_rn(hf[e], rinv), __fadd_rn(gf[e], a.weight_offset));
+                    qv[e] = __fmul_rn(y, inv_scale);
+                }
+                st_once(a.q + row_base + v, f32_to_e4m3x8(qv));
+                if (RES && CLUSTER) st_once(a.res_out + row_base + v, h[k]);
+            }
+        }
+        if (tid == 0 && rank == 0) a.scales[row] = scale;
     }
-    if (tid == 0 && rank == 0) a.scales[row] = scale;
 }
 
-template <int RB, int VPT, bool RES, bool CLUSTER, bool ASYNC>
+template <int RB, int VPT, bool RES, bool CLUSTER, bool ASYNC, bool MX>
 cudaError_t launch_one(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
                        cudaStream_t stream) {
-    auto kernel = fused_kernel<RB, VPT, RES, CLUSTER, ASYNC>;
+    auto kernel = fused_kernel<RB, VPT, RES, CLUSTER, ASYNC, MX>;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(rows * l.cluster), 1, 1);
     cfg.blockDim = dim3((unsigned)l.threads, 1, 1);
@@ -203,24 +249,32 @@ cudaError_t launch_one(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
     return cudaLaunchKernelEx(&cfg, kernel, a);
 }
 
-template <int RB, bool RES, bool CLUSTER, bool ASYNC>
+template <int RB, bool RES, bool CLUSTER, bool ASYNC, bool MX>
 cudaError_t launch_vpt(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
                        cudaStream_t stream) {
     switch (l.vecs_per_thread) {
-        case 1: return launch_one<RB, 1, RES, CLUSTER, ASYNC>(a, rows, l, stream);
-        case 2: return launch_one<RB, 2, RES, CLUSTER, ASYNC>(a, rows, l, stream);
-        case 4: return launch_one<RB, 4, RES, CLUSTER, ASYNC>(a, rows, l, stream);
-        case 8: return launch_one<RB, 8, RES, CLUSTER, ASYNC>(a, rows, l, stream);
+        case 1: return launch_one<RB, 1, RES, CLUSTER, ASYNC, MX>(a, rows, l, stream);
+        case 2: return launch_one<RB, 2, RES, CLUSTER, ASYNC, MX>(a, rows, l, stream);
+        case 4: return launch_one<RB, 4, RES, CLUSTER, ASYNC, MX>(a, rows, l, stream);
+        case 8: return launch_one<RB, 8, RES, CLUSTER, ASYNC, MX>(a, rows, l, stream);
         default: return cudaErrorInvalidValue;
     }
 }
 
+// The MX output exists with one block per row or the transaction-counted
+// cluster exchange (the library's choice); the barrier exchange is a test
+// and benchmark option of the row-scaled output only.
 template <int RB, bool RES>
 cudaError_t launch_shape(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
                          cudaStream_t stream) {
-    if (l.cluster == 1) return launch_vpt<RB, RES, false, false>(a, rows, l, stream);
-    return l.async_exchange ? launch_vpt<RB, RES, true, true>(a, rows, l, stream)
-                            : launch_vpt<RB, RES, true, false>(a, rows, l, stream);
+    if (l.mx) {
+        if (l.cluster == 1) return launch_vpt<RB, RES, false, false, true>(a, rows, l, stream);
+        if (!l.async_exchange) return cudaErrorInvalidValue;
+        return launch_vpt<RB, RES, true, true, true>(a, rows, l, stream);
+    }
+    if (l.cluster == 1) return launch_vpt<RB, RES, false, false, false>(a, rows, l, stream);
+    return l.async_exchange ? launch_vpt<RB, RES, true, true, false>(a, rows, l, stream)
+                            : launch_vpt<RB, RES, true, false, false>(a, rows, l, stream);
 }
 
 }  // namespace

@@ -41,6 +41,8 @@ struct FusedArgs {
     int stats_only;
     float2* stats;         // [rows]
     uint4* h_out;          // [rows, cols] or null (with a residual, res_out holds h)
+    // MX output: one E8M0 scale code per 32 elements instead of scales
+    uint8_t* scales_mx;    // [rows, cols / 32]
 };
 
 // The second phase of the sharded norm: quantise one column shard from the
@@ -119,6 +121,7 @@ struct FusedLaunch {
     int vecs_per_thread;  // 1, 2, 4 or 8
     bool pdl;             // launch with programmatic stream serialization
     bool async_exchange;  // clusters meet through st.async + mbarrier waits
+    bool mx = false;      // MX output (per-32-element scales)
 };
 
 // The fused kernel is compiled for input-count bounds RB in {2, 4, 8, 16}

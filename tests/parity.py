@@ -108,3 +108,51 @@ def assert_fused_parity(gpu: dict, ref: dict, label: str = "", cap_at_ties: bool
         step = np.abs((qg[diff] & 0x7F).astype(int) - (qr[diff] & 0x7F).astype(int))
         assert same_sign.all() and (step == 1).all(), f"{label}: a code differs by > 1 step"
     return {"scale_max_rel": float(rel.max()), "codes_differing": n_diff}
+
+
+def oracle_mx(case: workloads.Case, rows=None) -> dict:
+    """The oracle's MX output on the case (all rows, or the listed rows)."""
+    bits = workloads.bits
+    if rows is None:
+        xs = [bits(x) for x in case.inputs]
+        res = None if case.residual is None else bits(case.residual)
+        n = case.rows
+    else:
+        idx = torch.as_tensor(np.asarray(rows), device=case.inputs[0].device)
+        xs = [bits(x.index_select(0, idx)) for x in case.inputs]
+        res = None if case.residual is None else bits(case.residual.index_select(0, idx))
+        n = len(rows)
+    return oracle.sum_rmsnorm_mxfp8(xs, n, case.cols, bits(case.gamma), case.eps,
+                                    case.weight_offset, residual=res, detail=True)
+
+
+def assert_mx_parity(gpu: dict, ref: dict, label: str = "", cap_at_ties: bool = False) -> dict:
+    """MX output: the residual bit for bit; the E8M0 codes equal except in
+    blocks whose max |y| lies within 1e-6 of a power of two (where the last
+    bit of r decides floor(log2)), and there at most one step apart; within
+    blocks of equal codes, the element codes as for the row-scaled output
+    (one step, at an e4m3 midpoint, on at most 0.1% of them)."""
+    if "res_out" in ref:
+        assert np.array_equal(gpu["res_out"], ref["res_out"]), f"{label}: residual_out differs"
+    sg, sr = gpu["scales_mx"].astype(int), ref["scales_mx"].astype(int)
+    rows, nb = sr.shape
+    vmax = np.abs(ref["v"].astype(np.float64)).reshape(rows, nb, 32).max(axis=2)
+    edge = (vmax * (1 - CODE_MIDPOINT_RTOL) < 256.0) | (vmax * (1 + CODE_MIDPOINT_RTOL) >= 512.0)
+    diff = sg != sr
+    assert not np.any(diff & ~edge), f"{label}: a block scale differs away from a power of two"
+    assert np.all(np.abs(sg - sr)[diff] <= 1), f"{label}: a block scale differs by > 1"
+    same = np.repeat(~diff, 32, axis=1)
+    qg, qr = gpu["q"][same], ref["q"][same]
+    dq = qg != qr
+    n_diff = int(dq.sum())
+    if n_diff:
+        near = midpoint_distance(ref["v"][same]) <= CODE_MIDPOINT_RTOL
+        cap = CODE_MISMATCH_FRACTION * qr.size
+        if cap_at_ties:
+            cap = max(cap, int(near.sum()))
+        assert n_diff <= cap, f"{label}: {n_diff} codes differ"
+        assert near[dq].all(), f"{label}: a code differs away from a rounding midpoint"
+        step = np.abs((qg[dq] & 0x7F).astype(int) - (qr[dq] & 0x7F).astype(int))
+        assert ((qg[dq] & 0x80) == (qr[dq] & 0x80)).all() and (step == 1).all(), \
+            f"{label}: a code differs by > 1 step"
+    return {"scale_blocks_differing": int(diff.sum()), "codes_differing": n_diff}

@@ -404,3 +404,20 @@ def test_scaled_mm_validation(rrf):
         kw = dict(ok)
         kw.update(change)
         assert rrf.rrf_check_scaled_mm_args(**kw) == rrf.Status[status], change
+
+
+def test_mxfp8_validation(rrf):
+    ins = [A, 2 * A]
+    ok = dict(input_ptrs=ins, rows=8, cols=64, residual_in=0, residual_out=0, gamma=3 * A,
+              eps=1e-5, weight_offset=0.0, q_out=4 * A, scales_mx_out=5 * A + 1)
+    assert rrf.rrf_check_mxfp8_args(**ok) == rrf.Status.OK  # scale codes are bytes
+    for change, status in [
+            (dict(cols=48), "ERR_SHAPE"),                    # not a multiple of 32
+            (dict(scales_mx_out=0), "ERR_NULL"),
+            (dict(q_out=4 * A + 8), "ERR_ALIGN"),
+            (dict(scales_mx_out=A + 100), "ERR_ALIAS"),      # inside an input
+            (dict(scales_mx_out=4 * A + 8 * 64 - 1), "ERR_ALIAS"),  # the codes' last byte
+            (dict(eps=-1.0), "ERR_VALUE")]:
+        kw = dict(ok)
+        kw.update(change)
+        assert rrf.rrf_check_mxfp8_args(**kw) == rrf.Status[status], change
