@@ -86,6 +86,8 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
     uint4 h[VPT];
     uint4 g[KEEP_GAMMA ? VPT : 1];
     RowStats st = stats_empty();
+    // MX: max |h * g'| over each vector's 32-element block (4 lanes)
+    float bkey[MX ? VPT : 1];
 
     // ---- pass 1: sum, residual, sum of squares, max |h * g'|
 #pragma unroll
@@ -127,8 +129,29 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
             float hf[8], gf[8];
             bf16x8_to_f32(s, hf);
             bf16x8_to_f32(gv, gf);
+            if constexpr (MX) {
+                RowStats vs = stats_empty();
 #pragma unroll
-            for (int e = 0; e < 8; ++e) stats_offer(st, hf[e], __fadd_rn(gf[e], a.weight_offset));
+                for (int e = 0; e < 8; ++e)
+                    stats_offer(vs, hf[e], __fadd_rn(gf[e], a.weight_offset));
+                bkey[k] = vs.key;
+                st.key = fmaxf(st.key, vs.key);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    stats_offer(st, hf[e], __fadd_rn(gf[e], a.weight_offset));
+            }
+        } else if constexpr (MX) {
+            bkey[k] = 0.0f;
+        }
+    }
+    if constexpr (MX) {
+        // A 32-element block is the vectors of lanes 4i .. 4i+3 (slices and
+        // block sizes are multiples of 4 vectors); every lane shuffles.
+#pragma unroll
+        for (int k = 0; k < VPT; ++k) {
+            bkey[k] = fmaxf(bkey[k], __shfl_xor_sync(0xFFFFFFFFu, bkey[k], 1));
+            bkey[k] = fmaxf(bkey[k], __shfl_xor_sync(0xFFFFFFFFu, bkey[k], 2));
         }
     }
 
@@ -154,33 +177,23 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
 
     // ---- last pass: quantise
     if constexpr (MX) {
-        // A block of 32 elements is the vectors of lanes 4i .. 4i+3 (slices
-        // and block sizes are multiples of 4 vectors): its max |y| by two
-        // shuffles, which every lane executes.
+        // The block's max |y| is r * its max |h * g'| (the same two products
+        // rounded in the other order, as for the row scale).
 #pragma unroll
         for (int k = 0; k < VPT; ++k) {
             const int v = v_begin + tid + k * T;
-            const bool live = v < v_end;  // the same for the 4 lanes of a block
-            float y[8];
-            float bmax = 0.0f;
-            if (live) {
-                float hf[8], gf[8];
+            if (v < v_end) {
+                const uint32_t code = mx_scale_code(__fmul_rn(bkey[k], rinv));
+                const float inv_x = __uint_as_float((254u - code) << 23);  // 2^(127 - code)
+                float hf[8], gf[8], qv[8];
                 bf16x8_to_f32(h[k], hf);
                 bf16x8_to_f32(KEEP_GAMMA ? g[k] : ld_shared_by_all(a.gamma + v), gf);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    y[e] = __fmul_rn(__fmul_rn(hf[e], rinv), __fadd_rn(gf[e], a.weight_offset));
-                    bmax = fmaxf(bmax, fabsf(y[e]));
+                    const float y =
+                        __fmul_rn(__fmul_rn(hf[e], rinv), __fadd_rn(gf[e], a.weight_offset));
+                    qv[e] = __fmul_rn(y, inv_x);
                 }
-            }
-            bmax = fmaxf(bmax, __shfl_xor_sync(0xFFFFFFFFu, bmax, 1));
-            bmax = fmaxf(bmax, __shfl_xor_sync(0xFFFFFFFFu, bmax, 2));
-            if (live) {
-                const uint32_t code = mx_scale_code(bmax);
-                const float inv_x = __uint_as_float((254u - code) << 23);  // 2^(127 - code)
-                float qv[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) qv[e] = __fmul_rn(y[e], inv_x);
                 st_once(a.q + row_base + v, f32_to_e4m3x8(qv));
                 if ((v & 3) == 0) a.scales_mx[(row_base + v) >> 2] = (uint8_t)code;
                 if (RES && CLUSTER) st_once(a.res_out + row_base + v, h[k]);
