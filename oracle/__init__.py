@@ -88,6 +88,10 @@ class Oracle:
         lib.oracle_sum_rmsnorm_mxfp8_rows.argtypes = [
             ctypes.POINTER(u16p), ctypes.c_int, i64, i64, i64, vp, vp, vp, ctypes.c_float,
             ctypes.c_float, vp, vp, vp, vp]
+        lib.oracle_e8m0_decode.restype = ctypes.c_double
+        lib.oracle_e8m0_decode.argtypes = [ctypes.c_uint8]
+        lib.oracle_scaled_mm_mx.restype = None
+        lib.oracle_scaled_mm_mx.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp, vp]
         lib.oracle_bf16_round_double.restype = ctypes.c_uint16
         lib.oracle_bf16_round_double.argtypes = [ctypes.c_double]
         lib.oracle_scaled_mm.restype = None
@@ -212,6 +216,31 @@ class Oracle:
             out["v"] = v[sl].copy()
         return out
 
+    def e8m0_decode(self, codes) -> np.ndarray:
+        """E8M0 codes -> float64 values (NaN for 0xFF)."""
+        c = np.asarray(codes, dtype=np.uint8)
+        return np.array([self.lib.oracle_e8m0_decode(int(k)) for k in c.ravel()],
+                        dtype=np.float64).reshape(c.shape)
+
+    def scaled_mm_mx(self, a, sa, b, sb, bias=None, exact: bool = False):
+        """The MX GEMM: a uint8 e4m3fn codes [M, K], b [N, K], sa / sb E8M0
+        codes [M, K / 32] / [N, K / 32], bias bf16 bits [N] or None.  Returns
+        out (bf16 bits [M, N]) and, with ``exact``, the float64 values."""
+        a = np.ascontiguousarray(a, dtype=np.uint8)
+        b = np.ascontiguousarray(b, dtype=np.uint8)
+        M, K = a.shape
+        N = b.shape[0]
+        if b.shape[1] != K or K % 32:
+            raise ValueError("a and b need the same K, a multiple of 32")
+        sa = np.ascontiguousarray(sa, dtype=np.uint8).reshape(M, K // 32)
+        sb = np.ascontiguousarray(sb, dtype=np.uint8).reshape(N, K // 32)
+        bi = None if bias is None else np.ascontiguousarray(bias, dtype=np.uint16).reshape(N)
+        out = np.empty((M, N), dtype=np.uint16)
+        ex = np.empty((M, N), dtype=np.float64) if exact else None
+        self.lib.oracle_scaled_mm_mx(_ptr(a), _ptr(sa), _ptr(b), _ptr(sb), _ptr(bi), M, N, K,
+                                     _ptr(out), _ptr(ex))
+        return (out, ex) if exact else out
+
     def bf16_round_double(self, values) -> np.ndarray:
         """float64 -> nearest bf16 (ties to even) in one rounding, as uint16."""
         v = np.asarray(values, dtype=np.float64)
@@ -278,3 +307,7 @@ def scaled_mm(*args, **kwargs):
 
 def sum_rmsnorm_mxfp8(*args, **kwargs):
     return default().sum_rmsnorm_mxfp8(*args, **kwargs)
+
+
+def scaled_mm_mx(*args, **kwargs):
+    return default().scaled_mm_mx(*args, **kwargs)

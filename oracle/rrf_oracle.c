@@ -354,3 +354,40 @@ void oracle_sum_rmsnorm_mxfp8_rows(const uint16_t* const* x, int R, int64_t row0
         }
     }
 }
+
+/* ------------------------------------------------------ the MX GEMM --- */
+
+/* Value of an E8M0 code: 2^(code - 127); 0xFF is NaN (OCP MX v1.0). */
+double oracle_e8m0_decode(uint8_t c) {
+    if (c == 0xFF) return NAN;
+    return ldexp(1.0, (int)c - 127);
+}
+
+/* The mx scenario of the Ascend aclnnAlltoAllQuantMatmul page:
+ * out = (x1 * x1Scale) @ (x2 * x2Scale) + bias with one scale per 32 values
+ * of K on both sides.  Here a is [M, K] and b is [N, K] e4m3fn codes,
+ * sa is [M, K / 32] and sb is [N, K / 32] E8M0 codes (row-major),
+ *   out[m][n] = RN_bf16( sum_k (e4m3(a[m][k]) * 2^(sa[m][k/32] - 127))
+ *                              * (e4m3(b[n][k]) * 2^(sb[n][k/32] - 127)) + bias[n] )
+ * in float64: every term is an exact power-of-two multiple of a product of
+ * two e4m3 values, and the sum is exact while the terms' exponents stay
+ * within float64's 53 bits (checked by the tests' magnitudes); one rounding to
+ * bf16.  exact (may be NULL) receives the float64 value before rounding. */
+void oracle_scaled_mm_mx(const uint8_t* a, const uint8_t* sa, const uint8_t* b,
+                         const uint8_t* sb, const uint16_t* bias, int64_t M, int64_t N,
+                         int64_t K, uint16_t* out, double* exact) {
+    const int64_t nb = K / MX_BLOCK;
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double S = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double x = oracle_e4m3_decode(a[m * K + k]) * oracle_e8m0_decode(sa[m * nb + k / MX_BLOCK]);
+                double y = oracle_e4m3_decode(b[n * K + k]) * oracle_e8m0_decode(sb[n * nb + k / MX_BLOCK]);
+                S += x * y;
+            }
+            if (bias != NULL) S += (double)oracle_bf16_to_float(bias[n]);
+            if (exact != NULL) exact[m * N + n] = S;
+            out[m * N + n] = oracle_bf16_round_double(S);
+        }
+    }
+}

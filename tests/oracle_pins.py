@@ -666,4 +666,55 @@ def pin_scaled_mm_k_split(o):
     assert np.array_equal(whole, lo + hi)
 
 
+# ----------------------------------------------------------------- MX GEMM ---
+# The Ascend page's mx scenario: out = (x1 * x1Scale) @ (x2 * x2Scale) +
+# bias, one E8M0 scale per 32 values of K on both operands.
+
+def rand_e8m0(seed: int, shape, lo: int = 120, hi: int = 134) -> np.ndarray:
+    return np.random.default_rng(seed).integers(lo, hi, size=shape).astype(np.uint8)
+
+
+def pin_scaled_mm_mx_vs_float64_matmul(o):
+    """Against numpy's float64 matmul of the dequantised operands (ml_dtypes'
+    e4m3fn and E8M0 decodings): the same float64 values, the same bf16."""
+    M, N, K = 4, 6, 160
+    a, b = rand_e4m3(61, (M, K), 2.0), rand_e4m3(62, (N, K), 2.0)
+    sa, sb = rand_e8m0(63, (M, K // 32)), rand_e8m0(64, (N, K // 32))
+    bias = lib_bf16(np.random.default_rng(65).normal(0, 1, N).astype(np.float32))
+    A = lib_e4m3_decode(a) * np.repeat(e8m0_value(sa), 32, axis=1)
+    B = lib_e4m3_decode(b) * np.repeat(e8m0_value(sb), 32, axis=1)
+    want = A @ B.T + f32(bias).astype(np.float64)[None, :]
+    out, ex = o.scaled_mm_mx(a, sa, b, sb, bias, exact=True)
+    assert np.array_equal(ex, want)
+    assert np.array_equal(out, brute_bf16_round_double(want))
+
+
+def pin_scaled_mm_mx_reduces_to_row_scales(o):
+    """With one scale code per row of a and per row of b, the MX GEMM is the
+    (pinned) per-token GEMM with scales 2^(code - 127)."""
+    M, N, K = 3, 5, 128
+    a, b = rand_e4m3(66, (M, K)), rand_e4m3(67, (N, K))
+    ca, cb = rand_e8m0(68, M), rand_e8m0(69, N)
+    sa, sb = np.repeat(ca[:, None], K // 32, axis=1), np.repeat(cb[:, None], K // 32, axis=1)
+    mx = o.scaled_mm_mx(a, sa, b, sb)
+    row = o.scaled_mm(a, e8m0_value(ca).astype(np.float32), b, e8m0_value(cb).astype(np.float32))
+    assert np.array_equal(mx, row)
+
+
+def pin_scaled_mm_mx_block_linearity(o):
+    """Raising one block's scale code of a by one adds exactly that block's
+    contribution once more (the blocks are the 32 values of K they cover)."""
+    M, N, K = 2, 3, 128
+    a, b = rand_e4m3(70, (M, K)), rand_e4m3(71, (N, K))
+    sa, sb = rand_e8m0(72, (M, K // 32)), rand_e8m0(73, (N, K // 32))
+    _, base = o.scaled_mm_mx(a, sa, b, sb, exact=True)
+    sa2 = sa.copy()
+    sa2[1, 2] += 1
+    _, up = o.scaled_mm_mx(a, sa2, b, sb, exact=True)
+    keep = np.zeros_like(a)
+    keep[1, 64:96] = a[1, 64:96]
+    _, blk = o.scaled_mm_mx(keep, sa, b, sb, exact=True)
+    assert np.array_equal(up[0], base[0]) and np.array_equal(up[1], base[1] + blk[1])
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

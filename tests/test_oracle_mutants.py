@@ -66,6 +66,10 @@ MUTANTS = [
      "if (k < 16 && fabsf(y[k]) > amax) amax = fabsf(y[k]);"),
     ("MX zero block scale 1", "if (!(amax > 0.0f)) return 0;", "if (!(amax > 0.0f)) return 127;"),
     ("MX scale applied as a multiplier", "float v = y[k] * inv_x;", "float v = y[k] / inv_x;"),
+    ("MX GEMM block shifted", "sa[m * nb + k / MX_BLOCK]", "sa[m * nb + (k / MX_BLOCK + 1) % nb]"),
+    ("MX GEMM b scaled by a's row", "sb[n * nb + k / MX_BLOCK]", "sb[(m % N) * nb + k / MX_BLOCK]"),
+    ("E8M0 bias 126", "return ldexp(1.0, (int)c - 127);", "return ldexp(1.0, (int)c - 126);"),
+    ("MX GEMM bias dropped", "if (bias != NULL) S += (double)oracle_bf16_to_float(bias[n]);", ""),
 ]
 
 
