@@ -481,6 +481,45 @@ def time_mx(rrf, label, rows, device, stream, l2, peak):
             "GB_s": round(nbytes / t / 1e9, 1), "frac": round(nbytes / t / 1e9 / peak, 4)}
 
 
+def time_gemm_mx(rrf, M, N, K, device, stream, l2, hbm_peak):
+    """The MX GEMM (rrf_scaled_mm_mxfp8) on operands with random E8M0 codes
+    in [120, 134), cycling through operand sets larger than 3 x L2."""
+    import numpy as np
+    import torch
+    nbytes = workloads.gemm_bytes(M, N, K) + (M + N) * K // 32
+    n = max(1, math.ceil(L2_FLUSH_FACTOR * l2 / nbytes))
+    sets = []
+    for i in range(n):
+        c = workloads.make_gemm_case(M, N, K, sub=i, device=device)
+        rng = np.random.default_rng(200 + i)
+        sa = rrf.mx_blocked(torch.from_numpy(
+            rng.integers(120, 134, (M, K // 32)).astype(np.uint8)).to(device))
+        sb = rrf.mx_blocked(torch.from_numpy(
+            rng.integers(120, 134, (N, K // 32)).astype(np.uint8)).to(device))
+        sets.append((c, sa, sb, torch.empty((M, N), dtype=torch.bfloat16, device=device)))
+
+    def call(k):
+        c, sa, sb, out = sets[k % n]
+        rrf.rrf_scaled_mm_mxfp8(c.a, sa, c.b, sb, c.bias, out=out)
+        return 1
+
+    for k in range(3):
+        call(k)
+    reps = max(n, 20 if M * N * K >= 2 ** 36 else 100)
+    g, _ = capture_steps(call, reps, device)
+    g.replay()
+    torch.cuda.synchronize(device)
+    t = time_region(lambda _: g.replay(), 1, device, stream) / reps
+    del g, sets
+    tf = workloads.gemm_flops(M, N, K) / t / 1e12
+    fp8_peak, fp8_kind = fp8_peak_tflops()
+    return {"shape": f"{M} x {N} x {K}", "us_per_call": round(t * 1e6, 3),
+            "TFLOP_s": round(tf, 1), "tensor_frac": round(tf / fp8_peak, 4),
+            "GB_s": round(nbytes / t / 1e9, 1), "hbm_frac": round(nbytes / t / 1e9 / hbm_peak, 4),
+            "fp8_peak_TFLOP_s": round(fp8_peak, 1), "fp8_peak_kind": fp8_kind,
+            "operand_sets": n, "device_error": rrf.rrf_device_error(clear=True)}
+
+
 def capture_steps(fn, n: int, device):
     """Capture fn(0) .. fn(n-1) into one CUDA graph; returns (graph, number
     of kernels fn launched)."""
@@ -833,11 +872,14 @@ def run_rrf(args):
                                   ("prefill", 8192))]
         torch.cuda.empty_cache()
 
-    # ---- the FP8 GEMM that consumes the per-row scales
-    gemm = None
+    # ---- the FP8 GEMMs that consume the per-row and the MX scales
+    gemm = gemm_mx = None
     if not args.no_secondary:
         gemm = [time_gemm(rrf, M, 7168, 7168, device, stream, l2, peak) for M in (1, 8, 32, 64)]
         gemm.append(time_gemm(rrf, 8192, 8192, 8192, device, stream, l2, peak))
+        torch.cuda.empty_cache()
+        gemm_mx = [time_gemm_mx(rrf, M, N, N, device, stream, l2, peak)
+                   for M, N in ((64, 7168), (8192, 8192))]
         torch.cuda.empty_cache()
 
     cpu = None
@@ -889,6 +931,7 @@ def run_rrf(args):
             "allreduce_emulated": emulated,
             "mx": mx,
             "gemm_fp8": gemm,
+            "gemm_mxfp8": gemm_mx,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

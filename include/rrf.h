@@ -214,6 +214,25 @@ rrf_status rrf_sum_rmsnorm_mxfp8(const void* const* inputs, int num_inputs, int6
                                  const void* gamma, float eps, float weight_offset, void* q_out,
                                  void* scales_mx_out, rrf_stream_t stream);
 
+/* The blocked order of MX scale codes, the order the tensor cores'
+ * block-scaled MMA reads them in (512-byte atoms of 128 rows x 4 blocks of
+ * 32 columns): the code of row r, block j (of cols / 32) lives at byte
+ *   ((r / 128) * (cols / 128) + j / 4) * 512 + (r % 32) * 16 + ((r / 32) % 4) * 4 + j % 4
+ * of a buffer of RRF_MX_BLOCKED_BYTES(rows, cols) bytes (rows rounded up to
+ * 128; cols a multiple of 128).  Bytes of the rounded-up rows are not
+ * written. */
+#define RRF_MX_BLOCKED_BYTES(rows, cols) ((((rows) + 127) / 128) * 128 * ((cols) / 32))
+
+/* rrf_sum_rmsnorm_mxfp8_blocked -- rrf_sum_rmsnorm_mxfp8 with the scale
+ * codes in the blocked order (cols a multiple of 128; scales_mx_out holds
+ * RRF_MX_BLOCKED_BYTES(rows, cols) bytes), ready for rrf_scaled_mm_mxfp8.
+ * Errors: as rrf_sum_rmsnorm_mxfp8. */
+rrf_status rrf_sum_rmsnorm_mxfp8_blocked(const void* const* inputs, int num_inputs,
+                                         int64_t rows, int64_t cols, const void* residual_in,
+                                         void* residual_out, const void* gamma, float eps,
+                                         float weight_offset, void* q_out, void* scales_mx_out,
+                                         rrf_stream_t stream);
+
 /* The host validation of rrf_sum_rmsnorm_mxfp8 alone (no GPU needed). */
 rrf_status rrf_check_mxfp8_args(const void* const* inputs, int num_inputs, int64_t rows,
                                 int64_t cols, const void* residual_in, const void* residual_out,
@@ -417,6 +436,30 @@ rrf_status rrf_plan_allreduce(int world, int64_t rows, int64_t cols, int residua
 rrf_status rrf_scaled_mm_fp8(const void* a, const float* a_scale, const void* b,
                              const float* b_scale, const void* bias, void* out, int64_t M,
                              int64_t N, int64_t K, rrf_stream_t stream);
+
+/* rrf_scaled_mm_mxfp8 -- the GEMM of the mx scenario of the same page:
+ * out = (x1 * x1Scale) @ (x2 * x2Scale) + bias with one E8M0 scale per 32
+ * values of K on both operands,
+ *   out[m][n] = RN_bf16( sum_k e4m3(a[m][k]) 2^(sa[m][k/32] - 127)
+ *                              e4m3(b[n][k]) 2^(sb[n][k/32] - 127) + bias[n] )
+ * on the tensor cores' block-scaled MMA (fp32 accumulation, one rounding).
+ * a, b      e4m3fn codes [M, K] and [N, K], row-major, 16-byte aligned
+ * sa, sb    E8M0 codes in the blocked order (RRF_MX_BLOCKED_BYTES(M, K) and
+ *           (N, K) bytes; rrf_sum_rmsnorm_mxfp8_blocked writes sa), 16-byte
+ *           aligned.  The codes of rounded-up rows may hold anything: they
+ *           only scale output rows and columns that are not stored.
+ * bias      bf16 [N] or NULL;  out  bf16 [M, N], 16-byte aligned
+ * M >= 0 (0 is a no-op); N >= 16 and a multiple of 16; K a multiple of 128
+ * Errors: RRF_ERR_NULL, RRF_ERR_SHAPE, RRF_ERR_ALIGN, RRF_ERR_ALIAS,
+ *         RRF_ERR_CUDA. */
+rrf_status rrf_scaled_mm_mxfp8(const void* a, const void* sa, const void* b, const void* sb,
+                               const void* bias, void* out, int64_t M, int64_t N, int64_t K,
+                               rrf_stream_t stream);
+
+/* The host validation of rrf_scaled_mm_mxfp8 alone (no GPU needed). */
+rrf_status rrf_check_scaled_mm_mx_args(const void* a, const void* sa, const void* b,
+                                       const void* sb, const void* bias, const void* out,
+                                       int64_t M, int64_t N, int64_t K);
 
 /* The host validation of rrf_scaled_mm_fp8 alone (no GPU needed). */
 rrf_status rrf_check_scaled_mm_args(const void* a, const float* a_scale, const void* b,

@@ -110,6 +110,12 @@ lib.rrf_sum_rmsnorm_mxfp8.argtypes = [_ptrs, _int, _i64, _i64, _vp, _vp, _vp, _f
 lib.rrf_check_mxfp8_args.restype = _int
 lib.rrf_check_mxfp8_args.argtypes = [_ptrs, _int, _i64, _i64, _vp, _vp, _vp, _f32, _f32, _vp,
                                      _vp]
+lib.rrf_sum_rmsnorm_mxfp8_blocked.restype = _int
+lib.rrf_sum_rmsnorm_mxfp8_blocked.argtypes = lib.rrf_sum_rmsnorm_mxfp8.argtypes
+lib.rrf_scaled_mm_mxfp8.restype = _int
+lib.rrf_scaled_mm_mxfp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]
+lib.rrf_check_scaled_mm_mx_args.restype = _int
+lib.rrf_check_scaled_mm_mx_args.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64]
 lib.rrf_scaled_mm_fp8.restype = _int
 lib.rrf_scaled_mm_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]
 lib.rrf_check_scaled_mm_args.restype = _int
@@ -322,28 +328,52 @@ def rrf_check_mxfp8_args(input_ptrs, rows, cols, residual_in, residual_out, gamm
                                     eps, weight_offset, q_out or None, scales_mx_out or None)
 
 
+def mx_blocked_bytes(rows: int, cols: int) -> int:
+    """Bytes of MX scale codes in the blocked order (rows rounded up to 128)."""
+    return -(-rows // 128) * 128 * (cols // 32)
+
+
+def mx_blocked(codes):
+    """Row-major MX scale codes [rows, cols / 32] (uint8 tensor) -> the
+    blocked order that the block-scaled GEMM reads (a flat uint8 tensor of
+    mx_blocked_bytes(rows, cols) bytes; rounded-up rows zero).  A layout
+    change for preparing weights once, not a step of the call."""
+    torch = _torch()
+    rows, nb = codes.shape
+    if nb % 4:
+        raise ValueError("cols must be a multiple of 128")
+    pad = -(-rows // 128) * 128
+    p = torch.zeros((pad, nb), dtype=torch.uint8, device=codes.device)
+    p[:rows] = codes
+    # [rows/128, 4 (r/32 % 4), 32 (r % 32), nb/4, 4 (j % 4)] -> [rows/128, nb/4, 32, 4, 4]
+    return p.view(pad // 128, 4, 32, nb // 4, 4).permute(0, 3, 2, 1, 4).contiguous().view(-1)
+
+
 def rrf_sum_rmsnorm_mxfp8(inputs, gamma, eps, weight_offset, residual_in=None,
-                          residual_out=None, q_out=None, scales_mx_out=None):
+                          residual_out=None, q_out=None, scales_mx_out=None, blocked=False):
     """The fused operation with MX output: one E8M0 scale code per 32
     elements.  Returns (q: float8_e4m3fn like the inputs, scales_mx: uint8
-    [..., cols / 32], residual_out or None)."""
+    [..., cols / 32] or, with ``blocked``, a flat uint8 tensor in the blocked
+    order for rrf_scaled_mm_mxfp8, residual_out or None)."""
     torch = _torch()
     rows, cols = _rows_cols(inputs)
     x0 = inputs[0]
     dev = x0.device
     if gamma.dtype != torch.bfloat16 or gamma.numel() != cols or gamma.device != dev:
         raise ValueError("gamma must be a bf16 tensor of length cols on the inputs' device")
-    if cols % 32:
-        raise ValueError("cols must be a multiple of 32")
+    if cols % (128 if blocked else 32):
+        raise ValueError(f"cols must be a multiple of {128 if blocked else 32}")
     if residual_in is not None and residual_out is None:
         residual_out = torch.empty_like(residual_in)
     if q_out is None:
         q_out = torch.empty(x0.shape, dtype=torch.float8_e4m3fn, device=dev)
     if scales_mx_out is None:
-        scales_mx_out = torch.empty(tuple(x0.shape[:-1]) + (cols // 32,), dtype=torch.uint8,
-                                    device=dev)
+        shape = (mx_blocked_bytes(rows, cols),) if blocked else \
+            tuple(x0.shape[:-1]) + (cols // 32,)
+        scales_mx_out = torch.empty(shape, dtype=torch.uint8, device=dev)
+    fn = lib.rrf_sum_rmsnorm_mxfp8_blocked if blocked else lib.rrf_sum_rmsnorm_mxfp8
     with torch.cuda.device(dev):
-        _raise_on(lib.rrf_sum_rmsnorm_mxfp8(
+        _raise_on(fn(
             _ptr_table([x.data_ptr() for x in inputs]), len(inputs), rows, cols,
             residual_in.data_ptr() if residual_in is not None else None,
             residual_out.data_ptr() if residual_out is not None else None, gamma.data_ptr(),
@@ -457,6 +487,45 @@ def rrf_scaled_mm_fp8(a, a_scale, b, b_scale, bias=None, out=None):
     with torch.cuda.device(dev):
         _raise_on(lib.rrf_scaled_mm_fp8(
             a.data_ptr(), a_scale.data_ptr(), b.data_ptr(), b_scale.data_ptr(),
+            bias.data_ptr() if bias is not None else None, out.data_ptr(), M, N, K,
+            _stream(dev)))
+    return out
+
+
+def rrf_check_scaled_mm_mx_args(a, sa, b, sb, bias, out, M, N, K) -> int:
+    """Host validation of the MX GEMM on raw pointers."""
+    return lib.rrf_check_scaled_mm_mx_args(a or None, sa or None, b or None, sb or None,
+                                           bias or None, out or None, M, N, K)
+
+
+def rrf_scaled_mm_mxfp8(a, sa, b, sb, bias=None, out=None):
+    """out = RN_bf16((a * 2^(sa - 127)) @ (b * 2^(sb - 127))^T + bias) on
+    the tensor cores' block-scaled MMA.  a: float8_e4m3fn [M, K], b:
+    float8_e4m3fn [N, K]; sa / sb: uint8 E8M0 codes in the blocked order
+    (rrf_sum_rmsnorm_mxfp8(..., blocked=True) for a, mx_blocked for a
+    weight); bias bf16 [N] or None.  Returns out, bf16 [M, N]."""
+    torch = _torch()
+    for t, name in ((a, "a"), (b, "b")):
+        if t.dtype != torch.float8_e4m3fn or t.dim() != 2 or not t.is_contiguous() or \
+                t.device.type != "cuda":
+            raise ValueError(f"{name} must be a contiguous 2-D float8_e4m3fn CUDA tensor")
+    M, K = a.shape
+    N = b.shape[0]
+    if b.shape[1] != K:
+        raise ValueError("a and b need the same K")
+    dev = a.device
+    for t, n, name in ((sa, M, "sa"), (sb, N, "sb")):
+        if t.dtype != torch.uint8 or t.numel() != mx_blocked_bytes(n, K) or \
+                not t.is_contiguous() or t.device != dev:
+            raise ValueError(f"{name} must hold the blocked scale codes of {n} rows")
+    if bias is not None and (bias.dtype != torch.bfloat16 or bias.numel() != N or
+                             bias.device != dev):
+        raise ValueError("bias must be a bf16 tensor of N values")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    with torch.cuda.device(dev):
+        _raise_on(lib.rrf_scaled_mm_mxfp8(
+            a.data_ptr(), sa.data_ptr(), b.data_ptr(), sb.data_ptr(),
             bias.data_ptr() if bias is not None else None, out.data_ptr(), M, N, K,
             _stream(dev)))
     return out

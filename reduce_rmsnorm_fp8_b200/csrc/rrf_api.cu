@@ -412,15 +412,30 @@ extern "C" rrf_status rrf_check_mxfp8_args(const void* const* inputs, int num_in
     return RRF_OK;
 }
 
-extern "C" rrf_status rrf_sum_rmsnorm_mxfp8(const void* const* inputs, int num_inputs,
-                                            int64_t rows, int64_t cols, const void* residual_in,
-                                            void* residual_out, const void* gamma, float eps,
-                                            float weight_offset, void* q_out,
-                                            void* scales_mx_out, rrf_stream_t stream) {
+static rrf_status mxfp8_call(const void* const* inputs, int num_inputs, int64_t rows,
+                             int64_t cols, const void* residual_in, void* residual_out,
+                             const void* gamma, float eps, float weight_offset, void* q_out,
+                             void* scales_mx_out, bool blocked, rrf_stream_t stream) {
     rrf_status st = rrf_check_mxfp8_args(inputs, num_inputs, rows, cols, residual_in,
                                          residual_out, gamma, eps, weight_offset, q_out,
                                          scales_mx_out);
-    if (st != RRF_OK || rows == 0) return st;
+    if (st != RRF_OK) return st;
+    if (blocked) {
+        if (cols % 128 != 0) return RRF_ERR_SHAPE;
+        if (rows == 0) return RRF_OK;
+        // the blocked buffer is larger than the row-major one (rows rounded
+        // up): it must not overlap the data either
+        const int64_t bf16_bytes = rows * cols * 2;
+        const Range sc = range_of(scales_mx_out, RRF_MX_BLOCKED_BYTES(rows, cols));
+        for (int r = 0; r < num_inputs; ++r)
+            if (overlap(sc, range_of(inputs[r], bf16_bytes))) return RRF_ERR_ALIAS;
+        if (overlap(sc, range_of(gamma, cols * 2)) || overlap(sc, range_of(q_out, rows * cols)))
+            return RRF_ERR_ALIAS;
+        if (residual_in != nullptr && (overlap(sc, range_of(residual_in, bf16_bytes)) ||
+                                       overlap(sc, range_of(residual_out, bf16_bytes))))
+            return RRF_ERR_ALIAS;
+    }
+    if (rows == 0) return RRF_OK;
     int sm_count = 0;
     if ((st = current_sm_count(&sm_count)) != RRF_OK) return st;
     FusedLaunch l = {};
@@ -438,6 +453,7 @@ extern "C" rrf_status rrf_sum_rmsnorm_mxfp8(const void* const* inputs, int num_i
     a.gamma = static_cast<const uint4*>(gamma);
     a.q = static_cast<uint2*>(q_out);
     a.scales_mx = static_cast<uint8_t*>(scales_mx_out);
+    a.mx_blocked = blocked ? 1 : 0;
     a.R = num_inputs;
     a.vecs = (int)vecs;
     a.cluster = l.cluster;
@@ -453,6 +469,25 @@ extern "C" rrf_status rrf_sum_rmsnorm_mxfp8(const void* const* inputs, int num_i
     if (!take_injected_failure(&e))
         e = launch_fused(a, rows, l, residual_in != nullptr, (cudaStream_t)stream);
     return e == cudaSuccess ? RRF_OK : cuda_fail(e);
+}
+
+extern "C" rrf_status rrf_sum_rmsnorm_mxfp8(const void* const* inputs, int num_inputs,
+                                            int64_t rows, int64_t cols, const void* residual_in,
+                                            void* residual_out, const void* gamma, float eps,
+                                            float weight_offset, void* q_out,
+                                            void* scales_mx_out, rrf_stream_t stream) {
+    return mxfp8_call(inputs, num_inputs, rows, cols, residual_in, residual_out, gamma, eps,
+                      weight_offset, q_out, scales_mx_out, false, stream);
+}
+
+extern "C" rrf_status rrf_sum_rmsnorm_mxfp8_blocked(const void* const* inputs, int num_inputs,
+                                                    int64_t rows, int64_t cols,
+                                                    const void* residual_in,
+                                                    void* residual_out, const void* gamma,
+                                                    float eps, float weight_offset, void* q_out,
+                                                    void* scales_mx_out, rrf_stream_t stream) {
+    return mxfp8_call(inputs, num_inputs, rows, cols, residual_in, residual_out, gamma, eps,
+                      weight_offset, q_out, scales_mx_out, true, stream);
 }
 
 // -------------------------------------------------------- sharded norm ---
@@ -835,6 +870,51 @@ extern "C" rrf_status rrf_scaled_mm_fp8(const void* a, const float* a_scale, con
     g.err = err;
     cudaError_t e;
     if (!take_injected_failure(&e)) e = launch_scaled_mm(g, a, b, sm_count, (cudaStream_t)stream);
+    return e == cudaSuccess ? RRF_OK : cuda_fail(e);
+}
+
+extern "C" rrf_status rrf_check_scaled_mm_mx_args(const void* a, const void* sa,
+                                                  const void* b, const void* sb,
+                                                  const void* bias, const void* out, int64_t M,
+                                                  int64_t N, int64_t K) {
+    if (M < 0 || N < 16 || K < 128 || N % 16 != 0 || K % 128 != 0) return RRF_ERR_SHAPE;
+    if (M > 65535LL * 128 || N > (int64_t)INT32_MAX / 2 || K > (int64_t)INT32_MAX / 2)
+        return RRF_ERR_SHAPE;
+    if (M == 0) return RRF_OK;
+    if (!a || !sa || !b || !sb || !out) return RRF_ERR_NULL;
+    if (!aligned(a, 16) || !aligned(b, 16) || !aligned(out, 16) || !aligned(sa, 16) ||
+        !aligned(sb, 16) || (bias != nullptr && !aligned(bias, 2)))
+        return RRF_ERR_ALIGN;
+    const Range o = range_of(out, M * N * 2);
+    const Range reads[5] = {range_of(a, M * K), range_of(b, N * K),
+                            range_of(sa, RRF_MX_BLOCKED_BYTES(M, K)),
+                            range_of(sb, RRF_MX_BLOCKED_BYTES(N, K)),
+                            bias != nullptr ? range_of(bias, N * 2) : Range{0, 0}};
+    for (const Range& r : reads)
+        if (overlap(o, r)) return RRF_ERR_ALIAS;
+    return RRF_OK;
+}
+
+extern "C" rrf_status rrf_scaled_mm_mxfp8(const void* a, const void* sa, const void* b,
+                                          const void* sb, const void* bias, void* out, int64_t M,
+                                          int64_t N, int64_t K, rrf_stream_t stream) {
+    rrf_status st = rrf_check_scaled_mm_mx_args(a, sa, b, sb, bias, out, M, N, K);
+    if (st != RRF_OK || M == 0) return st;
+    int sm_count = 0;
+    if ((st = current_sm_count(&sm_count)) != RRF_OK) return st;
+    unsigned int* err = nullptr;
+    if ((st = device_error_word(&err)) != RRF_OK) return st;
+    GemmArgs g = {};
+    g.bias = static_cast<const uint16_t*>(bias);
+    g.out = static_cast<uint16_t*>(out);
+    g.M = (int)M;
+    g.N = (int)N;
+    g.K = (int)K;
+    g.err = err;
+    cudaError_t e;
+    if (!take_injected_failure(&e))
+        e = launch_scaled_mm_mx(g, a, b, static_cast<const uint8_t*>(sa),
+                                static_cast<const uint8_t*>(sb), sm_count, (cudaStream_t)stream);
     return e == cudaSuccess ? RRF_OK : cuda_fail(e);
 }
 

@@ -195,7 +195,17 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
                     qv[e] = __fmul_rn(y, inv_x);
                 }
                 st_once(a.q + row_base + v, f32_to_e4m3x8(qv));
-                if ((v & 3) == 0) a.scales_mx[(row_base + v) >> 2] = (uint8_t)code;
+                if ((v & 3) == 0) {
+                    // row-major [rows, cols / 32], or the tensor cores' blocked
+                    // order (512-byte atoms of 128 rows x 4 blocks)
+                    const int64_t j = v >> 2;
+                    const int64_t off =
+                        a.mx_blocked
+                            ? ((row >> 7) * (a.vecs >> 4) + (j >> 2)) * 512 + (row & 31) * 16 +
+                                  ((row >> 5) & 3) * 4 + (j & 3)
+                            : (row_base + v) >> 2;
+                    a.scales_mx[off] = (uint8_t)code;
+                }
                 if (RES && CLUSTER) st_once(a.res_out + row_base + v, h[k]);
             }
         }

@@ -172,8 +172,12 @@ __device__ __forceinline__ void store_row_chunk(const GemmArgs& g, const float v
     uint32_t packed[16];
 #pragma unroll
     for (int i = 0; i < 32; i += 2) {
-        float y0 = __fmul_rn(__fmul_rn(v[i], sa), i < valid ? g.b_scale[n + i] : 0.0f);
-        float y1 = __fmul_rn(__fmul_rn(v[i + 1], sa), i + 1 < valid ? g.b_scale[n + i + 1] : 0.0f);
+        // (the MX GEMM has no column scales: its scales act inside the MMA)
+        const float s0 = i < valid ? (g.b_scale != nullptr ? g.b_scale[n + i] : 1.0f) : 0.0f;
+        const float s1 =
+            i + 1 < valid ? (g.b_scale != nullptr ? g.b_scale[n + i + 1] : 1.0f) : 0.0f;
+        float y0 = __fmul_rn(__fmul_rn(v[i], sa), s0);
+        float y1 = __fmul_rn(__fmul_rn(v[i + 1], sa), s1);
         if (g.bias != nullptr && i < valid) {
             y0 = __fadd_rn(y0, __uint_as_float((uint32_t)g.bias[n + i] << 16));
             y1 = __fadd_rn(y1, __uint_as_float((uint32_t)g.bias[n + i + 1] << 16));
@@ -610,6 +614,217 @@ __global__ void __launch_bounds__(kThreads, 1)
     cluster_wait_acquire();
 }
 
+// ------------------------------------------- MX (block-scaled) GEMM kernel --
+// out = (a * 2^(sa - 127)) @ (b * 2^(sb - 127))^T + bias with one E8M0 code
+// per 32 values of K (the mx scenario), on tcgen05.mma kind::mxf8f6f4 with
+// block scaling: the scale codes of a k-tile (128 rows x 4 codes, one
+// 512-byte atom of the blocked order) are loaded next to the A and B tiles,
+// copied into tensor memory with tcgen05.cp (32 lanes x 128 bits, repeated
+// in the 4 lane quarters: lane l holds rows l, l+32, l+64, l+96, 4 codes
+// each), and the k-tile's four MMAs take code (k-step) of each 32-bit word.
+
+// 1-D bulk copy of `bytes` (a multiple of 16, both addresses 16-byte
+// aligned) into shared memory, completing on `bar` (no multicast).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Shared -> tensor memory: 32 rows of 16 bytes, repeated in the 4 lane quarters.
+__device__ __forceinline__ void tmem_copy_32x128b_x4(uint32_t taddr, uint64_t src_desc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(src_desc)
+                 : "memory");
+}
+
+// Descriptor of a scale atom as tcgen05.cp's source: 32 rows of 16 bytes,
+// contiguous, no swizzle (8-row core matrices 128 bytes apart).
+__device__ __forceinline__ uint64_t sf_atom_desc(const void* atom) {
+    const uint64_t addr = smem_u32(atom);
+    return ((addr >> 4) & 0x3FFFull) | ((128ull >> 4) << 32) | (1ull << 46);
+}
+
+__device__ __forceinline__ void mma_mx(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate, uint32_t sfa,
+                                       uint32_t sfb) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa),
+           "r"(sfb)
+        : "memory");
+}
+
+// Instruction descriptor of the block-scaled MMA: A and B e4m3 (0), K-major,
+// N = bn, M = 128, E8M0 scales (bit 23), scale codes taken from byte `id` of
+// the A and B scale words.
+__host__ __device__ constexpr uint32_t mx_idesc(int bn, uint32_t id) {
+    return (id << 4) | ((uint32_t)(bn >> 3) << 17) | (1u << 23) | ((uint32_t)(kBM >> 4) << 24) |
+           (id << 29);
+}
+
+struct MxTile {
+    static constexpr int BN = 128;
+    static constexpr int kABytes = kBM * kBK;        // 16 KB
+    static constexpr int kBBytes = BN * kBK;         // 16 KB
+    static constexpr int kSfBytes = 512;             // one atom: 128 rows x 4 codes
+    static constexpr int kStageBytes = kABytes + kBBytes + 2 * kSfBytes;  // 33 KB
+    static constexpr int kStageStride = (kStageBytes + 1023) / 1024 * 1024;
+    static constexpr int kStages = 6;
+    static constexpr int kAccCols = 2 * BN;          // two accumulators
+    static constexpr int kTmemCols = 512;            // accumulators, then 4 + 4 scale columns
+    static constexpr int kBarriers = 2 * kStages + 4 + 1;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageStride + kBarriers * 8 + 16;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    scaled_mm_mx_kernel(const __grid_constant__ CUtensorMap tma_a,
+                        const __grid_constant__ CUtensorMap tma_b, const GemmArgs g,
+                        const uint8_t* sfa, const uint8_t* sfb) {
+    using T = MxTile;
+    constexpr int S = T::kStages;
+    constexpr int BN = T::BN;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * T::kStageStride);
+    uint64_t* empty = full + S;
+    uint64_t* acc_full = empty + S;
+    uint64_t* acc_empty = acc_full + 2;
+    uint64_t* drained = acc_empty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tiles_n = (g.N + BN - 1) / BN;
+    const int tiles = tiles_n * ((g.M + kBM - 1) / kBM);
+    const int ktiles = g.K / kBK;  // K is a multiple of 128
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 4);
+        }
+        mbar_init(drained, 1);
+        fence_mbar_init_cluster();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, T::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tmem_sfa = tmem + T::kAccCols, tmem_sfb = tmem + T::kAccCols + 4;
+
+    if (warp == 0) {
+        // ---- producer: A, B and their scale atoms of every k-tile
+        if (lane == 0) {
+            int it = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+                const int m0 = (t / tiles_n) * kBM, n0 = (t % tiles_n) * BN;
+                const uint8_t* sfa_tile = sfa + (int64_t)(m0 / 128) * ktiles * T::kSfBytes;
+                const uint8_t* sfb_tile = sfb + (int64_t)(n0 / 128) * ktiles * T::kSfBytes;
+                for (int kt = 0; kt < ktiles; ++kt, ++it) {
+                    const int s = it % S;
+                    if (!wait_phase(&empty[s], ((it / S) & 1) ^ 1, g.err)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* dst = smem + s * T::kStageStride;
+                    mbar_arrive_expect_tx(&full[s], T::kStageBytes);
+                    tma_load_2d(dst, &tma_a, &full[s], kt * kBK, m0);
+                    tma_load_2d(dst + T::kABytes, &tma_b, &full[s], kt * kBK, n0);
+                    bulk_load(dst + T::kABytes + T::kBBytes, sfa_tile + kt * T::kSfBytes,
+                              T::kSfBytes, &full[s]);
+                    bulk_load(dst + T::kABytes + T::kBBytes + T::kSfBytes,
+                              sfb_tile + kt * T::kSfBytes, T::kSfBytes, &full[s]);
+                }
+            }
+            for (int i = it > S ? it - S : 0; i < it; ++i)
+                wait_phase(&full[i % S], (i / S) & 1, g.err);
+        }
+    } else if (warp == 1) {
+        // ---- scale copies and MMAs
+        if (lane == 0) {
+            int it = 0, j = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++j) {
+                const int buf = j & 1;
+                if (!wait_phase(&acc_empty[buf], ((j >> 1) & 1) ^ 1, g.err)) break;
+                tc_fence_after_sync();
+                const uint32_t d = tmem + (uint32_t)(buf * BN);
+                for (int kt = 0; kt < ktiles; ++kt, ++it) {
+                    const int s = it % S;
+                    if (!wait_phase(&full[s], (it / S) & 1, g.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint8_t* tile = smem + s * T::kStageStride;
+                    // tcgen05 operations of this thread run in issue order: the
+                    // copies land before the MMAs below read the scales, and
+                    // the previous k-tile's MMAs have read theirs before these
+                    tmem_copy_32x128b_x4(tmem_sfa, sf_atom_desc(tile + T::kABytes + T::kBBytes));
+                    tmem_copy_32x128b_x4(tmem_sfb, sf_atom_desc(tile + T::kABytes + T::kBBytes +
+                                                                T::kSfBytes));
+                    const uint64_t ad = kmajor_sw128_desc(tile);
+                    const uint64_t bd = kmajor_sw128_desc(tile + T::kABytes);
+#pragma unroll
+                    for (int k = 0; k < kBK / kMmaK; ++k) {
+                        const uint64_t step = (uint64_t)(k * kMmaK) >> 4;
+                        mma_mx(d, ad + step, bd + step, mx_idesc(BN, (uint32_t)k), (kt | k) != 0,
+                               tmem_sfa, tmem_sfb);
+                    }
+                    mma_commit(&empty[s]);
+                }
+                mma_commit(&acc_full[buf]);
+            }
+            mma_commit(drained);
+        }
+        __syncwarp();
+    } else {
+        // ---- epilogue: the scales are inside the accumulator; bias, bf16
+        const int quarter = warp & 3;
+        int j = 0;
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
+            const int buf = j & 1;
+            const int m0 = (t / tiles_n) * kBM, n0 = (t % tiles_n) * BN;
+            bool have = wait_phase(&acc_full[buf], (j >> 1) & 1, g.err);
+            if (!__all_sync(0xFFFFFFFFu, have)) break;
+            tc_fence_after_sync();
+            const int row = m0 + quarter * 32 + lane;
+            const uint32_t base = tmem + (uint32_t)(buf * BN) + ((uint32_t)(quarter * 32) << 16);
+            for (int c = 0; c < BN; c += 32) {
+                float v[32];
+                tmem_load_32(base + (uint32_t)c, v);
+                const int n = n0 + c;
+                if (row >= g.M || n >= g.N) continue;
+                store_row_chunk(g, v, 1.0f, row, n);  // g.b_scale is null: no scaling
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        wait_phase(drained, 0, g.err);
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, T::kTmemCols);
+    }
+}
+
 // ------------------------------------------------------------------- host --
 
 using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -708,7 +923,36 @@ cudaError_t launch_pair(const GemmArgs& g, const void* a, const void* b, int sm_
     return cudaLaunchKernelEx(&cfg, scaled_mm_pair_kernel, ma, mb, g);
 }
 
+cudaError_t launch_mx(const GemmArgs& g, const void* a, const void* b, const uint8_t* sfa,
+                      const uint8_t* sfb, int sm_count, cudaStream_t stream) {
+    using T = MxTile;
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, a, g.M, g.K, kBM) || !make_map(&mb, b, g.N, g.K, T::BN))
+        return cudaErrorInvalidValue;
+    static std::atomic<uint64_t> enabled_on{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
+    if (bit == 0 || (enabled_on.load(std::memory_order_relaxed) & bit) == 0) {
+        e = cudaFuncSetAttribute(scaled_mm_mx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 T::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        enabled_on.fetch_or(bit, std::memory_order_relaxed);
+    }
+    const int64_t tiles = (int64_t)((g.N + T::BN - 1) / T::BN) * ((g.M + kBM - 1) / kBM);
+    const unsigned grid = (unsigned)(tiles < sm_count ? tiles : sm_count);
+    scaled_mm_mx_kernel<<<grid, kThreads, T::kSmemBytes, stream>>>(ma, mb, g, sfa, sfb);
+    return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_scaled_mm_mx(const GemmArgs& g, const void* a, const void* b,
+                                const uint8_t* sfa, const uint8_t* sfb, int sm_count,
+                                cudaStream_t stream) {
+    return launch_mx(g, a, b, sfa, sfb, sm_count, stream);
+}
 
 cudaError_t launch_scaled_mm(const GemmArgs& g, const void* a, const void* b, int sm_count,
                              cudaStream_t stream) {

@@ -42,7 +42,8 @@ struct FusedArgs {
     float2* stats;         // [rows]
     uint4* h_out;          // [rows, cols] or null (with a residual, res_out holds h)
     // MX output: one E8M0 scale code per 32 elements instead of scales
-    uint8_t* scales_mx;    // [rows, cols / 32]
+    uint8_t* scales_mx;    // [rows, cols / 32], or blocked (mx_blocked)
+    int mx_blocked;        // scales in the block-scaled MMA's 512-byte atom order
 };
 
 // The second phase of the sharded norm: quantise one column shard from the
@@ -160,6 +161,11 @@ cudaError_t launch_post(const PostArgs& a, int sm_count, bool pdl, cudaStream_t 
 cudaError_t launch_allreduce(const ArArgs& a, const ArLaunch& l, cudaStream_t stream);
 cudaError_t launch_scaled_mm(const GemmArgs& g, const void* a, const void* b, int sm_count,
                              cudaStream_t stream);
+// The MX GEMM: sfa / sfb are the scale codes in the blocked order; g.a_scale
+// and g.b_scale are null.
+cudaError_t launch_scaled_mm_mx(const GemmArgs& g, const void* a, const void* b,
+                                const uint8_t* sfa, const uint8_t* sfb, int sm_count,
+                                cudaStream_t stream);
 // Blocks of the launch shape `l` that can be resident on the current device
 // at once (the occupancy query; nothing is launched).
 cudaError_t allreduce_resident_blocks(const ArLaunch& l, int* resident);

@@ -421,3 +421,18 @@ def test_mxfp8_validation(rrf):
         kw = dict(ok)
         kw.update(change)
         assert rrf.rrf_check_mxfp8_args(**kw) == rrf.Status[status], change
+
+
+def test_scaled_mm_mx_validation(rrf):
+    ok = dict(a=A, sa=2 * A, b=3 * A, sb=4 * A, bias=5 * A, out=6 * A, M=64, N=256, K=512)
+    assert rrf.rrf_check_scaled_mm_mx_args(**ok) == rrf.Status.OK
+    assert rrf.rrf_check_scaled_mm_mx_args(0, 0, 0, 0, 0, 0, 0, 256, 512) == rrf.Status.OK
+    for change, status in [
+            (dict(K=384 + 64), "ERR_SHAPE"), (dict(K=0), "ERR_SHAPE"), (dict(N=264), "ERR_SHAPE"),
+            (dict(sa=0), "ERR_NULL"), (dict(sb=4 * A + 8), "ERR_ALIGN"),
+            (dict(sa=2 * A + 4), "ERR_ALIGN"),
+            (dict(out=2 * A + 16), "ERR_ALIAS"),          # over sa's blocked bytes
+            (dict(sb=6 * A + 64 * 256 * 2 - 16), "ERR_ALIAS")]:  # sb's start inside out
+        kw = dict(ok)
+        kw.update(change)
+        assert rrf.rrf_check_scaled_mm_mx_args(**kw) == rrf.Status[status], change
