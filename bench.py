@@ -988,17 +988,18 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
-def run_gemm_only(M: int, N: int, K: int):
-    """One GEMM shape through time_gemm (3 eager calls, then graph replays),
-    for profiling; prints its record."""
+def run_gemm_only(M: int, N: int, K: int, mx: bool = False):
+    """One GEMM shape through time_gemm or time_gemm_mx (3 eager calls, then
+    graph replays), for profiling; prints its record."""
     import torch
 
     import reduce_rmsnorm_fp8_b200 as rrf
     device = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream(device)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    rec = time_gemm(rrf, M, N, K, device, stream, l2, measured_peaks()[0])
-    print(json.dumps({"gemm_fp8": rec}), flush=True)
+    fn, key = (time_gemm_mx, "gemm_mxfp8") if mx else (time_gemm, "gemm_fp8")
+    rec = fn(rrf, M, N, K, device, stream, l2, measured_peaks()[0])
+    print(json.dumps({key: rec}), flush=True)
 
 
 def run_one_secondary(key, fn, *args):
@@ -1032,6 +1033,8 @@ def main(argv=None):
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--gemm", type=int, nargs=3, metavar=("M", "N", "K"), default=None,
                     help="time only the FP8 GEMM of this shape (profiling runs)")
+    ap.add_argument("--gemm-mx", type=int, nargs=3, metavar=("M", "N", "K"), default=None,
+                    help="time only the MX GEMM of this shape (profiling runs)")
     ap.add_argument("--allreduce", nargs=4, metavar=("WORKLOAD", "ROWS", "RANKS", "MODE"),
                     default=None, help="time only the multi-GPU call, all ranks in one launch "
                                        "(MODE 0 auto, 1 one-shot, 2 two-shot; profiling runs)")
@@ -1046,6 +1049,8 @@ def main(argv=None):
         ap.error("--warmup must be at least 3")
     if args.gemm is not None:
         run_gemm_only(*args.gemm)
+    elif args.gemm_mx is not None:
+        run_gemm_only(*args.gemm_mx, mx=True)
     elif args.allreduce is not None:
         w, rows, ranks, mode = args.allreduce
         run_one_secondary("allreduce_emulated", time_allreduce, w, int(rows), int(ranks),

@@ -825,6 +825,253 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// --------------------------------------------- MX GEMM on SM pairs (2 CTAs) --
+// The block-scaled MMA with cta_group::2 on 256 x 256 tiles, as the per-token
+// pair kernel: each CTA loads 128 rows of A and 128 rows of B per k-tile.
+// Scales: each CTA loads the atom of its own 128 A rows and both atoms of
+// the tile's 256 B rows (the MMA scales each CTA's half of the product with
+// the scale codes in that CTA's tensor memory, and every CTA's half spans
+// all 256 columns); the leader's tcgen05.cp.cta_group::2 copies each CTA's
+// atoms from its own shared memory into its own tensor memory.  The scale
+// atoms travel as 3-D TMA boxes, so that the odd CTA's copies, like its A
+// and B tiles, complete on the leader's stage barrier.
+//
+// Tensor memory (512 columns): the 256-column accumulator twice would leave
+// no room for the 12 scale columns, so the two accumulators overlap in 32
+// columns -- buffer 0 at [0, 256), buffer 1 at [224, 480), scales at
+// [480, 492).  The epilogue reads the shared 32 columns first and reports
+// that on `ovl_free`; the MMAs of the next tile wait for it.
+
+// A 3-D tiled load of the pair (no swizzle) completing on the leader's barrier.
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                                 int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];"
+        :
+        : "r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar) & 0xFEFFFFFFu), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
+// tcgen05.cp of the pair: in both CTAs, from the CTA's own shared memory at
+// the descriptor's address to its own tensor memory at `taddr`.
+__device__ __forceinline__ void tmem_copy_32x128b_x4_pair(uint32_t taddr, uint64_t src_desc) {
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(src_desc)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mma_mx_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate, uint32_t sfa,
+                                            uint32_t sfb) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa),
+           "r"(sfb)
+        : "memory");
+}
+
+// mx_idesc with M = 256.
+__host__ __device__ constexpr uint32_t mx_idesc_pair(int bn, uint32_t id) {
+    return (id << 4) | ((uint32_t)(bn >> 3) << 17) | (1u << 23) | ((uint32_t)(256 >> 4) << 24) |
+           (id << 29);
+}
+
+struct MxPairTile {
+    static constexpr int BN = 256;
+    static constexpr int kHalfBytes = 128 * kBK;                 // 16 KB: 128 rows of A or B
+    static constexpr int kSfaBytes = 512;                        // one atom
+    static constexpr int kSfbBytes = 1024;                       // two atoms: 256 rows of B
+    static constexpr int kSfOffset = 2 * kHalfBytes;
+    static constexpr int kStageBytes = 2 * kHalfBytes + kSfaBytes + kSfbBytes;  // 33.5 KB
+    static constexpr int kStageStride = (kStageBytes + 1023) / 1024 * 1024;     // 34 KB
+    static constexpr int kStages = 6;
+    static constexpr int kTmemCols = 512;
+    static constexpr uint32_t kBuf1 = 224;                       // buffer 1's first column
+    static constexpr uint32_t kSfaCol = kBuf1 + BN;              // 480
+    static constexpr uint32_t kSfbCol = kSfaCol + 4;             // 484 .. 491
+    // full / empty per stage, full / empty per accumulator, overlap, drain
+    static constexpr int kBarriers = 2 * kStages + 4 + 1 + 1;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageStride + kBarriers * 8 + 16;
+};
+static_assert(MxPairTile::kSfbCol + 8 <= MxPairTile::kTmemCols, "scale columns past the allocation");
+static_assert(MxPairTile::kSmemBytes <= 227 * 1024, "stages exceed the shared memory of a CTA");
+
+__global__ void __launch_bounds__(kThreads, 1)
+    scaled_mm_mx_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
+                             const __grid_constant__ CUtensorMap tma_b,
+                             const __grid_constant__ CUtensorMap tma_sfa,
+                             const __grid_constant__ CUtensorMap tma_sfb, const GemmArgs g) {
+    using T = MxPairTile;
+    constexpr int S = T::kStages;
+    constexpr int BN = T::BN;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * T::kStageStride);  // leader's are used
+    uint64_t* empty = full + S;
+    uint64_t* acc_full = empty + S;       // [2]
+    uint64_t* acc_empty = acc_full + 2;   // [2], the leader's: both CTAs' epilogue warps
+    uint64_t* ovl_free = acc_empty + 2;   // the leader's: the shared columns have been read
+    uint64_t* drained = ovl_free + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();  // 0: the leader
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int tiles_n = (g.N + 255) / 256, tiles_m = (g.M + 255) / 256;
+    const int tiles = tiles_n * tiles_m;
+    const int ktiles = g.K / kBK;  // K is a multiple of 128
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 8);  // 4 epilogue warps in each CTA of the pair
+        }
+        mbar_init(ovl_free, 8);
+        mbar_init(drained, 1);
+        fence_mbar_init_cluster();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, T::kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before_sync();
+    cluster_arrive_release();
+    cluster_wait_acquire();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---- producer (each CTA): its 128 rows of A and of B, its A scale
+        // atom and both B scale atoms of the tile, per k-tile
+        if (lane == 0) {
+            int it = 0;
+            bool ok = true;
+            for (int t = pair; t < tiles && ok; t += npairs) {
+                int tm, tn;
+                grouped_tile(t, tiles_m, tiles_n, tm, tn);
+                const int m0 = tm * 256 + (int)rank * 128;
+                const int n0 = tn * 256 + (int)rank * 128;
+                for (int kt = 0; kt < ktiles; ++kt, ++it) {
+                    const int s = it % S;
+                    if (!wait_phase(&empty[s], ((it / S) & 1) ^ 1, g.err)) {
+                        ok = false;
+                        break;
+                    }
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * T::kStageBytes);
+                    uint8_t* dst = smem + s * T::kStageStride;
+                    tma_load_2d_pair(dst, &tma_a, &full[s], kt * kBK, m0);
+                    tma_load_2d_pair(dst + T::kHalfBytes, &tma_b, &full[s], kt * kBK, n0);
+                    tma_load_3d_pair(dst + T::kSfOffset, &tma_sfa, &full[s], 0, kt, m0 / 128);
+                    tma_load_3d_pair(dst + T::kSfOffset + T::kSfaBytes, &tma_sfb, &full[s], 0, kt,
+                                     tn * 2);
+                }
+            }
+            for (int i = it > S ? it - S : 0; i < it; ++i)
+                wait_phase(&empty[i % S], (i / S) & 1, g.err);
+        }
+    } else if (warp == 1) {
+        // ---- scale copies and MMAs (the leader only)
+        if (rank == 0 && lane == 0) {
+            const uint32_t peer = 1;
+            int it = 0, j = 0;
+            bool ok = true;
+            for (int t = pair; t < tiles && ok; t += npairs, ++j) {
+                const int buf = j & 1;
+                // this buffer's previous tile has been drained, and the
+                // previous tile (the other buffer) no longer needs the
+                // shared columns
+                if (!wait_phase(&acc_empty[buf], ((j >> 1) & 1) ^ 1, g.err)) break;
+                if (j > 0 && !wait_phase(ovl_free, (j - 1) & 1, g.err)) break;
+                tc_fence_after_sync();
+                const uint32_t d = tmem + (buf ? T::kBuf1 : 0u);
+                for (int kt = 0; kt < ktiles; ++kt, ++it) {
+                    const int s = it % S;
+                    if (!wait_phase(&full[s], (it / S) & 1, g.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint8_t* tile = smem + s * T::kStageStride;
+                    const uint8_t* sf = tile + T::kSfOffset;
+                    tmem_copy_32x128b_x4_pair(tmem + T::kSfaCol, sf_atom_desc(sf));
+                    tmem_copy_32x128b_x4_pair(tmem + T::kSfbCol, sf_atom_desc(sf + T::kSfaBytes));
+                    tmem_copy_32x128b_x4_pair(tmem + T::kSfbCol + 4,
+                                              sf_atom_desc(sf + T::kSfaBytes + 512));
+                    const uint64_t ad = kmajor_sw128_desc(tile);
+                    const uint64_t bd = kmajor_sw128_desc(tile + T::kHalfBytes);
+#pragma unroll
+                    for (int k = 0; k < kBK / kMmaK; ++k) {
+                        const uint64_t step = (uint64_t)(k * kMmaK) >> 4;
+                        mma_mx_pair(d, ad + step, bd + step, mx_idesc_pair(BN, (uint32_t)k),
+                                    (kt | k) != 0, tmem + T::kSfaCol, tmem + T::kSfbCol);
+                    }
+                    mma_commit_pair(smem_u32(&empty[s]));
+                    mma_commit_pair(peer_smem(&empty[s], peer));
+                }
+                mma_commit_pair(smem_u32(&acc_full[buf]));
+                mma_commit_pair(peer_smem(&acc_full[buf], peer));
+            }
+            mma_commit_pair(smem_u32(drained));
+            mma_commit_pair(peer_smem(drained, peer));
+        }
+        __syncwarp();
+    } else {
+        // ---- epilogue (each CTA): its 128 accumulator rows; the 32 columns
+        // shared by the two buffers first
+        const int quarter = warp & 3;
+        const uint32_t leader_acc_empty[2] = {peer_smem(&acc_empty[0], 0),
+                                              peer_smem(&acc_empty[1], 0)};
+        const uint32_t leader_ovl_free = peer_smem(ovl_free, 0);
+        int j = 0;
+        for (int t = pair; t < tiles; t += npairs, ++j) {
+            const int buf = j & 1;
+            int tm, tn;
+            grouped_tile(t, tiles_m, tiles_n, tm, tn);
+            const int m0 = tm * 256 + (int)rank * 128, n0 = tn * 256;
+            bool have = wait_phase(&acc_full[buf], (j >> 1) & 1, g.err);
+            if (!__all_sync(0xFFFFFFFFu, have)) break;
+            tc_fence_after_sync();
+            const int row = m0 + quarter * 32 + lane;
+            const uint32_t base = tmem + (buf ? T::kBuf1 : 0u) + ((uint32_t)(quarter * 32) << 16);
+            // the shared columns are the last 32 of buffer 0, the first of buffer 1
+            const int first = buf ? 0 : BN - 32;
+            for (int i = 0; i < BN / 32; ++i) {
+                const int c = (first + 32 * i) % BN;
+                float v[32];
+                tmem_load_32(base + (uint32_t)c, v);
+                if (i == 0) {
+                    tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(leader_ovl_free);
+                }
+                const int n = n0 + c;
+                if (row >= g.M || n >= g.N) continue;
+                store_row_chunk(g, v, 1.0f, row, n);  // g.b_scale is null: no scaling
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(leader_acc_empty[buf]);
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        wait_phase(drained, 0, g.err);
+        tc_fence_after_sync();
+        tmem_dealloc_pair(tmem, T::kTmemCols);
+    }
+    cluster_arrive_release();
+    cluster_wait_acquire();
+}
+
 // ------------------------------------------------------------------- host --
 
 using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -859,6 +1106,23 @@ bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int b
     const cuuint32_t elem[2] = {1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
               elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+// Blocked scale codes of a [rows, K] operand as a 3-D array of 32-bit words:
+// 128 words (one 512-byte atom) x K/128 atoms along k x ceil(rows/128) row
+// blocks; a box is one atom (box_blocks 1) or the atoms of two consecutive
+// row blocks (2).  Row blocks past the operand read as zero.
+bool make_sf_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int box_blocks) {
+    EncodeTiled fn = encode_tiled();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[3] = {128, (cuuint64_t)(K / 128), (cuuint64_t)((rows + 127) / 128)};
+    const cuuint64_t strides[2] = {512, (cuuint64_t)(K / 128) * 512};
+    const cuuint32_t box[3] = {128, 1, (cuuint32_t)box_blocks};
+    const cuuint32_t elem[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), dims, strides, box,
+              elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
            CUDA_SUCCESS;
 }
@@ -946,11 +1210,50 @@ cudaError_t launch_mx(const GemmArgs& g, const void* a, const void* b, const uin
     return cudaGetLastError();
 }
 
+cudaError_t launch_mx_pair(const GemmArgs& g, const void* a, const void* b, const uint8_t* sfa,
+                           const uint8_t* sfb, int sm_count, cudaStream_t stream) {
+    using T = MxPairTile;
+    CUtensorMap ma, mb, msa, msb;
+    if (!make_map(&ma, a, g.M, g.K, 128) || !make_map(&mb, b, g.N, g.K, 128) ||
+        !make_sf_map(&msa, sfa, g.M, g.K, 1) || !make_sf_map(&msb, sfb, g.N, g.K, 2))
+        return cudaErrorInvalidValue;
+    static std::atomic<uint64_t> enabled_on{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
+    if (bit == 0 || (enabled_on.load(std::memory_order_relaxed) & bit) == 0) {
+        e = cudaFuncSetAttribute(scaled_mm_mx_pair_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, T::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        enabled_on.fetch_or(bit, std::memory_order_relaxed);
+    }
+    const int64_t tiles = (int64_t)((g.N + 255) / 256) * ((g.M + 255) / 256);
+    const int64_t pairs = tiles < sm_count / 2 ? tiles : sm_count / 2;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = T::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, scaled_mm_mx_pair_kernel, ma, mb, msa, msb, g);
+}
+
 }  // namespace
 
 cudaError_t launch_scaled_mm_mx(const GemmArgs& g, const void* a, const void* b,
                                 const uint8_t* sfa, const uint8_t* sfb, int sm_count,
                                 cudaStream_t stream) {
+    // 256 x 256 tiles on SM pairs once they fill every pair, as the
+    // per-token GEMM; else one CTA per 128 x 128 tile
+    if (((g.M + 255) / 256) * ((g.N + 255) / 256) >= sm_count / 2)
+        return launch_mx_pair(g, a, b, sfa, sfb, sm_count, stream);
     return launch_mx(g, a, b, sfa, sfb, sm_count, stream);
 }
 

@@ -148,7 +148,22 @@ def test_mx_gemm_matches_oracle(rrf, M, N, K, bias):
     check_mx_gemm(c, sa, sb, out, label=f"{M}x{N}x{K}")
 
 
-@pytest.mark.parametrize("M,N,K", [(64, 7168, 7168), (2000, 2560, 1024)])
+@pytest.mark.parametrize("bias", [True, False])
+def test_mx_gemm_pair_tiles_with_tails(rrf, bias):
+    """Enough 256 x 256 tiles for the SM-pair kernel (every pair takes two,
+    so both accumulators and their shared columns are used), with a row tail
+    inside the odd CTA's half and a column tail that leaves the odd CTA's B
+    half and the second B scale atom past the operand; every output checked."""
+    M, N, K = 2200, 2320, 384
+    c, sa, sb = mx_operands(M, N, K, 4, bias)
+    out = rrf.rrf_scaled_mm_mxfp8(c.a, rrf.mx_blocked(torch.from_numpy(sa).cuda()), c.b,
+                                  rrf.mx_blocked(torch.from_numpy(sb).cuda()), c.bias)
+    torch.cuda.synchronize()
+    check_mx_gemm(c, sa, sb, out, label=f"pair {M}x{N}x{K}")
+    assert rrf.rrf_device_error() == 0
+
+
+@pytest.mark.parametrize("M,N,K", [(64, 7168, 7168), (2000, 2560, 1024), (8192, 8192, 8192)])
 def test_mx_gemm_large_sampled_rows(rrf, M, N, K):
     c, sa, sb = mx_operands(M, N, K, 7)
     out = rrf.rrf_scaled_mm_mxfp8(c.a, rrf.mx_blocked(torch.from_numpy(sa).cuda()), c.b,
