@@ -666,27 +666,38 @@ __host__ __device__ constexpr uint32_t mx_idesc(int bn, uint32_t id) {
            (id << 29);
 }
 
+// BN 128 or 64 columns per tile; AROWS as for the per-token kernel (64 for
+// calls of at most 64 rows: the MMA's rows 64-127 then read the B tile that
+// follows and land in accumulator rows that are never stored).  A 64-column
+// tile uses half of its B scale atom: the MMA reads the scale columns from 2
+// further on for the odd half (column j of the atom holds rows 32j..32j+31).
+template <int BN, int AROWS>
 struct MxTile {
-    static constexpr int BN = 128;
-    static constexpr int kABytes = kBM * kBK;        // 16 KB
-    static constexpr int kBBytes = BN * kBK;         // 16 KB
+    static_assert(BN == 128 || BN == 64, "one scale atom covers 128 columns");
+    static_assert(AROWS == kBM || (AROWS == 64 && BN == 64),
+                  "the MMA's 128 rows of A must stay inside the stage");
+    static constexpr int kABytes = AROWS * kBK;
+    static constexpr int kBBytes = BN * kBK;
     static constexpr int kSfBytes = 512;             // one atom: 128 rows x 4 codes
-    static constexpr int kStageBytes = kABytes + kBBytes + 2 * kSfBytes;  // 33 KB
+    static constexpr int kStageBytes = kABytes + kBBytes + 2 * kSfBytes;
     static constexpr int kStageStride = (kStageBytes + 1023) / 1024 * 1024;
-    static constexpr int kStages = 6;
+    // as many stages as fit in 200 KB, at most 12: 6 at BN 128, 11 at 64
+    static constexpr int kStages =
+        (200 * 1024) / kStageStride > 12 ? 12 : (200 * 1024) / kStageStride;
     static constexpr int kAccCols = 2 * BN;          // two accumulators
-    static constexpr int kTmemCols = 512;            // accumulators, then 4 + 4 scale columns
+    // accumulators, then 4 + 4 scale columns (a power of two of at least 32)
+    static constexpr int kTmemCols = BN == 128 ? 512 : 256;
     static constexpr int kBarriers = 2 * kStages + 4 + 1;
     static constexpr int kSmemBytes = 1024 + kStages * kStageStride + kBarriers * 8 + 16;
 };
 
+template <int BN, int AROWS>
 __global__ void __launch_bounds__(kThreads, 1)
     scaled_mm_mx_kernel(const __grid_constant__ CUtensorMap tma_a,
                         const __grid_constant__ CUtensorMap tma_b, const GemmArgs g,
                         const uint8_t* sfa, const uint8_t* sfb) {
-    using T = MxTile;
+    using T = MxTile<BN, AROWS>;
     constexpr int S = T::kStages;
-    constexpr int BN = T::BN;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -762,6 +773,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!wait_phase(&acc_empty[buf], ((j >> 1) & 1) ^ 1, g.err)) break;
                 tc_fence_after_sync();
                 const uint32_t d = tmem + (uint32_t)(buf * BN);
+                // the odd 64-column half of a scale atom: 2 columns further on
+                const uint32_t sfb_cols =
+                    tmem_sfb + (BN == 64 ? (uint32_t)((t % tiles_n) & 1) * 2u : 0u);
                 for (int kt = 0; kt < ktiles; ++kt, ++it) {
                     const int s = it % S;
                     if (!wait_phase(&full[s], (it / S) & 1, g.err)) {
@@ -782,7 +796,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int k = 0; k < kBK / kMmaK; ++k) {
                         const uint64_t step = (uint64_t)(k * kMmaK) >> 4;
                         mma_mx(d, ad + step, bd + step, mx_idesc(BN, (uint32_t)k), (kt | k) != 0,
-                               tmem_sfa, tmem_sfb);
+                               tmem_sfa, sfb_cols);
                     }
                     mma_commit(&empty[s]);
                 }
@@ -1187,26 +1201,28 @@ cudaError_t launch_pair(const GemmArgs& g, const void* a, const void* b, int sm_
     return cudaLaunchKernelEx(&cfg, scaled_mm_pair_kernel, ma, mb, g);
 }
 
+template <int BN, int AROWS>
 cudaError_t launch_mx(const GemmArgs& g, const void* a, const void* b, const uint8_t* sfa,
                       const uint8_t* sfb, int sm_count, cudaStream_t stream) {
-    using T = MxTile;
+    using T = MxTile<BN, AROWS>;
     CUtensorMap ma, mb;
-    if (!make_map(&ma, a, g.M, g.K, kBM) || !make_map(&mb, b, g.N, g.K, T::BN))
+    if (!make_map(&ma, a, g.M, g.K, AROWS) || !make_map(&mb, b, g.N, g.K, BN))
         return cudaErrorInvalidValue;
+    auto kernel = scaled_mm_mx_kernel<BN, AROWS>;
     static std::atomic<uint64_t> enabled_on{0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
     if (bit == 0 || (enabled_on.load(std::memory_order_relaxed) & bit) == 0) {
-        e = cudaFuncSetAttribute(scaled_mm_mx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  T::kSmemBytes);
         if (e != cudaSuccess) return e;
         enabled_on.fetch_or(bit, std::memory_order_relaxed);
     }
-    const int64_t tiles = (int64_t)((g.N + T::BN - 1) / T::BN) * ((g.M + kBM - 1) / kBM);
+    const int64_t tiles = (int64_t)((g.N + BN - 1) / BN) * ((g.M + kBM - 1) / kBM);
     const unsigned grid = (unsigned)(tiles < sm_count ? tiles : sm_count);
-    scaled_mm_mx_kernel<<<grid, kThreads, T::kSmemBytes, stream>>>(ma, mb, g, sfa, sfb);
+    kernel<<<grid, kThreads, T::kSmemBytes, stream>>>(ma, mb, g, sfa, sfb);
     return cudaGetLastError();
 }
 
@@ -1251,10 +1267,15 @@ cudaError_t launch_scaled_mm_mx(const GemmArgs& g, const void* a, const void* b,
                                 const uint8_t* sfa, const uint8_t* sfb, int sm_count,
                                 cudaStream_t stream) {
     // 256 x 256 tiles on SM pairs once they fill every pair, as the
-    // per-token GEMM; else one CTA per 128 x 128 tile
+    // per-token GEMM
     if (((g.M + 255) / 256) * ((g.N + 255) / 256) >= sm_count / 2)
         return launch_mx_pair(g, a, b, sfa, sfb, sm_count, stream);
-    return launch_mx(g, a, b, sfa, sfb, sm_count, stream);
+    // else one CTA per 128 x 128 tile once those fill every SM; short, wide
+    // problems take 128 x 64 tiles (64-row A stages for at most 64 rows)
+    if (((g.M + kBM - 1) / kBM) * ((g.N + 127) / 128) >= sm_count)
+        return launch_mx<128, kBM>(g, a, b, sfa, sfb, sm_count, stream);
+    if (g.M <= 64) return launch_mx<64, 64>(g, a, b, sfa, sfb, sm_count, stream);
+    return launch_mx<64, kBM>(g, a, b, sfa, sfb, sm_count, stream);
 }
 
 cudaError_t launch_scaled_mm(const GemmArgs& g, const void* a, const void* b, int sm_count,
