@@ -196,37 +196,75 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_u32(bar)) : "memory");
 }
 
-// AROWS: rows of A loaded per stage.  128 normally; 64 for calls of at most
-// 64 rows, which halves the A stage and so deepens the ring (the MMA still
-// reads 128 rows: rows 64-127 come from the B half of the same stage, whose
-// 8 KB follow, and land in accumulator rows that are never stored).
-template <int BN, int AROWS>
+// AROWS: rows of A loaded per k-tile.  128 normally; 8, 16, 32 or 64 for
+// calls of at most that many rows, which shrinks the A stage (the MMA still
+// reads 128 rows: the rows past AROWS come from the bytes that follow -- the
+// next k-tiles' A rows or the stage's B tiles -- and land in accumulator
+// rows that are never stored).
+// Z: k-tiles per stage, loaded by one 3-D TMA box per operand (128 bytes x
+// rows x Z atoms of 128 values of K).  A TMA operation moves a few KB at a
+// fixed cost, and a CTA streams a weight only as fast as it issues them:
+// short, wide products (a decode batch against a weight) take Z = 4 or 2,
+// which needs K % 128 == 0 (k-atoms past K read as zero).
+template <int BN, int AROWS, int Z>
 struct Tile {
-    static_assert(AROWS == kBM || (AROWS == 64 && BN == 64),
+    static_assert(AROWS == kBM || (AROWS <= 64 && AROWS % 8 == 0 && BN == 64),
                   "the MMA's 128 rows of A must stay inside the stage");
-    static constexpr int kABytes = AROWS * kBK;
-    static constexpr int kBBytes = BN * kBK;
-    static constexpr int kStageBytes = kABytes + kBBytes;
-    // as many stages as fit in 200 KB, at most 12: 4 at BN 256, 6 at 128,
-    // 8 at 64, 12 with 64-row A stages
-    static constexpr int kStages =
-        (200 * 1024) / kStageBytes > 12 ? 12 : (200 * 1024) / kStageBytes;
+    static_assert((Z - 1) * AROWS * kBK + kBM * kBK <= Z * (AROWS + BN) * kBK,
+                  "the MMA's 128 rows of A must stay inside the stage");
+    static constexpr int kABytes = AROWS * kBK;        // one k-tile of A
+    static constexpr int kBBytes = BN * kBK;           // one k-tile of B
+    static constexpr int kBOffset = Z * kABytes;       // B tiles follow the Z A tiles
+    static constexpr int kStageBytes = Z * (kABytes + kBBytes);
+    // as many stages as fit in 200 KB (220 KB with several k-tiles per
+    // stage), at most 12: 4 at BN 256, 6 at 128, 8 at 64, 12 with 64-row A
+    // stages, 3 with four k-tiles of 64 rows
+    static constexpr int kBudget = (Z > 1 ? 220 : 200) * 1024;
+    static constexpr int kStages = kBudget / kStageBytes > 12 ? 12 : kBudget / kStageBytes;
     static constexpr int kTmemCols = 2 * BN;  // two accumulators
     // full / empty per stage, full / empty per accumulator, one for the drain
     static constexpr int kBarriers = 2 * kStages + 4 + 1;
     // 1 KB of slack aligns the stages to the 1024-byte swizzle atom
     static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarriers * 8 + 16;
+    static_assert(kSmemBytes <= 227 * 1024, "stages exceed the shared memory of a CTA");
 };
+
+// 3-D tiled load of box {x, y, z} at coordinates (x, y, z), completing on
+// `bar` (no multicast).
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];"
+        :
+        : "r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
+// The loads of stage group kg (k-tiles kg*Z ...) of A rows m0.. and B rows
+// n0..: 2-D boxes for Z = 1, else one 3-D box of Z atoms per operand.
+template <int Z, int ABYTES, int BOFFSET>
+__device__ __forceinline__ void load_group(uint8_t* dst, const CUtensorMap* ma,
+                                           const CUtensorMap* mb, uint64_t* bar, int kg, int m0,
+                                           int n0) {
+    if constexpr (Z == 1) {
+        tma_load_2d(dst, ma, bar, kg * kBK, m0);
+        tma_load_2d(dst + BOFFSET, mb, bar, kg * kBK, n0);
+    } else {
+        tma_load_3d(dst, ma, bar, 0, m0, kg * Z);
+        tma_load_3d(dst + BOFFSET, mb, bar, 0, n0, kg * Z);
+    }
+}
 
 // A persistent grid: CTA c takes tiles c, c + gridDim.x, ... (row-major over
 // the 128 x BN tiles, so the CTAs working at one time share A rows and B
 // columns in L2).  The accumulator is double-buffered in tensor memory: the
 // MMAs of a CTA's next tile run while the epilogue warps drain this one.
-template <int BN, int AROWS>
+template <int BN, int AROWS, int Z>
 __global__ void __launch_bounds__(kThreads, 1)
     scaled_mm_kernel(const __grid_constant__ CUtensorMap tma_a,
                      const __grid_constant__ CUtensorMap tma_b, const GemmArgs g) {
-    using T = Tile<BN, AROWS>;
+    using T = Tile<BN, AROWS, Z>;
     constexpr int S = T::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -242,6 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tiles_n = (g.N + BN - 1) / BN;
     const int tiles = tiles_n * ((g.M + kBM - 1) / kBM);
     const int ktiles = (g.K + kBK - 1) / kBK;
+    const int kgroups = (ktiles + Z - 1) / Z;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -271,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
                 const int m0 = (t / tiles_n) * kBM, n0 = (t % tiles_n) * BN;
-                for (int kt = 0; kt < ktiles; ++kt, ++it) {
+                for (int kg = 0; kg < kgroups; ++kg, ++it) {
                     const int s = it % S;
                     // a fresh barrier counts as having completed the phase
                     // before phase 0: the first pass over the ring does not wait
@@ -279,10 +318,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    uint8_t* dst = smem + s * T::kStageBytes;
                     mbar_arrive_expect_tx(&full[s], T::kStageBytes);
-                    tma_load_2d(dst, &tma_a, &full[s], kt * kBK, m0);
-                    tma_load_2d(dst + T::kABytes, &tma_b, &full[s], kt * kBK, n0);
+                    load_group<Z, T::kABytes, T::kBOffset>(smem + s * T::kStageBytes, &tma_a,
+                                                           &tma_b, &full[s], kg, m0, n0);
                 }
             }
             // the loads still in flight land before the CTA may exit
@@ -301,21 +339,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!wait_phase(&acc_empty[buf], ((j >> 1) & 1) ^ 1, g.err)) break;
                 tc_fence_after_sync();
                 const uint32_t d = tmem + (uint32_t)(buf * BN);
-                for (int kt = 0; kt < ktiles; ++kt, ++it) {
+                for (int kg = 0; kg < kgroups; ++kg, ++it) {
                     const int s = it % S;
                     if (!wait_phase(&full[s], (it / S) & 1, g.err)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint8_t* tile = smem + s * T::kStageBytes;
-                    const uint64_t ad = kmajor_sw128_desc(tile);
-                    const uint64_t bd = kmajor_sw128_desc(tile + T::kABytes);
+                    const uint8_t* stage = smem + s * T::kStageBytes;
+                    // the k-tiles of the group that lie inside K
+                    const int nk = ktiles - kg * Z < Z ? ktiles - kg * Z : Z;
+                    for (int j = 0; j < nk; ++j) {
+                        const uint64_t ad = kmajor_sw128_desc(stage + j * T::kABytes);
+                        const uint64_t bd = kmajor_sw128_desc(stage + T::kBOffset + j * T::kBBytes);
 #pragma unroll
-                    for (int k = 0; k < kBK / kMmaK; ++k) {
-                        // advance the start address by k * 32 bytes in the swizzle row
-                        const uint64_t step = (uint64_t)(k * kMmaK) >> 4;
-                        mma_f8(d, ad + step, bd + step, idesc, (kt | k) != 0);
+                        for (int k = 0; k < kBK / kMmaK; ++k) {
+                            // advance the start address by k * 32 bytes in the swizzle row
+                            const uint64_t step = (uint64_t)(k * kMmaK) >> 4;
+                            mma_f8(d, ad + step, bd + step, idesc, (kg | j | k) != 0);
+                        }
                     }
                     mma_commit(&empty[s]);  // the stage is free once these are done
                 }
@@ -666,37 +708,46 @@ __host__ __device__ constexpr uint32_t mx_idesc(int bn, uint32_t id) {
            (id << 29);
 }
 
-// BN 128 or 64 columns per tile; AROWS as for the per-token kernel (64 for
-// calls of at most 64 rows: the MMA's rows 64-127 then read the B tile that
-// follows and land in accumulator rows that are never stored).  A 64-column
-// tile uses half of its B scale atom: the MMA reads the scale columns from 2
-// further on for the odd half (column j of the atom holds rows 32j..32j+31).
-template <int BN, int AROWS>
+// BN 128 or 64 columns per tile; AROWS and Z (k-tiles per stage, one 3-D
+// TMA box per operand) as for the per-token kernel (64-row A: the MMA's rows
+// 64-127 read the 8 KB that follow and land in accumulator rows that are
+// never stored).  A 64-column tile uses half of its B scale atom: the MMA
+// reads the scale columns from 2 further on for the odd half (column j of
+// the atom holds rows 32j..32j+31).  Stage: Z A tiles, Z B tiles, the Z A
+// scale atoms, the Z B scale atoms (consecutive in the blocked order).
+template <int BN, int AROWS, int Z>
 struct MxTile {
     static_assert(BN == 128 || BN == 64, "one scale atom covers 128 columns");
-    static_assert(AROWS == kBM || (AROWS == 64 && BN == 64),
+    static_assert(AROWS == kBM || (AROWS <= 64 && AROWS % 8 == 0 && BN == 64),
                   "the MMA's 128 rows of A must stay inside the stage");
-    static constexpr int kABytes = AROWS * kBK;
-    static constexpr int kBBytes = BN * kBK;
+    static_assert((Z - 1) * AROWS * kBK + kBM * kBK <= Z * (AROWS + BN) * kBK,
+                  "the MMA's 128 rows of A must stay inside the stage");
+    static constexpr int kABytes = AROWS * kBK;      // one k-tile of A
+    static constexpr int kBBytes = BN * kBK;         // one k-tile of B
     static constexpr int kSfBytes = 512;             // one atom: 128 rows x 4 codes
-    static constexpr int kStageBytes = kABytes + kBBytes + 2 * kSfBytes;
+    static constexpr int kBOffset = Z * kABytes;
+    static constexpr int kSfaOffset = Z * (kABytes + kBBytes);
+    static constexpr int kSfbOffset = kSfaOffset + Z * kSfBytes;
+    static constexpr int kStageBytes = Z * (kABytes + kBBytes + 2 * kSfBytes);
     static constexpr int kStageStride = (kStageBytes + 1023) / 1024 * 1024;
-    // as many stages as fit in 200 KB, at most 12: 6 at BN 128, 11 at 64
-    static constexpr int kStages =
-        (200 * 1024) / kStageStride > 12 ? 12 : (200 * 1024) / kStageStride;
+    // as many stages as fit in 200 KB (220 KB with several k-tiles per
+    // stage), at most 12: 6 at BN 128, 11 at 64, 3 with four 64-row k-tiles
+    static constexpr int kBudget = (Z > 1 ? 220 : 200) * 1024;
+    static constexpr int kStages = kBudget / kStageStride > 12 ? 12 : kBudget / kStageStride;
     static constexpr int kAccCols = 2 * BN;          // two accumulators
     // accumulators, then 4 + 4 scale columns (a power of two of at least 32)
     static constexpr int kTmemCols = BN == 128 ? 512 : 256;
     static constexpr int kBarriers = 2 * kStages + 4 + 1;
     static constexpr int kSmemBytes = 1024 + kStages * kStageStride + kBarriers * 8 + 16;
+    static_assert(kSmemBytes <= 227 * 1024, "stages exceed the shared memory of a CTA");
 };
 
-template <int BN, int AROWS>
+template <int BN, int AROWS, int Z>
 __global__ void __launch_bounds__(kThreads, 1)
     scaled_mm_mx_kernel(const __grid_constant__ CUtensorMap tma_a,
                         const __grid_constant__ CUtensorMap tma_b, const GemmArgs g,
                         const uint8_t* sfa, const uint8_t* sfb) {
-    using T = MxTile<BN, AROWS>;
+    using T = MxTile<BN, AROWS, Z>;
     constexpr int S = T::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -712,6 +763,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tiles_n = (g.N + BN - 1) / BN;
     const int tiles = tiles_n * ((g.M + kBM - 1) / kBM);
     const int ktiles = g.K / kBK;  // K is a multiple of 128
+    const int kgroups = (ktiles + Z - 1) / Z;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -744,20 +796,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int m0 = (t / tiles_n) * kBM, n0 = (t % tiles_n) * BN;
                 const uint8_t* sfa_tile = sfa + (int64_t)(m0 / 128) * ktiles * T::kSfBytes;
                 const uint8_t* sfb_tile = sfb + (int64_t)(n0 / 128) * ktiles * T::kSfBytes;
-                for (int kt = 0; kt < ktiles; ++kt, ++it) {
+                for (int kg = 0; kg < kgroups; ++kg, ++it) {
                     const int s = it % S;
                     if (!wait_phase(&empty[s], ((it / S) & 1) ^ 1, g.err)) {
                         ok = false;
                         break;
                     }
                     uint8_t* dst = smem + s * T::kStageStride;
-                    mbar_arrive_expect_tx(&full[s], T::kStageBytes);
-                    tma_load_2d(dst, &tma_a, &full[s], kt * kBK, m0);
-                    tma_load_2d(dst + T::kABytes, &tma_b, &full[s], kt * kBK, n0);
-                    bulk_load(dst + T::kABytes + T::kBBytes, sfa_tile + kt * T::kSfBytes,
-                              T::kSfBytes, &full[s]);
-                    bulk_load(dst + T::kABytes + T::kBBytes + T::kSfBytes,
-                              sfb_tile + kt * T::kSfBytes, T::kSfBytes, &full[s]);
+                    // the scale atoms of the group's k-tiles inside K (a 1-D
+                    // copy must not run past the row block's atoms); the A
+                    // and B boxes are whole (atoms past K read as zero)
+                    const int nk = ktiles - kg * Z < Z ? ktiles - kg * Z : Z;
+                    const uint32_t sf_bytes = (uint32_t)(nk * T::kSfBytes);
+                    mbar_arrive_expect_tx(&full[s],
+                                          Z * (T::kABytes + T::kBBytes) + 2 * sf_bytes);
+                    load_group<Z, T::kABytes, T::kBOffset>(dst, &tma_a, &tma_b, &full[s], kg,
+                                                           m0, n0);
+                    bulk_load(dst + T::kSfaOffset, sfa_tile + kg * Z * T::kSfBytes, sf_bytes,
+                              &full[s]);
+                    bulk_load(dst + T::kSfbOffset, sfb_tile + kg * Z * T::kSfBytes, sf_bytes,
+                              &full[s]);
                 }
             }
             for (int i = it > S ? it - S : 0; i < it; ++i)
@@ -776,27 +834,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // the odd 64-column half of a scale atom: 2 columns further on
                 const uint32_t sfb_cols =
                     tmem_sfb + (BN == 64 ? (uint32_t)((t % tiles_n) & 1) * 2u : 0u);
-                for (int kt = 0; kt < ktiles; ++kt, ++it) {
+                for (int kg = 0; kg < kgroups; ++kg, ++it) {
                     const int s = it % S;
                     if (!wait_phase(&full[s], (it / S) & 1, g.err)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint8_t* tile = smem + s * T::kStageStride;
-                    // tcgen05 operations of this thread run in issue order: the
-                    // copies land before the MMAs below read the scales, and
-                    // the previous k-tile's MMAs have read theirs before these
-                    tmem_copy_32x128b_x4(tmem_sfa, sf_atom_desc(tile + T::kABytes + T::kBBytes));
-                    tmem_copy_32x128b_x4(tmem_sfb, sf_atom_desc(tile + T::kABytes + T::kBBytes +
-                                                                T::kSfBytes));
-                    const uint64_t ad = kmajor_sw128_desc(tile);
-                    const uint64_t bd = kmajor_sw128_desc(tile + T::kABytes);
+                    const uint8_t* stage = smem + s * T::kStageStride;
+                    const int nk = ktiles - kg * Z < Z ? ktiles - kg * Z : Z;
+                    for (int kj = 0; kj < nk; ++kj) {
+                        // tcgen05 operations of this thread run in issue order:
+                        // the copies land before the MMAs below read the
+                        // scales, and the previous k-tile's MMAs have read
+                        // theirs before these
+                        tmem_copy_32x128b_x4(tmem_sfa,
+                                             sf_atom_desc(stage + T::kSfaOffset + kj * T::kSfBytes));
+                        tmem_copy_32x128b_x4(tmem_sfb,
+                                             sf_atom_desc(stage + T::kSfbOffset + kj * T::kSfBytes));
+                        const uint64_t ad = kmajor_sw128_desc(stage + kj * T::kABytes);
+                        const uint64_t bd = kmajor_sw128_desc(stage + T::kBOffset + kj * T::kBBytes);
 #pragma unroll
-                    for (int k = 0; k < kBK / kMmaK; ++k) {
-                        const uint64_t step = (uint64_t)(k * kMmaK) >> 4;
-                        mma_mx(d, ad + step, bd + step, mx_idesc(BN, (uint32_t)k), (kt | k) != 0,
-                               tmem_sfa, sfb_cols);
+                        for (int k = 0; k < kBK / kMmaK; ++k) {
+                            const uint64_t step = (uint64_t)(k * kMmaK) >> 4;
+                            mma_mx(d, ad + step, bd + step, mx_idesc(BN, (uint32_t)k),
+                                   (kg | kj | k) != 0, tmem_sfa, sfb_cols);
+                        }
                     }
                     mma_commit(&empty[s]);
                 }
@@ -1141,14 +1204,37 @@ bool make_sf_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, in
            CUDA_SUCCESS;
 }
 
-template <int BN, int AROWS>
+// A [rows, K] byte matrix (K % 128 == 0) as a 3-D array: 128 bytes x rows x
+// K/128 atoms; a box is box_rows rows of Z consecutive atoms, which land as
+// Z row-major tiles of box_rows x 128 bytes, 128-byte swizzle.  Rows and
+// atoms past the matrix read as zero.
+bool make_map3(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int box_rows, int z) {
+    EncodeTiled fn = encode_tiled();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)kBK, (cuuint64_t)rows, (cuuint64_t)(K / kBK)};
+    const cuuint64_t strides[2] = {(cuuint64_t)K, (cuuint64_t)kBK};
+    const cuuint32_t box[3] = {(cuuint32_t)kBK, (cuuint32_t)box_rows, (cuuint32_t)z};
+    const cuuint32_t elem[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
+              elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+// The operand maps of a kernel that loads Z k-tiles per stage.
+bool make_maps(CUtensorMap* ma, CUtensorMap* mb, const GemmArgs& g, const void* a, const void* b,
+               int arows, int brows, int z) {
+    if (z == 1) return make_map(ma, a, g.M, g.K, arows) && make_map(mb, b, g.N, g.K, brows);
+    return make_map3(ma, a, g.M, g.K, arows, z) && make_map3(mb, b, g.N, g.K, brows, z);
+}
+
+template <int BN, int AROWS, int Z>
 cudaError_t launch_bn(const GemmArgs& g, const void* a, const void* b, int sm_count,
                       cudaStream_t stream) {
-    using T = Tile<BN, AROWS>;
+    using T = Tile<BN, AROWS, Z>;
     CUtensorMap ma, mb;
-    if (!make_map(&ma, a, g.M, g.K, AROWS) || !make_map(&mb, b, g.N, g.K, BN))
-        return cudaErrorInvalidValue;
-    auto kernel = scaled_mm_kernel<BN, AROWS>;
+    if (!make_maps(&ma, &mb, g, a, b, AROWS, BN, Z)) return cudaErrorInvalidValue;
+    auto kernel = scaled_mm_kernel<BN, AROWS, Z>;
     // the dynamic shared memory above 48 KB is enabled once per device
     static std::atomic<uint64_t> enabled_on{0};
     int dev = 0;
@@ -1201,14 +1287,13 @@ cudaError_t launch_pair(const GemmArgs& g, const void* a, const void* b, int sm_
     return cudaLaunchKernelEx(&cfg, scaled_mm_pair_kernel, ma, mb, g);
 }
 
-template <int BN, int AROWS>
+template <int BN, int AROWS, int Z>
 cudaError_t launch_mx(const GemmArgs& g, const void* a, const void* b, const uint8_t* sfa,
                       const uint8_t* sfb, int sm_count, cudaStream_t stream) {
-    using T = MxTile<BN, AROWS>;
+    using T = MxTile<BN, AROWS, Z>;
     CUtensorMap ma, mb;
-    if (!make_map(&ma, a, g.M, g.K, AROWS) || !make_map(&mb, b, g.N, g.K, BN))
-        return cudaErrorInvalidValue;
-    auto kernel = scaled_mm_mx_kernel<BN, AROWS>;
+    if (!make_maps(&ma, &mb, g, a, b, AROWS, BN, Z)) return cudaErrorInvalidValue;
+    auto kernel = scaled_mm_mx_kernel<BN, AROWS, Z>;
     static std::atomic<uint64_t> enabled_on{0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -1273,9 +1358,13 @@ cudaError_t launch_scaled_mm_mx(const GemmArgs& g, const void* a, const void* b,
     // else one CTA per 128 x 128 tile once those fill every SM; short, wide
     // problems take 128 x 64 tiles (64-row A stages for at most 64 rows)
     if (((g.M + kBM - 1) / kBM) * ((g.N + 127) / 128) >= sm_count)
-        return launch_mx<128, kBM>(g, a, b, sfa, sfb, sm_count, stream);
-    if (g.M <= 64) return launch_mx<64, 64>(g, a, b, sfa, sfb, sm_count, stream);
-    return launch_mx<64, kBM>(g, a, b, sfa, sfb, sm_count, stream);
+        return launch_mx<128, kBM, 1>(g, a, b, sfa, sfb, sm_count, stream);
+    // (K % 128 == 0 here: several k-tiles per TMA box, as the per-token GEMM)
+    if (g.M <= 8) return launch_mx<64, 8, 4>(g, a, b, sfa, sfb, sm_count, stream);
+    if (g.M <= 16) return launch_mx<64, 16, 4>(g, a, b, sfa, sfb, sm_count, stream);
+    if (g.M <= 32) return launch_mx<64, 32, 4>(g, a, b, sfa, sfb, sm_count, stream);
+    if (g.M <= 64) return launch_mx<64, 64, 4>(g, a, b, sfa, sfb, sm_count, stream);
+    return launch_mx<64, kBM, 2>(g, a, b, sfa, sfb, sm_count, stream);
 }
 
 cudaError_t launch_scaled_mm(const GemmArgs& g, const void* a, const void* b, int sm_count,
@@ -1288,11 +1377,19 @@ cudaError_t launch_scaled_mm(const GemmArgs& g, const void* a, const void* b, in
     if (((g.M + 255) / 256) * ((g.N + 255) / 256) >= sm_count / 2)
         return launch_pair(g, a, b, sm_count, stream);
     if (row_tiles * ((g.N + 255) / 256) >= sm_count)
-        return launch_bn<256, kBM>(g, a, b, sm_count, stream);
+        return launch_bn<256, kBM, 1>(g, a, b, sm_count, stream);
     if (row_tiles * ((g.N + 127) / 128) >= sm_count)
-        return launch_bn<128, kBM>(g, a, b, sm_count, stream);
-    if (g.M <= 64) return launch_bn<64, 64>(g, a, b, sm_count, stream);
-    return launch_bn<64, kBM>(g, a, b, sm_count, stream);
+        return launch_bn<128, kBM, 1>(g, a, b, sm_count, stream);
+    // the weight-streaming shapes: several k-tiles per TMA box where K allows
+    const bool atoms = g.K % kBK == 0;
+    if (g.M <= 64 && !atoms) return launch_bn<64, 64, 1>(g, a, b, sm_count, stream);
+    // A stages of the fewest rows that hold the call's rows
+    if (g.M <= 8) return launch_bn<64, 8, 4>(g, a, b, sm_count, stream);
+    if (g.M <= 16) return launch_bn<64, 16, 4>(g, a, b, sm_count, stream);
+    if (g.M <= 32) return launch_bn<64, 32, 4>(g, a, b, sm_count, stream);
+    if (g.M <= 64) return launch_bn<64, 64, 4>(g, a, b, sm_count, stream);
+    return atoms ? launch_bn<64, kBM, 2>(g, a, b, sm_count, stream)
+                 : launch_bn<64, kBM, 1>(g, a, b, sm_count, stream);
 }
 
 }  // namespace rrf
