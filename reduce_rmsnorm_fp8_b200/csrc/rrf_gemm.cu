@@ -403,6 +403,190 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// ------------------------------------- short products: the operands swapped --
+// A call of at most 64 rows against a weight (a decode batch): the weight's
+// rows are the MMA's M side and the call's rows its N side, so the tensor
+// cores do 64 x NA x 32 per instruction (NA = the rows rounded up to 8, 16,
+// 32) instead of 128 x 64 x 32 with most rows empty.  A CTA streams a
+// 64-row weight tile (Z k-tiles per 3-D TMA box) against the call's rows
+// (an L2-resident box of NA rows per stage).  The accumulator
+// D[n][m] = out[m][n] lives in the M = 64 layout of tensor memory: weight
+// row 16 q + i in lane 32 q + i (q < 4, i < 16), row m of the call in
+// column m.
+
+// Instruction descriptor of kind::f8f6f4 with M = 64, N = na.
+__host__ __device__ constexpr uint32_t f8_idesc_m64(int na) {
+    return (1u << 4) | ((uint32_t)(na >> 3) << 17) | ((uint32_t)(64 >> 4) << 24);
+}
+
+template <int NA, int Z>
+struct SwapTile {
+    static_assert(NA % 8 == 0 && NA >= 8 && NA <= 64, "the call's rows: 8 .. 64 in steps of 8");
+    static constexpr int kWRows = 64;                  // weight rows per tile (the MMA's M)
+    static constexpr int kWBytes = kWRows * kBK;       // one k-tile of the weight: 8 KB
+    static constexpr int kXBytes = NA * kBK;           // one k-tile of the call's rows
+    static constexpr int kXOffset = Z * kWBytes;
+    static constexpr int kStageBytes = Z * (kWBytes + kXBytes);
+    static constexpr int kStages =
+        (220 * 1024) / kStageBytes > 12 ? 12 : (220 * 1024) / kStageBytes;
+    // two accumulators of NA columns, each at least 32 wide (the epilogue
+    // reads 32 columns at a time); a power of two of at least 32
+    static constexpr int kAccStride = NA < 32 ? 32 : NA;
+    static constexpr int kTmemCols = 2 * kAccStride;
+    static constexpr int kBarriers = 2 * kStages + 4 + 1;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarriers * 8 + 16;
+    static_assert(kSmemBytes <= 227 * 1024, "stages exceed the shared memory of a CTA");
+    static_assert(kXBytes % 1024 == 0, "each k-tile must start on a swizzle atom");
+};
+
+template <int NA, int Z>
+__global__ void __launch_bounds__(kThreads, 1)
+    scaled_mm_swap_kernel(const __grid_constant__ CUtensorMap tma_x,
+                          const __grid_constant__ CUtensorMap tma_w, const GemmArgs g) {
+    using T = SwapTile<NA, Z>;
+    constexpr int S = T::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(ring + S * T::kStageBytes);
+    uint64_t* empty = full + S;
+    uint64_t* acc_full = empty + S;
+    uint64_t* acc_empty = acc_full + 2;
+    uint64_t* drained = acc_empty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tiles = (g.N + T::kWRows - 1) / T::kWRows;
+    const int ktiles = g.K / kBK;  // K is a multiple of 128
+    const int kgroups = (ktiles + Z - 1) / Z;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 4);
+        }
+        mbar_init(drained, 1);
+        fence_mbar_init_cluster();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, T::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---- producer: Z k-tiles of the weight tile and of the call's rows
+        if (lane == 0) {
+            int it = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+                const int n0 = t * T::kWRows;
+                for (int kg = 0; kg < kgroups; ++kg, ++it) {
+                    const int s = it % S;
+                    if (!wait_phase(&empty[s], ((it / S) & 1) ^ 1, g.err)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* dst = ring + s * T::kStageBytes;
+                    mbar_arrive_expect_tx(&full[s], T::kStageBytes);
+                    tma_load_3d(dst, &tma_w, &full[s], 0, n0, kg * Z);
+                    tma_load_3d(dst + T::kXOffset, &tma_x, &full[s], 0, 0, kg * Z);
+                }
+            }
+            for (int i = it > S ? it - S : 0; i < it; ++i)
+                wait_phase(&full[i % S], (i / S) & 1, g.err);
+        }
+    } else if (warp == 1) {
+        // ---- MMA issue: D[64 x NA] += W[64 x 32] * X[NA x 32]^T
+        if (lane == 0) {
+            constexpr uint32_t idesc = f8_idesc_m64(NA);
+            int it = 0, j = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++j) {
+                const int buf = j & 1;
+                if (!wait_phase(&acc_empty[buf], ((j >> 1) & 1) ^ 1, g.err)) break;
+                tc_fence_after_sync();
+                const uint32_t d = tmem + (uint32_t)(buf * T::kAccStride);
+                for (int kg = 0; kg < kgroups; ++kg, ++it) {
+                    const int s = it % S;
+                    if (!wait_phase(&full[s], (it / S) & 1, g.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint8_t* stage = ring + s * T::kStageBytes;
+                    const int nk = ktiles - kg * Z < Z ? ktiles - kg * Z : Z;
+                    for (int kj = 0; kj < nk; ++kj) {
+                        const uint64_t wd = kmajor_sw128_desc(stage + kj * T::kWBytes);
+                        const uint64_t xd = kmajor_sw128_desc(stage + T::kXOffset + kj * T::kXBytes);
+#pragma unroll
+                        for (int k = 0; k < kBK / kMmaK; ++k) {
+                            const uint64_t step = (uint64_t)(k * kMmaK) >> 4;
+                            mma_f8(d, wd + step, xd + step, idesc, (kg | kj | k) != 0);
+                        }
+                    }
+                    mma_commit(&empty[s]);
+                }
+                mma_commit(&acc_full[buf]);
+            }
+            mma_commit(drained);
+        }
+        __syncwarp();
+    } else {
+        // ---- epilogue: lanes 0-15 of each warp hold 16 weight rows (output
+        // columns); column m of tensor memory is row m of the call
+        const int quarter = warp & 3;
+        int j = 0;
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
+            const int buf = j & 1;
+            const int n = t * T::kWRows + quarter * 16 + (lane & 15);
+            bool have = wait_phase(&acc_full[buf], (j >> 1) & 1, g.err);
+            if (!__all_sync(0xFFFFFFFFu, have)) break;
+            tc_fence_after_sync();
+            const bool mine = lane < 16 && n < g.N;
+            const float sb = mine ? g.b_scale[n] : 0.0f;
+            const float bias =
+                mine && g.bias != nullptr ? __uint_as_float((uint32_t)g.bias[n] << 16) : 0.0f;
+            const uint32_t base =
+                tmem + (uint32_t)(buf * T::kAccStride) + ((uint32_t)(quarter * 32) << 16);
+#pragma unroll
+            for (int c = 0; c < NA; c += 32) {
+                float v[32];
+                tmem_load_32(base + (uint32_t)c, v);
+                if (!mine) continue;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int m = c + i;
+                    if (m < NA && m < g.M) {
+                        float y = __fmul_rn(__fmul_rn(v[i], __ldg(g.a_scale + m)), sb);
+                        if (g.bias != nullptr) y = __fadd_rn(y, bias);
+                        // one rounding to bf16 (the low half of the packed pair)
+                        g.out[(int64_t)m * g.N + n] = (uint16_t)(f32x2_to_bf16x2(y, 0.0f) & 0xFFFFu);
+                    }
+                }
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        wait_phase(drained, 0, g.err);
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, T::kTmemCols);
+    }
+}
+
 // ------------------------------------------------- two-CTA (pair) kernel --
 // A cluster of two CTAs on neighbouring SMs computes a 256 x 256 tile with
 // tcgen05.mma.cta_group::2 (M = 256, N = 256): each CTA loads 128 rows of A
@@ -1253,6 +1437,31 @@ cudaError_t launch_bn(const GemmArgs& g, const void* a, const void* b, int sm_co
     return cudaGetLastError();
 }
 
+template <int NA, int Z>
+cudaError_t launch_swap(const GemmArgs& g, const void* a, const void* b, int sm_count,
+                        cudaStream_t stream) {
+    using T = SwapTile<NA, Z>;
+    CUtensorMap mx, mw;
+    if (!make_map3(&mx, a, g.M, g.K, NA, Z) || !make_map3(&mw, b, g.N, g.K, T::kWRows, Z))
+        return cudaErrorInvalidValue;
+    auto kernel = scaled_mm_swap_kernel<NA, Z>;
+    static std::atomic<uint64_t> enabled_on{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
+    if (bit == 0 || (enabled_on.load(std::memory_order_relaxed) & bit) == 0) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 T::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        enabled_on.fetch_or(bit, std::memory_order_relaxed);
+    }
+    const int64_t tiles = (g.N + T::kWRows - 1) / T::kWRows;
+    const unsigned grid = (unsigned)(tiles < sm_count ? tiles : sm_count);
+    kernel<<<grid, kThreads, T::kSmemBytes, stream>>>(mx, mw, g);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_pair(const GemmArgs& g, const void* a, const void* b, int sm_count,
                         cudaStream_t stream) {
     using T = PairTile;
@@ -1383,10 +1592,11 @@ cudaError_t launch_scaled_mm(const GemmArgs& g, const void* a, const void* b, in
     // the weight-streaming shapes: several k-tiles per TMA box where K allows
     const bool atoms = g.K % kBK == 0;
     if (g.M <= 64 && !atoms) return launch_bn<64, 64, 1>(g, a, b, sm_count, stream);
-    // A stages of the fewest rows that hold the call's rows
-    if (g.M <= 8) return launch_bn<64, 8, 4>(g, a, b, sm_count, stream);
-    if (g.M <= 16) return launch_bn<64, 16, 4>(g, a, b, sm_count, stream);
-    if (g.M <= 32) return launch_bn<64, 32, 4>(g, a, b, sm_count, stream);
+    // at most 32 rows: the operands swapped, the call's rows padded to 8, 16
+    // or 32 (at 64 the swapped MMA is no cheaper: measured slower)
+    if (g.M <= 8) return launch_swap<8, 4>(g, a, b, sm_count, stream);
+    if (g.M <= 16) return launch_swap<16, 4>(g, a, b, sm_count, stream);
+    if (g.M <= 32) return launch_swap<32, 4>(g, a, b, sm_count, stream);
     if (g.M <= 64) return launch_bn<64, 64, 4>(g, a, b, sm_count, stream);
     return atoms ? launch_bn<64, kBM, 2>(g, a, b, sm_count, stream)
                  : launch_bn<64, kBM, 1>(g, a, b, sm_count, stream);

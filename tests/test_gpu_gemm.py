@@ -56,7 +56,8 @@ def check(c, got, rows=None, label=""):
     return worst
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 256, 128), (37, 256, 256), (128, 128, 128),
+@pytest.mark.parametrize("M,N,K", [(1, 256, 128), (9, 512, 640), (24, 336, 1536),
+                                   (5, 256, 144), (37, 256, 256), (128, 128, 128),
                                    (200, 272, 384), (130, 400, 144), (64, 1024, 1024),
                                    (256, 512, 2048)])
 @pytest.mark.parametrize("bias", [True, False])
@@ -76,7 +77,7 @@ def test_wide_tiles_sampled_rows(rrf):
     check(c, out, rows=[0, 1, 127, 128, 255, 1000, 1919, 1920, 1999], label="wide")
 
 
-@pytest.mark.parametrize("M", [1, 8, 32, 64])
+@pytest.mark.parametrize("M", [1, 8, 16, 32, 64])
 def test_decode_projection_sampled_rows(rrf, M):
     N = K = 7168
     c = workloads.make_gemm_case(M, N, K, sub=M, device="cuda")
