@@ -1593,9 +1593,10 @@ cudaError_t launch_scaled_mm(const GemmArgs& g, const void* a, const void* b, in
     const bool atoms = g.K % kBK == 0;
     if (g.M <= 64 && !atoms) return launch_bn<64, 64, 1>(g, a, b, sm_count, stream);
     // at most 32 rows: the operands swapped, the call's rows padded to 8, 16
-    // or 32 (at 64 the swapped MMA is no cheaper: measured slower)
-    if (g.M <= 8) return launch_swap<8, 4>(g, a, b, sm_count, stream);
-    if (g.M <= 16) return launch_swap<16, 4>(g, a, b, sm_count, stream);
+    // or 32 (at 64 the swapped MMA is no cheaper: measured slower); 8 k-tiles
+    // per box up to 16 rows (measured faster than 4 or 2 there; equal at 32)
+    if (g.M <= 8) return launch_swap<8, 8>(g, a, b, sm_count, stream);
+    if (g.M <= 16) return launch_swap<16, 8>(g, a, b, sm_count, stream);
     if (g.M <= 32) return launch_swap<32, 4>(g, a, b, sm_count, stream);
     if (g.M <= 64) return launch_bn<64, 64, 4>(g, a, b, sm_count, stream);
     return atoms ? launch_bn<64, kBM, 2>(g, a, b, sm_count, stream)
