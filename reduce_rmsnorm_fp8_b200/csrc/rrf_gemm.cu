@@ -1568,7 +1568,8 @@ cudaError_t launch_scaled_mm_mx(const GemmArgs& g, const void* a, const void* b,
     // problems take 128 x 64 tiles (64-row A stages for at most 64 rows)
     if (((g.M + kBM - 1) / kBM) * ((g.N + 127) / 128) >= sm_count)
         return launch_mx<128, kBM, 1>(g, a, b, sfa, sfb, sm_count, stream);
-    // (K % 128 == 0 here: several k-tiles per TMA box, as the per-token GEMM)
+    // (K % 128 == 0 here: several k-tiles per TMA box, as the per-token GEMM;
+    // no swapped operands: the block-scaled MMA of one CTA has no M = 64 form)
     if (g.M <= 8) return launch_mx<64, 8, 4>(g, a, b, sfa, sfb, sm_count, stream);
     if (g.M <= 16) return launch_mx<64, 16, 4>(g, a, b, sfa, sfb, sm_count, stream);
     if (g.M <= 32) return launch_mx<64, 32, 4>(g, a, b, sfa, sfb, sm_count, stream);

@@ -137,7 +137,8 @@ def check_mx_gemm(c, sa, sb, got, rows=None, label=""):
     assert worst <= 1.0, f"{label}: beyond the bound (ratio {worst:.3g})"
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 128, 128), (37, 256, 256), (128, 128, 512),
+@pytest.mark.parametrize("M,N,K", [(1, 128, 128), (8, 384, 512), (13, 320, 1024),
+                                   (32, 448, 640), (37, 256, 256), (128, 128, 512),
                                    (200, 272, 384), (130, 400, 1024), (256, 512, 2048)])
 @pytest.mark.parametrize("bias", [True, False])
 def test_mx_gemm_matches_oracle(rrf, M, N, K, bias):
@@ -163,7 +164,8 @@ def test_mx_gemm_pair_tiles_with_tails(rrf, bias):
     assert rrf.rrf_device_error() == 0
 
 
-@pytest.mark.parametrize("M,N,K", [(64, 7168, 7168), (2000, 2560, 1024), (8192, 8192, 8192)])
+@pytest.mark.parametrize("M,N,K", [(8, 7168, 7168), (64, 7168, 7168), (2000, 2560, 1024),
+                                   (8192, 8192, 8192)])
 def test_mx_gemm_large_sampled_rows(rrf, M, N, K):
     c, sa, sb = mx_operands(M, N, K, 7)
     out = rrf.rrf_scaled_mm_mxfp8(c.a, rrf.mx_blocked(torch.from_numpy(sa).cuda()), c.b,
