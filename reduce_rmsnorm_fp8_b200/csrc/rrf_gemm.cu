@@ -4,8 +4,15 @@
 // aclnnAlltoAllQuantMatmul: per-token dynamic quantisation of the
 // activations, then (x1_q @ x2) * x1Scale * x2Scale + bias).
 //
+// Kernels (launch_scaled_mm and launch_scaled_mm_mx choose by shape):
+//   scaled_mm_pair_kernel / scaled_mm_mx_pair_kernel  256 x 256 tiles on SM
+//            pairs (tcgen05.mma.cta_group::2) for products that fill every pair;
+//   scaled_mm_kernel / scaled_mm_mx_kernel  persistent CTAs on 128 x BN tiles
+//            (BN 256, 128 or 64), Z k-tiles per TMA box for short products;
+//   scaled_mm_swap_kernel  at most 32 rows against a weight, the operands
+//            swapped (the weight's rows on the MMA's M = 64 side).
 // A persistent CTA per SM walks 128 x BN tiles of out (BN 256, 128 or 64).
-// Warp roles:
+// Warp roles (the same in every kernel):
 //   warp 0   one thread issues the TMA loads of the A (128 x 128 bytes) and
 //            B (BN x 128 bytes) k-tiles into a ring of shared-memory stages
 //            (128-byte swizzle, the layout the MMA descriptors name);
