@@ -76,7 +76,7 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, unsig
 // ---------------------------------------------------------------------- TMA --
 
 // 2-D tiled load of box {x, y} at coordinates (x, y) into shared memory,
-// completing `bytes` on `bar` (no multicast).
+// completing `bytes` on `bar` (this CTA's shared memory only).
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int x, int y) {
     asm volatile(
@@ -237,7 +237,7 @@ struct Tile {
 };
 
 // 3-D tiled load of box {x, y, z} at coordinates (x, y, z), completing on
-// `bar` (no multicast).
+// `bar` (this CTA's shared memory only).
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int x, int y, int z) {
     asm volatile(
@@ -857,7 +857,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // each), and the k-tile's four MMAs take code (k-step) of each 32-bit word.
 
 // 1-D bulk copy of `bytes` (a multiple of 16, both addresses 16-byte
-// aligned) into shared memory, completing on `bar` (no multicast).
+// aligned) into this CTA's shared memory, completing on `bar`.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
                                           uint64_t* bar) {
     asm volatile(
