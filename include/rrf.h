@@ -515,6 +515,16 @@ int rrf_last_cuda_error(void);
  * the RRF_ERR_CUDA path can be tested without making a GPU fail. */
 void rrf_debug_fail_next_launch(int cuda_error);
 
+/* Test hook for the GEMMs' bounded waits: the next rrf_scaled_mm_fp8 or
+ * rrf_scaled_mm_mxfp8 call on this host thread launches normally, but its
+ * epilogue, after each accumulator it drains, also waits for that
+ * accumulator's next completion, which cannot come before the epilogue
+ * releases it.  The wait runs out (100 ms), the kernel sets
+ * RRF_DEVICE_ERROR_GEMM_TIMEOUT in the device error word and finishes; the
+ * output of that call is incomplete.  So the failure path is tested without
+ * making a GPU fault or hang. */
+void rrf_debug_starve_next_gemm(void);
+
 /* Library version, "major.minor.patch". */
 const char* rrf_version(void);
 

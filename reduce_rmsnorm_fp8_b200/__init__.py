@@ -30,7 +30,7 @@ _EXPORTS = (
     "RRF_VARIANT_ROW", "RRF_FLAG_NO_PDL", "RRF_FLAG_BARRIER_EXCHANGE",
     "RRF_FLAG_DEBUG_STARVE_EXCHANGE", "RRF_DEVICE_ERROR_EXCHANGE_TIMEOUT", "RrfError",
     "Status", "lib", "rrf_check_fused_args", "rrf_check_sum_args",
-    "rrf_debug_fail_next_launch", "rrf_device_error", "rrf_last_cuda_error", "rrf_plan_fused",
+    "rrf_debug_fail_next_launch", "rrf_debug_starve_next_gemm", "rrf_device_error", "rrf_last_cuda_error", "rrf_plan_fused",
     "rrf_status_string", "rrf_sum", "rrf_sum_ptr", "rrf_sum_rmsnorm_fp8",
     "rrf_sum_rmsnorm_fp8_ex", "rrf_sum_rmsnorm_fp8_ptr", "rrf_version", "RRF_MAX_SHARDS",
     "rrf_sum_rmsnorm_fp8_pre", "rrf_rmsnorm_fp8_post", "rrf_check_pre_args",

@@ -85,6 +85,8 @@ lib.rrf_last_cuda_error.restype = _int
 lib.rrf_last_cuda_error.argtypes = []
 lib.rrf_debug_fail_next_launch.restype = None
 lib.rrf_debug_fail_next_launch.argtypes = [_int]
+lib.rrf_debug_starve_next_gemm.restype = None
+lib.rrf_debug_starve_next_gemm.argtypes = []
 lib.rrf_sum_rmsnorm_fp8_pre.restype = _int
 lib.rrf_sum_rmsnorm_fp8_pre.argtypes = [_ptrs, _int, _i64, _i64, _vp, _vp, _vp, _vp, _f32, _vp,
                                         _vp]
@@ -136,6 +138,12 @@ def rrf_last_cuda_error() -> int:
 
 def rrf_debug_fail_next_launch(cuda_error: int) -> None:
     lib.rrf_debug_fail_next_launch(int(cuda_error))
+
+
+def rrf_debug_starve_next_gemm() -> None:
+    """The next GEMM call on this thread runs its epilogue's bounded wait
+    out (test hook; see include/rrf.h)."""
+    lib.rrf_debug_starve_next_gemm()
 
 
 def rrf_device_error(clear: bool = False) -> int:

@@ -17,6 +17,7 @@ namespace {
 
 thread_local int t_last_cuda_error = 0;
 thread_local int t_fail_next_launch = 0;
+thread_local bool t_starve_next_gemm = false;
 
 // The library's device error word: kernels set bits in it (a wait that ran
 // out); rrf_device_error reads and clears it.  Static device memory, one per
@@ -79,6 +80,12 @@ bool take_injected_failure(cudaError_t* e) {
     *e = (cudaError_t)t_fail_next_launch;
     t_fail_next_launch = 0;
     return true;
+}
+
+int take_starve_gemm() {
+    const bool s = t_starve_next_gemm;
+    t_starve_next_gemm = false;
+    return s ? 1 : 0;
 }
 
 bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
@@ -868,6 +875,7 @@ extern "C" rrf_status rrf_scaled_mm_fp8(const void* a, const float* a_scale, con
     g.N = (int)N;
     g.K = (int)K;
     g.err = err;
+    g.starve = take_starve_gemm();
     cudaError_t e;
     if (!take_injected_failure(&e)) e = launch_scaled_mm(g, a, b, sm_count, (cudaStream_t)stream);
     return e == cudaSuccess ? RRF_OK : cuda_fail(e);
@@ -911,6 +919,7 @@ extern "C" rrf_status rrf_scaled_mm_mxfp8(const void* a, const void* sa, const v
     g.N = (int)N;
     g.K = (int)K;
     g.err = err;
+    g.starve = take_starve_gemm();
     cudaError_t e;
     if (!take_injected_failure(&e))
         e = launch_scaled_mm_mx(g, a, b, static_cast<const uint8_t*>(sa),
@@ -961,5 +970,7 @@ extern "C" rrf_status rrf_device_error(unsigned int* flags, int clear) {
 }
 
 extern "C" void rrf_debug_fail_next_launch(int cuda_error) { t_fail_next_launch = cuda_error; }
+
+extern "C" void rrf_debug_starve_next_gemm(void) { t_starve_next_gemm = true; }
 
 extern "C" const char* rrf_version(void) { return "0.1.0"; }

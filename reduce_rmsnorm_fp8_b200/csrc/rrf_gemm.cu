@@ -73,6 +73,16 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, unsig
     return true;
 }
 
+// The epilogue's wait for its accumulator (phase `parity` of `bar`).  Under
+// the test hook (g.starve) it then also waits for the accumulator's next
+// completion, which cannot come before this epilogue releases it: the
+// bounded wait runs out and reports RRF_DEVICE_ERROR_GEMM_TIMEOUT, so the
+// failure path runs on a GPU without a fault or a hang.
+__device__ __forceinline__ bool epilogue_wait(uint64_t* bar, uint32_t parity, const GemmArgs& g) {
+    if (!wait_phase(bar, parity, g.err)) return false;
+    return g.starve == 0 || wait_phase(bar, parity ^ 1u, g.err);
+}
+
 // ---------------------------------------------------------------------- TMA --
 
 // 2-D tiled load of box {x, y} at coordinates (x, y) into shared memory,
@@ -380,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
             const int buf = j & 1;
             const int m0 = (t / tiles_n) * kBM, n0 = (t % tiles_n) * BN;
-            bool have = wait_phase(&acc_full[buf], (j >> 1) & 1, g.err);
+            bool have = epilogue_wait(&acc_full[buf], (j >> 1) & 1, g);
             if (!__all_sync(0xFFFFFFFFu, have)) break;
             tc_fence_after_sync();
             const int row = m0 + quarter * 32 + lane;
@@ -554,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
             const int buf = j & 1;
             const int n = t * T::kWRows + quarter * 16 + (lane & 15);
-            bool have = wait_phase(&acc_full[buf], (j >> 1) & 1, g.err);
+            bool have = epilogue_wait(&acc_full[buf], (j >> 1) & 1, g);
             if (!__all_sync(0xFFFFFFFFu, have)) break;
             tc_fence_after_sync();
             const bool mine = lane < 16 && n < g.N;
@@ -815,7 +825,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int tm, tn;
             grouped_tile(t, tiles_m, tiles_n, tm, tn);
             const int m0 = tm * 256 + (int)rank * 128, n0 = tn * 256;
-            bool have = wait_phase(&acc_full[buf], (j >> 1) & 1, g.err);
+            bool have = epilogue_wait(&acc_full[buf], (j >> 1) & 1, g);
             if (!__all_sync(0xFFFFFFFFu, have)) break;
             tc_fence_after_sync();
             const int row = m0 + quarter * 32 + lane;
@@ -1066,7 +1076,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
             const int buf = j & 1;
             const int m0 = (t / tiles_n) * kBM, n0 = (t % tiles_n) * BN;
-            bool have = wait_phase(&acc_full[buf], (j >> 1) & 1, g.err);
+            bool have = epilogue_wait(&acc_full[buf], (j >> 1) & 1, g);
             if (!__all_sync(0xFFFFFFFFu, have)) break;
             tc_fence_after_sync();
             const int row = m0 + quarter * 32 + lane;
@@ -1303,7 +1313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int tm, tn;
             grouped_tile(t, tiles_m, tiles_n, tm, tn);
             const int m0 = tm * 256 + (int)rank * 128, n0 = tn * 256;
-            bool have = wait_phase(&acc_full[buf], (j >> 1) & 1, g.err);
+            bool have = epilogue_wait(&acc_full[buf], (j >> 1) & 1, g);
             if (!__all_sync(0xFFFFFFFFu, have)) break;
             tc_fence_after_sync();
             const int row = m0 + quarter * 32 + lane;

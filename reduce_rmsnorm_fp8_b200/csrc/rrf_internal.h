@@ -114,6 +114,7 @@ struct GemmArgs {
     uint16_t* out;         // bf16 [M, N]
     int M, N, K;
     unsigned int* err;
+    int starve;            // test hook: the epilogue's extra wait runs out
 };
 
 struct FusedLaunch {

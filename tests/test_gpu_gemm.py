@@ -116,3 +116,35 @@ def test_deterministic_and_empty(rrf):
     out = rrf.rrf_scaled_mm_fp8(e.a, e.a_scale, e.b, e.b_scale, e.bias)
     assert out.shape == (0, 256)
     assert rrf.rrf_device_error() == 0
+
+
+@pytest.mark.parametrize("M,N,K,mx", [(96, 512, 512, False), (8, 1024, 1024, False),
+                                      (2048, 2048, 512, False), (4096, 4096, 512, False),
+                                      (96, 512, 512, True), (4096, 4096, 512, True)])
+def test_wait_timeout_is_reported(rrf, M, N, K, mx):
+    """The test hook makes the epilogue's bounded wait run out (one CTA's
+    tile, several tiles per CTA, SM pairs; per-token and MX): the call
+    finishes, reports RRF_DEVICE_ERROR_GEMM_TIMEOUT, and the next call on the
+    same operands matches the oracle."""
+    import test_gpu_mx
+    rrf.rrf_device_error(clear=True)
+    if mx:
+        c, sa, sb = test_gpu_mx.mx_operands(M, N, K, 6)
+        args = (c.a, rrf.mx_blocked(torch.from_numpy(sa).cuda()), c.b,
+                rrf.mx_blocked(torch.from_numpy(sb).cuda()), c.bias)
+        call = lambda: rrf.rrf_scaled_mm_mxfp8(*args)
+    else:
+        c = workloads.make_gemm_case(M, N, K, sub=6, device="cuda")
+        call = lambda: rrf.rrf_scaled_mm_fp8(c.a, c.a_scale, c.b, c.b_scale, c.bias)
+    rrf.rrf_debug_starve_next_gemm()
+    call()
+    torch.cuda.synchronize()
+    assert rrf.rrf_device_error(clear=True) & rrf.RRF_DEVICE_ERROR_GEMM_TIMEOUT
+    out = call()
+    torch.cuda.synchronize()
+    assert rrf.rrf_device_error() == 0
+    rows = [0, M // 2, M - 1]
+    if mx:
+        test_gpu_mx.check_mx_gemm(c, sa, sb, out, rows=rows, label="after the timeout")
+    else:
+        check(c, out, rows=rows, label="after the timeout")
