@@ -1587,8 +1587,10 @@ cudaError_t launch_scaled_mm_mx(const GemmArgs& g, const void* a, const void* b,
         return launch_mx<128, kBM, 1>(g, a, b, sfa, sfb, sm_count, stream);
     // (K % 128 == 0 here: several k-tiles per TMA box, as the per-token GEMM;
     // no swapped operands: the block-scaled MMA of one CTA has no M = 64 form)
-    if (g.M <= 8) return launch_mx<64, 8, 4>(g, a, b, sfa, sfb, sm_count, stream);
-    if (g.M <= 16) return launch_mx<64, 16, 4>(g, a, b, sfa, sfb, sm_count, stream);
+    // 8 k-tiles per stage up to 16 rows (2 stages; measured 7% faster than 4
+    // at 8 rows, 2 k-tiles slower)
+    if (g.M <= 8) return launch_mx<64, 8, 8>(g, a, b, sfa, sfb, sm_count, stream);
+    if (g.M <= 16) return launch_mx<64, 16, 8>(g, a, b, sfa, sfb, sm_count, stream);
     if (g.M <= 32) return launch_mx<64, 32, 4>(g, a, b, sfa, sfb, sm_count, stream);
     if (g.M <= 64) return launch_mx<64, 64, 4>(g, a, b, sfa, sfb, sm_count, stream);
     return launch_mx<64, kBM, 2>(g, a, b, sfa, sfb, sm_count, stream);
