@@ -731,12 +731,16 @@ def run_rrf(args):
         gi, _ = capture_steps(lambda k: cp.call(rrf, 3 + k, 0), reps, device)
         gi.replay()
         torch.cuda.synchronize(device)
-        tc = time_region(lambda _: gi.replay(), 1, device, stream)
+        # eleven timed replays: the median is the figure, p10/p90 its spread
+        tcs = sorted(time_region(lambda _: gi.replay(), 1, device, stream) for _ in range(11))
+        tc = tcs[5]
         del gi, cp
         b = workloads.fused_bytes(w.R, c.rows, c.cols, c.residual is not None)
         launch = rrf.rrf_plan_fused(w.R, c.rows, c.cols, props.multi_processor_count,
                                     residual=c.residual is not None)
         cases.append({"rows": c.rows, "us_per_call": round(tc / reps * 1e6, 3),
+                      "us_p10": round(tcs[1] / reps * 1e6, 3),
+                      "us_p90": round(tcs[9] / reps * 1e6, 3),
                       "GB_s": round(b * reps / tc / 1e9, 1),
                       "frac": round(b * reps / tc / 1e9 / peak, 4),
                       "rows_per_s": round(c.rows * reps / tc, 1),
