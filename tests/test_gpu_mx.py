@@ -149,13 +149,15 @@ def test_mx_gemm_matches_oracle(rrf, M, N, K, bias):
     check_mx_gemm(c, sa, sb, out, label=f"{M}x{N}x{K}")
 
 
-@pytest.mark.parametrize("bias", [True, False])
-def test_mx_gemm_pair_tiles_with_tails(rrf, bias):
+@pytest.mark.parametrize("M,N,K,bias", [(2200, 2320, 384, True), (2200, 2320, 384, False),
+                                        (2100, 2336, 256, True)])
+def test_mx_gemm_pair_tiles_with_tails(rrf, M, N, K, bias):
     """Enough 256 x 256 tiles for the SM-pair kernel (every pair takes two,
     so both accumulators and their shared columns are used), with a row tail
-    inside the odd CTA's half and a column tail that leaves the odd CTA's B
-    half and the second B scale atom past the operand; every output checked."""
-    M, N, K = 2200, 2320, 384
+    inside the odd CTA's half (2200) or inside the even CTA's half with the
+    odd CTA's rows and scale atom wholly past the operand (2100), and a
+    column tail that leaves the odd CTA's B half and the second B scale atom
+    past the operand; every output checked."""
     c, sa, sb = mx_operands(M, N, K, 4, bias)
     out = rrf.rrf_scaled_mm_mxfp8(c.a, rrf.mx_blocked(torch.from_numpy(sa).cuda()), c.b,
                                   rrf.mx_blocked(torch.from_numpy(sb).cuda()), c.bias)
