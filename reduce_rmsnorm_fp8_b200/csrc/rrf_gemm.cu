@@ -1373,6 +1373,40 @@ EncodeTiled encode_tiled() {
     return fn;
 }
 
+// Dynamic shared memory above 48 KB is enabled once per device for each
+// kernel (KERNEL: the kernel's address; its devices done in a bitmask).
+template <auto KERNEL>
+cudaError_t enable_dynamic_smem(int bytes) {
+    static std::atomic<uint64_t> enabled_on{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
+    if (bit != 0 && (enabled_on.load(std::memory_order_relaxed) & bit) != 0) return cudaSuccess;
+    e = cudaFuncSetAttribute(KERNEL, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) enabled_on.fetch_or(bit, std::memory_order_relaxed);
+    return e;
+}
+
+// A launch of `pairs` clusters of two CTAs, one SM pair each.
+template <class... Params, class... Args>
+cudaError_t launch_on_pairs(void (*kernel)(Params...), int64_t pairs, int smem_bytes,
+                            cudaStream_t stream, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem_bytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // A [rows, K] byte matrix, box of 128 bytes x box_rows rows, 128-byte swizzle;
 // rows and columns past the matrix read as zero.
 bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int box_rows) {
@@ -1435,19 +1469,9 @@ cudaError_t launch_bn(const GemmArgs& g, const void* a, const void* b, int sm_co
     using T = Tile<BN, AROWS, Z>;
     CUtensorMap ma, mb;
     if (!make_maps(&ma, &mb, g, a, b, AROWS, BN, Z)) return cudaErrorInvalidValue;
-    auto kernel = scaled_mm_kernel<BN, AROWS, Z>;
-    // the dynamic shared memory above 48 KB is enabled once per device
-    static std::atomic<uint64_t> enabled_on{0};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    constexpr auto kernel = scaled_mm_kernel<BN, AROWS, Z>;
+    const cudaError_t e = enable_dynamic_smem<kernel>(T::kSmemBytes);
     if (e != cudaSuccess) return e;
-    const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
-    if (bit == 0 || (enabled_on.load(std::memory_order_relaxed) & bit) == 0) {
-        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 T::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        enabled_on.fetch_or(bit, std::memory_order_relaxed);
-    }
     const int64_t tiles = (int64_t)((g.N + BN - 1) / BN) * ((g.M + kBM - 1) / kBM);
     const unsigned grid = (unsigned)(tiles < sm_count ? tiles : sm_count);  // one CTA per SM
     kernel<<<grid, kThreads, T::kSmemBytes, stream>>>(ma, mb, g);
@@ -1461,18 +1485,9 @@ cudaError_t launch_swap(const GemmArgs& g, const void* a, const void* b, int sm_
     CUtensorMap mx, mw;
     if (!make_map3(&mx, a, g.M, g.K, NA, Z) || !make_map3(&mw, b, g.N, g.K, T::kWRows, Z))
         return cudaErrorInvalidValue;
-    auto kernel = scaled_mm_swap_kernel<NA, Z>;
-    static std::atomic<uint64_t> enabled_on{0};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    constexpr auto kernel = scaled_mm_swap_kernel<NA, Z>;
+    const cudaError_t e = enable_dynamic_smem<kernel>(T::kSmemBytes);
     if (e != cudaSuccess) return e;
-    const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
-    if (bit == 0 || (enabled_on.load(std::memory_order_relaxed) & bit) == 0) {
-        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 T::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        enabled_on.fetch_or(bit, std::memory_order_relaxed);
-    }
     const int64_t tiles = (g.N + T::kWRows - 1) / T::kWRows;
     const unsigned grid = (unsigned)(tiles < sm_count ? tiles : sm_count);
     kernel<<<grid, kThreads, T::kSmemBytes, stream>>>(mx, mw, g);
@@ -1485,32 +1500,11 @@ cudaError_t launch_pair(const GemmArgs& g, const void* a, const void* b, int sm_
     CUtensorMap ma, mb;
     if (!make_map(&ma, a, g.M, g.K, 128) || !make_map(&mb, b, g.N, g.K, 128))
         return cudaErrorInvalidValue;
-    static std::atomic<uint64_t> enabled_on{0};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    const cudaError_t e = enable_dynamic_smem<scaled_mm_pair_kernel>(T::kSmemBytes);
     if (e != cudaSuccess) return e;
-    const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
-    if (bit == 0 || (enabled_on.load(std::memory_order_relaxed) & bit) == 0) {
-        e = cudaFuncSetAttribute(scaled_mm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 T::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        enabled_on.fetch_or(bit, std::memory_order_relaxed);
-    }
     const int64_t tiles = (int64_t)((g.N + 255) / 256) * ((g.M + 255) / 256);
     const int64_t pairs = tiles < sm_count / 2 ? tiles : sm_count / 2;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = T::kSmemBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, scaled_mm_pair_kernel, ma, mb, g);
+    return launch_on_pairs(scaled_mm_pair_kernel, pairs, T::kSmemBytes, stream, ma, mb, g);
 }
 
 template <int BN, int AROWS, int Z>
@@ -1519,18 +1513,9 @@ cudaError_t launch_mx(const GemmArgs& g, const void* a, const void* b, const uin
     using T = MxTile<BN, AROWS, Z>;
     CUtensorMap ma, mb;
     if (!make_maps(&ma, &mb, g, a, b, AROWS, BN, Z)) return cudaErrorInvalidValue;
-    auto kernel = scaled_mm_mx_kernel<BN, AROWS, Z>;
-    static std::atomic<uint64_t> enabled_on{0};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    constexpr auto kernel = scaled_mm_mx_kernel<BN, AROWS, Z>;
+    const cudaError_t e = enable_dynamic_smem<kernel>(T::kSmemBytes);
     if (e != cudaSuccess) return e;
-    const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
-    if (bit == 0 || (enabled_on.load(std::memory_order_relaxed) & bit) == 0) {
-        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 T::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        enabled_on.fetch_or(bit, std::memory_order_relaxed);
-    }
     const int64_t tiles = (int64_t)((g.N + BN - 1) / BN) * ((g.M + kBM - 1) / kBM);
     const unsigned grid = (unsigned)(tiles < sm_count ? tiles : sm_count);
     kernel<<<grid, kThreads, T::kSmemBytes, stream>>>(ma, mb, g, sfa, sfb);
@@ -1544,32 +1529,12 @@ cudaError_t launch_mx_pair(const GemmArgs& g, const void* a, const void* b, cons
     if (!make_map(&ma, a, g.M, g.K, 128) || !make_map(&mb, b, g.N, g.K, 128) ||
         !make_sf_map(&msa, sfa, g.M, g.K, 1) || !make_sf_map(&msb, sfb, g.N, g.K, 2))
         return cudaErrorInvalidValue;
-    static std::atomic<uint64_t> enabled_on{0};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    const cudaError_t e = enable_dynamic_smem<scaled_mm_mx_pair_kernel>(T::kSmemBytes);
     if (e != cudaSuccess) return e;
-    const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
-    if (bit == 0 || (enabled_on.load(std::memory_order_relaxed) & bit) == 0) {
-        e = cudaFuncSetAttribute(scaled_mm_mx_pair_kernel,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, T::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        enabled_on.fetch_or(bit, std::memory_order_relaxed);
-    }
     const int64_t tiles = (int64_t)((g.N + 255) / 256) * ((g.M + 255) / 256);
     const int64_t pairs = tiles < sm_count / 2 ? tiles : sm_count / 2;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = T::kSmemBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, scaled_mm_mx_pair_kernel, ma, mb, msa, msb, g);
+    return launch_on_pairs(scaled_mm_mx_pair_kernel, pairs, T::kSmemBytes, stream, ma, mb, msa,
+                           msb, g);
 }
 
 }  // namespace
