@@ -516,7 +516,8 @@ int rrf_last_cuda_error(void);
 void rrf_debug_fail_next_launch(int cuda_error);
 
 /* Test hook for the GEMMs' bounded waits: the next rrf_scaled_mm_fp8 or
- * rrf_scaled_mm_mxfp8 call on this host thread launches normally, but its
+ * rrf_scaled_mm_mxfp8 call on this host thread that launches (a call
+ * rejected on the host, or with M == 0, leaves the hook set) runs, but its
  * epilogue, after each accumulator it drains, also waits for that
  * accumulator's next completion, which cannot come before the epilogue
  * releases it.  The wait runs out (100 ms), the kernel sets
