@@ -436,3 +436,31 @@ def test_scaled_mm_mx_validation(rrf):
         kw = dict(ok)
         kw.update(change)
         assert rrf.rrf_check_scaled_mm_mx_args(**kw) == rrf.Status[status], change
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 128), (37, 256), (128, 512), (200, 384), (300, 1024)])
+def test_mx_blocked_layout_is_the_header_formula(rrf, rows, cols):
+    """The host helper that puts a weight's MX scale codes in the blocked
+    order, against the byte position include/rrf.h states, written out as a
+    plain loop; the size against RRF_MX_BLOCKED_BYTES."""
+    import numpy as np
+    import torch
+    rng = np.random.default_rng(rows * 7 + cols)
+    nb = cols // 32
+    codes = rng.integers(0, 256, (rows, nb)).astype(np.uint8)
+    got = rrf.mx_blocked(torch.from_numpy(codes)).numpy()
+    size = -(-rows // 128) * 128 * nb
+    assert got.size == size == rrf.mx_blocked_bytes(rows, cols)
+    want = np.zeros(size, dtype=np.uint8)
+    for r in range(rows):
+        for j in range(nb):
+            pos = ((r // 128) * (cols // 128) + j // 4) * 512 + (r % 32) * 16 + \
+                ((r // 32) % 4) * 4 + j % 4
+            want[pos] = codes[r, j]
+    assert np.array_equal(got, want)
+
+
+def test_mx_blocked_rejects_partial_atoms(rrf):
+    import torch
+    with pytest.raises(ValueError):
+        rrf.mx_blocked(torch.zeros((4, 6), dtype=torch.uint8))
