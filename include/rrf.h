@@ -404,6 +404,50 @@ rrf_status rrf_plan_allreduce(int world, int64_t rows, int64_t cols, int residua
                               int* block_threads, int* vecs_per_thread);
 
 /* ------------------------------------------------------------------------
+ * The multi-GPU form without any allocation by the caller.
+ *
+ * No page has a counterpart to this entry point; it is a library service.
+ * Some callers cannot allocate device memory: a program whose device memory
+ * is all owned by another allocator (a framework's caching pool that has
+ * reserved the GPU, where an outside cudaMalloc can fail or fragment the
+ * pool), code that must not call cudaMalloc / cudaFree because they may
+ * synchronise the whole device (a latency-bound serving loop), or a plug-in
+ * whose host forbids allocation after start-up.  Such a caller still owns
+ * and passes every input and output; the signal pads, the call's only
+ * scratch memory, come from a fixed array inside the library.
+ * ---------------------------------------------------------------------- */
+
+/* Ranks whose signal pads the library's fixed array holds:
+ * RRF_AR_STATIC_MAX_WORLD * RRF_AR_SIGNAL_WORDS 32-bit words (544 KiB),
+ * held on every GPU that loads the library until the process exits. */
+#define RRF_AR_STATIC_MAX_WORLD 8
+
+/* rrf_allreduce_rmsnorm_fp8_static -- rrf_allreduce_rmsnorm_fp8 with every
+ * rank in one launch on the current GPU (local_ranks == world, rank 0) and
+ * the signal pads taken from the library's fixed array: the call allocates
+ * no memory (no cudaMalloc, cudaFree or allocating library routine).
+ * Arguments, results and errors are those of rrf_allreduce_rmsnorm_fp8
+ * without `signals`, `rank` and `local_ranks`; every pointer entry is a
+ * buffer of this GPU.
+ * world    1..RRF_AR_STATIC_MAX_WORLD; a larger world is rejected with
+ *          RRF_ERR_RANKS before any CUDA call.
+ * Set-up: the first call on a device (with that device current) looks up
+ * the array's device address once and keeps it; make that first call
+ * before any stream capture.  Failing look-up: RRF_ERR_CUDA.
+ * Sharing: every call uses the same array, which keeps the last call's
+ * contents; each call zeroes the pads it uses, in stream order, before its
+ * kernel.  Calls that overlap on the GPU (on two streams, or from two host
+ * threads without ordering between their streams) race on the pads; order
+ * them on one stream or with events. */
+rrf_status rrf_allreduce_rmsnorm_fp8_static(const void* const* inputs,
+                                            const void* const* residual_in,
+                                            void* const* residual_out, void* const* q_out,
+                                            float* const* scales_out, int world, int64_t rows,
+                                            int64_t cols, const void* gamma, float eps,
+                                            float weight_offset, float scale_ub, int mode,
+                                            uint64_t timeout_ns, rrf_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * A consumer of the per-row scales: the FP8 GEMM that follows the
  * quantisation in a transformer layer.
  *

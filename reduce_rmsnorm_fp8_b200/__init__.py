@@ -40,6 +40,7 @@ _EXPORTS = (
     "rrf_allreduce_rmsnorm_fp8_ptr", "RRF_DEVICE_ERROR_GEMM_TIMEOUT", "rrf_scaled_mm_fp8",
     "rrf_check_scaled_mm_args", "rrf_sum_rmsnorm_mxfp8", "rrf_check_mxfp8_args",
     "mx_blocked", "mx_blocked_bytes", "rrf_scaled_mm_mxfp8", "rrf_check_scaled_mm_mx_args",
+    "RRF_AR_STATIC_MAX_WORLD", "rrf_allreduce_rmsnorm_fp8_static_ptr",
 )
 
 __all__ = list(_EXPORTS)

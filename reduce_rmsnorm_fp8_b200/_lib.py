@@ -22,6 +22,7 @@ RRF_DEVICE_ERROR_PEER_TIMEOUT = 2
 RRF_AR_MAX_WORLD = 8
 RRF_AR_MAX_BLOCKS = 1024
 RRF_AR_SIGNAL_WORDS = (2 * RRF_AR_MAX_WORLD + 1) * RRF_AR_MAX_BLOCKS
+RRF_AR_STATIC_MAX_WORLD = 8  # ranks whose pads the library's fixed array holds
 RRF_AR_AUTO = 0
 RRF_AR_ONE_SHOT = 1
 RRF_AR_TWO_SHOT = 2
@@ -102,6 +103,9 @@ _ar_args = [_ptrs, _ptrs, _ptrs, _ptrs, _ptrs, _ptrs, _int, _int, _int, _i64, _i
             _f32, _f32, _int]
 lib.rrf_allreduce_rmsnorm_fp8.restype = _int
 lib.rrf_allreduce_rmsnorm_fp8.argtypes = _ar_args + [ctypes.c_uint64, _vp]
+lib.rrf_allreduce_rmsnorm_fp8_static.restype = _int
+lib.rrf_allreduce_rmsnorm_fp8_static.argtypes = [_ptrs] * 5 + [_int, _i64, _i64, _vp, _f32, _f32,
+                                                               _f32, _int, ctypes.c_uint64, _vp]
 lib.rrf_check_allreduce_args.restype = _int
 lib.rrf_check_allreduce_args.argtypes = _ar_args
 lib.rrf_plan_allreduce.restype = _int
@@ -225,6 +229,18 @@ def rrf_allreduce_rmsnorm_fp8_ptr(inputs, residual_in, residual_out, q_out, scal
     _raise_on(lib.rrf_allreduce_rmsnorm_fp8(
         *_ar_tables(inputs, residual_in, residual_out, q_out, scales_out, signals), len(inputs),
         rank, local_ranks, rows, cols, gamma or None, eps, weight_offset, scale_ub, mode,
+        timeout_ns, stream or None))
+
+
+def rrf_allreduce_rmsnorm_fp8_static_ptr(inputs, residual_in, residual_out, q_out, scales_out,
+                                         rows, cols, gamma, eps, weight_offset, scale_ub,
+                                         mode=0, timeout_ns=0, stream=0) -> None:
+    """rrf_allreduce_rmsnorm_fp8_static on raw pointers: every rank's buffers
+    on the current GPU, all ranks in one launch, the signal pads held by the
+    library (nothing is allocated)."""
+    tables = _ar_tables(inputs, residual_in, residual_out, q_out, scales_out, None)[:5]
+    _raise_on(lib.rrf_allreduce_rmsnorm_fp8_static(
+        *tables, len(inputs), rows, cols, gamma or None, eps, weight_offset, scale_ub, mode,
         timeout_ns, stream or None))
 
 

@@ -29,7 +29,7 @@ NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
 # (source, extra flags, object name)
 UNITS = [("rrf_api.cu", [], "rrf_api.o"), ("rrf_sum.cu", [], "rrf_sum.o"),
          ("rrf_post.cu", [], "rrf_post.o"), ("rrf_allreduce.cu", [], "rrf_allreduce.o"),
-         ("rrf_gemm.cu", [], "rrf_gemm.o")] + [
+         ("rrf_gemm.cu", [], "rrf_gemm.o"), ("rrf_noalloc.cu", [], "rrf_noalloc.o")] + [
     ("rrf_fused.cu", [f"-DRRF_RB={rb}"], f"rrf_fused_rb{rb}.o") for rb in (2, 4, 8, 16)]
 
 

@@ -201,6 +201,8 @@ rrf_status plan_fused(int R, int64_t rows, int64_t cols, int sm_count, bool resi
     return shape_launch(R, rows, cols, sm_count, 0, 0, residual, out);
 }
 
+rrf_status record_cuda_error(cudaError_t e) { return cuda_fail(e); }
+
 cudaError_t launch_fused(const FusedArgs& a, int64_t rows, const FusedLaunch& l, bool residual,
                          cudaStream_t stream) {
     switch (input_bound(a.R)) {

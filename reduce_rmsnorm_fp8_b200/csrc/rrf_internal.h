@@ -171,6 +171,10 @@ cudaError_t launch_scaled_mm_mx(const GemmArgs& g, const void* a, const void* b,
 // at once (the occupancy query; nothing is launched).
 cudaError_t allreduce_resident_blocks(const ArLaunch& l, int* resident);
 
+// Keep `e` as this host thread's last CUDA error (rrf_last_cuda_error) and
+// return RRF_ERR_CUDA.
+rrf_status record_cuda_error(cudaError_t e);
+
 // The launch shape the library picks (pure host arithmetic).
 rrf_status plan_fused(int R, int64_t rows, int64_t cols, int sm_count, bool residual,
                       FusedLaunch* out);
