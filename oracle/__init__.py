@@ -21,6 +21,8 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "rrf_oracle.c")
+# the row-parallel driver (no arithmetic of its own), linked into the same library
+_SRC_MT = os.path.join(_HERE, "rrf_oracle_mt.c")
 _BUILD_DIR = os.path.join(_HERE, "_build")
 _LIB_PATH = os.path.join(_BUILD_DIR, "liboracle.so")
 
@@ -33,12 +35,15 @@ _default = None
 
 
 def build(force: bool = False, src: str = _SRC, out: str = _LIB_PATH) -> str:
-    """Compile ``src`` (default ``rrf_oracle.c``) into a shared library (gcc)."""
+    """Compile ``src`` (default ``rrf_oracle.c``) and the row-parallel driver
+    ``rrf_oracle_mt.c`` into a shared library (gcc)."""
     os.makedirs(os.path.dirname(out), exist_ok=True)
-    stale = not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src)
+    srcs = [src, _SRC_MT]
+    stale = not os.path.exists(out) or any(os.path.getmtime(out) < os.path.getmtime(f)
+                                           for f in srcs)
     if force or stale:
         tmp = out + f".tmp{os.getpid()}"
-        subprocess.run(["gcc", *CFLAGS, "-o", tmp, src, "-lm"], check=True)
+        subprocess.run(["gcc", *CFLAGS, "-o", tmp, *srcs, "-lm", "-lpthread"], check=True)
         os.replace(tmp, out)
     return out
 
@@ -82,6 +87,12 @@ class Oracle:
         lib.oracle_sum_rmsnorm_fp8_rows.argtypes = [
             ctypes.POINTER(u16p), ctypes.c_int, i64, i64, i64, vp, vp, vp,
             ctypes.c_float, ctypes.c_float, ctypes.c_float, vp, vp, vp, vp]
+        lib.oracle_cores.restype = ctypes.c_int
+        lib.oracle_cores.argtypes = []
+        lib.oracle_sum_rmsnorm_fp8_mt.restype = ctypes.c_int
+        lib.oracle_sum_rmsnorm_fp8_mt.argtypes = [
+            ctypes.POINTER(u16p), ctypes.c_int, i64, i64, vp, vp, vp, ctypes.c_float,
+            ctypes.c_float, ctypes.c_float, vp, vp, ctypes.c_int]
         lib.oracle_mx_scale_code.restype = ctypes.c_uint8
         lib.oracle_mx_scale_code.argtypes = [ctypes.c_float]
         lib.oracle_sum_rmsnorm_mxfp8_rows.restype = None
@@ -176,6 +187,34 @@ class Oracle:
             out["v"] = v[sl].copy()
         return out
 
+
+    def cores(self) -> int:
+        """Cores this process may run on (its CPU affinity)."""
+        return int(self.lib.oracle_cores())
+
+    def sum_rmsnorm_fp8_mt(self, inputs, rows: int, cols: int, gamma, eps: float,
+                           weight_offset: float, scale_ub: float, residual=None,
+                           threads: int = 0) -> dict:
+        """sum_rmsnorm_fp8 over all rows, the rows split into contiguous
+        chunks over ``threads`` POSIX threads (0: one per core).  Returns the
+        outputs of sum_rmsnorm_fp8 and ``threads``, the number used."""
+        arrs, table = self._table(inputs, rows, cols)
+        g = np.ascontiguousarray(gamma, dtype=np.uint16).reshape(cols)
+        q = np.zeros((rows, cols), dtype=np.uint8)
+        scales = np.zeros(rows, dtype=np.float32)
+        res_in = res_out = None
+        if residual is not None:
+            res_in = _bf16_rows(residual, rows, cols)
+            res_out = np.zeros((rows, cols), dtype=np.uint16)
+        used = self.lib.oracle_sum_rmsnorm_fp8_mt(
+            table, len(arrs), rows, cols, _ptr(res_in), _ptr(res_out), _ptr(g), eps,
+            weight_offset, scale_ub, _ptr(q), _ptr(scales), threads)
+        if used < 0:
+            raise RuntimeError("a worker thread could not be started")
+        out = {"q": q, "scales": scales, "threads": int(used)}
+        if res_out is not None:
+            out["res_out"] = res_out
+        return out
 
     def mx_scale_code(self, amax: float) -> int:
         """E8M0 code of a block's shared scale from its max |V| (OCP MX)."""
