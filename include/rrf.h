@@ -147,6 +147,9 @@ rrf_status rrf_sum_rmsnorm_fp8(const void* const* inputs, int num_inputs,
 #define RRF_FLAG_NO_PDL 1            /* launch without programmatic dependent launch */
 #define RRF_FLAG_BARRIER_EXCHANGE 2  /* clusters meet at a cluster barrier phase
                                         instead of the transaction-counted exchange */
+#define RRF_FLAG_NO_PREFETCH 4       /* no L2 prefetch before the wait for the
+                                        previous kernel (see below)              */
+#define RRF_FLAG_PREFETCH 8          /* the L2 prefetch whatever the planner says */
 #define RRF_FLAG_DEBUG_STARVE_EXCHANGE 0x100 /* test hook: every block of a cluster
                                         waits for one value more than its peers
                                         send, so its bounded wait runs out (about
@@ -158,8 +161,8 @@ rrf_status rrf_sum_rmsnorm_fp8(const void* const* inputs, int num_inputs,
 
 /* rrf_sum_rmsnorm_fp8_ex -- rrf_sum_rmsnorm_fp8 with the launch forced, for
  * tests and benchmarks.  variant is one of RRF_VARIANT_*; cluster_size is
- * 2, 4, 8 or 16 for RRF_VARIANT_CLUSTER (0 = automatic) and ignored
- * otherwise; block_threads is a multiple of 32 in [32, 1024] or 0
+ * 2..16 for RRF_VARIANT_CLUSTER (0 = automatic; sizes above 8 are the
+ * non-portable cluster sizes B200 allows) and ignored otherwise; block_threads is a multiple of 32 in [32, 1024] or 0
  * (automatic); flags combines RRF_FLAG_*.  Results are bit-identical across
  * variants for the bf16 outputs and agree within the stated tolerance for
  * scales and codes.
@@ -178,6 +181,16 @@ rrf_status rrf_sum_rmsnorm_fp8(const void* const* inputs, int num_inputs,
  * still finishing; each kernel waits for that kernel (its completion and the
  * visibility of its writes) before it touches global memory, so stream order
  * is kept for every producer.  RRF_FLAG_NO_PDL launches the plain way.
+ *
+ * L2 prefetch: where the planner expects the grid to be resident at once
+ * (decode-sized batches), each block first asks L2 for its slice of the
+ * inputs, the residual and gamma (cp.async.bulk.prefetch.L2), then waits for
+ * the previous kernel: the HBM fetch overlaps that kernel's tail.  A
+ * prefetch returns no data and changes no value the kernel reads after the
+ * wait (L2 is the point of coherence of the GPU's own memory), so this is
+ * safe whatever the previous kernel writes; it gains nothing for data that
+ * kernel has not yet written.  RRF_FLAG_NO_PREFETCH and RRF_FLAG_PREFETCH
+ * override the planner.
  * Errors: those of rrf_sum_rmsnorm_fp8, and RRF_ERR_UNSUPPORTED when the
  * forced launch cannot cover the row or flags holds an unknown bit. */
 rrf_status rrf_sum_rmsnorm_fp8_ex(const void* const* inputs, int num_inputs,
@@ -510,6 +523,26 @@ rrf_status rrf_check_scaled_mm_args(const void* a, const float* a_scale, const v
                                     const float* b_scale, const void* bias, const void* out,
                                     int64_t M, int64_t N, int64_t K);
 
+/* GEMM kernels (rrf_plan_scaled_mm). */
+#define RRF_GEMM_KERNEL_PAIR 1 /* 256 x 256 tiles on SM pairs (two-CTA MMA)           */
+#define RRF_GEMM_KERNEL_TILE 2 /* one persistent CTA per SM walking 128 x tile_n output
+                                  tiles, its A stages a_rows rows                     */
+#define RRF_GEMM_KERNEL_SWAP 3 /* per-token only: operands swapped, 64 weight rows on
+                                  the MMA's M side, the call's rows padded to a_rows  */
+
+/* rrf_plan_scaled_mm -- the kernel rrf_scaled_mm_fp8 (mx == 0) or
+ * rrf_scaled_mm_mxfp8 (mx != 0) runs for an M x N x K product on a GPU with
+ * sm_count SMs, without touching the GPU: its RRF_GEMM_KERNEL_*, the rows of
+ * an A stage, the output columns of a tile (for RRF_GEMM_KERNEL_SWAP the 64
+ * weight rows of a tile), the k-tiles of 128 bytes per TMA box, the output
+ * tiles and the CTAs launched (ctas < tiles: CTAs walk several tiles).
+ * M == 0 launches nothing: kernel 0, tiles and ctas 0.
+ * Errors: RRF_ERR_NULL (an output pointer), RRF_ERR_SHAPE (a shape the call
+ * rejects), RRF_ERR_UNSUPPORTED (sm_count < 2). */
+rrf_status rrf_plan_scaled_mm(int64_t M, int64_t N, int64_t K, int mx, int sm_count,
+                              int* kernel, int* a_rows, int* tile_n, int* k_tiles_per_stage,
+                              int64_t* tiles, int64_t* ctas);
+
 /* rrf_plan_fused -- the launch rrf_sum_rmsnorm_fp8 would use on a GPU with
  * sm_count SMs for a call with (residual != 0) or without a residual,
  * without touching the GPU.  Writes the cluster size (1 = one
@@ -520,6 +553,16 @@ rrf_status rrf_check_scaled_mm_args(const void* a, const float* a_scale, const v
 rrf_status rrf_plan_fused(int num_inputs, int64_t rows, int64_t cols, int residual,
                           int sm_count, int* cluster_size, int* block_threads,
                           int* vecs_per_thread);
+
+/* rrf_plan_fused_ex -- rrf_plan_fused with the launch's L2-prefetch choice
+ * (1: each block prefetches its slice before waiting for the previous
+ * kernel; see rrf_sum_rmsnorm_fp8_ex).  The launch comes from the library's
+ * table of measured launches (the entry nearest to the shape), adjusted so
+ * that every block keeps at least 32 vectors and fits its slice.
+ * Errors: those of rrf_plan_fused. */
+rrf_status rrf_plan_fused_ex(int num_inputs, int64_t rows, int64_t cols, int residual,
+                             int sm_count, int* cluster_size, int* block_threads,
+                             int* vecs_per_thread, int* prefetch);
 
 /* rrf_check_sum_args / rrf_check_fused_args -- the host-side validation of
  * rrf_sum / rrf_sum_rmsnorm_fp8 alone: the status those calls would return
@@ -539,6 +582,10 @@ rrf_status rrf_check_fused_args(const void* const* inputs, int num_inputs, int64
                                             rank ran out                      */
 #define RRF_DEVICE_ERROR_GEMM_TIMEOUT 4u /* a wait of the FP8 GEMM's operand
                                             pipeline ran out                  */
+#define RRF_DEVICE_ERROR_BOUNDS 8u /* the bounds-checking build (librrf_debug.so,
+                                      compiled with RRF_DEBUG) found an index
+                                      outside its buffer and skipped that
+                                      access; never set by the normal build    */
 
 /* rrf_device_error -- the device error word of the current device: the OR
  * of RRF_DEVICE_ERROR_* bits that kernels of this library have set since it

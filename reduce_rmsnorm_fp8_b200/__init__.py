@@ -41,6 +41,9 @@ _EXPORTS = (
     "rrf_check_scaled_mm_args", "rrf_sum_rmsnorm_mxfp8", "rrf_check_mxfp8_args",
     "mx_blocked", "mx_blocked_bytes", "rrf_scaled_mm_mxfp8", "rrf_check_scaled_mm_mx_args",
     "RRF_AR_STATIC_MAX_WORLD", "rrf_allreduce_rmsnorm_fp8_static_ptr",
+    "rrf_plan_scaled_mm", "RRF_GEMM_KERNEL_PAIR", "RRF_GEMM_KERNEL_TILE",
+    "RRF_GEMM_KERNEL_SWAP", "RRF_FLAG_NO_PREFETCH", "RRF_FLAG_PREFETCH", "rrf_plan_fused_ex",
+    "RRF_DEVICE_ERROR_BOUNDS",
 )
 
 __all__ = list(_EXPORTS)

@@ -6,7 +6,9 @@ import enum
 import os
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "librrf.so")
+# RRF_DEBUG_LIBRARY=1 selects the bounds-checking build (librrf_debug.so).
+LIB_PATH = os.path.join(_PKG, "librrf_debug.so" if os.environ.get("RRF_DEBUG_LIBRARY") == "1"
+                        else "librrf.so")
 
 RRF_MAX_INPUTS = 16
 RRF_MAX_COLS = 16 * 256 * 8 * 8
@@ -16,6 +18,8 @@ RRF_VARIANT_CLUSTER = 2
 RRF_FLAG_NO_PDL = 1
 RRF_FLAG_BARRIER_EXCHANGE = 2
 RRF_FLAG_DEBUG_STARVE_EXCHANGE = 0x100
+RRF_FLAG_NO_PREFETCH = 4
+RRF_FLAG_PREFETCH = 8
 RRF_DEVICE_ERROR_EXCHANGE_TIMEOUT = 1
 RRF_MAX_SHARDS = 64
 RRF_DEVICE_ERROR_PEER_TIMEOUT = 2
@@ -27,6 +31,10 @@ RRF_AR_AUTO = 0
 RRF_AR_ONE_SHOT = 1
 RRF_AR_TWO_SHOT = 2
 RRF_DEVICE_ERROR_GEMM_TIMEOUT = 4
+RRF_DEVICE_ERROR_BOUNDS = 8
+RRF_GEMM_KERNEL_PAIR = 1
+RRF_GEMM_KERNEL_TILE = 2
+RRF_GEMM_KERNEL_SWAP = 3
 
 
 class Status(enum.IntEnum):
@@ -76,6 +84,8 @@ lib.rrf_sum_rmsnorm_fp8_ex.argtypes = _fused_args + [_int, _int, _int, _int, _vp
 lib.rrf_plan_fused.restype = _int
 lib.rrf_plan_fused.argtypes = [_int, _i64, _i64, _int, _int, ctypes.POINTER(_int),
                                ctypes.POINTER(_int), ctypes.POINTER(_int)]
+lib.rrf_plan_fused_ex.restype = _int
+lib.rrf_plan_fused_ex.argtypes = [_int, _i64, _i64, _int, _int] + [ctypes.POINTER(_int)] * 4
 lib.rrf_check_sum_args.restype = _int
 lib.rrf_check_sum_args.argtypes = [_ptrs, _int, _i64, _i64, _vp]
 lib.rrf_check_fused_args.restype = _int
@@ -126,6 +136,9 @@ lib.rrf_scaled_mm_fp8.restype = _int
 lib.rrf_scaled_mm_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]
 lib.rrf_check_scaled_mm_args.restype = _int
 lib.rrf_check_scaled_mm_args.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64]
+lib.rrf_plan_scaled_mm.restype = _int
+lib.rrf_plan_scaled_mm.argtypes = [_i64, _i64, _i64, _int, _int] + [ctypes.POINTER(_int)] * 4 + \
+    [ctypes.POINTER(_i64)] * 2
 lib.rrf_device_error.restype = _int
 lib.rrf_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), _int]
 lib.rrf_version.restype = ctypes.c_char_p
@@ -193,6 +206,15 @@ def rrf_plan_fused(num_inputs: int, rows: int, cols: int, sm_count: int, residua
     _raise_on(lib.rrf_plan_fused(num_inputs, rows, cols, int(bool(residual)), sm_count,
                                  ctypes.byref(c), ctypes.byref(t), ctypes.byref(v)))
     return c.value, t.value, v.value
+
+
+def rrf_plan_fused_ex(num_inputs: int, rows: int, cols: int, sm_count: int, residual=True):
+    """The launch the library would pick, with its L2-prefetch choice:
+    (cluster_size, block_threads, vecs_per_thread, prefetch)."""
+    out = [_int() for _ in range(4)]
+    _raise_on(lib.rrf_plan_fused_ex(num_inputs, rows, cols, int(bool(residual)), sm_count,
+                                    *[ctypes.byref(o) for o in out]))
+    return tuple(o.value for o in out)
 
 
 def _ar_tables(inputs, residual_in, residual_out, q_out, scales_out, signals):
@@ -482,6 +504,20 @@ def rrf_check_scaled_mm_args(a, a_scale, b, b_scale, bias, out, M, N, K) -> int:
     """Host validation of the FP8 GEMM on raw pointers."""
     return lib.rrf_check_scaled_mm_args(a or None, a_scale or None, b or None, b_scale or None,
                                         bias or None, out or None, M, N, K)
+
+
+def rrf_plan_scaled_mm(M: int, N: int, K: int, sm_count: int, mx: bool = False) -> dict:
+    """The GEMM kernel rrf_scaled_mm_fp8 (or, mx=True, rrf_scaled_mm_mxfp8)
+    runs for an M x N x K product on sm_count SMs (host only)."""
+    ints = [_int() for _ in range(4)]
+    longs = [_i64() for _ in range(2)]
+    _raise_on(lib.rrf_plan_scaled_mm(M, N, K, int(bool(mx)), sm_count,
+                                     *[ctypes.byref(o) for o in ints + longs]))
+    names = {RRF_GEMM_KERNEL_PAIR: "pair", RRF_GEMM_KERNEL_TILE: "tile",
+             RRF_GEMM_KERNEL_SWAP: "swap"}
+    return {"kernel": names.get(ints[0].value), "a_rows": ints[1].value,
+            "tile_n": ints[2].value, "k_tiles_per_stage": ints[3].value,
+            "tiles": longs[0].value, "ctas": longs[1].value}
 
 
 def rrf_scaled_mm_fp8(a, a_scale, b, b_scale, bias=None, out=None):

@@ -39,9 +39,6 @@
 namespace rrf {
 namespace {
 
-constexpr float kE4m3Max = 448.0f;
-constexpr float kScaleFloor = 1e-12f;
-
 // ------------------------------------------------------------- signal pads --
 
 // Word (phase, src, block) of a rank's pad: block `block` of rank `src` has
@@ -91,7 +88,10 @@ __device__ void peer_barrier(const ArArgs& a, int phase, int rank, int block,
                              unsigned int call) {
     __syncthreads();
     const int t = threadIdx.x;
-    if (t < a.world) {
+    // (the pads' words: world <= RRF_AR_MAX_WORLD ranks, block < RRF_AR_MAX_BLOCKS)
+    if (t < a.world && RRF_IN_BOUNDS(a.world <= RRF_AR_MAX_WORLD && rank < a.world &&
+                                         block < RRF_AR_MAX_BLOCKS,
+                                     a.err)) {
         unsigned int* theirs = flag_word(a.sig[t], phase, rank, block);
         if (phase == 0) st_relaxed_sys(theirs, call);
         else st_release_sys(theirs, call);
@@ -150,7 +150,10 @@ __global__ void __launch_bounds__(kArMaxThreads, VPT <= 2 ? 2 : 1) ar_kernel(con
     // on its rank's pad (written by this block at the end of the previous
     // call, an earlier kernel of the stream).
     __shared__ unsigned int call_s;
-    if (tid == 0) call_s = ld_relaxed_gpu(counter_word(a.sig[rank], block)) + 1u;
+    if (tid == 0)
+        call_s = RRF_IN_BOUNDS(rank < a.world && block < RRF_AR_MAX_BLOCKS, a.err)
+                     ? ld_relaxed_gpu(counter_word(a.sig[rank], block)) + 1u
+                     : 0u;
     __syncthreads();
     const unsigned int call = call_s;
 
@@ -160,7 +163,9 @@ __global__ void __launch_bounds__(kArMaxThreads, VPT <= 2 ? 2 : 1) ar_kernel(con
     peer_barrier(a, 0, rank, block, call);
     if (CLUSTER) cluster_wait_acquire();
 
-    const int64_t first = a.two_shot ? (int64_t)rank * a.rows_per_rank : 0;
+    // every address below derives from `first`, taken after the start
+    // barrier's acquire (the peers' loads must not move above it)
+    const int64_t first = opaque(a.two_shot ? (int64_t)rank * a.rows_per_rank : (int64_t)0);
     const int64_t stop = a.two_shot ? min(first + a.rows_per_rank, a.rows) : a.rows;
     const int nclusters = a.blocks / C;
     const uint4* res_in = RES ? a.res_in[rank] : nullptr;
@@ -174,7 +179,7 @@ __global__ void __launch_bounds__(kArMaxThreads, VPT <= 2 ? 2 : 1) ar_kernel(con
 #pragma unroll
         for (int k = 0; k < VPT; ++k) {
             const int v = v_begin + tid + k * T;
-            if (v < v_end) {
+            if (v < v_end && RRF_IN_BOUNDS(v >= 0 && v < a.vecs && row < a.rows, a.err)) {
                 uint4 x[W];
 #pragma unroll
                 for (int j = 0; j < W; ++j)
@@ -213,17 +218,14 @@ __global__ void __launch_bounds__(kArMaxThreads, VPT <= 2 ? 2 : 1) ar_kernel(con
             cluster_wait_acquire();
             st = stats_butterfly(slots[par][lane & (C - 1)], C);
         }
-        const float ms = st.ss / a.cols_f;
-        const float rinv = 1.0f / sqrtf(ms + a.eps);
-        const float amax = __fmul_rn(st.key, rinv);
-        const float scale = fmaxf(fminf(amax, a.scale_ub), kScaleFloor) / kE4m3Max;
-        const float inv_scale = 1.0f / scale;
+        const RowScale rs = row_scale(st.ss, st.key, a.inv_cols, a.eps, a.scale_ub);
+        const float rinv = rs.rinv, scale = rs.scale, inv_scale = rs.inv_scale;
         // ---- pass 2: codes; the outputs go to this rank (one-shot) or to
         // every rank (two-shot)
 #pragma unroll
         for (int k = 0; k < VPT; ++k) {
             const int v = v_begin + tid + k * T;
-            if (v < v_end) {
+            if (v < v_end && RRF_IN_BOUNDS(v >= 0 && v < a.vecs && row < a.rows, a.err)) {
                 float hf[8], gf[8], qv[8];
                 bf16x8_to_f32(h[k], hf);
                 bf16x8_to_f32(KEEP_GAMMA ? g[k] : ld_shared_by_all(a.gamma + v), gf);
@@ -248,7 +250,7 @@ __global__ void __launch_bounds__(kArMaxThreads, VPT <= 2 ? 2 : 1) ar_kernel(con
                 }
             }
         }
-        if (tid == 0 && crank == 0) {
+        if (tid == 0 && crank == 0 && RRF_IN_BOUNDS(row < a.rows, a.err)) {
             if (a.two_shot) {
 #pragma unroll
                 for (int j = 0; j < W; ++j)
@@ -259,7 +261,8 @@ __global__ void __launch_bounds__(kArMaxThreads, VPT <= 2 ? 2 : 1) ar_kernel(con
         }
     }
     peer_barrier(a, 1, rank, block, call);
-    if (tid == 0) *counter_word(a.sig[rank], block) = call;
+    if (tid == 0 && RRF_IN_BOUNDS(rank < a.world && block < RRF_AR_MAX_BLOCKS, a.err))
+        *counter_word(a.sig[rank], block) = call;
 }
 
 // Clusters of up to 8 (the portable size) only.

@@ -150,19 +150,63 @@ static bool pick_block(int R, int64_t slice, int forced_threads, FusedLaunch* l)
     return false;
 }
 
-// The cluster choice, from launch-shape sweeps on B200 (148 SMs; 1-256 rows
-// of 4096-8192 columns, 4-8 inputs, with and without a residual; graph
-// replays over buffer sets larger than L2):
-//   * a batch of at least one row per SM, or rows under ~48 KB of traffic,
-//     runs best with one block per row (a block streams a 37 KB row in about
-//     the time a cluster round trip costs);
-//   * longer rows of smaller batches run best split over clusters of 8
-//     (150 KB rows: 2.53 us at 1 row vs 4.53 us unsplit), or of 4 once 4
-//     blocks per row already give two blocks per SM.
-constexpr double kSplitRowBytes = 48.0 * 1024.0;
+// ------------------------------------------------------------ launch table --
+// The fused call's launch is read from a table of measured launches
+// (rrf_plan_table.inc, written by `bench.py --plan-sweep` on a B200): for
+// input bounds 2/4/8/16, with and without a residual, over row lengths and
+// batch sizes, the cluster size and L2-prefetch setting whose graph-replayed
+// calls over buffer sets larger than L2 ran fastest.  A call takes the entry
+// of its input bound and residual flag nearest to its shape (row length
+// weighted 4x against batch size, both on a log scale; batch sizes scaled to
+// the table's 148 SMs), then adjusts the cluster so that every block keeps
+// at least 32 vectors and fits its slice.
+struct PlanEntry {
+    int rb;        // input bound
+    int residual;  // 0 / 1
+    int cols;
+    int rows;
+    int cluster;   // blocks per row
+    int prefetch;  // L2 prefetch before the wait for the previous kernel
+    float us;      // measured time per call of this launch
+};
 
-static int cluster_choice(int64_t rows, double row_bytes, int sm_count) {
-    if (rows >= sm_count || row_bytes < kSplitRowBytes) return 1;
+static const PlanEntry kPlanTable[] = {
+#define RRF_PLAN(rb, res, cols, rows, cluster, prefetch, us) \
+    {rb, res, cols, rows, cluster, prefetch, us},
+#include "rrf_plan_table.inc"
+#undef RRF_PLAN
+    {0, 0, 0, 0, 0, 0, 0.0f}};
+
+constexpr int kPlanTableSms = 148;
+
+static const PlanEntry* table_entry(int R, int64_t rows, int64_t cols, int sm_count,
+                                    bool residual) {
+    const int rb = input_bound(R);
+    const double r = (double)(rows > 0 ? rows : 1) * kPlanTableSms / sm_count;
+    const PlanEntry* best = nullptr;
+    double best_d = 0.0;
+    for (const PlanEntry* e = kPlanTable; e->rb != 0; ++e) {
+        if (e->rb != rb || e->residual != (residual ? 1 : 0)) continue;
+        const double d = 4.0 * std::fabs(std::log2((double)cols / e->cols)) +
+                         std::fabs(std::log2(r / e->rows));
+        if (best == nullptr || d < best_d) {
+            best = e;
+            best_d = d;
+        }
+    }
+    return best;
+}
+
+// The cluster size by formula, from earlier launch-shape sweeps on B200: one
+// block per row when the batch has a row per SM or a row moves under ~48 KB
+// (a block streams a 37 KB row in about the time a cluster round trip
+// costs), else clusters of 8 (150 KB rows: 2.53 us at 1 row vs 4.53 us
+// unsplit), or of 4 once 4 blocks per row give two blocks per SM.  The
+// multi-GPU kernel uses it; the fused call uses it only without a table
+// entry, and then prefetches when its grid is resident at once (at most 4
+// blocks per SM).
+static int cluster_formula(int64_t rows, double row_bytes, int sm_count) {
+    if (rows >= sm_count || row_bytes < 48.0 * 1024.0) return 1;
     return rows * 4 >= 2 * (int64_t)sm_count ? 4 : 8;
 }
 
@@ -174,20 +218,29 @@ static rrf_status shape_launch(int R, int64_t rows, int64_t cols, int sm_count, 
     if (st != RRF_OK) return st;
     if (sm_count < 1) sm_count = 1;
     const int64_t vecs = cols / 8;
-    int c = cluster;
-    if (c == 0) {
-        // The measured choice (see cluster_choice), at least 32 vectors per
-        // block; then split further, up to 16, while one block cannot hold
-        // its slice.
+    int c = 0;
+    bool prefetch = false;
+    if (const PlanEntry* e = table_entry(R, rows, cols, sm_count, residual)) {
+        c = e->cluster;
+        prefetch = e->prefetch != 0;
+    } else {
         const double row_bytes = (double)cols * (2.0 * R + (residual ? 4.0 : 0.0) + 1.0);
-        c = cluster_choice(rows, row_bytes, sm_count);
-        while (c > 1 && vecs / c < 32) c /= 2;
-        while (c < 16 && !pick_block(R, (vecs + c - 1) / c, forced_threads, out)) c *= 2;
+        c = cluster_formula(rows, row_bytes, sm_count);
+        prefetch = rows * c <= 4 * (int64_t)sm_count;
+    }
+    if (cluster != 0) {
+        c = cluster;
+    } else {
+        // at least 32 vectors per block; then split further, up to 16, while
+        // one block cannot hold its slice
+        while (c > 1 && vecs / c < 32) --c;
+        while (c < 16 && !pick_block(R, (vecs + c - 1) / c, forced_threads, out)) ++c;
     }
     if (!pick_block(R, (vecs + c - 1) / c, forced_threads, out))
         return cluster == 0 && forced_threads == 0 ? RRF_ERR_SHAPE : RRF_ERR_UNSUPPORTED;
     out->cluster = c;
     out->pdl = true;
+    out->prefetch = prefetch;
     // Exchange: measured on B200 (residual stores after the exchange in both
     // forms), the st.async + mbarrier exchange ties the cluster barrier at 1-8
     // rows and beats it from 32 rows on (4.03 vs 4.39 us at 64 rows of 7168
@@ -308,13 +361,14 @@ extern "C" rrf_status rrf_sum_rmsnorm_fp8_ex(const void* const* inputs, int num_
                                          q_out, scales_out);
     if (st != RRF_OK) return st;
     if (variant < RRF_VARIANT_AUTO || variant > RRF_VARIANT_CLUSTER) return RRF_ERR_UNSUPPORTED;
-    if ((flags & ~(RRF_FLAG_NO_PDL | RRF_FLAG_BARRIER_EXCHANGE | RRF_FLAG_DEBUG_STARVE_EXCHANGE)) !=
-        0)
+    if ((flags & ~(RRF_FLAG_NO_PDL | RRF_FLAG_BARRIER_EXCHANGE | RRF_FLAG_NO_PREFETCH |
+                   RRF_FLAG_PREFETCH | RRF_FLAG_DEBUG_STARVE_EXCHANGE)) != 0 ||
+        (flags & RRF_FLAG_NO_PREFETCH && flags & RRF_FLAG_PREFETCH))
         return RRF_ERR_UNSUPPORTED;
     if (block_threads != 0 && (block_threads < 32 || block_threads > 1024 || block_threads % 32))
         return RRF_ERR_UNSUPPORTED;
-    if (variant == RRF_VARIANT_CLUSTER && cluster_size != 0 && cluster_size != 2 &&
-        cluster_size != 4 && cluster_size != 8 && cluster_size != 16)
+    if (variant == RRF_VARIANT_CLUSTER && cluster_size != 0 &&
+        (cluster_size < 2 || cluster_size > 16))
         return RRF_ERR_UNSUPPORTED;
     if (rows == 0) return RRF_OK;
 
@@ -338,6 +392,8 @@ extern "C" rrf_status rrf_sum_rmsnorm_fp8_ex(const void* const* inputs, int num_
         return st;
     const int64_t vecs = cols / 8;
     l.pdl = (flags & RRF_FLAG_NO_PDL) == 0;
+    if (flags & RRF_FLAG_NO_PREFETCH) l.prefetch = false;
+    if (flags & RRF_FLAG_PREFETCH) l.prefetch = true;
     if (flags & RRF_FLAG_BARRIER_EXCHANGE) l.async_exchange = false;
     if (flags & RRF_FLAG_DEBUG_STARVE_EXCHANGE) {
         // the hook exercises the bounded wait of the transaction-counted exchange
@@ -356,14 +412,16 @@ extern "C" rrf_status rrf_sum_rmsnorm_fp8_ex(const void* const* inputs, int num_
     a.scales = scales_out;
     a.R = num_inputs;
     a.vecs = (int)vecs;
+    a.rows = rows;
     a.cluster = l.cluster;
     a.slice_vecs = (int)((vecs + l.cluster - 1) / l.cluster);
-    a.cols_f = (float)cols;
+    a.inv_cols = (float)(1.0 / (double)cols);
     a.eps = eps;
     a.weight_offset = weight_offset;
     a.scale_ub = scale_ub;
     a.err = err;
     a.starve = (flags & RRF_FLAG_DEBUG_STARVE_EXCHANGE) ? 1 : 0;
+    a.prefetch = l.prefetch ? 1 : 0;
     cudaError_t e;
     if (!take_injected_failure(&e))
         e = launch_fused(a, rows, l, residual_in != nullptr, (cudaStream_t)stream);
@@ -463,13 +521,15 @@ static rrf_status mxfp8_call(const void* const* inputs, int num_inputs, int64_t 
     a.q = static_cast<uint2*>(q_out);
     a.scales_mx = static_cast<uint8_t*>(scales_mx_out);
     a.mx_blocked = blocked ? 1 : 0;
+    a.prefetch = l.prefetch ? 1 : 0;
     a.R = num_inputs;
     a.vecs = (int)vecs;
+    a.rows = rows;
     a.cluster = l.cluster;
     // a cluster block's slice starts on a 32-element block (4 vectors); the
     // block's threads (a multiple of 32) x vectors per thread still cover it
     a.slice_vecs = (int)(((vecs + l.cluster - 1) / l.cluster + 3) / 4 * 4);
-    a.cols_f = (float)cols;
+    a.inv_cols = (float)(1.0 / (double)cols);
     a.eps = eps;
     a.weight_offset = weight_offset;
     a.scale_ub = 1.0f;
@@ -564,13 +624,15 @@ extern "C" rrf_status rrf_sum_rmsnorm_fp8_pre(const void* const* inputs, int num
     a.gamma = static_cast<const uint4*>(gamma);
     a.R = num_inputs;
     a.vecs = (int)vecs;
+    a.rows = rows;
     a.cluster = l.cluster;
     a.slice_vecs = (int)((vecs + l.cluster - 1) / l.cluster);
-    a.cols_f = (float)cols;
+    a.inv_cols = (float)(1.0 / (double)cols);
     a.weight_offset = weight_offset;
     a.scale_ub = 1.0f;
     a.err = err;
     a.stats_only = 1;
+    a.prefetch = l.prefetch ? 1 : 0;
     a.stats = reinterpret_cast<float2*>(stats_out);
     a.h_out = static_cast<uint4*>(h_out);
     cudaError_t e;
@@ -631,10 +693,11 @@ extern "C" rrf_status rrf_rmsnorm_fp8_post(const void* h, int64_t rows, int64_t 
     a.rows = rows;
     a.vecs = (int)(cols / 8);
     a.shards = shards;
-    a.total_cols_f = (float)total_cols;
+    a.inv_total_cols = (float)(1.0 / (double)total_cols);
     a.eps = eps;
     a.weight_offset = weight_offset;
     a.scale_ub = scale_ub;
+    if ((st = device_error_word(&a.err)) != RRF_OK) return st;
     cudaError_t e;
     if (!take_injected_failure(&e)) e = launch_post(a, sm_count, true, (cudaStream_t)stream);
     return e == cudaSuccess ? RRF_OK : cuda_fail(e);
@@ -657,7 +720,7 @@ int ar_mode(int world, int64_t rows, int mode) {
 }
 
 // The row shape for the rows one rank computes, chosen as for the single-GPU
-// kernel (cluster_choice), then the fewest vectors per thread (at most 4)
+// kernel's formula (cluster_formula), then the fewest vectors per thread (at most 4)
 // that keep a block at <= 512 threads, splitting the row further (up to
 // clusters of 8) while none does.
 rrf_status plan_allreduce(int world, int64_t rows, int64_t cols, bool residual, int mode,
@@ -671,7 +734,7 @@ rrf_status plan_allreduce(int world, int64_t rows, int64_t cols, bool residual, 
     const int64_t mine = l->two_shot ? (rows + world - 1) / world : rows;
     const int64_t vecs = cols / 8;
     const double row_bytes = (double)cols * (2.0 * world + (residual ? 4.0 : 0.0) + 1.0);
-    int c = cluster_choice(mine, row_bytes, sm_count);
+    int c = cluster_formula(mine, row_bytes, sm_count);
     while (c > 1 && vecs / c < 32) c /= 2;
     for (;;) {
         const int64_t slice = (vecs + c - 1) / c;
@@ -809,7 +872,7 @@ extern "C" rrf_status rrf_allreduce_rmsnorm_fp8(
     a.vecs = (int)(cols / 8);
     a.cluster = l.cluster;
     a.slice_vecs = (int)((cols / 8 + l.cluster - 1) / l.cluster);
-    a.cols_f = (float)cols;
+    a.inv_cols = (float)(1.0 / (double)cols);
     a.eps = eps;
     a.weight_offset = weight_offset;
     a.scale_ub = scale_ub;
@@ -883,6 +946,34 @@ extern "C" rrf_status rrf_scaled_mm_fp8(const void* a, const float* a_scale, con
     return e == cudaSuccess ? RRF_OK : cuda_fail(e);
 }
 
+extern "C" rrf_status rrf_plan_scaled_mm(int64_t M, int64_t N, int64_t K, int mx, int sm_count,
+                                         int* kernel, int* a_rows, int* tile_n,
+                                         int* k_tiles_per_stage, int64_t* tiles,
+                                         int64_t* ctas) {
+    if (!kernel || !a_rows || !tile_n || !k_tiles_per_stage || !tiles || !ctas)
+        return RRF_ERR_NULL;
+    // the calls' own shape rules, checked without operands
+    const rrf_status st = mx ? rrf_check_scaled_mm_mx_args(nullptr, nullptr, nullptr, nullptr,
+                                                            nullptr, nullptr, M, N, K)
+                             : rrf_check_scaled_mm_args(nullptr, nullptr, nullptr, nullptr,
+                                                        nullptr, nullptr, M, N, K);
+    if (st != RRF_OK && st != RRF_ERR_NULL) return st;
+    if (sm_count < 2) return RRF_ERR_UNSUPPORTED;
+    if (M == 0) {
+        *kernel = *a_rows = *tile_n = *k_tiles_per_stage = 0;
+        *tiles = *ctas = 0;
+        return RRF_OK;
+    }
+    const GemmPlan p = plan_scaled_mm(M, N, K, mx != 0, sm_count);
+    *kernel = p.kernel;
+    *a_rows = p.a_rows;
+    *tile_n = p.tile_n;
+    *k_tiles_per_stage = p.k_tiles_per_stage;
+    *tiles = p.tiles;
+    *ctas = p.ctas;
+    return RRF_OK;
+}
+
 extern "C" rrf_status rrf_check_scaled_mm_mx_args(const void* a, const void* sa,
                                                   const void* b, const void* sb,
                                                   const void* bias, const void* out, int64_t M,
@@ -929,17 +1020,27 @@ extern "C" rrf_status rrf_scaled_mm_mxfp8(const void* a, const void* sa, const v
     return e == cudaSuccess ? RRF_OK : cuda_fail(e);
 }
 
-extern "C" rrf_status rrf_plan_fused(int num_inputs, int64_t rows, int64_t cols, int residual,
-                                     int sm_count, int* cluster_size, int* block_threads,
-                                     int* vecs_per_thread) {
-    if (!cluster_size || !block_threads || !vecs_per_thread) return RRF_ERR_NULL;
+extern "C" rrf_status rrf_plan_fused_ex(int num_inputs, int64_t rows, int64_t cols,
+                                        int residual, int sm_count, int* cluster_size,
+                                        int* block_threads, int* vecs_per_thread,
+                                        int* prefetch) {
+    if (!cluster_size || !block_threads || !vecs_per_thread || !prefetch) return RRF_ERR_NULL;
     FusedLaunch l = {};
     rrf_status st = plan_fused(num_inputs, rows, cols, sm_count, residual != 0, &l);
     if (st != RRF_OK) return st;
     *cluster_size = l.cluster;
     *block_threads = l.threads;
     *vecs_per_thread = l.vecs_per_thread;
+    *prefetch = l.prefetch ? 1 : 0;
     return RRF_OK;
+}
+
+extern "C" rrf_status rrf_plan_fused(int num_inputs, int64_t rows, int64_t cols, int residual,
+                                     int sm_count, int* cluster_size, int* block_threads,
+                                     int* vecs_per_thread) {
+    int prefetch = 0;
+    return rrf_plan_fused_ex(num_inputs, rows, cols, residual, sm_count, cluster_size,
+                             block_threads, vecs_per_thread, &prefetch);
 }
 
 extern "C" const char* rrf_status_string(rrf_status status) {

@@ -31,15 +31,36 @@
 namespace rrf {
 namespace {
 
-constexpr float kE4m3Max = 448.0f;
-constexpr float kScaleFloor = 1e-12f;
-
 // E8M0 code of an MX block's shared scale 2^(floor(log2(amax)) - 8) (OCP MX
 // v1.0, e4m3 elements: 448 = 1.75 * 2^8): the biased exponent field of
 // amax minus 8, clamped at 0 (zero, subnormal and tiny maxima).
 __device__ __forceinline__ uint32_t mx_scale_code(float amax) {
     const int e = (int)((__float_as_uint(amax) >> 23) & 0xFFu);
     return e > 8 ? (uint32_t)(e - 8) : 0u;
+}
+
+// The 8 codes of one vector: y = (h * r) * (gamma + weight_offset), then
+// y * m (m = 1 / scale, or 1 / X of an MX block), each product rounded once.
+template <bool PACKED>
+__device__ __forceinline__ uint2 quantise_vector(uint4 h, uint4 g, float r, float wo, float m) {
+    if constexpr (PACKED) {
+        const float2 r2 = make_float2(r, r), w2 = make_float2(wo, wo), m2 = make_float2(m, m);
+        float2 hf[4], gf[4], qv[4];
+        bf16x8_to_f32x2(h, hf);
+        bf16x8_to_f32x2(g, gf);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            qv[e] = __fmul2_rn(__fmul2_rn(__fmul2_rn(hf[e], r2), __fadd2_rn(gf[e], w2)), m2);
+        return f32x2_to_e4m3x8(qv);
+    } else {
+        float hf[8], gf[8], qv[8];
+        bf16x8_to_f32(h, hf);
+        bf16x8_to_f32(g, gf);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            qv[e] = __fmul_rn(__fmul_rn(__fmul_rn(hf[e], r), __fadd_rn(gf[e], wo)), m);
+        return f32_to_e4m3x8(qv);
+    }
 }
 
 // ASYNC (cluster rows only): the blocks of a cluster meet through the
@@ -66,22 +87,44 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
         // into a peer's shared memory.
         cluster_arrive_relaxed();
     }
+    const int tid = threadIdx.x;
+    const int T = blockDim.x;
+    const uint32_t rank = CLUSTER ? cluster_rank() : 0u;
+    const int64_t row = CLUSTER ? (int64_t)(blockIdx.x / a.cluster) : (int64_t)blockIdx.x;
+    if (a.prefetch) {
+        // Ask L2 for this block's slice of every input, the residual and
+        // gamma while the previous kernel may still run: a hint that changes
+        // no value read after the wait, and the fetch from HBM overlaps that
+        // kernel's tail instead of following it.
+        const int pb = (int)rank * a.slice_vecs;
+        const int pn = min(a.slice_vecs, a.vecs - pb);
+        if (pn > 0) {
+            const int64_t off = row * (int64_t)a.vecs + pb;
+            const uint32_t bytes = (uint32_t)pn * 16u;
+            if (tid < a.R) prefetch_l2(a.in[tid] + off, bytes);
+            else if (RES && tid == a.R) prefetch_l2(a.res_in + off, bytes);
+            else if (tid == a.R + 1) prefetch_l2(a.gamma + pb, bytes);
+        }
+    }
     // With programmatic dependent launch this block may run ahead of the
     // previous kernel: wait for it before any global access, then let the
     // next kernel launch early (it waits for this grid the same way).
     wait_for_previous_grid();
     allow_next_grid();
 
-    const int tid = threadIdx.x;
-    const int T = blockDim.x;
-    const uint32_t rank = CLUSTER ? cluster_rank() : 0u;
-    const int64_t row = CLUSTER ? (int64_t)(blockIdx.x / a.cluster) : (int64_t)blockIdx.x;
-    const int v_begin = (int)rank * a.slice_vecs;
+    // Every address below derives from these two, taken after the wait.
+    const int v_begin = opaque((int)rank * a.slice_vecs);
     const int v_end = min(v_begin + a.slice_vecs, a.vecs);
-    const int64_t row_base = row * (int64_t)a.vecs;
+    const int64_t row_base = opaque(row * (int64_t)a.vecs);
     // One vector per thread keeps gamma in registers between the passes;
     // longer slices re-read it (an L1 hit) to save registers.
     constexpr bool KEEP_GAMMA = VPT == 1;
+    // Packed fp32 pairs (the scalar operations' bits in half the
+    // instructions) where a thread holds one vector: the decode-sized calls
+    // are bound by that chain (0.05-0.17 us per call less on B200).  With
+    // several vectors per thread (prefill rows) the scalar form measured
+    // faster (209 against 220-230 us at 8 x 8192 x 8192).
+    constexpr bool PACKED = VPT == 1;
 
     uint4 h[VPT];
     uint4 g[KEEP_GAMMA ? VPT : 1];
@@ -93,7 +136,7 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
         const int v = v_begin + tid + k * T;
-        if (v < v_end) {
+        if (v < v_end && RRF_IN_BOUNDS(v >= 0 && v < a.vecs && row < a.rows, a.err)) {
             uint4 x[RB];
 #pragma unroll
             for (int r = 0; r < RB; ++r)
@@ -103,17 +146,34 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
             const uint4 gv = ld_shared_by_all(a.gamma + v);
             if (KEEP_GAMMA) g[k] = gv;
 
-            float acc[8];
-            bf16x8_to_f32(x[0], acc);
+            uint4 s;
+            if constexpr (PACKED) {
+                float2 acc[4];
+                bf16x8_to_f32x2(x[0], acc);
 #pragma unroll
-            for (int r = 1; r < RB; ++r)
-                if (r < a.R) add_bf16x8(acc, x[r]);
-            uint4 s = f32_to_bf16x8(acc);
+                for (int r = 1; r < RB; ++r)
+                    if (r < a.R) add_bf16x8_x2(acc, x[r]);
+                s = f32x2_to_bf16x8(acc);
+            } else {
+                float acc[8];
+                bf16x8_to_f32(x[0], acc);
+#pragma unroll
+                for (int r = 1; r < RB; ++r)
+                    if (r < a.R) add_bf16x8(acc, x[r]);
+                s = f32_to_bf16x8(acc);
+            }
             if (RES) {
-                float t[8];
-                bf16x8_to_f32(s, t);
-                add_bf16x8(t, res);
-                s = f32_to_bf16x8(t);
+                if constexpr (PACKED) {
+                    float2 t[4];
+                    bf16x8_to_f32x2(s, t);
+                    add_bf16x8_x2(t, res);
+                    s = f32x2_to_bf16x8(t);
+                } else {
+                    float t[8];
+                    bf16x8_to_f32(s, t);
+                    add_bf16x8(t, res);
+                    s = f32_to_bf16x8(t);
+                }
                 // Cluster rows store the residual in the last pass, after the
                 // exchange: with the barrier exchange its release would
                 // otherwise wait for the store to land, and with either
@@ -125,22 +185,30 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
                 st_once(a.h_out + row_base + v, s);
             }
             h[k] = s;
-            st.ss += sumsq_bf16x8(s);
-            float hf[8], gf[8];
-            bf16x8_to_f32(s, hf);
-            bf16x8_to_f32(gv, gf);
-            if constexpr (MX) {
-                RowStats vs = stats_empty();
+            // max |h * g'| of the vector's 8 elements, g' = gamma + weight_offset
+            float vkey = 0.0f;
+            if constexpr (PACKED) {
+                float2 hf[4], gf[4];
+                bf16x8_to_f32x2(s, hf);
+                bf16x8_to_f32x2(gv, gf);
+                st.ss += sumsq_bf16x8_x2(hf);
+                const float2 wo2 = make_float2(a.weight_offset, a.weight_offset);
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    stats_offer(vs, hf[e], __fadd_rn(gf[e], a.weight_offset));
-                bkey[k] = vs.key;
-                st.key = fmaxf(st.key, vs.key);
+                for (int e = 0; e < 4; ++e) {
+                    const float2 p = __fmul2_rn(hf[e], __fadd2_rn(gf[e], wo2));
+                    vkey = fmaxf(vkey, fmaxf(fabsf(p.x), fabsf(p.y)));
+                }
             } else {
+                float hf[8], gf[8];
+                bf16x8_to_f32(s, hf);
+                bf16x8_to_f32(gv, gf);
+                st.ss += sumsq_bf16x8(s);
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
-                    stats_offer(st, hf[e], __fadd_rn(gf[e], a.weight_offset));
+                    vkey = fmaxf(vkey, fabsf(__fmul_rn(hf[e], __fadd_rn(gf[e], a.weight_offset))));
             }
+            if constexpr (MX) bkey[k] = vkey;
+            st.key = fmaxf(st.key, vkey);
         } else if constexpr (MX) {
             bkey[k] = 0.0f;
         }
@@ -156,24 +224,27 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
     }
 
     // ---- reduction of the statistics: block, then cluster
+    // (a block has at most 32 warps: their slots in warp_stats)
+    (void)RRF_IN_BOUNDS(blockDim.x <= 1024, a.err);
     st = block_stats(st, warp_stats);
     if (CLUSTER) {
+        // the cluster's slots: C <= 16 blocks, this block's slot inside them
+        // (a failed check leaves the exchange to run out its bounded wait)
+        (void)RRF_IN_BOUNDS(a.cluster <= 16 && rank < (uint32_t)a.cluster, a.err);
         cluster_wait_acquire();  // phase 0 done: every block of the cluster runs
         st = ASYNC ? cluster_stats_async(st, cluster_stats, &exchange_bar, rank, a.cluster, a.err)
                    : cluster_stats_combine(st, cluster_stats, rank, a.cluster);
     }
     if (a.stats_only) {
         // first phase of the sharded norm: this shard's row statistics
-        if (tid == 0 && rank == 0) a.stats[row] = make_float2(st.ss, st.key);
+        if (tid == 0 && rank == 0 && RRF_IN_BOUNDS(row < a.rows, a.err))
+            a.stats[row] = make_float2(st.ss, st.key);
         return;
     }
-    const float ms = st.ss / a.cols_f;
-    const float rinv = 1.0f / sqrtf(ms + a.eps);
     // max_j |y_j| = max_j |(h_j * r) * g'_j| = r * max_j |h_j * g'_j| up to the
-    // order of the two roundings.
-    const float amax = __fmul_rn(st.key, rinv);
-    const float scale = fmaxf(fminf(amax, a.scale_ub), kScaleFloor) / kE4m3Max;
-    const float inv_scale = 1.0f / scale;
+    // order of the two roundings (row_scale)
+    const RowScale rs = row_scale(st.ss, st.key, a.inv_cols, a.eps, a.scale_ub);
+    const float rinv = rs.rinv, scale = rs.scale, inv_scale = rs.inv_scale;
 
     // ---- last pass: quantise
     if constexpr (MX) {
@@ -182,19 +253,13 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
 #pragma unroll
         for (int k = 0; k < VPT; ++k) {
             const int v = v_begin + tid + k * T;
-            if (v < v_end) {
+            if (v < v_end && RRF_IN_BOUNDS(v >= 0 && v < a.vecs && row < a.rows, a.err)) {
                 const uint32_t code = mx_scale_code(__fmul_rn(bkey[k], rinv));
                 const float inv_x = __uint_as_float((254u - code) << 23);  // 2^(127 - code)
-                float hf[8], gf[8], qv[8];
-                bf16x8_to_f32(h[k], hf);
-                bf16x8_to_f32(KEEP_GAMMA ? g[k] : ld_shared_by_all(a.gamma + v), gf);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float y =
-                        __fmul_rn(__fmul_rn(hf[e], rinv), __fadd_rn(gf[e], a.weight_offset));
-                    qv[e] = __fmul_rn(y, inv_x);
-                }
-                st_once(a.q + row_base + v, f32_to_e4m3x8(qv));
+                st_once(a.q + row_base + v,
+                        quantise_vector<PACKED>(h[k],
+                                                KEEP_GAMMA ? g[k] : ld_shared_by_all(a.gamma + v),
+                                                rinv, a.weight_offset, inv_x));
                 if ((v & 3) == 0) {
                     // row-major [rows, cols / 32], or the tensor cores' blocked
                     // order (512-byte atoms of 128 rows x 4 blocks)
@@ -204,7 +269,12 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
                             ? ((row >> 7) * (a.vecs >> 4) + (j >> 2)) * 512 + (row & 31) * 16 +
                                   ((row >> 5) & 3) * 4 + (j & 3)
                             : (row_base + v) >> 2;
-                    a.scales_mx[off] = (uint8_t)code;
+                    // (the scale buffer: rows, or rows rounded up to 128, of cols / 32)
+                    if (RRF_IN_BOUNDS(off >= 0 && off < (a.mx_blocked ? (a.rows + 127) / 128 * 128
+                                                                      : a.rows) *
+                                                             (a.vecs >> 2),
+                                      a.err))
+                        a.scales_mx[off] = (uint8_t)code;
                 }
                 if (RES && CLUSTER) st_once(a.res_out + row_base + v, h[k]);
             }
@@ -213,21 +283,15 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
 #pragma unroll
         for (int k = 0; k < VPT; ++k) {
             const int v = v_begin + tid + k * T;
-            if (v < v_end) {
-                float hf[8], gf[8], qv[8];
-                bf16x8_to_f32(h[k], hf);
-                bf16x8_to_f32(KEEP_GAMMA ? g[k] : ld_shared_by_all(a.gamma + v), gf);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float y =
-                        __fmul_rn(__fmul_rn(hf[e], rinv), __fadd_rn(gf[e], a.weight_offset));
-                    qv[e] = __fmul_rn(y, inv_scale);
-                }
-                st_once(a.q + row_base + v, f32_to_e4m3x8(qv));
+            if (v < v_end && RRF_IN_BOUNDS(v >= 0 && v < a.vecs && row < a.rows, a.err)) {
+                st_once(a.q + row_base + v,
+                        quantise_vector<PACKED>(h[k],
+                                                KEEP_GAMMA ? g[k] : ld_shared_by_all(a.gamma + v),
+                                                rinv, a.weight_offset, inv_scale));
                 if (RES && CLUSTER) st_once(a.res_out + row_base + v, h[k]);
             }
         }
-        if (tid == 0 && rank == 0) a.scales[row] = scale;
+        if (tid == 0 && rank == 0 && RRF_IN_BOUNDS(row < a.rows, a.err)) a.scales[row] = scale;
     }
 }
 

@@ -4,14 +4,14 @@
 // aclnnAlltoAllQuantMatmul: per-token dynamic quantisation of the
 // activations, then (x1_q @ x2) * x1Scale * x2Scale + bias).
 //
-// Kernels (launch_scaled_mm and launch_scaled_mm_mx choose by shape):
+// Kernels (plan_scaled_mm chooses by shape; the launchers follow its plan):
 //   scaled_mm_pair_kernel / scaled_mm_mx_pair_kernel  256 x 256 tiles on SM
 //            pairs (tcgen05.mma.cta_group::2) for products that fill every pair;
 //   scaled_mm_kernel / scaled_mm_mx_kernel  persistent CTAs on 128 x BN tiles
-//            (BN 256, 128 or 64), Z k-tiles per TMA box for short products;
+//            (BN 128 or 64), Z k-tiles per TMA box for short products;
 //   scaled_mm_swap_kernel  at most 32 rows against a weight, the operands
 //            swapped (the weight's rows on the MMA's M = 64 side).
-// A persistent CTA per SM walks 128 x BN tiles of out (BN 256, 128 or 64).
+// A persistent CTA per SM walks 128 x BN tiles of out (BN 128 or 64).
 // Warp roles (the same in every kernel):
 //   warp 0   one thread issues the TMA loads of the A (128 x 128 bytes) and
 //            B (BN x 128 bytes) k-tiles into a ring of shared-memory stages
@@ -185,6 +185,7 @@ __host__ __device__ constexpr uint32_t f8_idesc(int bn) {
 // 32 columns valid: N % 16 == 0).
 __device__ __forceinline__ void store_row_chunk(const GemmArgs& g, const float v[32], float sa,
                                                 int row, int n) {
+    if (!RRF_IN_BOUNDS(row >= 0 && row < g.M && n >= 0 && n < g.N, g.err)) return;
     const int valid = g.N - n < 32 ? g.N - n : 32;
     uint32_t packed[16];
 #pragma unroll
@@ -319,6 +320,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    // Programmatic dependent launch: the set-up above overlapped the previous
+    // kernel of the stream; the operands, scales and output are touched only
+    // after that kernel has completed.  (Measured on B200 at 1-64 x 7168 x
+    // 7168: 0.4-0.6 us per call faster than a plain launch; an L2 prefetch of
+    // the CTA's weight tile before the wait made the same calls 2 us slower
+    // and was dropped.)
+    wait_for_previous_grid();
+    allow_next_grid();
 
     if (warp == 0) {
         // ---- producer: TMA loads of every k-tile of every tile of this CTA
@@ -447,7 +456,9 @@ struct SwapTile {
     static constexpr int kStages =
         (220 * 1024) / kStageBytes > 12 ? 12 : (220 * 1024) / kStageBytes;
     // two accumulators of NA columns, each at least 32 wide (the epilogue
-    // reads 32 columns at a time); a power of two of at least 32
+    // reads 32 columns at a time); a power of two of at least 32.  (Spreading
+    // a tile's MMAs over 4 accumulators summed in the epilogue, to break the
+    // chain of dependent updates, measured 2 us slower at 1-32 x 7168 x 7168.)
     static constexpr int kAccStride = NA < 32 ? 32 : NA;
     static constexpr int kTmemCols = 2 * kAccStride;
     static constexpr int kBarriers = 2 * kStages + 4 + 1;
@@ -497,6 +508,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    // Programmatic dependent launch (see scaled_mm_kernel).
+    wait_for_previous_grid();
+    allow_next_grid();
 
     if (warp == 0) {
         // ---- producer: Z k-tiles of the weight tile and of the call's rows
@@ -581,7 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int m = c + i;
-                    if (m < NA && m < g.M) {
+                    if (m < NA && m < g.M && RRF_IN_BOUNDS(n >= 0 && n < g.N, g.err)) {
                         float y = __fmul_rn(__fmul_rn(v[i], __ldg(g.a_scale + m)), sb);
                         if (g.bias != nullptr) y = __fadd_rn(y, bias);
                         // one rounding to bf16 (the low half of the packed pair)
@@ -746,6 +760,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     cluster_wait_acquire();
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    // Programmatic dependent launch (see scaled_mm_kernel).
+    wait_for_previous_grid();
+    allow_next_grid();
 
     if (warp == 0) {
         // ---- producer (each CTA): its 128 rows of A and of B per k-tile
@@ -986,6 +1003,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    // Programmatic dependent launch (see scaled_mm_kernel).
+    wait_for_previous_grid();
+    allow_next_grid();
     const uint32_t tmem_sfa = tmem + T::kAccCols, tmem_sfb = tmem + T::kAccCols + 4;
 
     if (warp == 0) {
@@ -1224,6 +1244,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     cluster_wait_acquire();
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    // Programmatic dependent launch (see scaled_mm_kernel).
+    wait_for_previous_grid();
+    allow_next_grid();
 
     if (warp == 0) {
         // ---- producer (each CTA): its 128 rows of A and of B, its A scale
@@ -1397,11 +1420,31 @@ cudaError_t launch_on_pairs(void (*kernel)(Params...), int64_t pairs, int smem_b
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem_bytes;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// One CTA per SM (at most `ctas`), launched with programmatic dependent
+// launch: the kernel's set-up may overlap the previous kernel of the stream.
+template <class... Params, class... Args>
+cudaError_t launch_persistent(void (*kernel)(Params...), unsigned ctas, int smem_bytes,
+                              cudaStream_t stream, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(ctas, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem_bytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kernel, args...);
@@ -1474,8 +1517,7 @@ cudaError_t launch_bn(const GemmArgs& g, const void* a, const void* b, int sm_co
     if (e != cudaSuccess) return e;
     const int64_t tiles = (int64_t)((g.N + BN - 1) / BN) * ((g.M + kBM - 1) / kBM);
     const unsigned grid = (unsigned)(tiles < sm_count ? tiles : sm_count);  // one CTA per SM
-    kernel<<<grid, kThreads, T::kSmemBytes, stream>>>(ma, mb, g);
-    return cudaGetLastError();
+    return launch_persistent(kernel, grid, T::kSmemBytes, stream, ma, mb, g);
 }
 
 template <int NA, int Z>
@@ -1490,8 +1532,7 @@ cudaError_t launch_swap(const GemmArgs& g, const void* a, const void* b, int sm_
     if (e != cudaSuccess) return e;
     const int64_t tiles = (g.N + T::kWRows - 1) / T::kWRows;
     const unsigned grid = (unsigned)(tiles < sm_count ? tiles : sm_count);
-    kernel<<<grid, kThreads, T::kSmemBytes, stream>>>(mx, mw, g);
-    return cudaGetLastError();
+    return launch_persistent(kernel, grid, T::kSmemBytes, stream, mx, mw, g);
 }
 
 cudaError_t launch_pair(const GemmArgs& g, const void* a, const void* b, int sm_count,
@@ -1518,8 +1559,7 @@ cudaError_t launch_mx(const GemmArgs& g, const void* a, const void* b, const uin
     if (e != cudaSuccess) return e;
     const int64_t tiles = (int64_t)((g.N + BN - 1) / BN) * ((g.M + kBM - 1) / kBM);
     const unsigned grid = (unsigned)(tiles < sm_count ? tiles : sm_count);
-    kernel<<<grid, kThreads, T::kSmemBytes, stream>>>(ma, mb, g, sfa, sfb);
-    return cudaGetLastError();
+    return launch_persistent(kernel, grid, T::kSmemBytes, stream, ma, mb, g, sfa, sfb);
 }
 
 cudaError_t launch_mx_pair(const GemmArgs& g, const void* a, const void* b, const uint8_t* sfa,
@@ -1539,53 +1579,92 @@ cudaError_t launch_mx_pair(const GemmArgs& g, const void* a, const void* b, cons
 
 }  // namespace
 
+GemmPlan plan_scaled_mm(int64_t M, int64_t N, int64_t K, bool mx, int sm_count) {
+    auto tile = [&](int kernel, int arows, int bn, int z) {
+        GemmPlan p;
+        p.kernel = kernel;
+        p.a_rows = arows;
+        p.tile_n = bn;
+        p.k_tiles_per_stage = z;
+        if (kernel == kGemmPair) {
+            p.tiles = ((M + 255) / 256) * ((N + 255) / 256);
+            const int64_t pairs = p.tiles < sm_count / 2 ? p.tiles : sm_count / 2;
+            p.ctas = 2 * pairs;
+        } else {
+            // the swapped kernel's tiles are 64 weight rows by all the call's rows
+            p.tiles = kernel == kGemmSwap ? (N + 63) / 64 : ((N + bn - 1) / bn) * ((M + kBM - 1) / kBM);
+            p.ctas = p.tiles < sm_count ? p.tiles : sm_count;  // one CTA per SM
+        }
+        return p;
+    };
+    const int64_t row_tiles = (M + kBM - 1) / kBM;
+    // large products: 256 x 256 tiles on SM pairs once they fill every pair
+    if (((M + 255) / 256) * ((N + 255) / 256) >= sm_count / 2) return tile(kGemmPair, 256, 256, 1);
+    if (mx) {
+        // else one CTA per 128 x 128 tile once those fill every SM; short, wide
+        // problems take 128 x 64 tiles (A stages of the call's rows, up to 64)
+        if (row_tiles * ((N + 127) / 128) >= sm_count) return tile(kGemmTile, kBM, 128, 1);
+        // (K % 128 == 0 here: several k-tiles per TMA box, as the per-token GEMM;
+        // no swapped operands: the block-scaled MMA of one CTA has no M = 64 form)
+        // 8 k-tiles per stage up to 16 rows (2 stages; measured 7% faster than 4
+        // at 8 rows, 2 k-tiles slower)
+        if (M <= 8) return tile(kGemmTile, 8, 64, 8);
+        if (M <= 16) return tile(kGemmTile, 16, 64, 8);
+        if (M <= 32) return tile(kGemmTile, 32, 64, 4);
+        if (M <= 64) return tile(kGemmTile, 64, 64, 4);
+        return tile(kGemmTile, kBM, 64, 2);
+    }
+    // One CTA per 128 x 128 tile once those fill every SM (a 128 x 256 tile
+    // never would: ceil(M/128) * ceil(N/256) <= 2 * ceil(M/256) * ceil(N/256),
+    // which is below the SM count whenever the pairs are not all busy); short,
+    // wide problems (decode batches against a weight) take 64-column tiles,
+    // the most CTAs streaming the weight.
+    if (row_tiles * ((N + 127) / 128) >= sm_count) return tile(kGemmTile, kBM, 128, 1);
+    // the weight-streaming shapes: several k-tiles per TMA box where K allows
+    const bool atoms = K % kBK == 0;
+    if (M <= 64 && !atoms) return tile(kGemmTile, 64, 64, 1);
+    // at most 32 rows: the operands swapped, the call's rows padded to 8, 16
+    // or 32 (at 64 the swapped MMA is no cheaper: measured slower); 8 k-tiles
+    // per box up to 16 rows (measured faster than 4 or 2 there; equal at 32)
+    if (M <= 8) return tile(kGemmSwap, 8, 64, 8);
+    if (M <= 16) return tile(kGemmSwap, 16, 64, 8);
+    if (M <= 32) return tile(kGemmSwap, 32, 64, 4);
+    if (M <= 64) return tile(kGemmTile, 64, 64, 4);
+    return tile(kGemmTile, kBM, 64, atoms ? 2 : 1);
+}
+
 cudaError_t launch_scaled_mm_mx(const GemmArgs& g, const void* a, const void* b,
                                 const uint8_t* sfa, const uint8_t* sfb, int sm_count,
                                 cudaStream_t stream) {
-    // 256 x 256 tiles on SM pairs once they fill every pair, as the
-    // per-token GEMM
-    if (((g.M + 255) / 256) * ((g.N + 255) / 256) >= sm_count / 2)
-        return launch_mx_pair(g, a, b, sfa, sfb, sm_count, stream);
-    // else one CTA per 128 x 128 tile once those fill every SM; short, wide
-    // problems take 128 x 64 tiles (64-row A stages for at most 64 rows)
-    if (((g.M + kBM - 1) / kBM) * ((g.N + 127) / 128) >= sm_count)
-        return launch_mx<128, kBM, 1>(g, a, b, sfa, sfb, sm_count, stream);
-    // (K % 128 == 0 here: several k-tiles per TMA box, as the per-token GEMM;
-    // no swapped operands: the block-scaled MMA of one CTA has no M = 64 form)
-    // 8 k-tiles per stage up to 16 rows (2 stages; measured 7% faster than 4
-    // at 8 rows, 2 k-tiles slower)
-    if (g.M <= 8) return launch_mx<64, 8, 8>(g, a, b, sfa, sfb, sm_count, stream);
-    if (g.M <= 16) return launch_mx<64, 16, 8>(g, a, b, sfa, sfb, sm_count, stream);
-    if (g.M <= 32) return launch_mx<64, 32, 4>(g, a, b, sfa, sfb, sm_count, stream);
-    if (g.M <= 64) return launch_mx<64, 64, 4>(g, a, b, sfa, sfb, sm_count, stream);
-    return launch_mx<64, kBM, 2>(g, a, b, sfa, sfb, sm_count, stream);
+    const GemmPlan p = plan_scaled_mm(g.M, g.N, g.K, true, sm_count);
+    if (p.kernel == kGemmPair) return launch_mx_pair(g, a, b, sfa, sfb, sm_count, stream);
+    if (p.tile_n == 128) return launch_mx<128, kBM, 1>(g, a, b, sfa, sfb, sm_count, stream);
+    switch (p.a_rows) {
+        case 8: return launch_mx<64, 8, 8>(g, a, b, sfa, sfb, sm_count, stream);
+        case 16: return launch_mx<64, 16, 8>(g, a, b, sfa, sfb, sm_count, stream);
+        case 32: return launch_mx<64, 32, 4>(g, a, b, sfa, sfb, sm_count, stream);
+        case 64: return launch_mx<64, 64, 4>(g, a, b, sfa, sfb, sm_count, stream);
+        default: return launch_mx<64, kBM, 2>(g, a, b, sfa, sfb, sm_count, stream);
+    }
 }
 
 cudaError_t launch_scaled_mm(const GemmArgs& g, const void* a, const void* b, int sm_count,
                              cudaStream_t stream) {
-    // The widest tile that still gives every SM a tile; short, wide
-    // problems (decode batches against a weight) take 128 x 64 tiles, the
-    // most CTAs streaming the weight.
-    const int64_t row_tiles = (g.M + kBM - 1) / kBM;
-    // large products: 256 x 256 tiles on SM pairs once they fill every pair
-    if (((g.M + 255) / 256) * ((g.N + 255) / 256) >= sm_count / 2)
-        return launch_pair(g, a, b, sm_count, stream);
-    if (row_tiles * ((g.N + 255) / 256) >= sm_count)
-        return launch_bn<256, kBM, 1>(g, a, b, sm_count, stream);
-    if (row_tiles * ((g.N + 127) / 128) >= sm_count)
-        return launch_bn<128, kBM, 1>(g, a, b, sm_count, stream);
-    // the weight-streaming shapes: several k-tiles per TMA box where K allows
-    const bool atoms = g.K % kBK == 0;
-    if (g.M <= 64 && !atoms) return launch_bn<64, 64, 1>(g, a, b, sm_count, stream);
-    // at most 32 rows: the operands swapped, the call's rows padded to 8, 16
-    // or 32 (at 64 the swapped MMA is no cheaper: measured slower); 8 k-tiles
-    // per box up to 16 rows (measured faster than 4 or 2 there; equal at 32)
-    if (g.M <= 8) return launch_swap<8, 8>(g, a, b, sm_count, stream);
-    if (g.M <= 16) return launch_swap<16, 8>(g, a, b, sm_count, stream);
-    if (g.M <= 32) return launch_swap<32, 4>(g, a, b, sm_count, stream);
-    if (g.M <= 64) return launch_bn<64, 64, 4>(g, a, b, sm_count, stream);
-    return atoms ? launch_bn<64, kBM, 2>(g, a, b, sm_count, stream)
-                 : launch_bn<64, kBM, 1>(g, a, b, sm_count, stream);
+    const GemmPlan p = plan_scaled_mm(g.M, g.N, g.K, false, sm_count);
+    if (p.kernel == kGemmPair) return launch_pair(g, a, b, sm_count, stream);
+    if (p.kernel == kGemmSwap) {
+        switch (p.a_rows) {
+            case 8: return launch_swap<8, 8>(g, a, b, sm_count, stream);
+            case 16: return launch_swap<16, 8>(g, a, b, sm_count, stream);
+            default: return launch_swap<32, 4>(g, a, b, sm_count, stream);
+        }
+    }
+    if (p.tile_n == 128) return launch_bn<128, kBM, 1>(g, a, b, sm_count, stream);
+    if (p.a_rows == 64)
+        return p.k_tiles_per_stage == 4 ? launch_bn<64, 64, 4>(g, a, b, sm_count, stream)
+                                        : launch_bn<64, 64, 1>(g, a, b, sm_count, stream);
+    return p.k_tiles_per_stage == 2 ? launch_bn<64, kBM, 2>(g, a, b, sm_count, stream)
+                                    : launch_bn<64, kBM, 1>(g, a, b, sm_count, stream);
 }
 
 }  // namespace rrf

@@ -29,7 +29,7 @@ struct FusedArgs {
     int vecs;              // cols / 8 (vectors per row)
     int slice_vecs;        // vectors per block of a row's cluster: ceil(vecs / C)
     int cluster;           // C, blocks per row (1 = no cluster)
-    float cols_f;          // cols as fp32, the mean's divisor
+    float inv_cols;        // 1 / cols rounded to fp32: the mean square is sum * inv_cols
     float eps;
     float weight_offset;
     float scale_ub;
@@ -44,6 +44,8 @@ struct FusedArgs {
     // MX output: one E8M0 scale code per 32 elements instead of scales
     uint8_t* scales_mx;    // [rows, cols / 32], or blocked (mx_blocked)
     int mx_blocked;        // scales in the block-scaled MMA's 512-byte atom order
+    int prefetch;          // prefetch the block's slice into L2 before the PDL wait
+    int64_t rows;          // rows of the call (the bounds-checking build's limit)
 };
 
 // The second phase of the sharded norm: quantise one column shard from the
@@ -57,10 +59,11 @@ struct PostArgs {
     int64_t rows;
     int vecs;              // cols / 8
     int shards;
-    float total_cols_f;    // columns of the whole row (all shards), the mean's divisor
+    float inv_total_cols;  // 1 / (columns of the whole row, all shards), rounded to fp32
     float eps;
     float weight_offset;
     float scale_ub;
+    unsigned int* err;     // the library's device error word
 };
 
 // The multi-GPU form (rrf_allreduce.cu).  Pointer arrays are indexed by rank
@@ -83,7 +86,7 @@ struct ArArgs {
     int vecs;
     int slice_vecs;
     int cluster;
-    float cols_f;
+    float inv_cols;        // 1 / cols rounded to fp32
     float eps;
     float weight_offset;
     float scale_ub;
@@ -124,6 +127,7 @@ struct FusedLaunch {
     bool pdl;             // launch with programmatic stream serialization
     bool async_exchange;  // clusters meet through st.async + mbarrier waits
     bool mx = false;      // MX output (per-32-element scales)
+    bool prefetch = false;  // L2 prefetch of each block's slice before the PDL wait
 };
 
 // The fused kernel is compiled for input-count bounds RB in {2, 4, 8, 16}
@@ -160,6 +164,24 @@ cudaError_t launch_fused(const FusedArgs& a, int64_t rows, const FusedLaunch& l,
 cudaError_t launch_post(const PostArgs& a, int sm_count, bool pdl, cudaStream_t stream);
 
 cudaError_t launch_allreduce(const ArArgs& a, const ArLaunch& l, cudaStream_t stream);
+// The GEMM kernel a shape takes (pure host arithmetic; the launchers follow
+// it).  kernel: kGemmPair (256 x 256 tiles on SM pairs), kGemmTile (a
+// persistent CTA per SM walking a_rows-row A stages of 128 x tile_n tiles)
+// or kGemmSwap (operands swapped: 64 weight rows on the MMA's M side, the
+// call's rows padded to a_rows on its N side); k_tiles_per_stage k-tiles of
+// 128 per TMA box; tiles output tiles over ctas CTAs.
+constexpr int kGemmPair = RRF_GEMM_KERNEL_PAIR;
+constexpr int kGemmTile = RRF_GEMM_KERNEL_TILE;
+constexpr int kGemmSwap = RRF_GEMM_KERNEL_SWAP;
+struct GemmPlan {
+    int kernel;
+    int a_rows;
+    int tile_n;
+    int k_tiles_per_stage;
+    int64_t tiles;
+    int64_t ctas;
+};
+GemmPlan plan_scaled_mm(int64_t M, int64_t N, int64_t K, bool mx, int sm_count);
 cudaError_t launch_scaled_mm(const GemmArgs& g, const void* a, const void* b, int sm_count,
                              cudaStream_t stream);
 // The MX GEMM: sfa / sfb are the scale codes in the blocked order; g.a_scale

@@ -40,8 +40,9 @@ __global__ void __launch_bounds__(kPostThreads) post_kernel(const PostArgs a, in
     allow_next_grid();
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t row0 = (int64_t)(blockIdx.x / chunks) * RB;
-    const int v0 = (int)(blockIdx.x % chunks) * kPostChunkVecs;
+    // every address derives from these two, taken after the wait
+    const int64_t row0 = opaque((int64_t)(blockIdx.x / chunks) * RB);
+    const int v0 = opaque((int)(blockIdx.x % chunks) * kPostChunkVecs);
     const int64_t left = a.rows - row0;
     const int nrows = left < RB ? (int)left : RB;
 
@@ -60,13 +61,18 @@ __global__ void __launch_bounds__(kPostThreads) post_kernel(const PostArgs a, in
 #pragma unroll
         for (int j = 0; j < kPostVecsPerLane; ++j) {
             const int v = v0 + lane + 32 * j;
-            if (r < nrows && v < a.vecs) hv[k][j] = ld_once(a.h + (row0 + r) * a.vecs + v);
+            if (r < nrows && v < a.vecs &&
+                RRF_IN_BOUNDS(row0 + r < a.rows && v >= 0, a.err))
+                hv[k][j] = ld_once(a.h + (row0 + r) * a.vecs + v);
         }
     }
     // the statistics of the block's rows, coalesced per shard
     for (int i = tid; i < a.shards * RB; i += kPostThreads) {
         const int s = i / RB, r = i % RB;
-        stage[i] = r < nrows ? a.stats[(int64_t)s * a.rows + row0 + r] : make_float2(0.0f, 0.0f);
+        if (!RRF_IN_BOUNDS(i < RRF_MAX_SHARDS * RB, a.err)) break;  // the stage's size
+        stage[i] = r < nrows && RRF_IN_BOUNDS(row0 + r < a.rows, a.err)
+                       ? a.stats[(int64_t)s * a.rows + row0 + r]
+                       : make_float2(0.0f, 0.0f);
     }
     __syncthreads();
     if (tid < nrows) {
@@ -76,12 +82,11 @@ __global__ void __launch_bounds__(kPostThreads) post_kernel(const PostArgs a, in
             ss = ss + p.x;
             key = fmaxf(key, p.y);
         }
-        const float ms = ss / a.total_cols_f;
-        const float rinv = 1.0f / sqrtf(ms + a.eps);
-        const float amax = __fmul_rn(key, rinv);
-        const float scale = fmaxf(fminf(amax, a.scale_ub), 1e-12f) / 448.0f;
-        rowval[tid] = make_float3(rinv, scale, 1.0f / scale);
-        if (v0 == 0 && a.scales != nullptr) a.scales[row0 + tid] = scale;
+        const RowScale rs = row_scale(ss, key, a.inv_total_cols, a.eps, a.scale_ub);
+        const float scale = rs.scale;
+        rowval[tid] = make_float3(rs.rinv, scale, rs.inv_scale);
+        if (v0 == 0 && a.scales != nullptr && RRF_IN_BOUNDS(row0 + tid < a.rows, a.err))
+            a.scales[row0 + tid] = scale;
     }
     __syncthreads();
 
@@ -93,7 +98,7 @@ __global__ void __launch_bounds__(kPostThreads) post_kernel(const PostArgs a, in
 #pragma unroll
         for (int j = 0; j < kPostVecsPerLane; ++j) {
             const int v = v0 + lane + 32 * j;
-            if (v < a.vecs) {
+            if (v < a.vecs && RRF_IN_BOUNDS(row0 + r < a.rows && v >= 0, a.err)) {
                 float hf[8], gf[8], qv[8];
                 bf16x8_to_f32(hv[k][j], hf);
                 bf16x8_to_f32(gv[j], gf);

@@ -18,7 +18,9 @@ __global__ void __launch_bounds__(256) sum_kernel(const SumArgs a) {
     wait_for_previous_grid();  // see rrf_device.cuh: programmatic dependent launch
     allow_next_grid();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < a.n_vecs; i += stride) {
+    // every address derives from the first index, taken after the wait
+    const int64_t first = opaque((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+    for (int64_t i = first; i < a.n_vecs; i += stride) {
         uint4 x[RB];
 #pragma unroll
         for (int r = 0; r < RB; ++r)

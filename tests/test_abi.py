@@ -174,25 +174,60 @@ def test_sum_validation(rrf):
 
 # -------------------------------------------------------------- planner ---
 
-@pytest.mark.parametrize("R,rows,cols,res,want", [
-    (8, 8192, 8192, True, (1, 512, 2)),   # prefill: one block per row
-    (8, 1, 7168, True, (8, 128, 1)),      # decode: clusters of 8
-    (8, 8, 7168, True, (8, 128, 1)),
-    (8, 32, 7168, True, (8, 128, 1)),
-    (8, 64, 7168, True, (8, 128, 1)),
-    (4, 37, 7168, True, (8, 128, 1)),
-    (4, 16, 4096, False, (1, 512, 1)),    # 37 KB rows: one block streams a row
-    (4, 64, 4096, False, (1, 512, 1)),
-    (4, 256, 4096, False, (1, 512, 1)),
-    (2, 4, 256, False, (1, 32, 1)),       # too short to split
-    (4, 1, 8, False, (1, 32, 1)),
-    (4, 4, 262144, True, (8, 512, 8)),    # the longest row: 8 blocks of 512 x 8
-    (16, 1, 262144, True, (16, 512, 4)),  # with 16 inputs: 16 blocks of 512 x 4
-])
-def test_plan(rrf, R, rows, cols, res, want):
-    """The planner's choices for the workloads' shapes: the fastest launch of
-    the B200 sweeps that fitted its cost model."""
-    assert rrf.rrf_plan_fused(R, rows, cols, 148, residual=res) == want
+TABLE = os.path.join(ROOT, "reduce_rmsnorm_fp8_b200", "csrc", "rrf_plan_table.inc")
+
+
+def plan_table():
+    """The entries of the launch table compiled into the library:
+    (input bound, residual, cols, rows, cluster, prefetch, us)."""
+    text = re.sub(r"//.*", "", open(TABLE).read())
+    return [tuple(float(v) if "." in v else int(v) for v in m.replace("f", "").split(","))
+            for m in re.findall(r"RRF_PLAN\(([^)]*)\)", text)]
+
+
+def test_plan_table_is_measured_and_covers_the_grid():
+    """The table holds the sweep's grid: every input bound with and without
+    a residual, the workloads' row lengths and batch sizes."""
+    entries = plan_table()
+    assert entries, "no launch sweep recorded in rrf_plan_table.inc"
+    keys = {(e[0], e[1], e[2], e[3]) for e in entries}
+    assert len(keys) == len(entries)  # one entry per shape
+    for rb in (2, 4, 8, 16):
+        for res in (0, 1):
+            assert any(k[0] == rb and k[1] == res for k in keys), (rb, res)
+    for rb, res, cols, rows in ((8, 1, 7168, 1), (8, 1, 7168, 8), (8, 1, 7168, 32),
+                                (8, 1, 7168, 64), (4, 1, 7168, 37), (4, 1, 7168, 64),
+                                (2, 0, 1024, 4), (8, 1, 8192, 8192)):
+        assert (rb, res, cols, rows) in keys, (rb, res, cols, rows)
+    for e in entries:
+        assert 1 <= e[4] <= 16 and e[5] in (0, 1) and e[6] > 0
+
+
+def test_plan_follows_the_table(rrf):
+    """For every shape of the table the planner takes the launch measured
+    fastest there (cluster size and L2 prefetch)."""
+    for rb, res, cols, rows, cluster, prefetch, _ in plan_table():
+        c, t, v, p = rrf.rrf_plan_fused_ex(rb, rows, cols, 148, residual=bool(res))
+        assert (c, p) == (cluster, prefetch), (rb, res, cols, rows)
+        assert c * t * v * 8 >= cols
+
+
+def test_plan_takes_the_nearest_entry(rrf):
+    """Shapes between the table's: the entry of the same input bound and
+    residual flag nearest in log2(cols) (weighted 4x) + log2(rows)."""
+    import math
+    entries = plan_table()
+    for R, rows, cols, res in ((3, 5, 7168, True), (6, 40, 6144, False), (12, 300, 12288, True),
+                               (8, 100, 7168, True), (1, 3000, 1536, False)):
+        rb = 2 if R <= 2 else 4 if R <= 4 else 8 if R <= 8 else 16
+        cands = [e for e in entries if e[0] == rb and e[1] == int(res)]
+        best = min(cands, key=lambda e: 4 * abs(math.log2(cols / e[2])) +
+                   abs(math.log2(rows / e[3])))
+        c, t, v, p = rrf.rrf_plan_fused_ex(R, rows, cols, 148, residual=res)
+        want = best[4]
+        while want > 1 and cols // 8 // want < 32:
+            want -= 1
+        assert (c, p) == (want, best[5]), (R, rows, cols, res, c, best)
 
 
 def test_plan_covers_every_row(rrf):
@@ -200,7 +235,7 @@ def test_plan_covers_every_row(rrf):
         for cols in (8, 256, 2880, 7168, 7176, 8192, 8200, 16384, 131072, 262144):
             for rows in (1, 37, 4096):
                 c, t, v = rrf.rrf_plan_fused(R, rows, cols, 148)
-                assert c in (1, 2, 4, 8, 16) and 32 <= t <= 1024 and t % 32 == 0
+                assert 1 <= c <= 16 and 32 <= t <= 1024 and t % 32 == 0
                 assert v in (1, 2, 4, 8)
                 assert c * t * v * 8 >= cols, (R, rows, cols)
 
@@ -464,3 +499,48 @@ def test_mx_blocked_rejects_partial_atoms(rrf):
     import torch
     with pytest.raises(ValueError):
         rrf.mx_blocked(torch.zeros((4, 6), dtype=torch.uint8))
+
+
+@pytest.mark.parametrize("M,N,K,mx,want", [
+    (8, 16384, 7168, False, ("swap", 8, 64, 8, 256, 148)),
+    (16, 16384, 1024, False, ("swap", 16, 64, 8, 256, 148)),
+    (32, 16384, 7168, False, ("swap", 32, 64, 4, 256, 148)),
+    (64, 16384, 7168, False, ("tile", 64, 64, 4, 256, 148)),
+    (8, 16384, 1040, False, ("tile", 64, 64, 1, 256, 148)),   # K % 128 != 0: 2-D boxes
+    (100, 16384, 1024, False, ("tile", 128, 64, 2, 256, 148)),
+    (64, 7168, 7168, False, ("tile", 64, 64, 4, 112, 112)),
+    (2048, 2048, 512, False, ("tile", 128, 128, 1, 256, 148)),
+    (8192, 8192, 8192, False, ("pair", 256, 256, 1, 1024, 148)),
+    (8, 16384, 1024, True, ("tile", 8, 64, 8, 256, 148)),
+    (64, 16384, 7168, True, ("tile", 64, 64, 4, 256, 148)),
+    (100, 16384, 1024, True, ("tile", 128, 64, 2, 256, 148)),
+    (2048, 2048, 512, True, ("tile", 128, 128, 1, 256, 148)),
+    (8192, 8192, 8192, True, ("pair", 256, 256, 1, 1024, 148))])
+def test_gemm_plan(rrf, M, N, K, mx, want):
+    """The host-side GEMM plan on 148 SMs: the kernel a shape takes and how
+    many output tiles its CTAs walk (ctas < tiles: several per CTA)."""
+    p = rrf.rrf_plan_scaled_mm(M, N, K, 148, mx=mx)
+    assert (p["kernel"], p["a_rows"], p["tile_n"], p["k_tiles_per_stage"], p["tiles"],
+            p["ctas"]) == want
+
+
+def test_gemm_plan_invariants_and_rejections(rrf):
+    for M in (1, 7, 8, 9, 31, 33, 64, 65, 129, 300, 1000, 4096):
+        for N in (16, 256, 1024, 7168, 16384):
+            for K in (128, 1024, 7168):
+                for mx in (False, True):
+                    p = rrf.rrf_plan_scaled_mm(M, N, K, 148, mx=mx)
+                    assert 1 <= p["ctas"] <= min(p["tiles"] * (2 if p["kernel"] == "pair" else 1),
+                                                 148)
+                    assert p["kernel"] != "swap" or (not mx and M <= p["a_rows"] <= 32)
+                    if p["kernel"] == "pair":
+                        assert p["ctas"] % 2 == 0
+    p = rrf.rrf_plan_scaled_mm(0, 256, 256, 148)
+    assert (p["kernel"], p["tiles"], p["ctas"]) == (None, 0, 0)
+    for args, status in [((8, 8, 128, 148), "ERR_SHAPE"), ((8, 256, 8, 148), "ERR_SHAPE"),
+                         ((-1, 256, 256, 148), "ERR_SHAPE"), ((8, 256, 256, 1), "ERR_UNSUPPORTED")]:
+        with pytest.raises(rrf.RrfError) as e:
+            rrf.rrf_plan_scaled_mm(*args)
+        assert e.value.status == rrf.Status[status]
+    with pytest.raises(rrf.RrfError):
+        rrf.rrf_plan_scaled_mm(8, 256, 1040, 148, mx=True)  # MX needs K % 128 == 0

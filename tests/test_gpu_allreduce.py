@@ -88,12 +88,12 @@ def test_same_shape_same_bits_as_fused_call(rrf, allreduce, name, rows, world, m
     two reduce the statistics in the same order: identical bits."""
     c = rank_case(name, rows, world)
     sm = torch.cuda.get_device_properties(0).multi_processor_count
-    m, *shape = rrf.rrf_plan_allreduce(world, rows, c.cols, sm, c.residual is not None, mode)
-    mine = -(-rows // world) if m == TWO else rows
-    if tuple(shape) != rrf.rrf_plan_fused(world, mine, c.cols, sm, c.residual is not None):
-        pytest.skip("different row split from the single-GPU call's")
+    m, cluster, threads, vpt = rrf.rrf_plan_allreduce(world, rows, c.cols, sm,
+                                                       c.residual is not None, mode)
     outs = run_local(allreduce, c, mode)
-    fused = parity.gpu_fused(c)
+    # the single-GPU call forced to the same row split (cluster size, block size)
+    fused = parity.gpu_fused(c, variant=2 if cluster > 1 else 1,
+                             cluster_size=cluster if cluster > 1 else 0, block_threads=threads)
     for k in fused:
         assert np.array_equal(outs[0][k], fused[k]), k
 

@@ -69,8 +69,8 @@ def test_scaled_mm_matches_oracle(rrf, M, N, K, bias):
 
 
 def test_wide_tiles_sampled_rows(rrf):
-    """A grid large enough for the 128 x 256 tiles; sampled rows against the
-    oracle, including both tails."""
+    """A grid of 256 x 256 tiles on SM pairs with row and column tails;
+    sampled rows against the oracle, including both tails."""
     c = workloads.make_gemm_case(2000, 2576, 1040, sub=3, device="cuda")
     out = rrf.rrf_scaled_mm_fp8(c.a, c.a_scale, c.b, c.b_scale, c.bias)
     torch.cuda.synchronize()
@@ -84,6 +84,30 @@ def test_decode_projection_sampled_rows(rrf, M):
     out = rrf.rrf_scaled_mm_fp8(c.a, c.a_scale, c.b, c.b_scale, c.bias)
     torch.cuda.synchronize()
     check(c, out, rows=sorted({0, M // 2, M - 1}), label=f"decode {M}")
+
+
+def sm_count():
+    return torch.cuda.get_device_properties(0).multi_processor_count
+
+
+@pytest.mark.parametrize("M,N,K,kernel", [(1, 16384, 7168, "swap"), (8, 16384, 7168, "swap"),
+                                          (32, 16384, 7168, "swap"), (16, 16384, 1024, "swap"),
+                                          (9, 16384, 1024, "swap"), (64, 16384, 1024, "tile"),
+                                          (8, 16384, 1040, "tile"), (100, 16384, 1024, "tile")])
+def test_several_tiles_per_cta(rrf, M, N, K, kernel):
+    """Products with more 64-column weight tiles than CTAs, so every
+    persistent CTA walks several tiles and reuses its stage ring and both
+    accumulators: the swapped kernel at each row padding (8, 16, 32), the
+    64-row and 128-row A-stage kernels, and the one-k-tile-per-box form
+    (K % 128 != 0).  The plan query shows which kernel ran; sampled rows
+    with every column against the oracle."""
+    p = rrf.rrf_plan_scaled_mm(M, N, K, sm_count())
+    assert p["kernel"] == kernel and p["tiles"] > p["ctas"], p
+    c = workloads.make_gemm_case(M, N, K, sub=M % 5, device="cuda")
+    out = rrf.rrf_scaled_mm_fp8(c.a, c.a_scale, c.b, c.b_scale, c.bias)
+    torch.cuda.synchronize()
+    check(c, out, rows=sorted({0, M // 2, M - 1}), label=f"{M}x{N}x{K}")
+    assert rrf.rrf_device_error() == 0
 
 
 def test_prefill_sampled_rows(rrf):

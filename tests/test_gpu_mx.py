@@ -176,6 +176,25 @@ def test_mx_gemm_large_sampled_rows(rrf, M, N, K):
     check_mx_gemm(c, sa, sb, out, rows=sorted({0, 1, M // 2, M - 1}), label=f"{M}x{N}x{K}")
 
 
+@pytest.mark.parametrize("M,N,K", [(8, 16384, 1024), (16, 16384, 1024), (24, 16384, 1024),
+                                   (64, 16384, 7168), (100, 16384, 1024)])
+def test_mx_gemm_several_tiles_per_cta(rrf, M, N, K):
+    """More 128 x 64 output tiles than CTAs (N = 16384: 256 tiles on at most
+    one CTA per SM), so each persistent CTA walks several tiles with its
+    stage ring, both accumulators and the odd tiles' second scale column:
+    the 8-, 16-, 32-, 64- and 128-row A-stage kernels; sampled rows, every
+    column, against the oracle."""
+    sm = torch.cuda.get_device_properties(0).multi_processor_count
+    p = rrf.rrf_plan_scaled_mm(M, N, K, sm, mx=True)
+    assert p["kernel"] == "tile" and p["tile_n"] == 64 and p["tiles"] > p["ctas"], p
+    c, sa, sb = mx_operands(M, N, K, 8)
+    out = rrf.rrf_scaled_mm_mxfp8(c.a, rrf.mx_blocked(torch.from_numpy(sa).cuda()), c.b,
+                                  rrf.mx_blocked(torch.from_numpy(sb).cuda()), c.bias)
+    torch.cuda.synchronize()
+    check_mx_gemm(c, sa, sb, out, rows=sorted({0, 1, M // 2, M - 1}), label=f"{M}x{N}x{K}")
+    assert rrf.rrf_device_error() == 0
+
+
 def test_mx_quantizer_feeds_mx_gemm(rrf):
     """The fused call's MX codes and blocked scales feed the MX GEMM."""
     case = parity.to_device(workloads.make_case("decode", 64))

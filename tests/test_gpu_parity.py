@@ -91,10 +91,12 @@ def test_sum_prefill_size(rrf):
 
 @pytest.mark.parametrize("name,rows", [("decode", 64), ("odd", 37), ("decode", 1),
                                        ("sweep", 16)])
-@pytest.mark.parametrize("variant,cluster", [(1, 0), (2, 2), (2, 4), (2, 8), (2, 16)])
+@pytest.mark.parametrize("variant,cluster", [(1, 0), (2, 2), (2, 3), (2, 4), (2, 5), (2, 6),
+                                             (2, 7), (2, 8), (2, 12), (2, 14), (2, 16)])
 def test_forced_variants(rrf, name, rows, variant, cluster):
-    """Every cluster size (1 = one block per row) gives the same bf16 outputs
-    and matches the oracle within tolerance."""
+    """Every cluster size (1 = one block per row; powers of two reduce the
+    slots with the butterfly, the others in slot order) gives the same bf16
+    outputs and matches the oracle within tolerance."""
     c = dev_case(name, rows)
     gpu = parity.gpu_fused(c, variant=variant, cluster_size=cluster)
     parity.assert_fused_parity(gpu, parity.oracle_fused(c), f"{name} {rows} C={cluster}")
@@ -114,7 +116,7 @@ def test_forced_block_sizes(rrf, threads):
         parity.assert_fused_parity(gpu, ref, f"threads={threads} C={cluster}")
 
 
-@pytest.mark.parametrize("cluster", [2, 4, 8, 16])
+@pytest.mark.parametrize("cluster", [2, 3, 4, 7, 8, 16])
 @pytest.mark.parametrize("exchange", ["async", "barrier"])
 def test_cluster_exchanges(rrf, cluster, exchange):
     """Both ways for a cluster's blocks to share their statistics -- st.async
@@ -152,7 +154,7 @@ def test_starved_exchange_times_out_and_reports(rrf):
 def test_variants_bitwise_identical_bf16(rrf):
     c = dev_case("decode", 32)
     outs = [parity.gpu_fused(c, variant=v, cluster_size=k)
-            for v, k in ((1, 0), (2, 2), (2, 4), (2, 8), (2, 16))]
+            for v, k in ((1, 0), (2, 2), (2, 4), (2, 7), (2, 8), (2, 16))]
     for o in outs[1:]:
         assert np.array_equal(o["res_out"], outs[0]["res_out"])
 
@@ -186,6 +188,46 @@ def test_programmatic_dependent_launch_flag(rrf):
         expect = outs[i]
 
 
+@pytest.mark.parametrize("name,rows", [("decode", 64), ("decode", 1), ("odd", 37),
+                                       ("tiny", None), ("sweep", 256)])
+def test_prefetch_flags(rrf, name, rows):
+    """The L2 prefetch before the wait for the previous kernel, forced on and
+    off: the same bits either way, matching the oracle."""
+    c = dev_case(name, rows)
+    on = parity.gpu_fused(c, flags=rrf.RRF_FLAG_PREFETCH)
+    off = parity.gpu_fused(c, flags=rrf.RRF_FLAG_NO_PREFETCH)
+    for k in on:
+        assert np.array_equal(on[k], off[k]), k
+    parity.assert_fused_parity(on, parity.oracle_fused(c), f"{name} prefetch")
+    with pytest.raises(rrf.RrfError):
+        parity.gpu_fused(c, flags=rrf.RRF_FLAG_PREFETCH | rrf.RRF_FLAG_NO_PREFETCH)
+
+
+@pytest.mark.parametrize("cluster", [0, 7])
+def test_prefetch_of_data_the_previous_kernel_writes(rrf, cluster):
+    """A chain in which every call's inputs are the previous call's residual
+    output: each call prefetches (with PDL) the very rows the kernel before it
+    is still writing, and must still read the new values after its wait."""
+    c = dev_case("decode", 64, R=2)
+    x0 = c.inputs[0]
+    bufs = [c.inputs[1].clone()] + [torch.empty_like(x0) for _ in range(6)]
+    res = c.residual.clone()
+    for i in range(6):
+        # call i: inputs (x0, bufs[i]), residual res; writes bufs[i + 1]
+        rrf.rrf_sum_rmsnorm_fp8_ex([x0, bufs[i]], c.gamma, c.eps, c.weight_offset, c.scale_ub,
+                                   residual_in=res, residual_out=bufs[i + 1],
+                                   variant=2 if cluster else 0, cluster_size=cluster,
+                                   flags=rrf.RRF_FLAG_PREFETCH)
+    torch.cuda.synchronize()
+    bits = workloads.bits
+    prev = bufs[0]
+    for i in range(6):
+        step = workloads.Case(c.name, 2, c.rows, c.cols, [x0, prev], res, c.gamma, c.eps,
+                              c.weight_offset, c.scale_ub)
+        assert np.array_equal(bits(bufs[i + 1]), parity.oracle_fused(step)["res_out"]), i
+        prev = bufs[i + 1]
+
+
 # --------------------------------------------------------------- random shapes ---
 
 def test_random_shapes_and_launches(rrf):
@@ -204,9 +246,10 @@ def test_random_shapes_and_launches(rrf):
         c.weight_offset = float(rng.choice([0.0, 1.0, -0.5]))
         c.scale_ub = float(rng.choice([1200.0, 8.0, 0.5, float("inf")]))
         variant = int(rng.choice([0, 1, 2]))
-        cluster = int(rng.choice([2, 4, 8, 16])) if variant == 2 else 0
+        cluster = int(rng.integers(2, 17)) if variant == 2 else 0
         threads = int(rng.choice([0, 0, 32, 64, 128, 256, 512]))
-        flags = int(rng.choice([0, rrf.RRF_FLAG_BARRIER_EXCHANGE, rrf.RRF_FLAG_NO_PDL]))
+        flags = int(rng.choice([0, rrf.RRF_FLAG_BARRIER_EXCHANGE, rrf.RRF_FLAG_NO_PDL,
+                                rrf.RRF_FLAG_PREFETCH, rrf.RRF_FLAG_NO_PREFETCH]))
         in_place = c.residual is not None and bool(rng.integers(0, 2))
         try:
             gpu = parity.gpu_fused(c, variant=variant, cluster_size=cluster,
