@@ -1,26 +1,35 @@
 """Benchmark of the fused bf16 sum + residual + RMSNorm + per-row FP8 call.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--impl rrf|reference]
+                    [--replays N] [--impl rrf|reference]
+    python bench.py --plan-sweep reduce_rmsnorm_fp8_b200/csrc/rrf_plan_table.inc
 
 One step is one pass of the operation over one batch of the workload: for
-the default "decode" workload (R = 8 bf16 inputs, 7168 columns, residual on)
-the four calls at 1, 8, 32 and 64 rows.  Inputs are resident in HBM when the
-timed region starts and rotate over buffer sets whose total exceeds three
-times the L2 cache, so every step reads cold HBM.  K steps are timed with
-CUDA events on the launching stream, bracketed by a barrier and a device
-synchronisation on both sides; the time is the maximum over ranks.
+the default "prefill" workload, the largest single-GPU configuration, one
+call of R = 8 bf16 inputs of 8192 x 8192 with the residual on (1.41 GB of
+HBM traffic).  Inputs are resident in HBM when the timed region starts and
+rotate over buffer sets whose total exceeds three times the L2 cache, so
+every step reads cold HBM.  K steps are captured in one CUDA graph and timed
+with CUDA events on the launching stream, bracketed by a barrier and a
+device synchronisation on both sides; the value comes from the median of
+--replays timed replays, and the time is the maximum over ranks.
 
 value = algorithmic bytes of all ranks' steps / time, in GB/s, where one
 fused call moves R*rows*cols*2 + 4*rows*cols (residual read + write) +
 2*cols (gamma) + rows*cols (fp8 codes) + 4*rows (scales) bytes.
+
+Beside the headline: every configuration's calls timed one by one (decode
+1/8/32/64 x 7168, odd 37/64 x 7168, tiny, prefill), the launch floor of the
+call chain, the end-to-end figure through pinned host buffers, the oracle on
+one core and on all cores, and the other entry points.
 
 Multi-GPU (torchrun, one process per GPU, NCCL only for the barrier and the
 max-over-ranks timing): rows are independent, so every rank runs its own
 batch with no data-path collective (weak scaling).
 
 --impl reference times the CPU oracle (single-threaded C) on a bounded sample
-of the same workload, on rank 0 only.
+of the same workload, on rank 0 only.  --plan-sweep measures the fused call's
+launches on a grid of shapes and writes the library's launch table.
 """
 from __future__ import annotations
 
@@ -266,14 +275,19 @@ class DevicePool:
             self.big.append(b)
         self.eps, self.wo, self.ub = w.eps, w.weight_offset, w.scale_ub
 
-    def call(self, rrf, k: int, i: int) -> int:
-        """Enqueue call i of the workload on set k mod n_sets; returns 1."""
+    def call(self, rrf, k: int, i: int, flags: int = 0) -> int:
+        """Enqueue call i of the workload on set k mod n_sets (the library's
+        own launch; flags: RRF_FLAG_* overrides through the _ex entry);
+        returns 1."""
         b, s = self.big[i], k % self.n_sets
-        rrf.rrf_sum_rmsnorm_fp8(
-            [x[s] for x in b["inputs"]], b["gamma"][s], self.eps, self.wo, self.ub,
-            residual_in=None if b["residual"] is None else b["residual"][s],
-            residual_out=None if b["res_out"] is None else b["res_out"][s],
-            q_out=b["q"][s], scales_out=b["scales"][s])
+        args = ([x[s] for x in b["inputs"]], b["gamma"][s], self.eps, self.wo, self.ub)
+        kw = dict(residual_in=None if b["residual"] is None else b["residual"][s],
+                  residual_out=None if b["res_out"] is None else b["res_out"][s],
+                  q_out=b["q"][s], scales_out=b["scales"][s])
+        if flags:
+            rrf.rrf_sum_rmsnorm_fp8_ex(*args, **kw, flags=flags)
+        else:
+            rrf.rrf_sum_rmsnorm_fp8(*args, **kw)
         return 1
 
     def call_sum(self, rrf, k: int, i: int) -> int:
@@ -562,7 +576,7 @@ def e2e_measure(rrf, name: str, k_steps: int, warmup: int, device, stream):
     would run them, so one step's copies overlap the neighbouring steps'."""
     import torch
     w = workloads.WORKLOADS[name]
-    cases = [workloads.make_case(name, rows) for rows, _ in workload_cases(name)]
+    cases = [workloads.make_case(name, rows, device=device) for rows, _ in workload_cases(name)]
     ins, outs = _Arena(), _Arena()
     slots = []
     for c in cases:
@@ -638,40 +652,126 @@ def e2e_measure(rrf, name: str, k_steps: int, warmup: int, device, stream):
     return t, h2d, d2h
 
 
-def cpu_baseline(name: str, budget_s: float = 12.0):
-    """The oracle, as it stands, on a bounded sample of the workload: whole
-    steps of the workload (all its calls) until about budget_s seconds."""
+def _oracle_sample(name: str, rows: int):
+    """The workload's inputs for the oracle: one call of `rows` rows (drawn
+    with the workload's seeds), as bf16 bit patterns."""
+    bits = workloads.bits
+    c = workloads.make_case(name, rows, sub=0)
+    return ([bits(x) for x in c.inputs], None if c.residual is None else bits(c.residual),
+            bits(c.gamma), c)
+
+
+def cpu_baseline(name: str, budget_s: float = 10.0):
+    """The oracle, as it stands, on bounded samples of the workload: the
+    single-threaded C oracle on a block of rows per call until about budget_s
+    seconds, and the same per-row function on every core this process may use
+    (rows split into contiguous chunks, one POSIX thread each) on a larger
+    block.  Rows are independent, so GB/s over the sample is the oracle's
+    throughput on the workload."""
     import oracle
     w = workloads.WORKLOADS[name]
-    bits = workloads.bits
-    if name == "prefill":
-        # one full step is 1.4 GB; the sample is a block of 8 rows per call
-        calls = [(workloads.make_case(name, 8, sub=0), 8)]
-        sample = "8 of the 8192 rows per call, R=8 x 8192 cols + residual"
-        step_b = workloads.fused_bytes(w.R, 8, w.cols, w.residual)
-    else:
-        calls = [(workloads.make_case(name, rows), rows) for rows, _ in workload_cases(name)]
-        sample = "whole steps (every call of the workload)"
-        step_b = step_bytes(name)
-    prepared = [([bits(x) for x in c.inputs], None if c.residual is None else bits(c.residual),
-                 bits(c.gamma), c) for c, _ in calls]
+    o = oracle.default()
+    cores = o.cores()
+    calls = [r for r, _ in workload_cases(name)]
+    one_rows = [min(r, 8) for r in calls]
+    all_rows = [min(r, 16 * cores) for r in calls]
+    legs = {}
+    for leg, rows_list, threads in (("one", one_rows, 1), ("all", all_rows, cores)):
+        prepared = [_oracle_sample(name, r) for r in rows_list]
+        nbytes = sum(workloads.fused_bytes(w.R, r, w.cols, w.residual) for r in rows_list)
 
-    def one_step():
-        for xs, res, g, c in prepared:
-            oracle.sum_rmsnorm_fp8(xs, c.rows, c.cols, g, c.eps, c.weight_offset, c.scale_ub,
-                                   residual=res)
+        def one_step():
+            for xs, res, g, c in prepared:
+                if threads == 1:
+                    o.sum_rmsnorm_fp8(xs, c.rows, c.cols, g, c.eps, c.weight_offset,
+                                      c.scale_ub, residual=res)
+                else:
+                    o.sum_rmsnorm_fp8_mt(xs, c.rows, c.cols, g, c.eps, c.weight_offset,
+                                         c.scale_ub, residual=res, threads=threads)
 
-    one_step()  # builds the library and warms the caches
-    n, t0 = 0, time.perf_counter()
-    while True:
-        one_step()
-        n += 1
-        if time.perf_counter() - t0 >= budget_s:
-            break
-    dt = time.perf_counter() - t0
-    return {"value": round(step_b * n / dt / 1e9, 6), "unit": "GB/s", "cores": 1,
-            "kind": "oracle", "sample": f"{n} x ({sample}), {dt:.1f} s, single-threaded C",
-            "ms_per_step": round(dt / n * 1e3, 3)}
+        one_step()  # warms the caches
+        n, t0 = 0, time.perf_counter()
+        while True:
+            one_step()
+            n += 1
+            if time.perf_counter() - t0 >= budget_s:
+                break
+        dt = time.perf_counter() - t0
+        sample = (f"{n} x ({', '.join(str(r) for r in rows_list)} of the "
+                  f"{', '.join(str(r) for r in calls)} rows per call, R={w.R} x {w.cols} cols"
+                  f"{' + residual' if w.residual else ''}), {dt:.1f} s")
+        legs[leg] = {"value": round(nbytes * n / dt / 1e9, 6), "unit": "GB/s",
+                     "cores": threads, "kind": "oracle", "sample": sample,
+                     "rows_per_s": round(sum(rows_list) * n / dt, 1)}
+    out = dict(legs["one"])
+    out["sample"] += ", single-threaded C"
+    out["all_cores"] = legs["all"]
+    out["all_cores"]["sample"] += (f", {cores} POSIX threads (the cores of this process's "
+                                   f"CPU affinity), one contiguous row chunk each")
+    return out
+
+
+def time_calls(rrf, name, rows, device, stream, l2, peak, flags=0, replays=11):
+    """One call of a workload alone: a CUDA graph of back-to-back calls over
+    its own rotating buffer sets (> 3x L2, so every call reads cold HBM),
+    `replays` timed replays; the median per call, with p10 / p90."""
+    import torch
+    w = workloads.WORKLOADS[name]
+    cp = DevicePool(name, device, L2_FLUSH_FACTOR * l2, rows_list=[rows])
+    nbytes = workloads.fused_bytes(w.R, rows, w.cols, w.residual)
+    reps = max(cp.n_sets, 100) if nbytes < 64 << 20 else 20
+    for i in range(3):
+        cp.call(rrf, i, 0, flags)
+    g, _ = capture_steps(lambda k: cp.call(rrf, 3 + k, 0, flags), reps, device)
+    g.replay()
+    torch.cuda.synchronize(device)
+    ts = sorted(time_region(lambda _: g.replay(), 1, device, stream) for _ in range(replays))
+    del g, cp
+    tc = ts[len(ts) // 2]
+    return {"us_per_call": round(tc / reps * 1e6, 3),
+            "us_p10": round(ts[len(ts) // 10] / reps * 1e6, 3),
+            "us_p90": round(ts[-1 - len(ts) // 10] / reps * 1e6, 3),
+            "GB_s": round(nbytes * reps / tc / 1e9, 1),
+            "frac": round(nbytes * reps / tc / 1e9 / peak, 4),
+            "rows_per_s": round(rows * reps / tc, 1), "bytes": nbytes}
+
+
+def time_floor(rrf, device, stream, l2, replays=11):
+    """The floor of a call in this benchmark's chain: the library's smallest
+    kernel (rrf_sum of one 16-byte vector: one input, 8 columns) launched the
+    same way (programmatic dependent launch, graph replay), each call reading
+    a line of HBM that is not in L2 (a buffer larger than L2 is written
+    between replays): an empty PDL kernel chain plus one cold HBM round trip
+    per call."""
+    import torch
+    reps = 100
+    x = torch.randn((reps, 2048), device=device).to(torch.bfloat16)  # 4 KB apart
+    out = torch.empty((reps, 8), dtype=torch.bfloat16, device=device)
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=device)
+
+    def call(k):
+        rrf.rrf_sum([x[k, :8].view(1, 8)], out=out[k].view(1, 8))
+        return 1
+
+    for k in range(3):
+        call(k)
+    g, _ = capture_steps(call, reps, device)
+    ts = []
+    for _ in range(replays):
+        flush.fill_(1)
+        torch.cuda.synchronize(device)
+        ts.append(time_region(lambda _: g.replay(), 1, device, stream))
+    del g
+    ts.sort()
+    return {"us_per_call": round(ts[len(ts) // 2] / reps * 1e6, 3),
+            "what": "rrf_sum of one 16-byte vector per call, cold line each call, PDL, "
+                    "graph replay"}
+
+
+# The calls timed one by one beside the headline: every configuration's row
+# counts (decode and odd with the L2 prefetch also forced off).
+CASE_CONFIGS = (("decode", (1, 8, 32, 64)), ("odd", (37, 64)), ("tiny", (4,)),
+                ("prefill", (8192,)))
 
 
 def run_rrf(args):
@@ -692,140 +792,76 @@ def run_rrf(args):
     torch.cuda.set_device(device)
     props = torch.cuda.get_device_properties(device)
     l2 = props.L2_cache_size
+    sm = props.multi_processor_count
     peak, peak_kind = measured_peaks()
 
     name = args.workload
     w = workloads.WORKLOADS[name]
     pool = DevicePool(name, device, L2_FLUSH_FACTOR * l2)
     stream = torch.cuda.current_stream(device)
-    launches = 0
 
-    # ---- warm-up (eager), then K steps captured in one CUDA graph and timed
-    # as one replay: the step is launch-bound at decode sizes, and a graph
-    # removes the host's per-launch cost from the device timeline.
+    # ---- warm-up (eager), then K steps captured in one CUDA graph, timed
+    # as the median of several replays (the graph removes the host's
+    # per-launch cost from the device timeline)
     for i in range(args.warmup):
         pool.run_step(rrf, i)
     torch.cuda.synchronize(device)
     graph, launches = capture_steps(lambda i: pool.run_step(rrf, args.warmup + i),
                                     args.steps, device)
-    clocks = ClockSampler(device.index)
     graph.replay()  # one untimed replay: graph upload
     torch.cuda.synchronize(device)
-    t = time_region(lambda _: graph.replay(), 1, device, stream, clocks)
+    clocks = ClockSampler(device.index)
+    clocks.mark_start()
+    times = [time_region(lambda _: graph.replay(), 1, device, stream)
+             for _ in range(args.replays)]
+    clocks.mark_end()
     clock_info = clocks.summary()  # stops the poller
     del graph
+    t = statistics.median(times)
     n_sets = pool.n_sets
     per_step = step_bytes(name)
     value = world * per_step * args.steps / t / 1e9
     kernel_us = t / launches * 1e6
-
-    # ---- per-call breakdown: each row count alone, with its own rotating
-    # pool above 3 x L2 (a pool shared with the other calls would leave a
-    # small call's sets hot in L2 when it runs alone)
-    cases = []
-    reps = max(args.steps, 100)
-    for c in ([] if args.no_breakdown else pool.cases):
-        cp = DevicePool(name, device, L2_FLUSH_FACTOR * l2, rows_list=[c.rows])
-        for i in range(3):
-            cp.call(rrf, i, 0)
-        gi, _ = capture_steps(lambda k: cp.call(rrf, 3 + k, 0), reps, device)
-        gi.replay()
-        torch.cuda.synchronize(device)
-        # eleven timed replays: the median is the figure, p10/p90 its spread
-        tcs = sorted(time_region(lambda _: gi.replay(), 1, device, stream) for _ in range(11))
-        tc = tcs[5]
-        del gi, cp
-        b = workloads.fused_bytes(w.R, c.rows, c.cols, c.residual is not None)
-        launch = rrf.rrf_plan_fused(w.R, c.rows, c.cols, props.multi_processor_count,
-                                    residual=c.residual is not None)
-        cases.append({"rows": c.rows, "us_per_call": round(tc / reps * 1e6, 3),
-                      "us_p10": round(tcs[1] / reps * 1e6, 3),
-                      "us_p90": round(tcs[9] / reps * 1e6, 3),
-                      "GB_s": round(b * reps / tc / 1e9, 1),
-                      "frac": round(b * reps / tc / 1e9 / peak, 4),
-                      "rows_per_s": round(c.rows * reps / tc, 1),
-                      "launch": {"cluster": launch[0], "threads": launch[1],
-                                 "vecs_per_thread": launch[2]}})
+    calls_per_step = len(workload_cases(name))
+    del pool
     torch.cuda.empty_cache()
 
     # ---- end to end through host buffers
     e2e = None
     if not args.no_e2e:
-        te, h2d, d2h = e2e_measure(rrf, name, max(10, args.steps // 10), args.warmup, device,
-                                   torch.cuda.Stream(device))
-        ke = max(10, args.steps // 10)
+        ke = args.e2e_steps
+        te, h2d, d2h = e2e_measure(rrf, name, ke, 3, device, torch.cuda.Stream(device))
         e2e = {"value": round(world * per_step * ke / te / 1e9, 3), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": round(te / ke * 1e3, 4),
+               "ms_per_step": round(te / ke * 1e3, 4), "steps": ke,
                "how": "rrf_sum_rmsnorm_fp8 on device copies of pinned host buffers: one "
                       "H2D and one D2H copy per step, double-buffered over three streams"}
+        torch.cuda.empty_cache()
 
-    # ---- secondary: the prefill-size call, where the kernel can reach HBM speed
-    secondary = None
-    if not args.no_secondary and name != "prefill":
-        del pool
-        torch.cuda.empty_cache()
-        pf = DevicePool("prefill", device, 2 * l2)
-        for i in range(3):
-            pf.run_step(rrf, i)
-        kp = 20
-        gp, _ = capture_steps(lambda k: pf.run_step(rrf, k), kp, device)
-        gp.replay()
-        torch.cuda.synchronize(device)
-        tp = time_region(lambda _: gp.replay(), 1, device, stream)
-        del gp
-        bp = step_bytes("prefill")
-        secondary = {"workload": "prefill R=8 8192x8192 + residual, 2 rotating sets of 1.41 GB",
-                     "us_per_call": round(tp / kp * 1e6, 2),
-                     "GB_s": round(bp * kp / tp / 1e9, 1),
-                     "frac": round(bp * kp / tp / 1e9 / peak, 4), "calls": kp}
-        del pf
-        torch.cuda.empty_cache()
-        # the sum alone at the same size (8 inputs of 8192 x 8192)
-        pf = DevicePool("prefill", device, 2 * l2, with_sum=True)
-        for i in range(3):
-            pf.call_sum(rrf, i, 0)
-        gs, _ = capture_steps(lambda k: pf.call_sum(rrf, k, 0), kp, device)
-        gs.replay()
-        torch.cuda.synchronize(device)
-        ts = time_region(lambda _: gs.replay(), 1, device, stream)
-        del gs, pf
-        torch.cuda.empty_cache()
-        bs = workloads.sum_bytes(8, 8192, 8192)
-        secondary.update({"sum_us_per_call": round(ts / kp * 1e6, 2),
-                          "sum_GB_s": round(bs * kp / ts / 1e9, 1),
-                          "sum_frac": round(bs * kp / ts / 1e9 / peak, 4)})
-
-    # ---- the other configurations, each call alone over its own pool
-    others = None
-    if not args.no_secondary:
-        others = {}
-        for oname in ("tiny", "odd"):
-            if oname == name:
-                continue
-            recs = []
-            wo = workloads.WORKLOADS[oname]
-            for rows in wo.rows:
-                op = DevicePool(oname, device, L2_FLUSH_FACTOR * l2, rows_list=[rows])
-                for i in range(3):
-                    op.call(rrf, i, 0)
-                reps = 200
-                go, _ = capture_steps(lambda k: op.call(rrf, 3 + k, 0), reps, device)
-                go.replay()
-                torch.cuda.synchronize(device)
-                to = time_region(lambda _: go.replay(), 1, device, stream)
-                del go, op
-                bo = workloads.fused_bytes(wo.R, rows, wo.cols, wo.residual)
-                recs.append({"rows": rows, "us_per_call": round(to / reps * 1e6, 3),
-                             "GB_s": round(bo * reps / to / 1e9, 1),
-                             "frac": round(bo * reps / to / 1e9 / peak, 4)})
-            others[oname] = {"R": wo.R, "cols": wo.cols, "residual": wo.residual,
-                             "calls": recs}
-        torch.cuda.empty_cache()
+    # ---- every configuration's calls one by one, and the launch floor
+    cases = []
+    floor = None
+    if not args.no_breakdown:
+        for cname, rows_list in CASE_CONFIGS:
+            wc = workloads.WORKLOADS[cname]
+            for rows in rows_list:
+                rec = {"workload": cname, "R": wc.R, "rows": rows, "cols": wc.cols,
+                       "residual": wc.residual}
+                rec.update(time_calls(rrf, cname, rows, device, stream, l2, peak))
+                cl, th, vpt, pf = rrf.rrf_plan_fused_ex(wc.R, rows, wc.cols, sm,
+                                                        residual=wc.residual)
+                rec["launch"] = {"cluster": cl, "threads": th, "vecs_per_thread": vpt,
+                                 "prefetch": pf}
+                if cname in ("decode", "odd"):
+                    rec["no_prefetch"] = time_calls(rrf, cname, rows, device, stream, l2, peak,
+                                                    flags=rrf.RRF_FLAG_NO_PREFETCH)["us_per_call"]
+                cases.append(rec)
+                torch.cuda.empty_cache()
+        floor = time_floor(rrf, device, stream, l2)
 
     # ---- the sum-only / fused sweep over the b12x payload sizes (R=4, 4096 cols)
     sweep = None
-    if not args.no_secondary and name != "sweep":
+    if not args.no_secondary:
         sweep = []
         ws = workloads.WORKLOADS["sweep"]
         for rows in ws.rows:
@@ -841,13 +877,29 @@ def run_rrf(args):
                 gs, _ = capture_steps(lambda k, fn=fn: fn(rrf, 3 + k, 0), reps, device)
                 gs.replay()
                 torch.cuda.synchronize(device)
-                ts = time_region(lambda _: gs.replay(), 1, device, stream)
+                ts = sorted(time_region(lambda _: gs.replay(), 1, device, stream)
+                            for _ in range(5))
                 del gs
-                rec[f"{op}_us"] = round(ts / reps * 1e6, 3)
-                rec[f"{op}_GB_s"] = round(nbytes * reps / ts / 1e9, 1)
+                rec[f"{op}_us"] = round(ts[2] / reps * 1e6, 3)
+                rec[f"{op}_GB_s"] = round(nbytes * reps / ts[2] / 1e9, 1)
             sweep.append(rec)
             del sp
         torch.cuda.empty_cache()
+        # the sum alone at the prefill size (8 inputs of 8192 x 8192)
+        pf = DevicePool("prefill", device, 2 * l2, with_sum=True)
+        for i in range(3):
+            pf.call_sum(rrf, i, 0)
+        kp = 20
+        gs, _ = capture_steps(lambda k: pf.call_sum(rrf, k, 0), kp, device)
+        gs.replay()
+        torch.cuda.synchronize(device)
+        ts = sorted(time_region(lambda _: gs.replay(), 1, device, stream) for _ in range(5))
+        del gs, pf
+        torch.cuda.empty_cache()
+        bs = workloads.sum_bytes(8, 8192, 8192)
+        sweep.append({"rows": 8192, "cols": 8192, "R": 8, "sum_us": round(ts[2] / kp * 1e6, 2),
+                      "sum_GB_s": round(bs * kp / ts[2] / 1e9, 1),
+                      "sum_frac": round(bs * kp / ts[2] / 1e9 / peak, 4)})
 
     # ---- the sharded form, one shard of 8 (the all-gather between the phases
     # is not on one GPU): decode 32 x 7168 -> 896 columns, prefill 8192 x 8192
@@ -892,6 +944,7 @@ def run_rrf(args):
 
     if rank == 0:
         achieved = per_step * args.steps / t / 1e9
+        rows_list = [r for r, _ in workload_cases(name)]
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
@@ -900,37 +953,35 @@ def run_rrf(args):
             "io": "bf16 inputs/residual/gamma -> e4m3fn codes + f32 scales + bf16 residual",
             "data": "synthetic (seeded splitmix64 + Box-Muller, drawn on the GPU)",
             "impl": "rrf",
-            "config": {"workload": f"{name}: R={w.R}, cols={w.cols}, rows "
-                                   f"{[r for r, _ in workload_cases(name)]} per step, "
-                                   f"residual={'on' if w.residual else 'off'}",
-                       "R": w.R, "cols": w.cols, "rows": [r for r, _ in workload_cases(name)],
+            "config": {"workload": f"{name}: R={w.R}, cols={w.cols}, rows {rows_list} per "
+                                   f"step, residual={'on' if w.residual else 'off'}",
+                       "R": w.R, "cols": w.cols, "rows": rows_list,
                        "bytes_per_step": per_step,
                        "l2": f"inputs larger than L2: {n_sets} rotating buffer sets, "
                              f"{n_sets * per_step >> 20} MiB of traffic > "
                              f"{L2_FLUSH_FACTOR}x L2 ({l2 >> 20} MiB)",
                        "launch": "auto (rrf_sum_rmsnorm_fp8)",
-                       "timing": "K steps captured in one CUDA graph, one replay timed "
-                                 "with CUDA events",
+                       "timing": f"K steps captured in one CUDA graph; the median of "
+                                 f"{args.replays} timed replays (CUDA events)",
+                       "replay_ms": [round(x * 1e3, 4) for x in times],
                        "parallelism": f"dp{world}"},
             "us_per_call": round(t / launches * 1e6, 3),
-            "cases": cases,
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "traffic": recorded_traffic(name),
                          "traffic_note": "ncu dram__bytes_read.sum + dram__bytes_write.sum "
-                                         "per launch, averaged over the step's launches "
-                                         "(profiles/fused_kernel_traffic.txt); null when "
-                                         "not recorded for these kernel sources",
+                                         "per launch (profiles/fused_kernel_traffic.txt); "
+                                         "null when not recorded for these kernel sources",
                          "peak_kind": f"{peak_kind} hbm_gbs",
                          "kernel": "fused_kernel (rrf_fused.cu)",
                          "avg_launch_us": round(kernel_us, 3),
-                         "bytes_per_launch": round(per_step / len(workload_cases(name)))},
+                         "bytes_per_launch": round(per_step / calls_per_step)},
             "gpu_launches": launches,
             "clocks": clock_info,
             "e2e": e2e,
-            "prefill": secondary,
+            "cases": cases,
+            "floor": floor,
             "sweep": sweep,
-            "other_configs": others,
             "sharded": sharded,
             "allreduce_emulated": emulated,
             "mx": mx,
@@ -992,6 +1043,108 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------ launch sweep ---
+
+SWEEP_RB = (2, 4, 8, 16)
+SWEEP_COLS = (1024, 2048, 4096, 7168, 8192, 16384)
+SWEEP_ROWS = (1, 2, 4, 8, 16, 32, 37, 48, 64, 96, 128, 192, 256, 512, 1024, 2048, 8192)
+SWEEP_CLUSTERS = (1, 2, 3, 4, 5, 6, 7, 8, 12, 16)
+SWEEP_MAX_BYTES = 1600 << 20  # shapes moving more per call are left out
+
+
+def plan_sweep(out_inc: str, rbs=SWEEP_RB, cols_list=SWEEP_COLS, rows_list=SWEEP_ROWS):
+    """Measure every launch of the fused call (cluster size x L2 prefetch on
+    and off) on a grid of shapes and write the fastest per shape as the
+    library's launch table (rrf_plan_table.inc: one RRF_PLAN line per shape)
+    plus every measurement beside it (<out>.json).  Each launch is timed as
+    the median of five graph replays of back-to-back calls over rotating
+    buffer sets larger than 3x L2 (cold HBM, as the benchmark's calls).
+    Inputs: the sweep workload's distributions (N(0,1), gamma N(1, 0.1)),
+    R = the input bound."""
+    import torch
+    import reduce_rmsnorm_fp8_b200 as rrf
+    device = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(device)
+    props = torch.cuda.get_device_properties(device)
+    l2 = props.L2_cache_size
+    flags_of = {1: rrf.RRF_FLAG_PREFETCH, 0: rrf.RRF_FLAG_NO_PREFETCH}
+    records, best = [], []
+    t_start = time.perf_counter()
+    for rb in rbs:
+        for res in (0, 1):
+            for cols in cols_list:
+                for rows in rows_list:
+                    nbytes = workloads.fused_bytes(rb, rows, cols, bool(res))
+                    if nbytes > SWEEP_MAX_BYTES:
+                        continue
+                    c = workloads.make_case("sweep", rows, R=rb, cols=cols, residual=bool(res),
+                                            device=device)
+                    n_sets = max(2, math.ceil(L2_FLUSH_FACTOR * l2 / nbytes))
+                    shape = (n_sets, rows, cols)
+                    xs = [x.unsqueeze(0).expand(shape).contiguous() for x in c.inputs]
+                    rin = c.residual.unsqueeze(0).expand(shape).contiguous() if res else None
+                    rout = torch.empty(shape, dtype=torch.bfloat16, device=device) if res \
+                        else None
+                    q = torch.empty(shape, dtype=torch.float8_e4m3fn, device=device)
+                    sc = torch.empty((n_sets, rows, 1), dtype=torch.float32, device=device)
+                    calls = int(min(100, max(8, 1.5e-3 / (nbytes / 5e12 + 3e-6))))
+
+                    def call(k, C, pf):
+                        i = k % n_sets
+                        rrf.rrf_sum_rmsnorm_fp8_ex(
+                            [x[i] for x in xs], c.gamma, c.eps, c.weight_offset, c.scale_ub,
+                            residual_in=None if rin is None else rin[i],
+                            residual_out=None if rout is None else rout[i], q_out=q[i],
+                            scales_out=sc[i], variant=1 if C == 1 else 2,
+                            cluster_size=0 if C == 1 else C, flags=flags_of[pf])
+                        return 1
+
+                    meas = []
+                    for C in SWEEP_CLUSTERS:
+                        if C > 1 and cols // 8 // C < 32:
+                            continue
+                        for pf in (0, 1):
+                            try:
+                                for i in range(3):
+                                    call(i, C, pf)
+                            except rrf.RrfError:
+                                break  # the block cannot hold this cluster's slice
+                            g, _ = capture_steps(lambda k: call(3 + k, C, pf), calls, device)
+                            g.replay()
+                            torch.cuda.synchronize(device)
+                            ts = sorted(time_region(lambda _: g.replay(), 1, device, stream)
+                                        for _ in range(5))
+                            del g
+                            us = ts[2] / calls * 1e6
+                            meas.append((us, C, pf))
+                            records.append({"rb": rb, "residual": res, "cols": cols,
+                                            "rows": rows, "cluster": C, "prefetch": pf,
+                                            "us": round(us, 4),
+                                            "GB_s": round(nbytes / us / 1e3, 1)})
+                    us, C, pf = min(meas)
+                    best.append((rb, res, cols, rows, C, pf, us))
+                    del xs, rin, rout, q, sc, c
+                    print(f"sweep rb={rb} res={res} cols={cols} rows={rows}: C={C} "
+                          f"prefetch={pf} {us:.3f} us", file=sys.stderr, flush=True)
+                torch.cuda.empty_cache()
+    took = time.perf_counter() - t_start
+    with open(out_inc, "w") as fh:
+        fh.write(f"""// rrf_plan_table.inc -- measured launches of the fused call, one
+// RRF_PLAN(input bound, residual, cols, rows, cluster, prefetch, us per call)
+// per shape: the cluster size and L2-prefetch setting that ran fastest.
+// Written by `python bench.py --plan-sweep <this file>` on a {props.name}
+// ({props.multi_processor_count} SMs), {time.strftime('%Y-%m-%d')}, in {took:.0f} s; every
+// measurement is in the .json written beside the file.  Do not edit by hand.
+""")
+        for rb, res, cols, rows, C, pf, us in best:
+            fh.write(f"RRF_PLAN({rb}, {res}, {cols}, {rows}, {C}, {pf}, {us:.3f}f)\n")
+    with open(os.path.splitext(out_inc)[0] + ".json", "w") as fh:
+        json.dump({"gpu": props.name, "sms": props.multi_processor_count,
+                   "clusters": SWEEP_CLUSTERS, "records": records}, fh)
+    print(json.dumps({"plan_sweep": out_inc, "shapes": len(best), "measurements": len(records),
+                      "seconds": round(took, 1)}), flush=True)
+
+
 def run_gemm_only(M: int, N: int, K: int, mx: bool = False):
     """One GEMM shape through time_gemm or time_gemm_mx (3 eager calls, then
     graph replays), for profiling; prints its record."""
@@ -1027,7 +1180,10 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["rrf", "reference"], default="rrf")
-    ap.add_argument("--workload", choices=sorted(workloads.WORKLOADS), default="decode")
+    ap.add_argument("--workload", choices=sorted(workloads.WORKLOADS), default="prefill")
+    ap.add_argument("--replays", type=int, default=5,
+                    help="timed replays of the K-step graph (the value is their median)")
+    ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--rows", type=int, nargs="*", default=None,
                     help="only these row counts of the workload (profiling runs)")
     ap.add_argument("--no-breakdown", action="store_true",
@@ -1045,13 +1201,25 @@ def main(argv=None):
     ap.add_argument("--sharded", nargs=4, metavar=("WORKLOAD", "ROWS", "COLS", "SHARDS"),
                     default=None, help="time only the two phases of the sharded form on one "
                                        "shard (profiling runs)")
+    ap.add_argument("--plan-sweep", metavar="OUT_INC", default=None,
+                    help="measure the fused call's launches on a grid of shapes and write "
+                         "the launch table (reduce_rmsnorm_fp8_b200/csrc/rrf_plan_table.inc; "
+                         "rebuild the library afterwards) and OUT_INC's .json")
+    ap.add_argument("--plan-sweep-shapes", nargs=3, metavar=("RB", "COLS", "ROWS"),
+                    default=None, help="comma lists restricting the sweep's grid")
     args = ap.parse_args(argv)
     global ROWS_OVERRIDE
     if args.rows:
         ROWS_OVERRIDE = tuple(args.rows)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.gemm is not None:
+    if args.plan_sweep is not None:
+        grid = {}
+        if args.plan_sweep_shapes:
+            lists = [tuple(int(v) for v in x.split(",")) for x in args.plan_sweep_shapes]
+            grid = dict(rbs=lists[0], cols_list=lists[1], rows_list=lists[2])
+        plan_sweep(args.plan_sweep, **grid)
+    elif args.gemm is not None:
         run_gemm_only(*args.gemm)
     elif args.gemm_mx is not None:
         run_gemm_only(*args.gemm_mx, mx=True)
