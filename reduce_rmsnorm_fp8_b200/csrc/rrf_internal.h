@@ -64,6 +64,7 @@ struct PostArgs {
     float weight_offset;
     float scale_ub;
     unsigned int* err;     // the library's device error word
+    int prefetch;          // prefetch the block's h and gamma into L2 before the PDL wait
 };
 
 // The multi-GPU form (rrf_allreduce.cu).  Pointer arrays are indexed by rank

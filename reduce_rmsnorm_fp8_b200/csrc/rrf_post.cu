@@ -36,10 +36,22 @@ __global__ void __launch_bounds__(kPostThreads) post_kernel(const PostArgs a, in
     constexpr int RB = 4 * RPW;  // rows per block
     __shared__ float2 stage[RRF_MAX_SHARDS * RB];  // [shard][row]
     __shared__ float3 rowval[RB];                  // (1/r, scale, 1/scale)
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (a.prefetch) {
+        // This block's rows of h and its chunk of gamma to L2 while the
+        // previous kernel (normally the all-gather of the statistics; h was
+        // written before it) may still run: a hint, no value read after the
+        // wait changes.
+        const int64_t r0 = (int64_t)(blockIdx.x / chunks) * RB;
+        const int c0 = (int)(blockIdx.x % chunks) * kPostChunkVecs;
+        const int64_t rows_here = a.rows - r0 < RB ? a.rows - r0 : RB;
+        const int nv = a.vecs - c0 < kPostChunkVecs ? a.vecs - c0 : kPostChunkVecs;
+        if (tid < rows_here) prefetch_l2(a.h + (r0 + tid) * a.vecs + c0, (uint32_t)nv * 16u);
+        else if (tid == RB) prefetch_l2(a.gamma + c0, (uint32_t)nv * 16u);
+    }
     wait_for_previous_grid();  // see rrf_device.cuh: programmatic dependent launch
     allow_next_grid();
 
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     // every address derives from these two, taken after the wait
     const int64_t row0 = opaque((int64_t)(blockIdx.x / chunks) * RB);
     const int v0 = opaque((int)(blockIdx.x % chunks) * kPostChunkVecs);
@@ -135,10 +147,15 @@ cudaError_t launch_rpw(const PostArgs& a, int chunks, bool pdl, cudaStream_t str
 cudaError_t launch_post(const PostArgs& a, int sm_count, bool pdl, cudaStream_t stream) {
     const int chunks = (a.vecs + kPostChunkVecs - 1) / kPostChunkVecs;
     // Four rows per warp once that still gives every SM several blocks; one
-    // row per warp for small calls, which are latency-bound.
-    if ((a.rows + 15) / 16 * chunks >= 4 * (int64_t)sm_count)
-        return launch_rpw<4>(a, chunks, pdl, stream);
-    return launch_rpw<1>(a, chunks, pdl, stream);
+    // row per warp for small calls, which are latency-bound.  Small calls
+    // (every block resident at once) also prefetch before the wait.
+    PostArgs b = a;
+    if ((a.rows + 15) / 16 * chunks >= 4 * (int64_t)sm_count) {
+        b.prefetch = 0;
+        return launch_rpw<4>(b, chunks, pdl, stream);
+    }
+    b.prefetch = (a.rows + 3) / 4 * chunks <= 8 * (int64_t)sm_count ? 1 : 0;
+    return launch_rpw<1>(b, chunks, pdl, stream);
 }
 
 }  // namespace rrf
