@@ -63,6 +63,16 @@ __device__ __forceinline__ uint2 quantise_vector(uint4 h, uint4 g, float r, floa
     }
 }
 
+// The same from h and g' = gamma + weight_offset held as fp32 pairs.
+__device__ __forceinline__ uint2 quantise_pairs(const float2 hf[4], const float2 gp[4], float r,
+                                                float m) {
+    const float2 r2 = make_float2(r, r), m2 = make_float2(m, m);
+    float2 qv[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) qv[e] = __fmul2_rn(__fmul2_rn(__fmul2_rn(hf[e], r2), gp[e]), m2);
+    return f32x2_to_e4m3x8(qv);
+}
+
 // ASYNC (cluster rows only): the blocks of a cluster meet through the
 // transaction-counted exchange (st.async into the peers' shared memory,
 // bounded mbarrier waits) instead of a cluster barrier phase.
@@ -128,6 +138,9 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
 
     uint4 h[VPT];
     uint4 g[KEEP_GAMMA ? VPT : 1];
+    // PACKED: the vector's h and g' = gamma + weight_offset also stay as fp32
+    // pairs between the passes, so the last pass does not unpack them again
+    float2 hk[PACKED ? 4 : 1], gk[PACKED ? 4 : 1];
     RowStats st = stats_empty();
     // MX: max |h * g'| over each vector's 32-element block (4 lanes)
     float bkey[MX ? VPT : 1];
@@ -188,14 +201,15 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
             // max |h * g'| of the vector's 8 elements, g' = gamma + weight_offset
             float vkey = 0.0f;
             if constexpr (PACKED) {
-                float2 hf[4], gf[4];
-                bf16x8_to_f32x2(s, hf);
+                float2 gf[4];
+                bf16x8_to_f32x2(s, hk);
                 bf16x8_to_f32x2(gv, gf);
-                st.ss += sumsq_bf16x8_x2(hf);
+                st.ss += sumsq_bf16x8_x2(hk);
                 const float2 wo2 = make_float2(a.weight_offset, a.weight_offset);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float2 p = __fmul2_rn(hf[e], __fadd2_rn(gf[e], wo2));
+                    gk[e] = __fadd2_rn(gf[e], wo2);
+                    const float2 p = __fmul2_rn(hk[e], gk[e]);
                     vkey = fmaxf(vkey, fmaxf(fabsf(p.x), fabsf(p.y)));
                 }
             } else {
@@ -257,9 +271,10 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
                 const uint32_t code = mx_scale_code(__fmul_rn(bkey[k], rinv));
                 const float inv_x = __uint_as_float((254u - code) << 23);  // 2^(127 - code)
                 st_once(a.q + row_base + v,
-                        quantise_vector<PACKED>(h[k],
-                                                KEEP_GAMMA ? g[k] : ld_shared_by_all(a.gamma + v),
-                                                rinv, a.weight_offset, inv_x));
+                        PACKED ? quantise_pairs(hk, gk, rinv, inv_x)
+                               : quantise_vector<PACKED>(
+                                     h[k], KEEP_GAMMA ? g[k] : ld_shared_by_all(a.gamma + v),
+                                     rinv, a.weight_offset, inv_x));
                 if ((v & 3) == 0) {
                     // row-major [rows, cols / 32], or the tensor cores' blocked
                     // order (512-byte atoms of 128 rows x 4 blocks)
@@ -285,9 +300,10 @@ __global__ void __launch_bounds__(fused_max_threads(RB, VPT)) fused_kernel(const
             const int v = v_begin + tid + k * T;
             if (v < v_end && RRF_IN_BOUNDS(v >= 0 && v < a.vecs && row < a.rows, a.err)) {
                 st_once(a.q + row_base + v,
-                        quantise_vector<PACKED>(h[k],
-                                                KEEP_GAMMA ? g[k] : ld_shared_by_all(a.gamma + v),
-                                                rinv, a.weight_offset, inv_scale));
+                        PACKED ? quantise_pairs(hk, gk, rinv, inv_scale)
+                               : quantise_vector<PACKED>(
+                                     h[k], KEEP_GAMMA ? g[k] : ld_shared_by_all(a.gamma + v),
+                                     rinv, a.weight_offset, inv_scale));
                 if (RES && CLUSTER) st_once(a.res_out + row_base + v, h[k]);
             }
         }
