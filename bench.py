@@ -1052,6 +1052,23 @@ SWEEP_CLUSTERS = (1, 2, 3, 4, 5, 6, 7, 8, 12, 16)
 SWEEP_MAX_BYTES = 1600 << 20  # shapes moving more per call are left out
 
 
+def write_plan_table(out_inc: str, best, gpu: str, sms: int, seconds: float) -> None:
+    """The launch table the library compiles: a header comment, then one
+    RRF_PLAN(input bound, residual, cols, rows, cluster, prefetch, us) line
+    per (rb, residual, cols, rows, cluster, prefetch, us) of `best`."""
+    with open(out_inc, "w") as fh:
+        fh.write(f"""// rrf_plan_table.inc -- measured launches of the fused call, one
+// RRF_PLAN(input bound, residual, cols, rows, cluster, prefetch, us per call)
+// per shape: the cluster size and L2-prefetch setting that ran fastest.
+// Written by `python bench.py --plan-sweep <this file>` on a {gpu}
+// ({sms} SMs), {time.strftime('%Y-%m-%d')}, in {seconds:.0f} s; every
+// measurement is in the .json the sweep writes beside its output.  Do not
+// edit by hand.
+""")
+        for rb, res, cols, rows, C, pf, us in best:
+            fh.write(f"RRF_PLAN({rb}, {res}, {cols}, {rows}, {C}, {pf}, {us:.3f}f)\n")
+
+
 def plan_sweep(out_inc: str, rbs=SWEEP_RB, cols_list=SWEEP_COLS, rows_list=SWEEP_ROWS):
     """Measure every launch of the fused call (cluster size x L2 prefetch on
     and off) on a grid of shapes and write the fastest per shape as the
@@ -1128,16 +1145,7 @@ def plan_sweep(out_inc: str, rbs=SWEEP_RB, cols_list=SWEEP_COLS, rows_list=SWEEP
                           f"prefetch={pf} {us:.3f} us", file=sys.stderr, flush=True)
                 torch.cuda.empty_cache()
     took = time.perf_counter() - t_start
-    with open(out_inc, "w") as fh:
-        fh.write(f"""// rrf_plan_table.inc -- measured launches of the fused call, one
-// RRF_PLAN(input bound, residual, cols, rows, cluster, prefetch, us per call)
-// per shape: the cluster size and L2-prefetch setting that ran fastest.
-// Written by `python bench.py --plan-sweep <this file>` on a {props.name}
-// ({props.multi_processor_count} SMs), {time.strftime('%Y-%m-%d')}, in {took:.0f} s; every
-// measurement is in the .json written beside the file.  Do not edit by hand.
-""")
-        for rb, res, cols, rows, C, pf, us in best:
-            fh.write(f"RRF_PLAN({rb}, {res}, {cols}, {rows}, {C}, {pf}, {us:.3f}f)\n")
+    write_plan_table(out_inc, best, props.name, props.multi_processor_count, took)
     with open(os.path.splitext(out_inc)[0] + ".json", "w") as fh:
         json.dump({"gpu": props.name, "sms": props.multi_processor_count,
                    "clusters": SWEEP_CLUSTERS, "records": records}, fh)

@@ -544,3 +544,20 @@ def test_gemm_plan_invariants_and_rejections(rrf):
         assert e.value.status == rrf.Status[status]
     with pytest.raises(rrf.RrfError):
         rrf.rrf_plan_scaled_mm(8, 256, 1040, 148, mx=True)  # MX needs K % 128 == 0
+
+
+def test_sweep_writes_a_table_the_planner_reads(tmp_path):
+    """bench.py's table writer: the lines it writes parse back to its
+    entries, and the header is a C comment (the file is #included)."""
+    import bench
+    entries = [(2, 0, 1024, 1, 1, 1, 1.25), (8, 1, 7168, 64, 4, 1, 3.2262),
+               (16, 1, 16384, 2048, 1, 0, 198.5)]
+    out = tmp_path / "table.inc"
+    bench.write_plan_table(str(out), entries, "NVIDIA B200", 148, 181.0)
+    text = out.read_text()
+    assert all(l.startswith("//") or l.startswith("RRF_PLAN(") for l in text.splitlines() if l)
+    body = re.sub(r"//.*", "", text)
+    got = [tuple(float(v) if "." in v else int(v) for v in m.replace("f", "").split(","))
+           for m in re.findall(r"RRF_PLAN\(([^)]*)\)", body)]
+    assert [g[:6] for g in got] == [e[:6] for e in entries]
+    assert all(abs(g[6] - e[6]) < 5e-4 for g, e in zip(got, entries))
