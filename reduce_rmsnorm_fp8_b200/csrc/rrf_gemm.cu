@@ -9,8 +9,9 @@
 //            pairs (tcgen05.mma.cta_group::2) for products that fill every pair;
 //   scaled_mm_kernel / scaled_mm_mx_kernel  persistent CTAs on 128 x BN tiles
 //            (BN 128 or 64), Z k-tiles per TMA box for short products;
-//   scaled_mm_swap_kernel  at most 32 rows against a weight, the operands
-//            swapped (the weight's rows on the MMA's M = 64 side).
+//   scaled_mm_swap_pairk_kernel  at most 32 rows against a weight, the
+//            operands swapped (the weight's rows on the MMA's M side, two
+//            k-tiles of them per instruction).
 // A persistent CTA per SM walks 128 x BN tiles of out (BN 128 or 64).
 // Warp roles (the same in every kernel):
 //   warp 0   one thread issues the TMA loads of the A (128 x 128 bytes) and
@@ -430,58 +431,95 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------- short products: the operands swapped --
-// A call of at most 64 rows against a weight (a decode batch): the weight's
-// rows are the MMA's M side and the call's rows its N side, so the tensor
-// cores do 64 x NA x 32 per instruction (NA = the rows rounded up to 8, 16,
-// 32) instead of 128 x 64 x 32 with most rows empty.  A CTA streams a
-// 64-row weight tile (Z k-tiles per 3-D TMA box) against the call's rows
-// (an L2-resident box of NA rows per stage).  The accumulator
-// D[n][m] = out[m][n] lives in the M = 64 layout of tensor memory: weight
-// row 16 q + i in lane 32 q + i (q < 4, i < 16), row m of the call in
-// column m.
-
-// Instruction descriptor of kind::f8f6f4 with M = 64, N = na.
-__host__ __device__ constexpr uint32_t f8_idesc_m64(int na) {
-    return (1u << 4) | ((uint32_t)(na >> 3) << 17) | ((uint32_t)(64 >> 4) << 24);
-}
-
+// A call of at most 32 rows against a weight (a decode batch): the weight's
+// rows are the MMA's M side and the call's rows its N side (NA = the rows
+// rounded up to 8, 16 or 32), so no tensor-core row is spent on padding.  A
+// CTA streams a 64-row weight tile (Z k-tiles per 3-D TMA box) against the
+// call's rows (an L2-resident box of NA rows per stage).  One instruction
+// takes two k-tiles: A = the 128 rows of shared memory that hold weight
+// k-tiles kt and kt+1 (64 rows each, consecutive), B = the 2 NA rows that
+// hold the call's k-tiles kt and kt+1.  In D = A B^T (M = 128, N = 2 NA) the
+// block D[0:64, 0:NA] gets k-tile kt's partial product and D[64:128, NA:2NA]
+// k-tile kt+1's; the two off-diagonal blocks pair a weight k-tile with the
+// other k-tile of the call and are never read.  The epilogue adds the two
+// diagonal blocks (the even one first).  Against one M = 64, N = NA
+// instruction per k-tile this halves the instructions that hold each stage
+// back from the producer.  An odd number of k-tiles pairs the last one with
+// the zeros the TMA box holds past K.  D[w][m] of the M = 128 layout sits in
+// tensor-memory lane w, column m.
 template <int NA, int Z>
-struct SwapTile {
-    static_assert(NA % 8 == 0 && NA >= 8 && NA <= 64, "the call's rows: 8 .. 64 in steps of 8");
-    static constexpr int kWRows = 64;                  // weight rows per tile (the MMA's M)
+struct SwapPairTile {
+    static_assert(NA == 8 || NA == 16 || NA == 32, "the call's rows: 8, 16 or 32");
+    static_assert(Z % 2 == 0, "k-tiles go to the MMA in pairs");
+    static constexpr int kWRows = 64;                  // weight rows per tile
     static constexpr int kWBytes = kWRows * kBK;       // one k-tile of the weight: 8 KB
     static constexpr int kXBytes = NA * kBK;           // one k-tile of the call's rows
     static constexpr int kXOffset = Z * kWBytes;
     static constexpr int kStageBytes = Z * (kWBytes + kXBytes);
-    static constexpr int kStages =
-        (220 * 1024) / kStageBytes > 12 ? 12 : (220 * 1024) / kStageBytes;
-    // two accumulators of NA columns, each at least 32 wide (the epilogue
-    // reads 32 columns at a time); a power of two of at least 32.  (Spreading
-    // a tile's MMAs over 4 accumulators summed in the epilogue, to break the
-    // chain of dependent updates, measured 2 us slower at 1-32 x 7168 x 7168.)
-    static constexpr int kAccStride = NA < 32 ? 32 : NA;
+    static constexpr int kCombBytes = NA * kWRows * 4;  // the odd block, handed between warps
+    static constexpr int kStages = (218 * 1024 - kCombBytes) / kStageBytes > 12
+                                       ? 12
+                                       : (218 * 1024 - kCombBytes) / kStageBytes;
+    // two accumulators of 2 NA columns (a power of two of at least 32)
+    static constexpr int kAccStride = 2 * NA < 32 ? 32 : 2 * NA;
     static constexpr int kTmemCols = 2 * kAccStride;
-    static constexpr int kBarriers = 2 * kStages + 4 + 1;
-    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarriers * 8 + 16;
+    // full / empty per stage, full / empty per accumulator, the drain, and
+    // the odd block's full / empty
+    static constexpr int kBarriers = 2 * kStages + 4 + 1 + 2;
+    static constexpr int kSmemBytes =
+        1024 + kStages * kStageBytes + kCombBytes + kBarriers * 8 + 16;
     static_assert(kSmemBytes <= 227 * 1024, "stages exceed the shared memory of a CTA");
     static_assert(kXBytes % 1024 == 0, "each k-tile must start on a swizzle atom");
 };
 
+// NA consecutive fp32 accumulator columns of this thread's lane (NA = 8, 16
+// or 32).
+template <int NA>
+__device__ __forceinline__ void tmem_load_cols(uint32_t taddr, float v[NA]) {
+    uint32_t r[NA];
+    if constexpr (NA == 8) {
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                     : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                       "=r"(r[6]), "=r"(r[7])
+                     : "r"(taddr));
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+        for (int i = 0; i < NA; ++i) v[i] = __uint_as_float(r[i]);
+    } else if constexpr (NA == 16) {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, "
+            "%10, %11, %12, %13, %14, %15}, [%16];"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+              "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+              "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+            : "r"(taddr));
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+        for (int i = 0; i < NA; ++i) v[i] = __uint_as_float(r[i]);
+    } else {
+        static_assert(NA == 32, "8, 16 or 32 columns");
+        tmem_load_32(taddr, v);
+    }
+}
+
 template <int NA, int Z>
 __global__ void __launch_bounds__(kThreads, 1)
-    scaled_mm_swap_kernel(const __grid_constant__ CUtensorMap tma_x,
-                          const __grid_constant__ CUtensorMap tma_w, const GemmArgs g) {
-    using T = SwapTile<NA, Z>;
+    scaled_mm_swap_pairk_kernel(const __grid_constant__ CUtensorMap tma_x,
+                                const __grid_constant__ CUtensorMap tma_w, const GemmArgs g) {
+    using T = SwapPairTile<NA, Z>;
     constexpr int S = T::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(ring + S * T::kStageBytes);
+    float* comb = reinterpret_cast<float*>(ring + S * T::kStageBytes);  // [NA][64]
+    uint64_t* full = reinterpret_cast<uint64_t*>(ring + S * T::kStageBytes + T::kCombBytes);
     uint64_t* empty = full + S;
     uint64_t* acc_full = empty + S;
     uint64_t* acc_empty = acc_full + 2;
     uint64_t* drained = acc_empty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
+    uint64_t* comb_full = drained + 1;     // the odd block is in comb (64 threads arrive)
+    uint64_t* comb_empty = comb_full + 1;  // comb was read (64 threads arrive)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(comb_empty + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tiles = (g.N + T::kWRows - 1) / T::kWRows;
@@ -498,6 +536,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&acc_empty[b], 4);
         }
         mbar_init(drained, 1);
+        mbar_init(comb_full, 64);
+        mbar_init(comb_empty, 64);
         fence_mbar_init_cluster();
     }
     if (warp == 1) {
@@ -535,9 +575,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 wait_phase(&full[i % S], (i / S) & 1, g.err);
         }
     } else if (warp == 1) {
-        // ---- MMA issue: D[64 x NA] += W[64 x 32] * X[NA x 32]^T
+        // ---- MMA issue: D[128 x 2NA] += A[128 x 32] * B[2NA x 32]^T, A and B
+        // each spanning two k-tiles
         if (lane == 0) {
-            constexpr uint32_t idesc = f8_idesc_m64(NA);
+            constexpr uint32_t idesc = f8_idesc(2 * NA);  // M = 128, N = 2 NA
             int it = 0, j = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++j) {
@@ -554,7 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after_sync();
                     const uint8_t* stage = ring + s * T::kStageBytes;
                     const int nk = ktiles - kg * Z < Z ? ktiles - kg * Z : Z;
-                    for (int kj = 0; kj < nk; ++kj) {
+                    for (int kj = 0; kj < nk; kj += 2) {
                         const uint64_t wd = kmajor_sw128_desc(stage + kj * T::kWBytes);
                         const uint64_t xd = kmajor_sw128_desc(stage + T::kXOffset + kj * T::kXBytes);
 #pragma unroll
@@ -571,41 +612,59 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else {
-        // ---- epilogue: lanes 0-15 of each warp hold 16 weight rows (output
-        // columns); column m of tensor memory is row m of the call
+        // ---- epilogue: lane quarter q of tensor memory holds rows 32q ..
+        // 32q+31 of D: quarters 0, 1 the even block's weight rows 0-63,
+        // quarters 2, 3 the odd block's; the odd warps hand their NA values
+        // per row to the even warps through shared memory, which add them,
+        // scale and store (weight row w of the tile is output column n)
         const int quarter = warp & 3;
+        const bool odd = quarter >= 2;
+        const int w = (quarter & 1) * 32 + lane;
         int j = 0;
-        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
+        bool ok = true;
+        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++j) {
             const int buf = j & 1;
-            const int n = t * T::kWRows + quarter * 16 + (lane & 15);
+            const int n = t * T::kWRows + w;
             bool have = epilogue_wait(&acc_full[buf], (j >> 1) & 1, g);
             if (!__all_sync(0xFFFFFFFFu, have)) break;
             tc_fence_after_sync();
-            const bool mine = lane < 16 && n < g.N;
-            const float sb = mine ? g.b_scale[n] : 0.0f;
-            const float bias =
-                mine && g.bias != nullptr ? __uint_as_float((uint32_t)g.bias[n] << 16) : 0.0f;
-            const uint32_t base =
-                tmem + (uint32_t)(buf * T::kAccStride) + ((uint32_t)(quarter * 32) << 16);
-#pragma unroll
-            for (int c = 0; c < NA; c += 32) {
-                float v[32];
-                tmem_load_32(base + (uint32_t)c, v);
-                if (!mine) continue;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int m = c + i;
-                    if (m < NA && m < g.M && RRF_IN_BOUNDS(n >= 0 && n < g.N, g.err)) {
-                        float y = __fmul_rn(__fmul_rn(v[i], __ldg(g.a_scale + m)), sb);
-                        if (g.bias != nullptr) y = __fadd_rn(y, bias);
-                        // one rounding to bf16 (the low half of the packed pair)
-                        g.out[(int64_t)m * g.N + n] = (uint16_t)(f32x2_to_bf16x2(y, 0.0f) & 0xFFFFu);
-                    }
-                }
-            }
+            float v[NA];
+            tmem_load_cols<NA>(tmem + (uint32_t)(buf * T::kAccStride + (odd ? NA : 0)) +
+                                   ((uint32_t)(quarter * 32) << 16),
+                               v);
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[buf]);
+            if (odd) {
+                // comb is free once the even warps have read the previous tile's
+                if (j > 0 && !wait_phase(comb_empty, (j - 1) & 1, g.err)) ok = false;
+#pragma unroll
+                for (int m = 0; m < NA; ++m) comb[m * T::kWRows + w] = v[m];  // no bank conflicts
+                mbar_arrive(comb_full);  // each thread releases its own stores
+            } else {
+                if (!wait_phase(comb_full, j & 1, g.err)) ok = false;
+                float o[NA];
+#pragma unroll
+                for (int m = 0; m < NA; ++m) o[m] = comb[m * T::kWRows + w];
+                mbar_arrive(comb_empty);
+                if (ok && n < g.N && RRF_IN_BOUNDS(n >= 0, g.err)) {
+                    const float sb = g.b_scale[n];
+                    const float bias =
+                        g.bias != nullptr ? __uint_as_float((uint32_t)g.bias[n] << 16) : 0.0f;
+#pragma unroll
+                    for (int m = 0; m < NA; ++m) {
+                        if (m < g.M) {
+                            float y = __fmul_rn(__fmul_rn(__fadd_rn(v[m], o[m]),
+                                                          __ldg(g.a_scale + m)),
+                                                sb);
+                            if (g.bias != nullptr) y = __fadd_rn(y, bias);
+                            g.out[(int64_t)m * g.N + n] =
+                                (uint16_t)(f32x2_to_bf16x2(y, 0.0f) & 0xFFFFu);
+                        }
+                    }
+                }
+            }
+            if (!__all_sync(0xFFFFFFFFu, ok)) break;
         }
     }
 
@@ -1521,13 +1580,13 @@ cudaError_t launch_bn(const GemmArgs& g, const void* a, const void* b, int sm_co
 }
 
 template <int NA, int Z>
-cudaError_t launch_swap(const GemmArgs& g, const void* a, const void* b, int sm_count,
-                        cudaStream_t stream) {
-    using T = SwapTile<NA, Z>;
+cudaError_t launch_swap_pairk(const GemmArgs& g, const void* a, const void* b, int sm_count,
+                              cudaStream_t stream) {
+    using T = SwapPairTile<NA, Z>;
     CUtensorMap mx, mw;
     if (!make_map3(&mx, a, g.M, g.K, NA, Z) || !make_map3(&mw, b, g.N, g.K, T::kWRows, Z))
         return cudaErrorInvalidValue;
-    constexpr auto kernel = scaled_mm_swap_kernel<NA, Z>;
+    constexpr auto kernel = scaled_mm_swap_pairk_kernel<NA, Z>;
     const cudaError_t e = enable_dynamic_smem<kernel>(T::kSmemBytes);
     if (e != cudaSuccess) return e;
     const int64_t tiles = (g.N + T::kWRows - 1) / T::kWRows;
@@ -1625,9 +1684,11 @@ GemmPlan plan_scaled_mm(int64_t M, int64_t N, int64_t K, bool mx, int sm_count) 
     if (M <= 64 && !atoms) return tile(kGemmTile, 64, 64, 1);
     // at most 32 rows: the operands swapped, the call's rows padded to 8, 16
     // or 32 (at 64 the swapped MMA is no cheaper: measured slower); 8 k-tiles
-    // per box up to 16 rows (measured faster than 4 or 2 there; equal at 32)
+    // per box at 8 rows (3 stages), 4 at 16 and 32 rows (5 and 4 stages).
+    // Measured at 1-32 x 7168 x 7168: 8 beats 6 and 4 at 8 rows, 4 beats 8
+    // and 6 at 16 rows (12.2 against 13.4 us), 4 beats 2 at 32 rows.
     if (M <= 8) return tile(kGemmSwap, 8, 64, 8);
-    if (M <= 16) return tile(kGemmSwap, 16, 64, 8);
+    if (M <= 16) return tile(kGemmSwap, 16, 64, 4);
     if (M <= 32) return tile(kGemmSwap, 32, 64, 4);
     if (M <= 64) return tile(kGemmTile, 64, 64, 4);
     return tile(kGemmTile, kBM, 64, atoms ? 2 : 1);
@@ -1653,11 +1714,9 @@ cudaError_t launch_scaled_mm(const GemmArgs& g, const void* a, const void* b, in
     const GemmPlan p = plan_scaled_mm(g.M, g.N, g.K, false, sm_count);
     if (p.kernel == kGemmPair) return launch_pair(g, a, b, sm_count, stream);
     if (p.kernel == kGemmSwap) {
-        switch (p.a_rows) {
-            case 8: return launch_swap<8, 8>(g, a, b, sm_count, stream);
-            case 16: return launch_swap<16, 8>(g, a, b, sm_count, stream);
-            default: return launch_swap<32, 4>(g, a, b, sm_count, stream);
-        }
+        if (p.a_rows == 8) return launch_swap_pairk<8, 8>(g, a, b, sm_count, stream);
+        if (p.a_rows == 16) return launch_swap_pairk<16, 4>(g, a, b, sm_count, stream);
+        return launch_swap_pairk<32, 4>(g, a, b, sm_count, stream);
     }
     if (p.tile_n == 128) return launch_bn<128, kBM, 1>(g, a, b, sm_count, stream);
     if (p.a_rows == 64)

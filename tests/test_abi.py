@@ -503,7 +503,7 @@ def test_mx_blocked_rejects_partial_atoms(rrf):
 
 @pytest.mark.parametrize("M,N,K,mx,want", [
     (8, 16384, 7168, False, ("swap", 8, 64, 8, 256, 148)),
-    (16, 16384, 1024, False, ("swap", 16, 64, 8, 256, 148)),
+    (16, 16384, 1024, False, ("swap", 16, 64, 4, 256, 148)),
     (32, 16384, 7168, False, ("swap", 32, 64, 4, 256, 148)),
     (64, 16384, 7168, False, ("tile", 64, 64, 4, 256, 148)),
     (8, 16384, 1040, False, ("tile", 64, 64, 1, 256, 148)),   # K % 128 != 0: 2-D boxes

@@ -59,7 +59,10 @@ def check(c, got, rows=None, label=""):
 @pytest.mark.parametrize("M,N,K", [(1, 256, 128), (9, 512, 640), (24, 336, 1536),
                                    (5, 256, 144), (37, 256, 256), (128, 128, 128),
                                    (200, 272, 384), (130, 400, 144), (64, 1024, 1024),
-                                   (256, 512, 2048)])
+                                   (256, 512, 2048),
+                                   # an odd number of k-tiles after full boxes: the
+                                   # swapped kernel's last pair takes the box's zeros
+                                   (3, 320, 1152), (16, 208, 1408), (29, 128, 1664)])
 @pytest.mark.parametrize("bias", [True, False])
 def test_scaled_mm_matches_oracle(rrf, M, N, K, bias):
     c = workloads.make_gemm_case(M, N, K, sub=M % 7, bias=bias, device="cuda")
