@@ -527,9 +527,9 @@ rrf_status rrf_check_scaled_mm_args(const void* a, const float* a_scale, const v
 #define RRF_GEMM_KERNEL_PAIR 1 /* 256 x 256 tiles on SM pairs (two-CTA MMA)           */
 #define RRF_GEMM_KERNEL_TILE 2 /* one persistent CTA per SM walking 128 x tile_n output
                                   tiles, its A stages a_rows rows                     */
-#define RRF_GEMM_KERNEL_SWAP 3 /* per-token only: operands swapped, 64 weight rows of
-                                  each of two k-tiles on the MMA's M side, the call's
-                                  rows padded to a_rows                               */
+#define RRF_GEMM_KERNEL_SWAP 3 /* operands swapped, 64 weight rows of each of two
+                                  k-tiles on the MMA's M side, the call's rows padded
+                                  to a_rows (per-token and MX, at most 32 rows)       */
 
 /* rrf_plan_scaled_mm -- the kernel rrf_scaled_mm_fp8 (mx == 0) or
  * rrf_scaled_mm_mxfp8 (mx != 0) runs for an M x N x K product on a GPU with

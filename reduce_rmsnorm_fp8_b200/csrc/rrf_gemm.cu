@@ -11,7 +11,7 @@
 //            (BN 128 or 64), Z k-tiles per TMA box for short products;
 //   scaled_mm_swap_pairk_kernel  at most 32 rows against a weight, the
 //            operands swapped (the weight's rows on the MMA's M side, two
-//            k-tiles of them per instruction).
+//            k-tiles of them per instruction); per-token and MX forms.
 // A persistent CTA per SM walks 128 x BN tiles of out (BN 128 or 64).
 // Warp roles (the same in every kernel):
 //   warp 0   one thread issues the TMA loads of the A (128 x 128 bytes) and
@@ -430,6 +430,61 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// ------------------------------------------------ block-scaled MMA helpers --
+// The mx scenario's GEMM carries one E8M0 code per 32 values of K on both
+// operands, on tcgen05.mma kind::mxf8f6f4 with block scaling: the scale codes
+// of a k-tile (128 rows x 4 codes, one 512-byte atom of the blocked order:
+// row r's 4 codes at byte (r % 32) * 16 + (r / 32) * 4) are loaded next to
+// the A and B tiles, copied into tensor memory with tcgen05.cp (32 lanes x
+// 128 bits, repeated in the 4 lane quarters: lane l holds rows l, l+32,
+// l+64, l+96, 4 codes each, in 4 columns), and the k-tile's four MMAs take
+// code (k-step) of each 32-bit word.  Row r of an M = 128 operand reads
+// column r / 32 of lane r; column c of the N side reads column c / 32 of
+// lane c % 32.
+
+// 1-D bulk copy of `bytes` (a multiple of 16, both addresses 16-byte
+// aligned) into this CTA's shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Shared -> tensor memory: 32 rows of 16 bytes, repeated in the 4 lane quarters.
+__device__ __forceinline__ void tmem_copy_32x128b_x4(uint32_t taddr, uint64_t src_desc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(src_desc)
+                 : "memory");
+}
+
+// Descriptor of a scale atom as tcgen05.cp's source: 32 rows of 16 bytes,
+// contiguous, no swizzle (8-row core matrices 128 bytes apart).
+__device__ __forceinline__ uint64_t sf_atom_desc(const void* atom) {
+    const uint64_t addr = smem_u32(atom);
+    return ((addr >> 4) & 0x3FFFull) | ((128ull >> 4) << 32) | (1ull << 46);
+}
+
+__device__ __forceinline__ void mma_mx(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate, uint32_t sfa,
+                                       uint32_t sfb) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa),
+           "r"(sfb)
+        : "memory");
+}
+
+// Instruction descriptor of the block-scaled MMA: A and B e4m3 (0), K-major,
+// N = bn, M = 128, E8M0 scales (bit 23), scale codes taken from byte `id` of
+// the A and B scale words.
+__host__ __device__ constexpr uint32_t mx_idesc(int bn, uint32_t id) {
+    return (id << 4) | ((uint32_t)(bn >> 3) << 17) | (1u << 23) | ((uint32_t)(kBM >> 4) << 24) |
+           (id << 29);
+}
+
 // ------------------------------------- short products: the operands swapped --
 // A call of at most 32 rows against a weight (a decode batch): the weight's
 // rows are the MMA's M side and the call's rows its N side (NA = the rows
@@ -447,7 +502,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 // back from the producer.  An odd number of k-tiles pairs the last one with
 // the zeros the TMA box holds past K.  D[w][m] of the M = 128 layout sits in
 // tensor-memory lane w, column m.
-template <int NA, int Z>
+//
+// MX (block-scaled) form: the stage also holds the Z scale atoms of the
+// weight's 128-row block and the Z of the call's rows, and per pair of
+// k-tiles a seventh warp writes two atoms for the pair into the stage (off
+// the MMA issue path: the MMA thread waits for them per stage): the A
+// atom, line l = the weight tile's rows l and 32 + l for k-tile kt (the
+// tile's half of the block's atom), then the same rows for kt+1, so that A
+// row r reads its own k-tile's codes in column r / 32; and the B atom, whose
+// column c / 32, lane c % 32 holds call row c's codes for kt (c < NA) or row
+// c - NA's for kt+1.  The k-tile past an odd count takes kt's codes (its
+// data are zeros).
+template <int NA, int Z, bool MX = false>
 struct SwapPairTile {
     static_assert(NA == 8 || NA == 16 || NA == 32, "the call's rows: 8, 16 or 32");
     static_assert(Z % 2 == 0, "k-tiles go to the MMA in pairs");
@@ -455,22 +521,38 @@ struct SwapPairTile {
     static constexpr int kWBytes = kWRows * kBK;       // one k-tile of the weight: 8 KB
     static constexpr int kXBytes = NA * kBK;           // one k-tile of the call's rows
     static constexpr int kXOffset = Z * kWBytes;
-    static constexpr int kStageBytes = Z * (kWBytes + kXBytes);
+    static constexpr int kSfBytes = 512;               // one scale atom
+    static constexpr int kSfwOffset = Z * (kWBytes + kXBytes);   // the weight's atoms
+    static constexpr int kSfxOffset = kSfwOffset + Z * kSfBytes;  // the call's atoms
+    static constexpr int kPairOffset = kSfxOffset + Z * kSfBytes; // per pair: A, B atoms
+    static constexpr int kStageBytes =
+        MX ? kPairOffset + (Z / 2) * 2 * kSfBytes : Z * (kWBytes + kXBytes);
+    static constexpr int kStageStride = (kStageBytes + 1023) / 1024 * 1024;
     static constexpr int kCombBytes = NA * kWRows * 4;  // the odd block, handed between warps
-    static constexpr int kStages = (218 * 1024 - kCombBytes) / kStageBytes > 12
+    static constexpr int kStages = (218 * 1024 - kCombBytes) / kStageStride > 12
                                        ? 12
-                                       : (218 * 1024 - kCombBytes) / kStageBytes;
-    // two accumulators of 2 NA columns (a power of two of at least 32)
+                                       : (218 * 1024 - kCombBytes) / kStageStride;
+    // two accumulators of 2 NA columns (a power of two of at least 32), then
+    // (MX) 4 + 4 scale columns; the allocation a power of two
     static constexpr int kAccStride = 2 * NA < 32 ? 32 : 2 * NA;
-    static constexpr int kTmemCols = 2 * kAccStride;
-    // full / empty per stage, full / empty per accumulator, the drain, and
-    // the odd block's full / empty
-    static constexpr int kBarriers = 2 * kStages + 4 + 1 + 2;
+    static constexpr int kUsedCols = 2 * kAccStride + (MX ? 8 : 0);
+    static constexpr int kTmemCols = kUsedCols <= 64 ? 64 : kUsedCols <= 128 ? 128 : 256;
+    // full / empty per stage, full / empty per accumulator, the drain, the
+    // odd block's full / empty, and (MX) the pair atoms written per stage
+    static constexpr int kBarriers = (MX ? 3 : 2) * kStages + 4 + 1 + 2;
+    // the MX form adds a seventh warp that writes the pair atoms
+    static constexpr int kThreadsPerCta = MX ? kThreads + 32 : kThreads;
     static constexpr int kSmemBytes =
-        1024 + kStages * kStageBytes + kCombBytes + kBarriers * 8 + 16;
+        1024 + kStages * kStageStride + kCombBytes + kBarriers * 8 + 16;
     static_assert(kSmemBytes <= 227 * 1024, "stages exceed the shared memory of a CTA");
     static_assert(kXBytes % 1024 == 0, "each k-tile must start on a swizzle atom");
 };
+
+// Make this thread's shared-memory stores visible to the async proxy
+// (tcgen05.cp reads them).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 
 // NA consecutive fp32 accumulator columns of this thread's lane (NA = 8, 16
 // or 32).
@@ -502,24 +584,28 @@ __device__ __forceinline__ void tmem_load_cols(uint32_t taddr, float v[NA]) {
     }
 }
 
-template <int NA, int Z>
-__global__ void __launch_bounds__(kThreads, 1)
+// sfx, sfw: the MX form's scale codes of the call's rows and of the weight
+// (the blocked order); null in the per-token form.
+template <int NA, int Z, bool MX>
+__global__ void __launch_bounds__(SwapPairTile<NA, Z, MX>::kThreadsPerCta, 1)
     scaled_mm_swap_pairk_kernel(const __grid_constant__ CUtensorMap tma_x,
-                                const __grid_constant__ CUtensorMap tma_w, const GemmArgs g) {
-    using T = SwapPairTile<NA, Z>;
+                                const __grid_constant__ CUtensorMap tma_w, const GemmArgs g,
+                                const uint8_t* sfx, const uint8_t* sfw) {
+    using T = SwapPairTile<NA, Z, MX>;
     constexpr int S = T::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
-    float* comb = reinterpret_cast<float*>(ring + S * T::kStageBytes);  // [NA][64]
-    uint64_t* full = reinterpret_cast<uint64_t*>(ring + S * T::kStageBytes + T::kCombBytes);
+    float* comb = reinterpret_cast<float*>(ring + S * T::kStageStride);  // [NA][64]
+    uint64_t* full = reinterpret_cast<uint64_t*>(ring + S * T::kStageStride + T::kCombBytes);
     uint64_t* empty = full + S;
     uint64_t* acc_full = empty + S;
     uint64_t* acc_empty = acc_full + 2;
     uint64_t* drained = acc_empty + 2;
     uint64_t* comb_full = drained + 1;     // the odd block is in comb (64 threads arrive)
     uint64_t* comb_empty = comb_full + 1;  // comb was read (64 threads arrive)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(comb_empty + 1);
+    uint64_t* built = comb_empty + 1;      // (MX) a stage's pair atoms are written
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(built + (MX ? S : 0));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tiles = (g.N + T::kWRows - 1) / T::kWRows;
@@ -538,6 +624,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(drained, 1);
         mbar_init(comb_full, 64);
         mbar_init(comb_empty, 64);
+        if constexpr (MX)
+            for (int s = 0; s < S; ++s) mbar_init(&built[s], 32);
         fence_mbar_init_cluster();
     }
     if (warp == 1) {
@@ -565,14 +653,119 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    uint8_t* dst = ring + s * T::kStageBytes;
-                    mbar_arrive_expect_tx(&full[s], T::kStageBytes);
-                    tma_load_3d(dst, &tma_w, &full[s], 0, n0, kg * Z);
-                    tma_load_3d(dst + T::kXOffset, &tma_x, &full[s], 0, 0, kg * Z);
+                    uint8_t* dst = ring + s * T::kStageStride;
+                    if constexpr (MX) {
+                        // the scale atoms of the group's k-tiles inside K (a
+                        // 1-D copy must not run past the row block's atoms)
+                        const int nk = ktiles - kg * Z < Z ? ktiles - kg * Z : Z;
+                        const uint32_t sf_bytes = (uint32_t)(nk * T::kSfBytes);
+                        mbar_arrive_expect_tx(&full[s],
+                                              Z * (T::kWBytes + T::kXBytes) + 2 * sf_bytes);
+                        tma_load_3d(dst, &tma_w, &full[s], 0, n0, kg * Z);
+                        tma_load_3d(dst + T::kXOffset, &tma_x, &full[s], 0, 0, kg * Z);
+                        bulk_load(dst + T::kSfwOffset,
+                                  sfw + ((int64_t)(n0 / 128) * ktiles + kg * Z) * T::kSfBytes,
+                                  sf_bytes, &full[s]);
+                        bulk_load(dst + T::kSfxOffset, sfx + (int64_t)kg * Z * T::kSfBytes,
+                                  sf_bytes, &full[s]);
+                    } else {
+                        mbar_arrive_expect_tx(&full[s], T::kStageBytes);
+                        tma_load_3d(dst, &tma_w, &full[s], 0, n0, kg * Z);
+                        tma_load_3d(dst + T::kXOffset, &tma_x, &full[s], 0, 0, kg * Z);
+                    }
                 }
             }
             for (int i = it > S ? it - S : 0; i < it; ++i)
                 wait_phase(&full[i % S], (i / S) & 1, g.err);
+        }
+    } else if (warp == 1 && MX) {
+        // ---- MX: one thread copies each pair's scale atoms (written by the
+        // seventh warp) into tensor memory and issues the block-scaled MMAs
+        // D[128 x 2NA] += A[128 x 32] * B[2NA x 32]^T
+        if (lane == 0) {
+            const uint32_t tmem_sfw = tmem + 2 * T::kAccStride, tmem_sfx = tmem_sfw + 4;
+            int it = 0, j = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++j) {
+                const int buf = j & 1;
+                if (!wait_phase(&acc_empty[buf], ((j >> 1) & 1) ^ 1, g.err)) break;
+                tc_fence_after_sync();
+                const uint32_t d = tmem + (uint32_t)(buf * T::kAccStride);
+                for (int kg = 0; kg < kgroups; ++kg, ++it) {
+                    const int s = it % S;
+                    if (!wait_phase(&full[s], (it / S) & 1, g.err) ||
+                        !wait_phase(&built[s], (it / S) & 1, g.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint8_t* stage = ring + s * T::kStageStride;
+                    const int nk = ktiles - kg * Z < Z ? ktiles - kg * Z : Z;
+                    for (int kj = 0; kj < nk; kj += 2) {
+                        const uint8_t* pair = stage + T::kPairOffset + kj * T::kSfBytes;
+                        // tcgen05 operations of this thread run in issue order
+                        // (see scaled_mm_mx_kernel)
+                        tmem_copy_32x128b_x4(tmem_sfw, sf_atom_desc(pair));
+                        tmem_copy_32x128b_x4(tmem_sfx, sf_atom_desc(pair + T::kSfBytes));
+                        const uint64_t wd = kmajor_sw128_desc(stage + kj * T::kWBytes);
+                        const uint64_t xd = kmajor_sw128_desc(stage + T::kXOffset + kj * T::kXBytes);
+#pragma unroll
+                        for (int k = 0; k < kBK / kMmaK; ++k) {
+                            const uint64_t step = (uint64_t)(k * kMmaK) >> 4;
+                            mma_mx(d, wd + step, xd + step, mx_idesc(2 * NA, (uint32_t)k),
+                                   (kg | kj | k) != 0, tmem_sfw, tmem_sfx);
+                        }
+                    }
+                    mma_commit(&empty[s]);
+                }
+                mma_commit(&acc_full[buf]);
+            }
+            mma_commit(drained);
+        }
+        __syncwarp();
+    } else if (MX && warp == kThreads / 32) {
+        // ---- MX, the seventh warp: once a stage has landed, each lane writes
+        // line `lane` of every pair's A and B atoms, makes its stores visible
+        // to the async proxy and arrives on the stage's `built` barrier
+        int it = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+            const int half = t & 1;  // the tile's 64 rows in the weight's 128-row block
+            for (int kg = 0; kg < kgroups; ++kg, ++it) {
+                const int s = it % S;
+                if (!__all_sync(0xFFFFFFFFu, wait_phase(&full[s], (it / S) & 1, g.err))) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* stage = ring + s * T::kStageStride;
+                const int nk = ktiles - kg * Z < Z ? ktiles - kg * Z : Z;
+                constexpr int kWords = T::kSfBytes / 4;
+                for (int kj = 0; kj < nk; kj += 2) {
+                    const uint32_t* w0 =
+                        reinterpret_cast<const uint32_t*>(stage + T::kSfwOffset + kj * T::kSfBytes);
+                    const uint32_t* x0 =
+                        reinterpret_cast<const uint32_t*>(stage + T::kSfxOffset + kj * T::kSfBytes);
+                    const uint32_t* w1 = kj + 1 < nk ? w0 + kWords : w0;
+                    const uint32_t* x1 = kj + 1 < nk ? x0 + kWords : x0;
+                    uint32_t* pa =
+                        reinterpret_cast<uint32_t*>(stage + T::kPairOffset + kj * T::kSfBytes);
+                    uint32_t* pb = pa + kWords;
+                    // line `lane` of each atom (16 bytes: 4 words)
+                    pa[4 * lane + 0] = w0[4 * lane + 2 * half];
+                    pa[4 * lane + 1] = w0[4 * lane + 2 * half + 1];
+                    pa[4 * lane + 2] = w1[4 * lane + 2 * half];
+                    pa[4 * lane + 3] = w1[4 * lane + 2 * half + 1];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int c = 32 * q + lane;  // a column of B (call rows < 32: word 0)
+                        pb[4 * lane + q] = c < NA       ? x0[4 * c]
+                                           : c < 2 * NA ? x1[4 * (c - NA)]
+                                                        : 0x7F7F7F7Fu;  // unread: 2^0
+                    }
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&built[s]);  // each lane releases its own stores
+            }
         }
     } else if (warp == 1) {
         // ---- MMA issue: D[128 x 2NA] += A[128 x 32] * B[2NA x 32]^T, A and B
@@ -593,7 +786,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint8_t* stage = ring + s * T::kStageBytes;
+                    const uint8_t* stage = ring + s * T::kStageStride;
                     const int nk = ktiles - kg * Z < Z ? ktiles - kg * Z : Z;
                     for (int kj = 0; kj < nk; kj += 2) {
                         const uint64_t wd = kmajor_sw128_desc(stage + kj * T::kWBytes);
@@ -616,7 +809,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // 32q+31 of D: quarters 0, 1 the even block's weight rows 0-63,
         // quarters 2, 3 the odd block's; the odd warps hand their NA values
         // per row to the even warps through shared memory, which add them,
-        // scale and store (weight row w of the tile is output column n)
+        // scale (per-token form; the MX form's scales act inside the MMA)
+        // and store (weight row w of the tile is output column n)
         const int quarter = warp & 3;
         const bool odd = quarter >= 2;
         const int w = (quarter & 1) * 32 + lane;
@@ -648,15 +842,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int m = 0; m < NA; ++m) o[m] = comb[m * T::kWRows + w];
                 mbar_arrive(comb_empty);
                 if (ok && n < g.N && RRF_IN_BOUNDS(n >= 0, g.err)) {
-                    const float sb = g.b_scale[n];
+                    const float sb = MX ? 1.0f : g.b_scale[n];
                     const float bias =
                         g.bias != nullptr ? __uint_as_float((uint32_t)g.bias[n] << 16) : 0.0f;
 #pragma unroll
                     for (int m = 0; m < NA; ++m) {
                         if (m < g.M) {
-                            float y = __fmul_rn(__fmul_rn(__fadd_rn(v[m], o[m]),
-                                                          __ldg(g.a_scale + m)),
-                                                sb);
+                            float y = __fadd_rn(v[m], o[m]);
+                            if constexpr (!MX) y = __fmul_rn(__fmul_rn(y, __ldg(g.a_scale + m)), sb);
                             if (g.bias != nullptr) y = __fadd_rn(y, bias);
                             g.out[(int64_t)m * g.N + n] =
                                 (uint16_t)(f32x2_to_bf16x2(y, 0.0f) & 0xFFFFu);
@@ -935,55 +1128,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------- MX (block-scaled) GEMM kernel --
 // out = (a * 2^(sa - 127)) @ (b * 2^(sb - 127))^T + bias with one E8M0 code
-// per 32 values of K (the mx scenario), on tcgen05.mma kind::mxf8f6f4 with
-// block scaling: the scale codes of a k-tile (128 rows x 4 codes, one
-// 512-byte atom of the blocked order) are loaded next to the A and B tiles,
-// copied into tensor memory with tcgen05.cp (32 lanes x 128 bits, repeated
-// in the 4 lane quarters: lane l holds rows l, l+32, l+64, l+96, 4 codes
-// each), and the k-tile's four MMAs take code (k-step) of each 32-bit word.
-
-// 1-D bulk copy of `bytes` (a multiple of 16, both addresses 16-byte
-// aligned) into this CTA's shared memory, completing on `bar`.
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
-                                          uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-        :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
-// Shared -> tensor memory: 32 rows of 16 bytes, repeated in the 4 lane quarters.
-__device__ __forceinline__ void tmem_copy_32x128b_x4(uint32_t taddr, uint64_t src_desc) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(src_desc)
-                 : "memory");
-}
-
-// Descriptor of a scale atom as tcgen05.cp's source: 32 rows of 16 bytes,
-// contiguous, no swizzle (8-row core matrices 128 bytes apart).
-__device__ __forceinline__ uint64_t sf_atom_desc(const void* atom) {
-    const uint64_t addr = smem_u32(atom);
-    return ((addr >> 4) & 0x3FFFull) | ((128ull >> 4) << 32) | (1ull << 46);
-}
-
-__device__ __forceinline__ void mma_mx(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate, uint32_t sfa,
-                                       uint32_t sfb) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
-        :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa),
-           "r"(sfb)
-        : "memory");
-}
-
-// Instruction descriptor of the block-scaled MMA: A and B e4m3 (0), K-major,
-// N = bn, M = 128, E8M0 scales (bit 23), scale codes taken from byte `id` of
-// the A and B scale words.
-__host__ __device__ constexpr uint32_t mx_idesc(int bn, uint32_t id) {
-    return (id << 4) | ((uint32_t)(bn >> 3) << 17) | (1u << 23) | ((uint32_t)(kBM >> 4) << 24) |
-           (id << 29);
-}
+// per 32 values of K (the mx scenario), the scale atoms handled as the
+// block-scaled MMA helpers above describe.
 
 // BN 128 or 64 columns per tile; AROWS and Z (k-tiles per stage, one 3-D
 // TMA box per operand) as for the per-token kernel (64-row A: the MMA's rows
@@ -1491,14 +1637,15 @@ cudaError_t launch_on_pairs(void (*kernel)(Params...), int64_t pairs, int smem_b
     return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-// One CTA per SM (at most `ctas`), launched with programmatic dependent
-// launch: the kernel's set-up may overlap the previous kernel of the stream.
+// One CTA per SM (at most `ctas`) of `threads` threads, launched with
+// programmatic dependent launch: the kernel's set-up may overlap the previous
+// kernel of the stream.
 template <class... Params, class... Args>
-cudaError_t launch_persistent(void (*kernel)(Params...), unsigned ctas, int smem_bytes,
-                              cudaStream_t stream, Args... args) {
+cudaError_t launch_persistent_threads(void (*kernel)(Params...), unsigned ctas, int threads,
+                                      int smem_bytes, cudaStream_t stream, Args... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(ctas, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.blockDim = dim3(threads, 1, 1);
     cfg.dynamicSmemBytes = smem_bytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -1507,6 +1654,13 @@ cudaError_t launch_persistent(void (*kernel)(Params...), unsigned ctas, int smem
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// The same with the GEMM kernels' kThreads threads per CTA.
+template <class... Params, class... Args>
+cudaError_t launch_persistent(void (*kernel)(Params...), unsigned ctas, int smem_bytes,
+                              cudaStream_t stream, Args... args) {
+    return launch_persistent_threads(kernel, ctas, kThreads, smem_bytes, stream, args...);
 }
 
 // A [rows, K] byte matrix, box of 128 bytes x box_rows rows, 128-byte swizzle;
@@ -1579,19 +1733,23 @@ cudaError_t launch_bn(const GemmArgs& g, const void* a, const void* b, int sm_co
     return launch_persistent(kernel, grid, T::kSmemBytes, stream, ma, mb, g);
 }
 
-template <int NA, int Z>
+// sfa, sfb: the MX form's scale codes of a and b (the blocked order), else
+// null.
+template <int NA, int Z, bool MX = false>
 cudaError_t launch_swap_pairk(const GemmArgs& g, const void* a, const void* b, int sm_count,
-                              cudaStream_t stream) {
-    using T = SwapPairTile<NA, Z>;
+                              cudaStream_t stream, const uint8_t* sfa = nullptr,
+                              const uint8_t* sfb = nullptr) {
+    using T = SwapPairTile<NA, Z, MX>;
     CUtensorMap mx, mw;
     if (!make_map3(&mx, a, g.M, g.K, NA, Z) || !make_map3(&mw, b, g.N, g.K, T::kWRows, Z))
         return cudaErrorInvalidValue;
-    constexpr auto kernel = scaled_mm_swap_pairk_kernel<NA, Z>;
+    constexpr auto kernel = scaled_mm_swap_pairk_kernel<NA, Z, MX>;
     const cudaError_t e = enable_dynamic_smem<kernel>(T::kSmemBytes);
     if (e != cudaSuccess) return e;
     const int64_t tiles = (g.N + T::kWRows - 1) / T::kWRows;
     const unsigned grid = (unsigned)(tiles < sm_count ? tiles : sm_count);
-    return launch_persistent(kernel, grid, T::kSmemBytes, stream, mx, mw, g);
+    return launch_persistent_threads(kernel, grid, T::kThreadsPerCta, T::kSmemBytes, stream, mx,
+                                     mw, g, sfa, sfb);
 }
 
 cudaError_t launch_pair(const GemmArgs& g, const void* a, const void* b, int sm_count,
@@ -1663,13 +1821,12 @@ GemmPlan plan_scaled_mm(int64_t M, int64_t N, int64_t K, bool mx, int sm_count) 
         // else one CTA per 128 x 128 tile once those fill every SM; short, wide
         // problems take 128 x 64 tiles (A stages of the call's rows, up to 64)
         if (row_tiles * ((N + 127) / 128) >= sm_count) return tile(kGemmTile, kBM, 128, 1);
-        // (K % 128 == 0 here: several k-tiles per TMA box, as the per-token GEMM;
-        // no swapped operands: the block-scaled MMA of one CTA has no M = 64 form)
-        // 8 k-tiles per stage up to 16 rows (2 stages; measured 7% faster than 4
-        // at 8 rows, 2 k-tiles slower)
-        if (M <= 8) return tile(kGemmTile, 8, 64, 8);
-        if (M <= 16) return tile(kGemmTile, 16, 64, 8);
-        if (M <= 32) return tile(kGemmTile, 32, 64, 4);
+        // (K % 128 == 0 here: several k-tiles per TMA box, as the per-token GEMM)
+        // at most 32 rows: the operands swapped, two k-tiles per MMA (M = 128
+        // over two weight k-tiles, the scale atoms rebuilt per pair)
+        if (M <= 8) return tile(kGemmSwap, 8, 64, 4);
+        if (M <= 16) return tile(kGemmSwap, 16, 64, 4);
+        if (M <= 32) return tile(kGemmSwap, 32, 64, 4);
         if (M <= 64) return tile(kGemmTile, 64, 64, 4);
         return tile(kGemmTile, kBM, 64, 2);
     }
@@ -1699,14 +1856,15 @@ cudaError_t launch_scaled_mm_mx(const GemmArgs& g, const void* a, const void* b,
                                 cudaStream_t stream) {
     const GemmPlan p = plan_scaled_mm(g.M, g.N, g.K, true, sm_count);
     if (p.kernel == kGemmPair) return launch_mx_pair(g, a, b, sfa, sfb, sm_count, stream);
-    if (p.tile_n == 128) return launch_mx<128, kBM, 1>(g, a, b, sfa, sfb, sm_count, stream);
-    switch (p.a_rows) {
-        case 8: return launch_mx<64, 8, 8>(g, a, b, sfa, sfb, sm_count, stream);
-        case 16: return launch_mx<64, 16, 8>(g, a, b, sfa, sfb, sm_count, stream);
-        case 32: return launch_mx<64, 32, 4>(g, a, b, sfa, sfb, sm_count, stream);
-        case 64: return launch_mx<64, 64, 4>(g, a, b, sfa, sfb, sm_count, stream);
-        default: return launch_mx<64, kBM, 2>(g, a, b, sfa, sfb, sm_count, stream);
+    if (p.kernel == kGemmSwap) {
+        if (p.a_rows == 8) return launch_swap_pairk<8, 4, true>(g, a, b, sm_count, stream, sfa, sfb);
+        if (p.a_rows == 16)
+            return launch_swap_pairk<16, 4, true>(g, a, b, sm_count, stream, sfa, sfb);
+        return launch_swap_pairk<32, 4, true>(g, a, b, sm_count, stream, sfa, sfb);
     }
+    if (p.tile_n == 128) return launch_mx<128, kBM, 1>(g, a, b, sfa, sfb, sm_count, stream);
+    if (p.a_rows == 64) return launch_mx<64, 64, 4>(g, a, b, sfa, sfb, sm_count, stream);
+    return launch_mx<64, kBM, 2>(g, a, b, sfa, sfb, sm_count, stream);
 }
 
 cudaError_t launch_scaled_mm(const GemmArgs& g, const void* a, const void* b, int sm_count,

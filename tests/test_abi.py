@@ -511,7 +511,8 @@ def test_mx_blocked_rejects_partial_atoms(rrf):
     (64, 7168, 7168, False, ("tile", 64, 64, 4, 112, 112)),
     (2048, 2048, 512, False, ("tile", 128, 128, 1, 256, 148)),
     (8192, 8192, 8192, False, ("pair", 256, 256, 1, 1024, 148)),
-    (8, 16384, 1024, True, ("tile", 8, 64, 8, 256, 148)),
+    (8, 16384, 1024, True, ("swap", 8, 64, 4, 256, 148)),
+    (32, 7168, 7168, True, ("swap", 32, 64, 4, 112, 112)),
     (64, 16384, 7168, True, ("tile", 64, 64, 4, 256, 148)),
     (100, 16384, 1024, True, ("tile", 128, 64, 2, 256, 148)),
     (2048, 2048, 512, True, ("tile", 128, 128, 1, 256, 148)),
@@ -532,7 +533,7 @@ def test_gemm_plan_invariants_and_rejections(rrf):
                     p = rrf.rrf_plan_scaled_mm(M, N, K, 148, mx=mx)
                     assert 1 <= p["ctas"] <= min(p["tiles"] * (2 if p["kernel"] == "pair" else 1),
                                                  148)
-                    assert p["kernel"] != "swap" or (not mx and M <= p["a_rows"] <= 32)
+                    assert p["kernel"] != "swap" or M <= p["a_rows"] <= 32
                     if p["kernel"] == "pair":
                         assert p["ctas"] % 2 == 0
     p = rrf.rrf_plan_scaled_mm(0, 256, 256, 148)

@@ -139,7 +139,10 @@ def check_mx_gemm(c, sa, sb, got, rows=None, label=""):
 
 @pytest.mark.parametrize("M,N,K", [(1, 128, 128), (8, 384, 512), (13, 320, 1024),
                                    (32, 448, 640), (37, 256, 256), (128, 128, 512),
-                                   (200, 272, 384), (130, 400, 1024), (256, 512, 2048)])
+                                   (200, 272, 384), (130, 400, 1024), (256, 512, 2048),
+                                   # an odd number of k-tiles after full boxes: the
+                                   # swapped kernel's last pair takes the box's zeros
+                                   (3, 256, 1152), (24, 384, 1408)])
 @pytest.mark.parametrize("bias", [True, False])
 def test_mx_gemm_matches_oracle(rrf, M, N, K, bias):
     c, sa, sb = mx_operands(M, N, K, M % 5, bias)
@@ -179,14 +182,16 @@ def test_mx_gemm_large_sampled_rows(rrf, M, N, K):
 @pytest.mark.parametrize("M,N,K", [(8, 16384, 1024), (16, 16384, 1024), (24, 16384, 1024),
                                    (64, 16384, 7168), (100, 16384, 1024)])
 def test_mx_gemm_several_tiles_per_cta(rrf, M, N, K):
-    """More 128 x 64 output tiles than CTAs (N = 16384: 256 tiles on at most
+    """More 64-column output tiles than CTAs (N = 16384: 256 tiles on at most
     one CTA per SM), so each persistent CTA walks several tiles with its
-    stage ring, both accumulators and the odd tiles' second scale column:
-    the 8-, 16-, 32-, 64- and 128-row A-stage kernels; sampled rows, every
-    column, against the oracle."""
+    stage ring, both accumulators and the odd tiles' half of the weight's
+    scale atoms: the swapped kernel at 8, 16 and 32 rows, the 64- and
+    128-row A-stage kernels; sampled rows, every column, against the
+    oracle."""
     sm = torch.cuda.get_device_properties(0).multi_processor_count
     p = rrf.rrf_plan_scaled_mm(M, N, K, sm, mx=True)
-    assert p["kernel"] == "tile" and p["tile_n"] == 64 and p["tiles"] > p["ctas"], p
+    want = "swap" if M <= 32 else "tile"
+    assert p["kernel"] == want and p["tile_n"] == 64 and p["tiles"] > p["ctas"], p
     c, sa, sb = mx_operands(M, N, K, 8)
     out = rrf.rrf_scaled_mm_mxfp8(c.a, rrf.mx_blocked(torch.from_numpy(sa).cuda()), c.b,
                                   rrf.mx_blocked(torch.from_numpy(sb).cuda()), c.bias)
