@@ -935,7 +935,7 @@ def run_rrf(args):
         gemm.append(time_gemm(rrf, 8192, 8192, 8192, device, stream, l2, peak))
         torch.cuda.empty_cache()
         gemm_mx = [time_gemm_mx(rrf, M, N, N, device, stream, l2, peak)
-                   for M, N in ((64, 7168), (8192, 8192))]
+                   for M, N in ((1, 7168), (8, 7168), (32, 7168), (64, 7168), (8192, 8192))]
         torch.cuda.empty_cache()
 
     cpu = None
