@@ -997,28 +997,27 @@ def run_rrf(args):
 
 def run_reference(args):
     """The oracle as the reference arm: rank 0 times it on the host cores.
-    Each step is a bounded sample of one step of the workload: the first two
-    rows of every call (rows are independent, so GB/s over the sample is the
-    oracle's throughput on the workload)."""
+    Each step is a bounded sample of one step of the workload: the first
+    2 x cores rows of every call, split into contiguous chunks over one
+    POSIX thread per core (the oracle's row-parallel driver of its per-row
+    function; rows are independent, so GB/s over the sample is the oracle's
+    throughput on the workload)."""
     rank, _, world = dist_env()
     if rank != 0:
         return
     name = args.workload
     w = workloads.WORKLOADS[name]
     import oracle
-    bits = workloads.bits
-    cases = [workloads.make_case(name, rows) if name != "prefill" else
-             workloads.make_case(name, 8, sub=0) for rows, _ in workload_cases(name)]
-    prepared = [([bits(x[:2]) for x in c.inputs],
-                 None if c.residual is None else bits(c.residual[:2]), bits(c.gamma), c)
-                for c in cases]
-    per_step = sum(workloads.fused_bytes(w.R, min(2, c.rows), w.cols, w.residual)
-                   for c in cases)
+    o = oracle.default()
+    cores = o.cores()
+    rows_list = [min(r, 2 * cores) for r, _ in workload_cases(name)]
+    prepared = [_oracle_sample(name, r) for r in rows_list]
+    per_step = sum(workloads.fused_bytes(w.R, r, w.cols, w.residual) for r in rows_list)
 
     def step():
         for xs, res, g, c in prepared:
-            oracle.sum_rmsnorm_fp8(xs, min(2, c.rows), c.cols, g, c.eps, c.weight_offset,
-                                   c.scale_ub, residual=res)
+            o.sum_rmsnorm_fp8_mt(xs, c.rows, c.cols, g, c.eps, c.weight_offset, c.scale_ub,
+                                 residual=res, threads=cores)
 
     for _ in range(args.warmup):
         step()
@@ -1027,7 +1026,9 @@ def run_reference(args):
         step()
     dt = time.perf_counter() - t0
     value = per_step * args.steps / dt / 1e9
-    sample = f"first 2 rows of each of the {len(cases)} calls per step"
+    sample = (f"first {', '.join(str(r) for r in rows_list)} rows of the "
+              f"{len(rows_list)} call(s) per step, {cores} POSIX threads (the cores of this "
+              f"process's CPU affinity), one contiguous row chunk each")
     line = {"metric": METRIC, "value": round(value, 6), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
@@ -1036,7 +1037,7 @@ def run_reference(args):
             "config": {"workload": f"{name}: R={w.R}, cols={w.cols}, rows {list(w.rows)} "
                                    f"per step, residual={'on' if w.residual else 'off'}",
                        "sample": sample},
-            "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": 1,
+            "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": cores,
                              "kind": "oracle", "sample": f"{args.steps} steps, {sample}"},
             "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
