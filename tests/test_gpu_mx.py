@@ -142,7 +142,10 @@ def check_mx_gemm(c, sa, sb, got, rows=None, label=""):
                                    (200, 272, 384), (130, 400, 1024), (256, 512, 2048),
                                    # an odd number of k-tiles after full boxes: the
                                    # swapped kernel's last pair takes the box's zeros
-                                   (3, 256, 1152), (24, 384, 1408)])
+                                   (3, 256, 1152), (24, 384, 1408),
+                                   # a last weight tile in the odd half of its scale
+                                   # block, 16 of its 64 rows inside N
+                                   (5, 208, 256)])
 @pytest.mark.parametrize("bias", [True, False])
 def test_mx_gemm_matches_oracle(rrf, M, N, K, bias):
     c, sa, sb = mx_operands(M, N, K, M % 5, bias)
