@@ -13,7 +13,8 @@
 //            operands swapped (the weight's rows on the MMA's M side, two
 //            k-tiles of them per instruction); per-token and MX forms.
 // A persistent CTA per SM walks 128 x BN tiles of out (BN 128 or 64).
-// Warp roles (the same in every kernel):
+// Warp roles (the same in every kernel; the swapped kernel's MX form adds a
+// seventh warp that rearranges the scale codes of each stage):
 //   warp 0   one thread issues the TMA loads of the A (128 x 128 bytes) and
 //            B (BN x 128 bytes) k-tiles into a ring of shared-memory stages
 //            (128-byte swizzle, the layout the MMA descriptors name);
