@@ -53,7 +53,7 @@ def test_fused_call_alias_rule(rrf, R, rows, cols, residual, slots):
         res_out = res_in
     bf16 = rows * cols * 2
     reads = [(p, bf16) for p in inputs] + [(gamma, cols * 2)]
-    if residual == "separate":
+    if residual != "none" and res_in != res_out:  # equal pointers are in place
         reads.append((res_in, bf16))
     writes = [(q, rows * cols), (scales, rows * 4)]
     if residual != "none":
@@ -109,3 +109,50 @@ def test_fused_call_alignment_rule(rrf, rows, cols, which, offset):
                                   BASE + step, 1e-5, 0.0, 1200.0, BASE + 2 * step,
                                   BASE + 5 * step + 4 * (offset % 2 == 0))
     assert ok == rrf.Status.OK
+
+
+@SETTINGS
+@given(world=st.integers(1, 4), rows=st.integers(1, 4), cols=st.sampled_from([8, 16, 64]),
+       residual=st.sampled_from(["none", "separate", "in_place", "mixed"]),
+       near_signal=st.booleans(), slots=st.lists(addr, min_size=22, max_size=22))
+def test_allreduce_alias_rule(rrf, world, rows, cols, residual, near_signal, slots):
+    """The multi-GPU call: no write (codes, scales, signal pads, residual
+    outputs) may overlap a read (inputs, gamma, residual inputs not written
+    in place) or another write, and a residual written in place serves only
+    its own rank."""
+    sig_words = rrf.RRF_AR_SIGNAL_WORDS
+    gamma = slots[0]
+    inputs = slots[1:1 + world]
+    q = slots[5:5 + world]
+    scales = slots[9:9 + world]
+    res_in = slots[13:13 + world]
+    res_out = slots[17:17 + world]
+    # signal pads far apart (their 4 * RRF_AR_SIGNAL_WORDS bytes would cover
+    # the small space), or one of them inside it
+    signals = [BASE + (1 << 22) * (j + 1) for j in range(world)]
+    if near_signal:
+        signals[0] = slots[21]
+    if residual == "none":
+        res_in = res_out = None
+    elif residual == "in_place":
+        res_out = list(res_in)
+    elif residual == "mixed":
+        res_out = [res_in[j] if j % 2 == 0 else res_out[j] for j in range(world)]
+    bf16 = rows * cols * 2
+    reads = [(gamma, cols * 2)] + [(p, bf16) for p in inputs]
+    writes = []
+    for j in range(world):
+        if res_in is not None and res_in[j] != res_out[j]:
+            reads.append((res_in[j], bf16))
+        writes += [(q[j], rows * cols), (scales[j], rows * 4), (signals[j], sig_words * 4)]
+        if res_in is not None:
+            writes.append((res_out[j], bf16))
+    alias = any_alias(writes, reads)
+    if res_in is not None and not alias:
+        alias = any(i != j and overlaps((res_out[j], bf16), (res_in[i], bf16))
+                    for j in range(world) for i in range(world))
+    want = rrf.Status.ERR_ALIAS if alias else rrf.Status.OK
+    got = rrf.rrf_check_allreduce_args(inputs, res_in, res_out, q, scales, signals, 0, 1,
+                                       rows, cols, gamma, 1e-5, 0.0, 1200.0,
+                                       rrf.RRF_AR_AUTO, world=world)
+    assert got == want, (got, want)
