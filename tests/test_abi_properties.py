@@ -4,6 +4,8 @@ overlap often, and the library's verdict is compared with the rule the
 header states for each call -- an output may overlap no input and no other
 output, except the residual written in place (residual_out == residual_in).
 Validation never dereferences the pointers."""
+import os
+
 import pytest
 from hypothesis import HealthCheck, given, settings
 from hypothesis import strategies as st
@@ -11,7 +13,10 @@ from hypothesis import strategies as st
 BASE = 1 << 24   # fake addresses: BASE + 16 * slot
 SLOTS = 64       # a small space, so that overlaps are common
 
-SETTINGS = settings(max_examples=400, deadline=None,
+# a fixed seed, so that every run checks the same layouts (RRF_PROPERTY_EXAMPLES
+# raises the count for a longer search)
+SETTINGS = settings(max_examples=int(os.environ.get("RRF_PROPERTY_EXAMPLES", "400")),
+                    deadline=None, derandomize=True, database=None,
                     suppress_health_check=[HealthCheck.function_scoped_fixture])
 
 
